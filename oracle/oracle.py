@@ -1,0 +1,195 @@
+"""ctypes front end of the fp64 CPU oracle for the Gated DeltaNet mixer.
+
+TEST INFRASTRUCTURE ONLY: the test suite, the smoke check and the CPU-baseline
+leg of the benchmark call this module; the product path never does.  It shares
+no code with the CUDA library (it does not import the package), and everything
+it computes is double precision on the host.
+
+The arithmetic lives in ``gdr_oracle.c`` next to this file.  What it computes is
+the gated delta rule named in the Qwen3.5 Chat guide (soniqo.audio, section
+"Architektur") and on the Core AI Qwen3.6-35B-A3B card (GVA, first section):
+
+    S_t = exp(g_t) S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,  o_t = S_t q_t
+    y_t = RMSNorm(o_t) * w * SiLU(z_t)
+
+with the published definition of "Gated Delta Networks" (Yang, Kautz,
+Hatamizadeh, ICLR 2025).  Arrays are numpy float64 in the packed layout:
+
+    q, k  [n_tok, H_k, d_k]     v, z  [n_tok, H_v, d_v]     g, beta  [n_tok, H_v]
+    cu_seqlens [n_seq + 1] (int)  s0 [n_seq, H_v, d_v, d_k] or None   w [d_v] or None
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdr_oracle.c")
+_LIB = os.path.join(_HERE, "_build", "liboracle.so")
+
+_DP = ctypes.POINTER(ctypes.c_double)
+
+
+class _Problem(ctypes.Structure):
+    _fields_ = [
+        ("n_tok", ctypes.c_int64),
+        ("n_seq", ctypes.c_int32),
+        ("H_k", ctypes.c_int32),
+        ("H_v", ctypes.c_int32),
+        ("d_k", ctypes.c_int32),
+        ("d_v", ctypes.c_int32),
+        ("qk_l2norm", ctypes.c_int32),
+        ("scale", ctypes.c_double),
+        ("eps_l2", ctypes.c_double),
+        ("eps_norm", ctypes.c_double),
+        ("q", _DP), ("k", _DP), ("v", _DP), ("z", _DP),
+        ("g", _DP), ("beta", _DP), ("s0", _DP), ("w", _DP),
+        ("cu_seqlens", ctypes.POINTER(ctypes.c_int64)),
+    ]
+
+
+def build(src: str = _SRC, out: str = _LIB, force: bool = False, werror: bool = True) -> str:
+    """Compile the oracle with the host C compiler (plain -O2, no CPU-specific flags)."""
+    if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(src):
+        return out
+    os.makedirs(os.path.dirname(out), exist_ok=True)
+    tmp = out + f".tmp{os.getpid()}"
+    subprocess.run(
+        ["gcc", "-std=c11", "-O2", "-fPIC", "-shared", "-Wall", "-Wextra"]
+        + (["-Werror"] if werror else []) + ["-o", tmp, src, "-lm", "-lpthread"],
+        check=True,
+    )
+    os.replace(tmp, out)
+    return out
+
+
+_lib_cache: dict[str, ctypes.CDLL] = {}
+
+
+def load(path: str | None = None) -> ctypes.CDLL:
+    """Load (building first if needed) the oracle library; ``path`` selects a
+    specific build, which the mutation tests use."""
+    path = path or build()
+    if path in _lib_cache:
+        return _lib_cache[path]
+    lib = ctypes.CDLL(path)
+    pp = ctypes.POINTER(_Problem)
+    lib.orc_gdr_recurrent.argtypes = [pp, _DP, _DP, _DP, ctypes.c_int]
+    lib.orc_gdr_recurrent.restype = ctypes.c_int
+    lib.orc_gdr_chunked.argtypes = [pp, ctypes.c_int, _DP, _DP, _DP, ctypes.c_int]
+    lib.orc_gdr_chunked.restype = ctypes.c_int
+    lib.orc_gdr_bruteforce.argtypes = [pp, _DP, _DP, _DP]
+    lib.orc_gdr_bruteforce.restype = ctypes.c_int
+    lib.orc_rmsnorm_gated.argtypes = [_DP, _DP, _DP, ctypes.c_int64, ctypes.c_int,
+                                      ctypes.c_double, _DP]
+    lib.orc_rmsnorm_gated.restype = None
+    _lib_cache[path] = lib
+    return lib
+
+
+def _f64(a, shape=None):
+    if a is None:
+        return None
+    a = np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+    if shape is not None and a.shape != tuple(shape):
+        raise ValueError(f"expected shape {tuple(shape)}, got {a.shape}")
+    return a
+
+
+def _ptr(a):
+    return a.ctypes.data_as(_DP) if a is not None else None
+
+
+@dataclass
+class Result:
+    o: np.ndarray            # [n_tok, H_v, d_v] before the output gate
+    y: np.ndarray | None     # [n_tok, H_v, d_v] after RMSNormGated (None without z)
+    state: np.ndarray        # [n_seq, H_v, d_v, d_k] state after each sequence
+
+
+def _problem(q, k, v, g, beta, cu_seqlens, z, s0, w, scale, eps_l2, eps_norm, qk_l2norm):
+    q = _f64(q); k = _f64(k); v = _f64(v)
+    if q.ndim != 3 or k.shape != q.shape or v.ndim != 3:
+        raise ValueError("q, k must be [n_tok, H_k, d_k] and v [n_tok, H_v, d_v]")
+    n_tok, H_k, d_k = q.shape
+    _, H_v, d_v = v.shape
+    if v.shape[0] != n_tok or H_v % H_k:
+        raise ValueError("token counts differ or H_v is not a multiple of H_k")
+    g = _f64(g, (n_tok, H_v)); beta = _f64(beta, (n_tok, H_v))
+    z = _f64(z, (n_tok, H_v, d_v)) if z is not None else None
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    n_seq = cu.shape[0] - 1
+    if cu[0] != 0 or cu[-1] != n_tok or np.any(np.diff(cu) < 0):
+        raise ValueError("cu_seqlens must rise from 0 to n_tok")
+    s0 = _f64(s0, (n_seq, H_v, d_v, d_k)) if s0 is not None else None
+    w = _f64(w, (d_v,)) if w is not None else None
+    keep = (q, k, v, z, g, beta, s0, w, cu)
+    p = _Problem(n_tok, n_seq, H_k, H_v, d_k, d_v, int(bool(qk_l2norm)), float(scale),
+                 float(eps_l2), float(eps_norm), _ptr(q), _ptr(k), _ptr(v), _ptr(z),
+                 _ptr(g), _ptr(beta), _ptr(s0), _ptr(w),
+                 cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)))
+    return p, keep, (n_tok, n_seq, H_v, d_v, d_k)
+
+
+def _outputs(dims, want_y):
+    n_tok, n_seq, H_v, d_v, d_k = dims
+    o = np.zeros((n_tok, H_v, d_v))
+    y = np.zeros((n_tok, H_v, d_v)) if want_y else None
+    s = np.zeros((n_seq, H_v, d_v, d_k))
+    return o, y, s
+
+
+def gdr_recurrent(q, k, v, g, beta, cu_seqlens, *, z=None, s0=None, w=None, scale=1.0,
+                  eps_l2=1e-6, eps_norm=1e-6, qk_l2norm=True, threads=1,
+                  lib: ctypes.CDLL | None = None) -> Result:
+    """The definition, token by token, for every (sequence, value head)."""
+    p, keep, dims = _problem(q, k, v, g, beta, cu_seqlens, z, s0, w, scale, eps_l2,
+                             eps_norm, qk_l2norm)
+    o, y, s = _outputs(dims, z is not None)
+    (lib or load()).orc_gdr_recurrent(ctypes.byref(p), _ptr(o), _ptr(y), _ptr(s), int(threads))
+    del keep
+    return Result(o, y, s)
+
+
+def gdr_chunked(q, k, v, g, beta, cu_seqlens, *, chunk, z=None, s0=None, w=None,
+                scale=1.0, eps_l2=1e-6, eps_norm=1e-6, qk_l2norm=True, threads=1,
+                lib: ctypes.CDLL | None = None) -> Result:
+    """The chunkwise (WY / UT transform) form with chunks of ``chunk`` tokens."""
+    p, keep, dims = _problem(q, k, v, g, beta, cu_seqlens, z, s0, w, scale, eps_l2,
+                             eps_norm, qk_l2norm)
+    o, y, s = _outputs(dims, z is not None)
+    rc = (lib or load()).orc_gdr_chunked(ctypes.byref(p), int(chunk), _ptr(o), _ptr(y),
+                                         _ptr(s), int(threads))
+    if rc:
+        raise ValueError("chunk must be >= 1")
+    del keep
+    return Result(o, y, s)
+
+
+def gdr_bruteforce(q, k, v, g, beta, cu_seqlens, *, z=None, s0=None, w=None, scale=1.0,
+                   eps_l2=1e-6, eps_norm=1e-6, qk_l2norm=True,
+                   lib: ctypes.CDLL | None = None) -> Result:
+    """Explicit transition matrices multiplied out; every sequence at most 8 tokens."""
+    p, keep, dims = _problem(q, k, v, g, beta, cu_seqlens, z, s0, w, scale, eps_l2,
+                             eps_norm, qk_l2norm)
+    o, y, s = _outputs(dims, z is not None)
+    rc = (lib or load()).orc_gdr_bruteforce(ctypes.byref(p), _ptr(o), _ptr(y), _ptr(s))
+    if rc:
+        raise ValueError("brute force takes sequences of at most 8 tokens")
+    del keep
+    return Result(o, y, s)
+
+
+def rmsnorm_gated(o, z, w=None, eps=1e-6, lib: ctypes.CDLL | None = None) -> np.ndarray:
+    """y = o / sqrt(mean(o^2) + eps) * w * z * sigmoid(z) over the last axis."""
+    o = _f64(o); z = _f64(z, o.shape)
+    n = o.shape[-1]
+    w = _f64(w, (n,)) if w is not None else None
+    y = np.zeros_like(o)
+    (lib or load()).orc_rmsnorm_gated(_ptr(o), _ptr(z), _ptr(w), o.size // n, n, float(eps),
+                                      _ptr(y))
+    return y

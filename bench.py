@@ -1,0 +1,435 @@
+"""Benchmark of the Gated DeltaNet mixer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Headline workload (one "step"): one decode token through the GDN layers of a
+Qwen3.5-0.8B-shaped model -- 18 independent layer states, batch 32, 16 key and
+16 value heads, d_k = d_v = 128, bf16 q/k/v/z and outputs, fp32 state,
+S_0 ~ N(0, 0.02).  Each step launches the decode kernel once per layer (18
+launches, replayed from one CUDA graph per step).  Inputs are seeded and
+synthetic, drawn on the GPU; the 18 layer states (604 MB) rotate through HBM,
+far more than the 126 MB L2, so no step finds its state in L2.
+
+Metric: GB/s of algorithmic bytes (per (sequence, value head) and token: the
+fp32 state read and written once, q/k per key head, v/z/g/beta read once, the
+output written once).  The JSON line also carries the roofline of the decode
+kernel, a clock record of the timed region, an end-to-end figure through the
+same C ABI with inputs copied from pinned host memory every step, the
+chunked-prefill throughput (Qwen3.5-0.8B-shaped prefill: 4 x 4096 tokens,
+16 heads), and the fp64 CPU oracle timed on this host on a bounded sample.
+
+With N > 1 (torchrun), every rank runs the same workload on its own GPU
+(weak scaling: the batch grows with N, no data exchange between ranks); the
+timed region is bracketed by barriers and the maximum over ranks is used.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+# Workload: Qwen3.5-0.8B-shaped GDN decode.
+LAYERS, BATCH, H_K, H_V, D = 18, 32, 16, 16, 128
+SLOTS = 512  # distinct per-step inputs (the workload's 512 decode steps), cycled
+IN_BYTES, OUT_BYTES = 2, 2
+# Chunked prefill (reported beside the headline): Qwen3.5-0.8B-shaped prompt batch.
+P_SEQS, P_LEN, P_H, P_CHUNK = 4, 4096, 16, 64
+
+HEADLINE = "GDN decode state-update GB/s"
+
+
+def decode_bytes_per_layer_step(B, H_k, H_v, d, in_b=IN_BYTES, out_b=OUT_BYTES) -> int:
+    per_value_head = 2 * d * d * 4 + 2 * d * in_b + 2 * 4 + d * out_b  # state r+w, v, z, g, beta, out
+    per_key_head = 2 * d * in_b                                       # q, k
+    return B * H_v * per_value_head + B * H_k * per_key_head
+
+
+def prefill_flops_per_token_head(C, d, gva: bool) -> int:
+    # K K^T, Q K^T, U, W, P Delta at 2 C d each; W S^T, Q S^T, state update at 2 d^2 each.
+    kk_qk = 0 if gva else 4 * C * d
+    return kk_qk + 6 * C * d + 6 * d * d
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return None
+        self.file.flush()
+        with open(self.file.name) as f:
+            rows = [r.strip().split(", ") for r in f if r.strip()]
+        os.unlink(self.file.name)
+        rows = [r for r in rows if len(r) >= 9]
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        loaded = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()
+                  and r[3].replace(".", "").isdigit() and float(r[3]) > 200.0] or sm
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len(loaded)}
+
+
+# ----------------------------------------------------------------- decode
+
+class DecodeBench:
+    def __init__(self, device, seed=1, B=BATCH, layers=LAYERS, slots=SLOTS):
+        import linear_attention_recurrence_10_b200 as gdr
+        from linear_attention_recurrence_10_b200 import synth
+        self.gdr = gdr
+        self.B, self.L, self.T = B, layers, slots
+        x = synth.make_decode_inputs(layers, slots, B, H_K, H_V, D, seed=seed, s0_std=0.02,
+                                     device=device)
+        self.x = x
+        self.state = x.s0.clone()
+        self.out = torch.empty(layers, B, H_V, D, device=device, dtype=torch.bfloat16)
+        self.graphs = []
+        self.bytes_per_step = layers * decode_bytes_per_layer_step(B, H_K, H_V, D)
+        self.launches_per_step = layers
+
+    def launch_step(self, t, x=None, out=None):
+        x = x or self.x
+        out = self.out if out is None else out
+        for l in range(self.L):
+            self.gdr.decode_step(x.q[l, t], x.k[l, t], x.v[l, t], x.g[l, t], x.beta[l, t],
+                                 self.state[l], out[l], z=x.z[l, t], norm_w=x.w)
+
+    def capture(self):
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.launch_step(0)  # load the library and kernels before capture
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        for t in range(self.T):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self.launch_step(t)
+            self.graphs.append(g)
+        torch.cuda.synchronize()
+
+    def run(self, first, n):
+        for s in range(first, first + n):
+            self.graphs[s % self.T].replay()
+
+
+class DecodeE2E:
+    """Same steps through the same C ABI, with the step's inputs copied in from
+    pinned host memory and its outputs copied back every step."""
+
+    def __init__(self, bench: DecodeBench, host_slots=16):
+        self.b = bench
+        x = bench.x
+        self.host_slots = host_slots
+        pin = lambda t: t[:, :host_slots].transpose(0, 1).contiguous().cpu().pin_memory()
+        # host tensors [slot, L, ...]
+        self.h = {n: pin(getattr(x, n)) for n in ("q", "k", "v", "z", "g", "beta")}
+        dev = x.q.device
+        self.d = {n: torch.empty_like(t[0], device=dev) for n, t in self.h.items()}
+        self.h_out = torch.empty(bench.out.shape, dtype=bench.out.dtype).pin_memory()
+        self.h2d_bytes = sum(t[0].numel() * t[0].element_size() for t in self.h.values())
+        self.d2h_bytes = self.h_out.numel() * self.h_out.element_size()
+        import types
+        self.view = types.SimpleNamespace(
+            q=self.d["q"].unsqueeze(1), k=self.d["k"].unsqueeze(1), v=self.d["v"].unsqueeze(1),
+            z=self.d["z"].unsqueeze(1), g=self.d["g"].unsqueeze(1),
+            beta=self.d["beta"].unsqueeze(1), w=x.w)
+
+    def step(self, s):
+        slot = s % self.host_slots
+        for n, t in self.h.items():
+            self.d[n].copy_(t[slot], non_blocking=True)
+        self.b.launch_step(0, x=self.view)
+        self.h_out.copy_(self.b.out, non_blocking=True)
+
+
+def time_region(fn, n, ranks):
+    """CUDA-event time of fn() over a barrier-bracketed region; max over ranks (ms)."""
+    if ranks > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    fn()
+    e1.record()
+    torch.cuda.synchronize()
+    if ranks > 1:
+        torch.distributed.barrier()
+    ms = e0.elapsed_time(e1)
+    if ranks > 1:
+        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms
+
+
+# ---------------------------------------------------------------- prefill
+
+def prefill_measure(device, reps=5):
+    import linear_attention_recurrence_10_b200 as gdr
+    from linear_attention_recurrence_10_b200 import synth
+    inp = synth.make_inputs([P_LEN] * P_SEQS, P_H, P_H, D, seed=2, device=device)
+    cu = torch.tensor(inp.cu_seqlens, dtype=torch.int32, device=device)
+    out = torch.empty(inp.n_tok, P_H, D, device=device, dtype=torch.bfloat16)
+    final = torch.empty(P_SEQS, P_H, D, D, device=device)
+    ws_bytes = gdr.prefill_workspace_size(inp.q, inp.k, inp.v, inp.g, inp.beta, cu, out,
+                                          cu_seqlens_host=inp.cu_seqlens, z=inp.z, chunk=P_CHUNK)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device)
+
+    def call():
+        gdr.prefill_chunked(inp.q, inp.k, inp.v, inp.g, inp.beta, cu, out,
+                            cu_seqlens_host=inp.cu_seqlens, z=inp.z, norm_w=inp.w,
+                            final_state=final, chunk=P_CHUNK, workspace=ws)
+
+    for _ in range(2):
+        call()
+    torch.cuda.synchronize()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    times = []
+    for _ in range(reps):
+        flush.zero_()  # evict L2 between repetitions
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        call()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    n_tok = inp.n_tok
+    flops = n_tok * P_H * prefill_flops_per_token_head(P_CHUNK, D, gva=False)
+    peaks = load_peaks()
+    tflops = flops / (ms * 1e-3) / 1e12
+    return {"metric": "chunked-prefill tokens/s", "value": n_tok / (ms * 1e-3), "unit": "tokens/s",
+            "ms": ms, "workload": f"Qwen3.5-0.8B-shaped prefill: {P_SEQS} x {P_LEN} tokens, "
+                                  f"{P_H}/{P_H} heads, d={D}, bf16, chunk {P_CHUNK}, S_0=0",
+            "tflops": tflops, "tc_frac": tflops / peaks["bf16_tflops"],
+            "tc_peak_tflops": peaks["bf16_tflops"], "flops_per_token_head":
+                prefill_flops_per_token_head(P_CHUNK, D, gva=False),
+            "l2": "flushed (256 MB write) before each repetition", "reps": reps}
+
+
+# ------------------------------------------------------------- CPU oracle
+
+def oracle_sample(n_tokens=512, seed=1, threads=None):
+    """Time the fp64 oracle on one layer of the decode workload: B sequences x
+    16 heads x n_tokens steps, on every host core."""
+    import numpy as np
+    import oracle
+    from linear_attention_recurrence_10_b200 import synth
+    threads = threads or os.cpu_count() or 1
+    inp = synth.make_inputs([n_tokens] * BATCH, H_K, H_V, D, seed=seed, s0_std=0.02)
+    f = lambda t: t.to(torch.float64).numpy()
+    args = dict(q=f(inp.q), k=f(inp.k), v=f(inp.v), g=f(inp.g), beta=f(inp.beta),
+                cu_seqlens=np.array(inp.cu_seqlens), z=f(inp.z), s0=f(inp.s0), w=f(inp.w))
+    t0 = time.perf_counter()
+    oracle.gdr_recurrent(**args, threads=threads)
+    dt = time.perf_counter() - t0
+    nbytes = n_tokens * decode_bytes_per_layer_step(BATCH, H_K, H_V, D)
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "seconds": dt,
+            "sample": f"one layer of the decode workload: {BATCH} sequences x {H_V} heads x "
+                      f"{n_tokens} tokens, fp64 recurrence, {threads} threads"}
+
+
+def run_reference(args, rank, world):
+    """The fp64 oracle as the reference arm: each step is one decode token of one
+    layer for a sample of the batch's (sequence, head) pairs, on the host cores."""
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+    from linear_attention_recurrence_10_b200 import synth
+    threads = os.cpu_count() or 1
+    inp = synth.make_inputs([SLOTS] * BATCH, H_K, H_V, D, seed=1, s0_std=0.02)
+    f = lambda t: t.to(torch.float64).numpy()
+    q, k, v, z = (f(t).reshape(BATCH, SLOTS, -1, D) for t in (inp.q, inp.k, inp.v, inp.z))
+    g, beta = (f(t).reshape(BATCH, SLOTS, H_V) for t in (inp.g, inp.beta))
+    state = f(inp.s0)
+    w = f(inp.w)
+    cu = np.arange(BATCH + 1, dtype=np.int64)
+    lib = oracle.load()
+
+    def step(s):
+        nonlocal state
+        t = s % SLOTS
+        r = oracle.gdr_recurrent(q[:, t], k[:, t], v[:, t], g[:, t], beta[:, t], cu, z=z[:, t],
+                                 s0=state, w=w, threads=threads, lib=lib)
+        state = r.state
+
+    for s in range(args.warmup):
+        step(s)
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        step(args.warmup + s)
+    dt = time.perf_counter() - t0
+    nbytes = args.steps * decode_bytes_per_layer_step(BATCH, H_K, H_V, D)
+    value = nbytes / dt / 1e9
+    sample = (f"one decode token of one layer per step: {BATCH} sequences x {H_V} heads, "
+              f"fp64 recurrence, {threads} threads")
+    line = {"impl": "reference", "metric": HEADLINE, "value": value, "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "Qwen3.5-0.8B-shaped GDN decode (oracle sample)",
+                       "global_batch": BATCH, "seq_len": 1, "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__,
+                                 formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=8192)
+    ap.add_argument("--warmup", type=int, default=16)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--batch", type=int, default=BATCH)
+    ap.add_argument("--e2e-steps", type=int, default=1024)
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", device_id=device,
+                                             timeout=datetime.timedelta(seconds=120))
+
+    from linear_attention_recurrence_10_b200 import build
+    build.build(quiet=True)
+
+    bench = DecodeBench(device, seed=1 + rank, B=args.batch)
+    bench.capture()
+    bench.run(0, args.warmup)
+    torch.cuda.synchronize()
+    visible = [v.strip() for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+    gpu_index = int(visible[local]) if local < len(visible) and visible[local].isdigit() else local
+    with ClockSampler(gpu_index) as clocks:
+        ms = time_region(lambda: bench.run(args.warmup, args.steps), args.steps, world)
+    clock_info = clocks.summary()
+
+    peaks = load_peaks()
+    bytes_total = bench.bytes_per_step * args.steps * world
+    gbs = bytes_total / (ms * 1e-3) / 1e9
+    per_launch_ms = ms / (args.steps * bench.launches_per_step)
+    per_launch_bytes = decode_bytes_per_layer_step(args.batch, H_K, H_V, D)
+    achieved = per_launch_bytes / (per_launch_ms * 1e-3) / 1e9
+
+    # End to end through the same ABI with host buffers.
+    e2e = DecodeE2E(bench)
+    for s in range(4):
+        e2e.step(s)
+    ms_e2e = time_region(lambda: [e2e.step(s) for s in range(args.e2e_steps)], args.e2e_steps,
+                         world)
+    e2e_gbs = bench.bytes_per_step * args.e2e_steps * world / (ms_e2e * 1e-3) / 1e9
+
+    prefill = None if args.no_prefill else prefill_measure(device)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_sample()
+
+    line = {
+        "metric": HEADLINE, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {
+            "workload": f"Qwen3.5-0.8B-shaped GDN decode: {LAYERS} layers x B={args.batch}, "
+                        f"{H_K}/{H_V} heads, d={D}, bf16 q/k/v/z/out, fp32 state and math",
+            "global_batch": args.batch * world, "seq_len": 1, "layers": LAYERS,
+            "parallelism": f"replicas x{world}",
+            "l2": f"inputs larger than L2: {LAYERS} layer states "
+                  f"({LAYERS * args.batch * H_V * D * D * 4 / 1e6:.0f} MB) rotate every step",
+            "launch": "one CUDA graph per step (one decode launch per layer)"},
+        "tokens_per_s": args.batch * world * args.steps / (ms * 1e-3),
+        "hbm_frac": gbs / world / peaks["hbm_gbs"],
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "kernel": "decode_kernel<128, bf16, bf16>",
+                     "bytes_per_launch": per_launch_bytes, "us_per_launch": per_launch_ms * 1e3,
+                     "peak_source": peaks["source"] + " (hbm_gbs, of measured copy bandwidth)"},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": e2e.h2d_bytes,
+                "d2h_bytes_per_step": e2e.d2h_bytes, "steps": args.e2e_steps,
+                "ms_per_step": ms_e2e / args.e2e_steps},
+        "gpu_launches": args.steps * bench.launches_per_step,
+        "clocks": clock_info,
+        "prefill": prefill,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,211 @@
+/*
+ * gdr.h -- C ABI of the Gated DeltaNet (gated delta rule) token mixer for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The mixer: the pages name it as the "gated delta rule" recurrence with an
+ * RMSNormGated output (Qwen3.5 Chat guide, soniqo.audio/de/guides/chat,
+ * section "Architektur"), 18 of the 24 layers of Qwen3.5-0.8B; on the Core AI
+ * Qwen3.6-35B-A3B card (first section) it runs 32 value heads over 16 key
+ * heads, each key/query head shared by two value heads (GVA).  Its state is a
+ * fixed-size matrix per head, so memory does not grow with context (Swiftlet
+ * post, "How It Works").  The equations follow the published gated delta rule
+ * (Gated Delta Networks, Yang, Kautz, Hatamizadeh, ICLR 2025).  Per sequence,
+ * per value head h_v with key head h_k = floor(h_v * H_k / H_v):
+ *
+ *     q_hat = scale * q / sqrt(|q|^2 + eps_l2),   k_hat = k / sqrt(|k|^2 + eps_l2)
+ *     S_t   = exp(g_t) S_{t-1} (I - beta_t k_hat k_hat^T) + beta_t v_t k_hat^T
+ *     o_t   = S_t q_hat
+ *     y_t   = o_t / sqrt(mean(o_t^2) + eps_norm) * w * z_t * sigmoid(z_t)
+ *
+ * S is d_v x d_k fp32, row-major ([d_v][d_k]: row i is value dimension i).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Memory.  Every pointer is device memory owned by the caller unless its
+ *    comment says host.  The library allocates nothing and keeps no state
+ *    between calls; it only reads and writes the buffers it is given.
+ *  - Streams.  Work is queued on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream) and the call returns without waiting for it.
+ *  - Errors.  Arguments are checked on the host before anything is queued; a
+ *    failed check returns its status and queues nothing.  A launch the CUDA
+ *    runtime refuses returns GDR_ERR_CUDA (the runtime's own error is cleared
+ *    and not reported further).  Faults inside a running kernel surface on the
+ *    stream like any CUDA error.  No C++ exception crosses this ABI.
+ *  - Layout.  Activations are token-major and head-contiguous: element
+ *    (row, head, i) of a [rows, H, d] tensor is at row*row_stride + head*d + i,
+ *    where row_stride (in elements) defaults to H*d when passed as 0.
+ *  - Alignment.  Every pointer must be 16-byte aligned and every row stride a
+ *    multiple of 16 bytes (GDR_ERR_MISALIGNED otherwise).
+ *  - Threads.  Calls are independent and may be made from several host
+ *    threads at once.
+ */
+#ifndef GDR_H_
+#define GDR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gdr_status {
+    GDR_OK = 0,
+    GDR_ERR_INVALID_ARG = 1, /* null pointer, negative or inconsistent size */
+    GDR_ERR_UNSUPPORTED = 2, /* valid, but no kernel for this shape / dtype / chunk */
+    GDR_ERR_MISALIGNED = 3,  /* pointer or stride breaks the 16-byte rule */
+    GDR_ERR_WORKSPACE = 4,   /* workspace missing or smaller than required */
+    GDR_ERR_CUDA = 5,        /* the CUDA runtime refused a launch or query */
+    GDR_ERR_TIMEOUT = 6      /* a bounded device-side wait gave up */
+} gdr_status;
+
+typedef enum gdr_dtype { GDR_F32 = 0, GDR_BF16 = 1 } gdr_dtype;
+
+/* Opaque CUDA stream (binary-compatible with cudaStream_t). */
+typedef struct CUstream_st *gdr_stream_t;
+
+/* ------------------------------------------------------------------------
+ * One decode step: every sequence in the batch advances by one token.
+ *
+ * The pages' decoder is a single-step model that owns the recurrent state, so
+ * the caller advances one token per call (Core ML card for Qwen3.5-0.8B,
+ * section "Model"); the state is held across the generation loop (same card,
+ * "Usage").  Here the caller owns the state buffer and this call updates it.
+ *
+ *   q, k       [batch, H_k, d_k]   in_dtype    row strides q_stride, k_stride
+ *   v, z       [batch, H_v, d_v]   in_dtype    row strides v_stride, z_stride
+ *   g, beta    [batch, H_v]        fp32        row stride  gb_stride (both)
+ *   state_in   [batch, H_v, d_v, d_k] fp32    batch stride state_stride
+ *   state_out  same layout; may be the same buffer as state_in (in place).
+ *              Any other overlap between them is undefined.
+ *   norm_w     [d_v] fp32, shared by all heads; NULL means all ones
+ *   out        [batch, H_v, d_v]   out_dtype   row stride out_stride
+ *
+ *   z == NULL skips the output gate: out receives o_t itself.
+ *   qk_l2norm == 0 uses q and k as given (the caller has normalised them);
+ *   `scale` still multiplies q.  g = -inf is allowed (state reset).
+ *   Supported: d_k == d_v in {16, 32, 64, 128}, H_v a multiple of H_k.
+ *   batch == 0 is a no-op.  state_stride must be >= H_v*d_v*d_k (0 = that).
+ * ------------------------------------------------------------------------ */
+typedef struct gdr_decode_args {
+    int32_t batch, H_k, H_v, d_k, d_v;
+    int32_t in_dtype;  /* gdr_dtype of q, k, v, z */
+    int32_t out_dtype; /* gdr_dtype of out */
+    int32_t qk_l2norm; /* 1: normalise q, k in the kernel */
+    float scale;       /* multiplies q_hat; 1.0 for the plain o_t = S_t q_t */
+    float eps_l2;      /* under the square root of the q/k norms */
+    float eps_norm;    /* added to mean(o^2) in RMSNormGated */
+    int32_t reserved;  /* must be 0 */
+    int64_t q_stride, k_stride, v_stride, z_stride, gb_stride, out_stride;
+    int64_t state_stride;
+    const void *q, *k, *v, *z;
+    const float *g, *beta;
+    const float *state_in;
+    float *state_out;
+    const float *norm_w;
+    void *out;
+} gdr_decode_args;
+
+gdr_status gdr_decode_step(const gdr_decode_args *args, gdr_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Chunked prefill over packed variable-length sequences.
+ *
+ * The pages' Core ML build pairs a prefill model with the decode model
+ * (Qwen3.5 Chat guide, "Architektur"), and the Swiftlet post checks that
+ * incremental decoding matches whole-sequence processing ("Correctness &
+ * Validation").  This call processes whole prompts with the chunkwise
+ * (WY / UT transform) form of the same recurrence: within a chunk of C tokens,
+ *   A_rs  = beta_r exp(gamma_r - gamma_s) (k_r . k_s)            s < r
+ *   Delta = (I + A)^{-1} (diag(beta) V - diag(beta e^gamma) K S_0^T)
+ *   O     = diag(e^gamma) Q S_0^T + (exp(gamma_r - gamma_s) q_r . k_s)_{s<=r} Delta
+ *   S_C   = e^{gamma_C} S_0 + Delta^T diag(e^{gamma_C - gamma}) K
+ * with gamma the running sum of g inside the chunk.  The result equals the
+ * token-by-token recurrence up to rounding.
+ *
+ *   q, k        [n_tok, H_k, d_k]  in_dtype   row strides q_stride, k_stride
+ *   v, z        [n_tok, H_v, d_v]  in_dtype   row strides v_stride, z_stride
+ *   g, beta     [n_tok, H_v]       fp32       row stride gb_stride
+ *   cu_seqlens       device int32 [n_seq + 1]: sequence s is tokens
+ *                    [cu_seqlens[s], cu_seqlens[s+1]); chunks never cross it.
+ *   cu_seqlens_host  HOST int32 [n_seq + 1], the same values; read during the
+ *                    call (validation, work ordering), not kept.
+ *   initial_state    [n_seq, H_v, d_v, d_k] fp32, or NULL for zeros
+ *   final_state      same layout, or NULL; may equal initial_state (in place)
+ *   norm_w, out, z, qk_l2norm, scale, eps_*: as for gdr_decode_step;
+ *   out is [n_tok, H_v, d_v] with row stride out_stride.
+ *
+ *   g is clamped below at -64 inside chunks (exp(-64) ~ 1.6e-28): the chunk
+ *   form takes differences of running sums of g, which a g of -inf would turn
+ *   into NaN.  Empty sequences are allowed (their final state = initial state).
+ *   chunk: 16, 32 or 64, or 0 for the library's choice.
+ *   Supported: d_k == d_v in {16, 32, 64, 128}; bf16 inputs with d = 128 and
+ *   chunk 64 (or 0) run on the tensor cores, everything else on CUDA cores
+ *   (chunk 64 with d = 128 needs the tensor-core path).
+ *   workspace: device memory of at least gdr_prefill_workspace_size() bytes,
+ *   16-byte aligned, owned by the caller, free for reuse once the queued work
+ *   has finished.
+ * ------------------------------------------------------------------------ */
+typedef struct gdr_prefill_args {
+    int32_t n_seq, H_k, H_v, d_k, d_v;
+    int32_t chunk;
+    int32_t in_dtype, out_dtype;
+    int32_t qk_l2norm;
+    float scale, eps_l2, eps_norm;
+    int64_t n_tok;
+    int64_t q_stride, k_stride, v_stride, z_stride, gb_stride, out_stride;
+    const void *q, *k, *v, *z;
+    const float *g, *beta;
+    const int32_t *cu_seqlens;
+    const int32_t *cu_seqlens_host;
+    const float *initial_state;
+    float *final_state;
+    const float *norm_w;
+    void *out;
+} gdr_prefill_args;
+
+/* Bytes of workspace gdr_prefill_chunked needs for these arguments (the same
+ * struct that will be passed to it; only sizes, dtypes and chunk are read).
+ * Returns 0 and sets *bytes on success; an invalid or unsupported shape
+ * returns the status gdr_prefill_chunked would. */
+gdr_status gdr_prefill_workspace_size(const gdr_prefill_args *args, size_t *bytes);
+
+gdr_status gdr_prefill_chunked(const gdr_prefill_args *args, void *workspace,
+                               size_t workspace_bytes, gdr_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * RMSNormGated on its own (the output gate of the mixer; Qwen3.5 Chat guide,
+ * "Architektur"):  y = o / sqrt(mean(o^2) + eps) * w * z * sigmoid(z), one
+ * row of d values at a time.
+ *
+ *   o    [rows, d] o_dtype, row stride o_stride
+ *   z    [rows, d] z_dtype, row stride z_stride
+ *   w    [d] fp32 or NULL (ones)
+ *   out  [rows, d] out_dtype, row stride out_stride; may equal o when the
+ *        dtypes and strides match (in place).
+ *   d in {16, 32, 64, 128}; rows == 0 is a no-op.
+ * ------------------------------------------------------------------------ */
+typedef struct gdr_norm_args {
+    int64_t rows;
+    int32_t d;
+    int32_t o_dtype, z_dtype, out_dtype;
+    float eps;
+    int32_t reserved; /* must be 0 */
+    int64_t o_stride, z_stride, out_stride;
+    const void *o, *z;
+    const float *w;
+    void *out;
+} gdr_norm_args;
+
+gdr_status gdr_rmsnorm_gated(const gdr_norm_args *args, gdr_stream_t stream);
+
+/* Static, human-readable name of a status (never NULL). */
+const char *gdr_status_string(gdr_status status);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+int gdr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GDR_H_ */

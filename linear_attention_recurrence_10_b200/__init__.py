@@ -1,0 +1,223 @@
+"""Gated DeltaNet (gated delta rule) token mixer for B200 -- Python binding.
+
+Thin wrappers over the C ABI of include/gdr.h (libgdr.so, built in-tree by
+``python -m linear_attention_recurrence_10_b200.build``).  Each wrapper only
+turns torch tensors into pointers, strides and dtype codes and passes the
+current CUDA stream; every step of the computation runs in the library's
+kernels.  PyTorch is used for device memory and streams only.
+
+    decode_step(q, k, v, g, beta, state, out, ...)        one token per sequence
+    prefill_chunked(q, k, v, g, beta, cu_seqlens, out, ...)  packed varlen prompts
+    rmsnorm_gated(o, z, out, ...)                          the output gate alone
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _abi
+from ._abi import GDR_BF16, GDR_F32
+
+__all__ = ["GdrError", "decode_step", "prefill_chunked", "prefill_workspace_size",
+           "rmsnorm_gated", "version", "status_string"]
+
+
+class GdrError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        name = _abi.STATUS_NAMES.get(self.status, f"status {status}")
+        super().__init__(f"{where}: {name}")
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise GdrError(status, where)
+
+
+def _dtype_code(t: torch.Tensor, what: str) -> int:
+    if t.dtype == torch.bfloat16:
+        return GDR_BF16
+    if t.dtype == torch.float32:
+        return GDR_F32
+    raise TypeError(f"{what}: dtype {t.dtype} is not bf16 or fp32")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _row_stride(t: torch.Tensor, what: str) -> int:
+    """Row stride of a [rows, H, d] (or [rows, d]) tensor whose inner dims are packed."""
+    if t.dim() >= 2:
+        inner = 1
+        for size, stride in zip(reversed(t.shape[1:]), reversed(t.stride()[1:])):
+            if size > 1 and stride != inner:
+                raise ValueError(f"{what}: inner dimensions must be contiguous")
+            inner *= size
+    return int(t.stride(0)) if t.shape[0] > 1 else 0
+
+
+def _stream(stream, device) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _f32_tensor(t, what):
+    if t is not None and t.dtype != torch.float32:
+        raise TypeError(f"{what} must be fp32")
+    return t
+
+
+def version() -> int:
+    return _abi.lib().gdr_version()
+
+
+def status_string(status: int) -> str:
+    return _abi.lib().gdr_status_string(int(status)).decode()
+
+
+def decode_step(q, k, v, g, beta, state, out, *, z=None, norm_w=None, state_out=None,
+                scale: float = 1.0, eps_l2: float = 1e-6, eps_norm: float = 1e-6,
+                qk_l2norm: bool = True, stream=None) -> torch.Tensor:
+    """Advance every sequence of the batch by one token (gdr_decode_step).
+
+    q, k [B, H_k, d]; v, z [B, H_v, d] (bf16 or fp32, same dtype); g, beta
+    [B, H_v] fp32; state [B, H_v, d, d] fp32, updated in place unless
+    ``state_out`` is given; out [B, H_v, d] bf16 or fp32.  Batch rows may be
+    strided views (e.g. one step of a [B, T, H, d] tensor).
+    """
+    B, H_k, d = q.shape
+    H_v = v.shape[1]
+    for t, name in ((g, "g"), (beta, "beta"), (state, "state"), (norm_w, "norm_w")):
+        _f32_tensor(t, name)
+    if g.stride() != beta.stride():
+        raise ValueError("g and beta must share one layout")
+    so = state if state_out is None else _f32_tensor(state_out, "state_out")
+    if state.stride() != so.stride():
+        raise ValueError("state and state_out must share one layout")
+    a = _abi.DecodeArgs()
+    a.batch, a.H_k, a.H_v, a.d_k, a.d_v = B, H_k, H_v, d, v.shape[2]
+    a.in_dtype = _dtype_code(q, "q")
+    for t, name in ((k, "k"), (v, "v"), (z, "z")):
+        if t is not None and _dtype_code(t, name) != a.in_dtype:
+            raise TypeError(f"{name} must have the dtype of q")
+    a.out_dtype = _dtype_code(out, "out")
+    a.qk_l2norm = int(bool(qk_l2norm))
+    a.scale, a.eps_l2, a.eps_norm = float(scale), float(eps_l2), float(eps_norm)
+    a.q_stride, a.k_stride = _row_stride(q, "q"), _row_stride(k, "k")
+    a.v_stride = _row_stride(v, "v")
+    a.z_stride = _row_stride(z, "z") if z is not None else 0
+    a.gb_stride = _row_stride(g, "g")
+    a.out_stride = _row_stride(out, "out")
+    a.state_stride = _row_stride(state, "state")
+    a.q, a.k, a.v, a.z = _ptr(q), _ptr(k), _ptr(v), _ptr(z)
+    a.g, a.beta = _ptr(g), _ptr(beta)
+    a.state_in, a.state_out = _ptr(state), _ptr(so)
+    a.norm_w, a.out = _ptr(norm_w), _ptr(out)
+    _check(_abi.lib().gdr_decode_step(ctypes.byref(a), _stream(stream, q.device)),
+           "gdr_decode_step")
+    return out
+
+
+def _prefill_args(q, k, v, g, beta, cu_seqlens, out, cu_seqlens_host, z, norm_w,
+                  initial_state, final_state, chunk, scale, eps_l2, eps_norm, qk_l2norm):
+    n_tok, H_k, d = q.shape
+    H_v = v.shape[1]
+    if cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    if cu_seqlens_host is None:
+        cu_seqlens_host = cu_seqlens.cpu()
+    host = (ctypes.c_int32 * len(cu_seqlens_host))(*[int(x) for x in cu_seqlens_host])
+    for t, name in ((g, "g"), (beta, "beta"), (initial_state, "initial_state"),
+                    (final_state, "final_state"), (norm_w, "norm_w")):
+        _f32_tensor(t, name)
+    if g.stride() != beta.stride():
+        raise ValueError("g and beta must share one layout")
+    a = _abi.PrefillArgs()
+    a.n_seq = len(cu_seqlens_host) - 1
+    a.H_k, a.H_v, a.d_k, a.d_v = H_k, H_v, d, v.shape[2]
+    a.chunk = int(chunk)
+    a.in_dtype = _dtype_code(q, "q")
+    for t, name in ((k, "k"), (v, "v"), (z, "z")):
+        if t is not None and _dtype_code(t, name) != a.in_dtype:
+            raise TypeError(f"{name} must have the dtype of q")
+    a.out_dtype = _dtype_code(out, "out")
+    a.qk_l2norm = int(bool(qk_l2norm))
+    a.scale, a.eps_l2, a.eps_norm = float(scale), float(eps_l2), float(eps_norm)
+    a.n_tok = n_tok
+    a.q_stride, a.k_stride = _row_stride(q, "q"), _row_stride(k, "k")
+    a.v_stride = _row_stride(v, "v")
+    a.z_stride = _row_stride(z, "z") if z is not None else 0
+    a.gb_stride = _row_stride(g, "g")
+    a.out_stride = _row_stride(out, "out")
+    a.q, a.k, a.v, a.z = _ptr(q), _ptr(k), _ptr(v), _ptr(z)
+    a.g, a.beta = _ptr(g), _ptr(beta)
+    a.cu_seqlens = _ptr(cu_seqlens)
+    a.cu_seqlens_host = ctypes.cast(host, ctypes.POINTER(ctypes.c_int32))
+    a.initial_state, a.final_state = _ptr(initial_state), _ptr(final_state)
+    a.norm_w, a.out = _ptr(norm_w), _ptr(out)
+    return a, host
+
+
+def prefill_workspace_size(q, k, v, g, beta, cu_seqlens, out, *, cu_seqlens_host=None,
+                           z=None, chunk: int = 0, **_) -> int:
+    a, host = _prefill_args(q, k, v, g, beta, cu_seqlens, out, cu_seqlens_host, z, None, None,
+                            None, chunk, 1.0, 1e-6, 1e-6, True)
+    n = ctypes.c_size_t(0)
+    _check(_abi.lib().gdr_prefill_workspace_size(ctypes.byref(a), ctypes.byref(n)),
+           "gdr_prefill_workspace_size")
+    del host
+    return int(n.value)
+
+
+def prefill_chunked(q, k, v, g, beta, cu_seqlens, out, *, cu_seqlens_host=None, z=None,
+                    norm_w=None, initial_state=None, final_state=None, chunk: int = 0,
+                    workspace=None, scale: float = 1.0, eps_l2: float = 1e-6,
+                    eps_norm: float = 1e-6, qk_l2norm: bool = True, stream=None) -> torch.Tensor:
+    """Chunked prefill of packed variable-length sequences (gdr_prefill_chunked).
+
+    q, k [n_tok, H_k, d]; v, z, out [n_tok, H_v, d]; g, beta [n_tok, H_v] fp32;
+    cu_seqlens int32 [n_seq + 1] on the device (``cu_seqlens_host``: the same
+    values on the host, read during the call); initial_state / final_state
+    [n_seq, H_v, d, d] fp32 or None.  ``workspace``: a uint8 device tensor of
+    at least prefill_workspace_size() bytes; allocated here when None.
+    """
+    a, host = _prefill_args(q, k, v, g, beta, cu_seqlens, out, cu_seqlens_host, z, norm_w,
+                            initial_state, final_state, chunk, scale, eps_l2, eps_norm,
+                            qk_l2norm)
+    L = _abi.lib()
+    n = ctypes.c_size_t(0)
+    _check(L.gdr_prefill_workspace_size(ctypes.byref(a), ctypes.byref(n)),
+           "gdr_prefill_workspace_size")
+    if workspace is None and n.value:
+        workspace = torch.empty(int(n.value), dtype=torch.uint8, device=q.device)
+    ws_ptr = _ptr(workspace)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(L.gdr_prefill_chunked(ctypes.byref(a), ws_ptr, ws_bytes, _stream(stream, q.device)),
+           "gdr_prefill_chunked")
+    del host
+    return out
+
+
+def rmsnorm_gated(o, z, out, *, w=None, eps: float = 1e-6, stream=None) -> torch.Tensor:
+    """y = o / sqrt(mean(o^2) + eps) * w * z * sigmoid(z) over the last dim (gdr_rmsnorm_gated).
+
+    o, z, out: [..., d] with packed rows; w [d] fp32 or None."""
+    d = o.shape[-1]
+    o2, z2, out2 = o.reshape(-1, d), z.reshape(-1, d), out.reshape(-1, d)
+    if out2.data_ptr() != out.data_ptr():
+        raise ValueError("out must be viewable as [rows, d]")
+    _f32_tensor(w, "w")
+    a = _abi.NormArgs()
+    a.rows, a.d = o2.shape[0], d
+    a.o_dtype, a.z_dtype = _dtype_code(o, "o"), _dtype_code(z, "z")
+    a.out_dtype = _dtype_code(out, "out")
+    a.eps = float(eps)
+    a.o_stride, a.z_stride = _row_stride(o2, "o"), _row_stride(z2, "z")
+    a.out_stride = _row_stride(out2, "out")
+    a.o, a.z, a.w, a.out = _ptr(o2), _ptr(z2), _ptr(w), _ptr(out2)
+    _check(_abi.lib().gdr_rmsnorm_gated(ctypes.byref(a), _stream(stream, o.device)),
+           "gdr_rmsnorm_gated")
+    return out

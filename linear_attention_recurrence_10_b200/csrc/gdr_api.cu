@@ -1,0 +1,233 @@
+// gdr_api.cu -- the C ABI declared in include/gdr.h: argument checks on the
+// host, then one kernel launch per call on the caller's stream.  Nothing here
+// allocates, synchronises or keeps state between calls.
+#include <stdint.h>
+#include <string.h>
+
+#include "gdr.h"
+#include "gdr_common.cuh"
+
+namespace gdr {
+cudaError_t launch_decode(const DecodeParams &p, int d, int in_bf16, int out_bf16, cudaStream_t s);
+cudaError_t launch_rmsnorm_gated(const NormParams &p, int d, int o_bf16, int z_bf16, int y_bf16,
+                                 cudaStream_t s);
+cudaError_t launch_prefill_simt(const PrefillParams &p, int d, int chunk, int in_bf16,
+                                int out_bf16, cudaStream_t s);
+}  // namespace gdr
+
+namespace {
+
+using gdr::DecodeParams;
+using gdr::NormParams;
+using gdr::PrefillParams;
+
+bool dtype_ok(int32_t t) { return t == GDR_F32 || t == GDR_BF16; }
+size_t dtype_bytes(int32_t t) { return t == GDR_BF16 ? 2 : 4; }
+bool head_dim_ok(int32_t d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+bool aligned4(const void *p) { return ((uintptr_t)p & 3u) == 0; }
+
+// Row stride: 0 selects the packed default; otherwise it must not let rows
+// overlap.  The byte stride must keep every row 16-byte aligned.
+gdr_status resolve_stride(int64_t given, int64_t packed, size_t elem, int64_t *out) {
+    if (given < 0) return GDR_ERR_INVALID_ARG;
+    const int64_t s = given == 0 ? packed : given;
+    if (s < packed) return GDR_ERR_INVALID_ARG;
+    if (((uint64_t)s * elem) % 16 != 0) return GDR_ERR_MISALIGNED;
+    *out = s;
+    return GDR_OK;
+}
+
+gdr_status from_cuda(cudaError_t e) { return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA; }
+
+#define GDR_TRY(expr)                         \
+    do {                                      \
+        gdr_status _st = (expr);              \
+        if (_st != GDR_OK) return _st;        \
+    } while (0)
+
+// Common shape checks of the mixer (decode and prefill).
+gdr_status check_heads(int32_t H_k, int32_t H_v, int32_t d_k, int32_t d_v) {
+    if (H_k <= 0 || H_v <= 0 || d_k <= 0 || d_v <= 0) return GDR_ERR_INVALID_ARG;
+    if (H_v % H_k != 0) return GDR_ERR_INVALID_ARG;
+    if (d_k != d_v || !head_dim_ok(d_k)) return GDR_ERR_UNSUPPORTED;
+    return GDR_OK;
+}
+
+bool ranges_overlap(const void *a, size_t an, const void *b, size_t bn) {
+    const uintptr_t a0 = (uintptr_t)a, b0 = (uintptr_t)b;
+    return a0 < b0 + bn && b0 < a0 + an;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *gdr_status_string(gdr_status s) {
+    switch (s) {
+        case GDR_OK: return "GDR_OK";
+        case GDR_ERR_INVALID_ARG: return "GDR_ERR_INVALID_ARG: invalid argument";
+        case GDR_ERR_UNSUPPORTED: return "GDR_ERR_UNSUPPORTED: shape, dtype or chunk not supported";
+        case GDR_ERR_MISALIGNED: return "GDR_ERR_MISALIGNED: pointer or stride not 16-byte aligned";
+        case GDR_ERR_WORKSPACE: return "GDR_ERR_WORKSPACE: workspace missing or too small";
+        case GDR_ERR_CUDA: return "GDR_ERR_CUDA: the CUDA runtime refused the launch";
+        case GDR_ERR_TIMEOUT: return "GDR_ERR_TIMEOUT: a bounded device wait gave up";
+        default: return "GDR_ERR_UNKNOWN: not a gdr_status value";
+    }
+}
+
+int gdr_version(void) { return 100; }
+
+gdr_status gdr_decode_step(const gdr_decode_args *a, gdr_stream_t stream) {
+    if (!a) return GDR_ERR_INVALID_ARG;
+    if (a->batch < 0 || a->reserved != 0) return GDR_ERR_INVALID_ARG;
+    if (!dtype_ok(a->in_dtype) || !dtype_ok(a->out_dtype)) return GDR_ERR_INVALID_ARG;
+    GDR_TRY(check_heads(a->H_k, a->H_v, a->d_k, a->d_v));
+    if (a->batch == 0) return GDR_OK;
+    if (!a->q || !a->k || !a->v || !a->g || !a->beta || !a->state_in || !a->state_out || !a->out)
+        return GDR_ERR_INVALID_ARG;
+    const int d = a->d_k;
+    const size_t ein = dtype_bytes(a->in_dtype), eout = dtype_bytes(a->out_dtype);
+    DecodeParams p;
+    memset(&p, 0, sizeof(p));
+    GDR_TRY(resolve_stride(a->q_stride, (int64_t)a->H_k * d, ein, &p.q_stride));
+    GDR_TRY(resolve_stride(a->k_stride, (int64_t)a->H_k * d, ein, &p.k_stride));
+    GDR_TRY(resolve_stride(a->v_stride, (int64_t)a->H_v * d, ein, &p.v_stride));
+    GDR_TRY(resolve_stride(a->z_stride, (int64_t)a->H_v * d, ein, &p.z_stride));
+    GDR_TRY(resolve_stride(a->out_stride, (int64_t)a->H_v * d, eout, &p.out_stride));
+    GDR_TRY(resolve_stride(a->state_stride, (int64_t)a->H_v * d * d, 4, &p.state_stride));
+    if (a->gb_stride < 0 || (a->gb_stride != 0 && a->gb_stride < a->H_v)) return GDR_ERR_INVALID_ARG;
+    p.gb_stride = a->gb_stride == 0 ? a->H_v : a->gb_stride;
+    const void *p16[] = {a->q, a->k, a->v, a->z, a->state_in, a->state_out, a->out};
+    for (const void *ptr : p16)
+        if (ptr && !aligned16(ptr)) return GDR_ERR_MISALIGNED;
+    if (!aligned4(a->g) || !aligned4(a->beta) || (a->norm_w && !aligned4(a->norm_w)))
+        return GDR_ERR_MISALIGNED;
+    if ((int64_t)a->batch * a->H_v > 0x7fffffffLL) return GDR_ERR_UNSUPPORTED;
+    if (a->state_in != a->state_out) {
+        const size_t span = ((size_t)(a->batch - 1) * p.state_stride + (size_t)a->H_v * d * d) * 4;
+        if (ranges_overlap(a->state_in, span, a->state_out, span)) return GDR_ERR_INVALID_ARG;
+    }
+    p.batch = a->batch;
+    p.H_k = a->H_k;
+    p.H_v = a->H_v;
+    p.hv_per_hk = a->H_v / a->H_k;
+    p.qk_l2norm = a->qk_l2norm ? 1 : 0;
+    p.scale = a->scale;
+    p.eps_l2 = a->eps_l2;
+    p.eps_norm = a->eps_norm;
+    p.q = a->q; p.k = a->k; p.v = a->v; p.z = a->z;
+    p.g = a->g; p.beta = a->beta;
+    p.state_in = a->state_in; p.state_out = a->state_out;
+    p.norm_w = a->norm_w; p.out = a->out;
+    return from_cuda(gdr::launch_decode(p, d, a->in_dtype == GDR_BF16, a->out_dtype == GDR_BF16,
+                                        (cudaStream_t)stream));
+}
+
+gdr_status gdr_rmsnorm_gated(const gdr_norm_args *a, gdr_stream_t stream) {
+    if (!a) return GDR_ERR_INVALID_ARG;
+    if (a->rows < 0 || a->reserved != 0) return GDR_ERR_INVALID_ARG;
+    if (!dtype_ok(a->o_dtype) || !dtype_ok(a->z_dtype) || !dtype_ok(a->out_dtype))
+        return GDR_ERR_INVALID_ARG;
+    if (a->d <= 0) return GDR_ERR_INVALID_ARG;
+    if (!head_dim_ok(a->d)) return GDR_ERR_UNSUPPORTED;
+    if (a->rows == 0) return GDR_OK;
+    if (!a->o || !a->z || !a->out) return GDR_ERR_INVALID_ARG;
+    NormParams p;
+    memset(&p, 0, sizeof(p));
+    GDR_TRY(resolve_stride(a->o_stride, a->d, dtype_bytes(a->o_dtype), &p.o_stride));
+    GDR_TRY(resolve_stride(a->z_stride, a->d, dtype_bytes(a->z_dtype), &p.z_stride));
+    GDR_TRY(resolve_stride(a->out_stride, a->d, dtype_bytes(a->out_dtype), &p.out_stride));
+    if (!aligned16(a->o) || !aligned16(a->z) || !aligned16(a->out) ||
+        (a->w && !aligned16(a->w)))
+        return GDR_ERR_MISALIGNED;
+    if (a->out == a->o && (a->out_dtype != a->o_dtype || p.out_stride != p.o_stride))
+        return GDR_ERR_INVALID_ARG;
+    p.rows = a->rows;
+    p.eps = a->eps;
+    p.o = a->o; p.z = a->z; p.w = a->w; p.out = a->out;
+    return from_cuda(gdr::launch_rmsnorm_gated(p, a->d, a->o_dtype == GDR_BF16,
+                                               a->z_dtype == GDR_BF16,
+                                               a->out_dtype == GDR_BF16, (cudaStream_t)stream));
+}
+
+// Shape checks shared by the workspace query and the prefill call.  Fills
+// *chunk_out with the chunk the launch will use.
+static gdr_status check_prefill(const gdr_prefill_args *a, int *chunk_out) {
+    if (!a) return GDR_ERR_INVALID_ARG;
+    if (a->n_seq < 0 || a->n_tok < 0) return GDR_ERR_INVALID_ARG;
+    if (!dtype_ok(a->in_dtype) || !dtype_ok(a->out_dtype)) return GDR_ERR_INVALID_ARG;
+    GDR_TRY(check_heads(a->H_k, a->H_v, a->d_k, a->d_v));
+    int chunk = a->chunk;
+    if (chunk == 0) chunk = 64;
+    if (chunk != 16 && chunk != 32 && chunk != 64) return GDR_ERR_UNSUPPORTED;
+    if (a->n_tok > 0x7fffffffLL) return GDR_ERR_UNSUPPORTED;
+    if ((int64_t)a->n_seq * a->H_v > 0x7fffffffLL) return GDR_ERR_UNSUPPORTED;
+    *chunk_out = chunk;
+    return GDR_OK;
+}
+
+gdr_status gdr_prefill_workspace_size(const gdr_prefill_args *a, size_t *bytes) {
+    if (!bytes) return GDR_ERR_INVALID_ARG;
+    int chunk = 0;
+    GDR_TRY(check_prefill(a, &chunk));
+    *bytes = 0;
+    return GDR_OK;
+}
+
+gdr_status gdr_prefill_chunked(const gdr_prefill_args *a, void *workspace, size_t ws_bytes,
+                               gdr_stream_t stream) {
+    int chunk = 0;
+    GDR_TRY(check_prefill(a, &chunk));
+    (void)workspace;
+    (void)ws_bytes;
+    if (a->n_seq == 0) return GDR_OK;
+    if (!a->cu_seqlens || !a->cu_seqlens_host) return GDR_ERR_INVALID_ARG;
+    // The host copy of the offsets must start at 0, never fall, and end at n_tok.
+    if (a->cu_seqlens_host[0] != 0 || a->cu_seqlens_host[a->n_seq] != a->n_tok)
+        return GDR_ERR_INVALID_ARG;
+    for (int s = 0; s < a->n_seq; ++s)
+        if (a->cu_seqlens_host[s + 1] < a->cu_seqlens_host[s]) return GDR_ERR_INVALID_ARG;
+    if (a->n_tok > 0 && (!a->q || !a->k || !a->v || !a->g || !a->beta || !a->out))
+        return GDR_ERR_INVALID_ARG;
+    const int d = a->d_k;
+    const size_t ein = dtype_bytes(a->in_dtype), eout = dtype_bytes(a->out_dtype);
+    PrefillParams p;
+    memset(&p, 0, sizeof(p));
+    GDR_TRY(resolve_stride(a->q_stride, (int64_t)a->H_k * d, ein, &p.q_stride));
+    GDR_TRY(resolve_stride(a->k_stride, (int64_t)a->H_k * d, ein, &p.k_stride));
+    GDR_TRY(resolve_stride(a->v_stride, (int64_t)a->H_v * d, ein, &p.v_stride));
+    GDR_TRY(resolve_stride(a->z_stride, (int64_t)a->H_v * d, ein, &p.z_stride));
+    GDR_TRY(resolve_stride(a->out_stride, (int64_t)a->H_v * d, eout, &p.out_stride));
+    if (a->gb_stride < 0 || (a->gb_stride != 0 && a->gb_stride < a->H_v)) return GDR_ERR_INVALID_ARG;
+    p.gb_stride = a->gb_stride == 0 ? a->H_v : a->gb_stride;
+    const void *p16[] = {a->q, a->k, a->v, a->z, a->initial_state, a->final_state, a->out};
+    for (const void *ptr : p16)
+        if (ptr && !aligned16(ptr)) return GDR_ERR_MISALIGNED;
+    if ((a->g && !aligned4(a->g)) || (a->beta && !aligned4(a->beta)) ||
+        (a->norm_w && !aligned4(a->norm_w)) || !aligned4(a->cu_seqlens))
+        return GDR_ERR_MISALIGNED;
+    if (a->initial_state && a->final_state && a->initial_state != a->final_state) {
+        const size_t span = (size_t)a->n_seq * a->H_v * d * d * 4;
+        if (ranges_overlap(a->initial_state, span, a->final_state, span)) return GDR_ERR_INVALID_ARG;
+    }
+    p.n_seq = a->n_seq;
+    p.H_k = a->H_k;
+    p.H_v = a->H_v;
+    p.hv_per_hk = a->H_v / a->H_k;
+    p.qk_l2norm = a->qk_l2norm ? 1 : 0;
+    p.scale = a->scale;
+    p.eps_l2 = a->eps_l2;
+    p.eps_norm = a->eps_norm;
+    p.q = a->q; p.k = a->k; p.v = a->v; p.z = a->z;
+    p.g = a->g; p.beta = a->beta;
+    p.cu_seqlens = a->cu_seqlens;
+    p.initial_state = a->initial_state;
+    p.final_state = a->final_state;
+    p.norm_w = a->norm_w;
+    p.out = a->out;
+    return from_cuda(gdr::launch_prefill_simt(p, d, chunk, a->in_dtype == GDR_BF16,
+                                              a->out_dtype == GDR_BF16, (cudaStream_t)stream));
+}
+
+}  // extern "C"

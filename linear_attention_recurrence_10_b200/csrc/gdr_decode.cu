@@ -1,0 +1,166 @@
+// gdr_decode.cu -- one decode step of the gated delta rule, fused end to end.
+//
+// The decoder the pages describe advances one token per call against a state
+// it keeps across the generation loop (Core ML card for Qwen3.5-0.8B, sections
+// "Model" and "Usage"); the state is a fixed-size matrix per head, so nothing
+// grows with context (Swiftlet post, "How It Works").  Per (sequence b, value
+// head h) this kernel computes, with S the d x d fp32 state (row i = value dim i):
+//
+//   q_hat, k_hat  L2-normalised (q also scaled)
+//   alpha = exp(g),  a = S k_hat,  c = S q_hat            (one pass over S)
+//   delta = beta (v - alpha a)
+//   S'    = alpha S + delta k_hat^T                        (written once)
+//   o     = S' q_hat = alpha c + delta (k_hat . q_hat)
+//   y     = o / sqrt(mean(o^2) + eps) * w * z * sigmoid(z)
+//
+// which is S' = exp(g) S (I - beta k k^T) + beta v k^T, o = S' q expanded so
+// that S is read exactly once and written exactly once: the kernel is bound by
+// HBM bandwidth on the 2 d^2 * 4 bytes of state per head.
+//
+// Thread layout (one CTA per (b, h), 2d threads): each lane owns one float4 of
+// a state row; LPR = d/4 lanes share a row, and every lane holds NS = LPR/2
+// rows of its warp's 16.  The partial sums for a and c (2 NS = LPR values per
+// lane) are reduced with a reduce-scatter butterfly over the LPR lanes, which
+// leaves exactly one finished value per lane (LPR - 1 shuffles instead of
+// 2 NS log2(LPR)): lane gl < NS ends with a of its row, lane gl >= NS with c.
+#include "gdr_common.cuh"
+
+namespace gdr {
+
+template <int D, typename TIN, typename TOUT>
+__global__ void __launch_bounds__(2 * D) decode_kernel(const DecodeParams p) {
+    constexpr int NW = 2 * D / 32;  // warps; each owns 16 state rows
+    constexpr int LPR = D / 4;      // lanes per state row (one float4 each)
+    constexpr int RPP = 32 / LPR;   // rows one warp-wide pass covers
+    constexpr int NS = LPR / 2;     // rows held per lane
+    static_assert(NS * RPP == 16, "each warp owns 16 rows");
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int gl = lane % LPR, rg = lane / LPR;
+    const int b = blockIdx.x / p.H_v;
+    const int hv = blockIdx.x - b * p.H_v;
+    const int hk = hv / p.hv_per_hk;
+    const int col = 4 * gl;
+    const int row0 = warp * 16 + rg;  // row of slot s is row0 + s * RPP
+
+    const size_t head_off = (size_t)hv * D * D;
+    const float *sin = p.state_in + (size_t)b * p.state_stride + head_off;
+    float *sout = p.state_out + (size_t)b * p.state_stride + head_off;
+
+    // Issue every state load first so the whole tile is in flight at once.
+    float4 S[NS];
+#pragma unroll
+    for (int s = 0; s < NS; ++s) S[s] = ld_state4(sin + (size_t)(row0 + s * RPP) * D + col);
+
+    const TIN *qp = static_cast<const TIN *>(p.q) + (size_t)b * p.q_stride + hk * D;
+    const TIN *kp = static_cast<const TIN *>(p.k) + (size_t)b * p.k_stride + hk * D;
+    float4 q4 = Elem<TIN>::load4(qp + col);
+    float4 k4 = Elem<TIN>::load4(kp + col);
+    const float g = __ldg(p.g + (size_t)b * p.gb_stride + hv);
+    const float beta = __ldg(p.beta + (size_t)b * p.gb_stride + hv);
+
+    // Row this lane finishes: lanes gl < NS need v of it, lanes gl >= NS need z.
+    const bool is_a = gl < NS;
+    const int my_row = row0 + (gl % NS) * RPP;
+    float vz = 0.f;
+    if (is_a) {
+        vz = Elem<TIN>::load1(static_cast<const TIN *>(p.v) + (size_t)b * p.v_stride + hv * D +
+                              my_row);
+    } else if (p.z) {
+        vz = Elem<TIN>::load1(static_cast<const TIN *>(p.z) + (size_t)b * p.z_stride + hv * D +
+                              my_row);
+    }
+
+    float qs = p.scale, ks = 1.f;
+    if (p.qk_l2norm) {
+        const float qq = group_sum<LPR>(dot4(q4, q4));
+        const float kk = group_sum<LPR>(dot4(k4, k4));
+        qs *= rsqrtf(qq + p.eps_l2);
+        ks = rsqrtf(kk + p.eps_l2);
+    }
+    q4 = scale4(q4, qs);
+    k4 = scale4(k4, ks);
+    const float kq = group_sum<LPR>(dot4(k4, q4));
+    const float alpha = expf(g);
+
+    // Partial S k and S q over this lane's 4 columns, for each held row.
+    float x[LPR];
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+        x[s] = dot4(S[s], k4);
+        x[NS + s] = dot4(S[s], q4);
+    }
+    // Reduce-scatter: at offset o a lane keeps the half of its 2o values picked
+    // by bit o of gl and adds the partner's copy of that half.
+#pragma unroll
+    for (int o = LPR / 2; o >= 1; o >>= 1) {
+        const bool up = (gl & o) != 0;
+#pragma unroll
+        for (int j = 0; j < o; ++j) {
+            const float send = up ? x[j] : x[j + o];
+            const float keep = up ? x[j + o] : x[j];
+            x[j] = keep + __shfl_xor_sync(kFullMask, send, o);
+        }
+    }
+    // x[0]: a = (S k)_row on lanes gl < NS, c = (S q)_row on lanes gl >= NS.
+    const float delta = beta * (vz - alpha * x[0]);                      // valid where is_a
+    const float delta_c = __shfl_xor_sync(kFullMask, delta, NS);         // row's delta on c-lanes
+    const float o_val = fmaf(alpha, x[0], delta_c * kq);                 // valid where !is_a
+
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+        const float d = __shfl_sync(kFullMask, delta, rg * LPR + s);
+        S[s] = axpby4(S[s], alpha, k4, d);
+        st_state4(sout + (size_t)(row0 + s * RPP) * D + col, S[s]);
+    }
+
+    TOUT *op = static_cast<TOUT *>(p.out) + (size_t)b * p.out_stride + hv * D;
+    if (p.z == nullptr) {
+        if (!is_a) Elem<TOUT>::store1(op + my_row, o_val);
+        return;
+    }
+    __shared__ float red[NW];
+    float ss = is_a ? 0.f : o_val * o_val;
+    ss = group_sum<32>(ss);
+    if (lane == 0) red[warp] = ss;
+    __syncthreads();
+    float tot = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) tot += red[w];
+    if (!is_a) {
+        const float rstd = rsqrtf(tot * (1.0f / D) + p.eps_norm);
+        const float wv = p.norm_w ? __ldg(p.norm_w + my_row) : 1.0f;
+        Elem<TOUT>::store1(op + my_row, o_val * rstd * wv * silu(vz));
+    }
+}
+
+template <int D, typename TIN, typename TOUT>
+static cudaError_t launch_decode_t(const DecodeParams &p, cudaStream_t stream) {
+    const unsigned grid = (unsigned)((int64_t)p.batch * p.H_v);
+    decode_kernel<D, TIN, TOUT><<<grid, 2 * D, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_decode_d(const DecodeParams &p, int in_bf16, int out_bf16,
+                                   cudaStream_t s) {
+    if (in_bf16) {
+        return out_bf16 ? launch_decode_t<D, __nv_bfloat16, __nv_bfloat16>(p, s)
+                        : launch_decode_t<D, __nv_bfloat16, float>(p, s);
+    }
+    return out_bf16 ? launch_decode_t<D, float, __nv_bfloat16>(p, s)
+                    : launch_decode_t<D, float, float>(p, s);
+}
+
+cudaError_t launch_decode(const DecodeParams &p, int d, int in_bf16, int out_bf16,
+                          cudaStream_t s) {
+    switch (d) {
+        case 16: return launch_decode_d<16>(p, in_bf16, out_bf16, s);
+        case 32: return launch_decode_d<32>(p, in_bf16, out_bf16, s);
+        case 64: return launch_decode_d<64>(p, in_bf16, out_bf16, s);
+        case 128: return launch_decode_d<128>(p, in_bf16, out_bf16, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace gdr

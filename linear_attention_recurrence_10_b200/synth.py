@@ -118,3 +118,40 @@ def make_inputs(seqlens, H_k, H_v, d, *, seed, dtype=torch.bfloat16, g_mode="sof
     w = torch.ones(d, dtype=torch.float32, device=device)
     return Inputs(q, k, v, z, g.contiguous(), beta.contiguous(), s0, w, cu, H_k, H_v, d,
                   seed, {"g_mode": g_mode, "s0_std": s0_std, "dtype": str(dtype)})
+
+
+@dataclass
+class DecodeInputs:
+    """Per-step decode inputs for L independent layers: slot t of every tensor is
+    the token that step t feeds to each of the B sequences.
+
+    q, k [L, T, B, H_k, d]   v, z [L, T, B, H_v, d]   g, beta [L, T, B, H_v] fp32
+    s0 [L, B, H_v, d, d] fp32   w [d] fp32
+    """
+    q: torch.Tensor
+    k: torch.Tensor
+    v: torch.Tensor
+    z: torch.Tensor
+    g: torch.Tensor
+    beta: torch.Tensor
+    s0: torch.Tensor
+    w: torch.Tensor
+
+
+def make_decode_inputs(L, T, B, H_k, H_v, d, *, seed, dtype=torch.bfloat16, s0_std=0.02,
+                       g_mode="softplus", device="cpu") -> DecodeInputs:
+    """Same value recipe as make_inputs, in the [layer, step, batch, head, dim] layout."""
+    q = normal((L, T, B, H_k, d), seed, "q", device=device).to(dtype)
+    k = normal((L, T, B, H_k, d), seed, "k", device=device).to(dtype)
+    v = normal((L, T, B, H_v, d), seed, "v", device=device).to(dtype)
+    z = normal((L, T, B, H_v, d), seed, "z", device=device).to(dtype)
+    beta = torch.sigmoid(normal((L, T, B, H_v), seed, "beta", device=device))
+    if g_mode == "softplus":
+        g = -torch.nn.functional.softplus(normal((L, T, B, H_v), seed, "g", device=device))
+    elif g_mode == "long":
+        g = torch.log(uniform((L, T, B, H_v), seed, "g", 0.9, 1.0, device=device))
+    else:
+        raise ValueError(f"unknown g_mode {g_mode!r}")
+    s0 = normal((L, B, H_v, d, d), seed, "s0", std=s0_std, device=device)
+    w = torch.ones(d, dtype=torch.float32, device=device)
+    return DecodeInputs(q, k, v, z, g.contiguous(), beta.contiguous(), s0, w)

@@ -1,0 +1,146 @@
+"""Chunked prefill (gdr_prefill_chunked) against the fp64 oracle on seeded inputs.
+
+Besides direct parity, two equivalences from the Swiftlet post ("Correctness &
+Validation": incremental decoding matches whole-sequence processing):
+decode steps after a prefill equal one longer prefill, and a prefill split in
+two with the state handed over equals the whole prefill.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import linear_attention_recurrence_10_b200 as gdr
+import oracle
+from gdr_testutil import TOL, f64, oracle_full, rel_l2, run_decode, run_prefill, sub_problem
+from linear_attention_recurrence_10_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _check(inp, out, final, dtype, ref=None):
+    ref = ref or oracle_full(inp)
+    e_out = rel_l2(f64(out), ref.y)
+    e_state = rel_l2(f64(final), ref.state)
+    assert e_out <= TOL[dtype]["out"], f"output rel-L2 {e_out:.3e}"
+    assert e_state <= TOL[dtype]["state"], f"state rel-L2 {e_state:.3e}"
+    return ref
+
+
+def test_tiny_fp32_chunk16():
+    """B=1, 2 heads, d=16, T=64, fp32, chunk 16, seed 0: chunked vs the recurrence."""
+    inp = synth.make_inputs([64], 2, 2, 16, seed=0, dtype=torch.float32)
+    out, final = run_prefill(inp, chunk=16)
+    _check(inp, out, final, torch.float32)
+
+
+@pytest.mark.parametrize("d", [16, 32, 64, 128])
+@pytest.mark.parametrize("chunk", [16, 32, 64])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_shapes_ragged(d, chunk, dtype):
+    """Several chunks, ragged last chunks, an empty sequence, GVA heads."""
+    lens = [1, chunk + 3, 0, 2 * chunk, 3 * chunk - 5]
+    inp = synth.make_inputs(lens, 2, 4, d, seed=200 + d + chunk, dtype=dtype, s0_std=0.02)
+    out, final = run_prefill(inp, chunk=chunk)
+    _check(inp, out, final, dtype)
+
+
+def test_no_initial_state_and_no_gate():
+    inp = synth.make_inputs([70, 33], 2, 2, 128, seed=21, dtype=torch.bfloat16)
+    ref = oracle_full(inp)
+    out, final = run_prefill(inp, chunk=64, initial_state=None)
+    _check(inp, out, final, torch.bfloat16, ref=ref)
+    raw, _ = run_prefill(inp, chunk=64, initial_state=None, with_z=False)
+    assert rel_l2(f64(raw), ref.o) <= 2e-3
+
+
+def test_in_place_state():
+    inp = synth.make_inputs([40, 90], 1, 2, 64, seed=22, dtype=torch.float32, s0_std=0.02)
+    ref = oracle_full(inp)
+    x = inp.to("cuda")
+    cu = torch.tensor(inp.cu_seqlens, dtype=torch.int32, device="cuda")
+    out = torch.empty(inp.n_tok, 2, 64, device="cuda")
+    st = x.s0.clone()
+    gdr.prefill_chunked(x.q, x.k, x.v, x.g, x.beta, cu, out, z=x.z, norm_w=x.w,
+                        initial_state=st, final_state=st, chunk=32)
+    torch.cuda.synchronize()
+    assert rel_l2(f64(st), ref.state) <= 1e-5
+    assert rel_l2(f64(out), ref.y) <= 1e-5
+
+
+def test_reset_clamp():
+    """g = -inf inside chunks: the chunk form clamps g at -64, which changes
+    nothing visible next to O(1) terms."""
+    inp = synth.make_inputs([100], 2, 2, 128, seed=23, dtype=torch.float32, s0_std=0.02)
+    g = inp.g.clone()
+    g[[3, 64, 99]] = -math.inf
+    inp.g = g
+    out, final = run_prefill(inp, chunk=64)
+    _check(inp, out, final, torch.float32)
+
+
+def test_decode_after_prefill_equals_longer_prefill():
+    T1, T2 = 100, 12
+    inp = synth.make_inputs([T1 + T2] * 2, 2, 2, 128, seed=24, dtype=torch.bfloat16,
+                            s0_std=0.02)
+    whole_out, whole_state = run_prefill(inp, chunk=64)
+    # Prefill the first T1 tokens, then T2 decode steps from its final state.
+    idx = torch.cat([torch.arange(s * (T1 + T2), s * (T1 + T2) + T1) for s in range(2)])
+    tail = torch.cat([torch.arange(s * (T1 + T2) + T1, (s + 1) * (T1 + T2)) for s in range(2)])
+    a = synth.Inputs(inp.q[idx], inp.k[idx], inp.v[idx], inp.z[idx], inp.g[idx], inp.beta[idx],
+                     inp.s0, inp.w, [0, T1, 2 * T1], inp.H_k, inp.H_v, inp.d, inp.seed)
+    a_out, a_state = run_prefill(a, chunk=64)
+    b = synth.Inputs(inp.q[tail], inp.k[tail], inp.v[tail], inp.z[tail], inp.g[tail],
+                     inp.beta[tail], a_state.cpu(), inp.w, [0, T2, 2 * T2], inp.H_k, inp.H_v,
+                     inp.d, inp.seed)
+    b_out, b_state = run_decode(b, T2)
+    assert rel_l2(f64(b_state), f64(whole_state)) <= 1e-5
+    w = f64(whole_out).reshape(2, T1 + T2, 2, 128)
+    assert rel_l2(f64(b_out).reshape(2, T2, 2, 128), w[:, T1:]) <= 1e-5
+    assert rel_l2(f64(a_out).reshape(2, T1, 2, 128), w[:, :T1]) <= 1e-6
+
+
+def test_split_prefill_equals_whole():
+    T, m = 300, 129
+    inp = synth.make_inputs([T], 2, 4, 128, seed=25, dtype=torch.bfloat16, s0_std=0.02)
+    whole_out, whole_state = run_prefill(inp)
+    parts = []
+    s0 = inp.s0
+    for lo, hi in ((0, m), (m, T)):
+        sl = slice(lo, hi)
+        p = synth.Inputs(inp.q[sl], inp.k[sl], inp.v[sl], inp.z[sl], inp.g[sl], inp.beta[sl],
+                         s0, inp.w, [0, hi - lo], inp.H_k, inp.H_v, inp.d, inp.seed)
+        o, s = run_prefill(p)
+        parts.append(o)
+        s0 = s.cpu()
+    assert rel_l2(f64(s0), f64(whole_state)) <= 1e-5
+    assert rel_l2(f64(torch.cat(parts)), f64(whole_out)) <= 1e-5
+
+
+@pytest.mark.slow
+def test_qwen35_prefill_full():
+    """Qwen3.5-0.8B-shaped prefill: B=4, T=4096, 16 heads, d=128, bf16, chunk 64,
+    S_0 = 0; sampled (sequence, head) pairs against the oracle."""
+    inp = synth.make_inputs([4096] * 4, 16, 16, 128, seed=2, dtype=torch.bfloat16)
+    out, final = run_prefill(inp, chunk=64)
+    for s, h in [(0, 0), (3, 15), (1, 7), (2, 12)]:
+        ref = oracle.gdr_recurrent(**sub_problem(inp, s, h))
+        t0, t1 = inp.cu_seqlens[s], inp.cu_seqlens[s + 1]
+        assert rel_l2(f64(out[t0:t1, h]), ref.y[:, 0]) <= 2e-3, (s, h)
+        assert rel_l2(f64(final[s, h]), ref.state[0, 0]) <= 1e-3, (s, h)
+
+
+@pytest.mark.slow
+def test_long_context_gva_prefill_full():
+    """Long-context GVA prefill: 8 sequences, lengths U{1024..32768} (seed 4),
+    16 key / 32 value heads, d=128, bf16, chunk 64, exp(g) in [0.9, 1)."""
+    lens = synth.lengths(8, 4, 1024, 32768)
+    inp = synth.make_inputs(lens, 16, 32, 128, seed=4, dtype=torch.bfloat16, g_mode="long")
+    out, final = run_prefill(inp, chunk=64)
+    shortest = int(np.argmin(lens))
+    for s, h in [(shortest, 0), (shortest, 31), (int(np.argmax(lens)), 5)]:
+        ref = oracle.gdr_recurrent(**sub_problem(inp, s, h))
+        t0, t1 = inp.cu_seqlens[s], inp.cu_seqlens[s + 1]
+        assert rel_l2(f64(out[t0:t1, h]), ref.y[:, 0]) <= 2e-3, (s, h)
+        assert rel_l2(f64(final[s, h]), ref.state[0, 0]) <= 1e-3, (s, h)

@@ -139,6 +139,7 @@ class DecodeBench:
         self.state = x.s0.clone()
         self.out = torch.empty(layers, B, H_V, D, device=device, dtype=torch.bfloat16)
         self.graphs = []
+        self.overlap = layers > 1
         self.bytes_per_step = layers * decode_bytes_per_layer_step(B, H_K, H_V, D)
         self.launches_per_step = layers
 
@@ -146,8 +147,11 @@ class DecodeBench:
         x = x or self.x
         out = self.out if out is None else out
         for l in range(self.L):
+            # Consecutive launches touch different layers' states, so each may
+            # start loading its state while the previous layer's kernel drains.
             self.gdr.decode_step(x.q[l, t], x.k[l, t], x.v[l, t], x.g[l, t], x.beta[l, t],
-                                 self.state[l], out[l], z=x.z[l, t], norm_w=x.w)
+                                 self.state[l], out[l], z=x.z[l, t], norm_w=x.w,
+                                 overlap_state_load=self.overlap)
 
     def capture(self):
         s = torch.cuda.Stream()

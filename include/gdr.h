@@ -34,8 +34,10 @@
  *  - Layout.  Activations are token-major and head-contiguous: element
  *    (row, head, i) of a [rows, H, d] tensor is at row*row_stride + head*d + i,
  *    where row_stride (in elements) defaults to H*d when passed as 0.
- *  - Alignment.  Every pointer must be 16-byte aligned and every row stride a
- *    multiple of 16 bytes (GDR_ERR_MISALIGNED otherwise).
+ *  - Alignment.  Pointers to rows of d values (q, k, v, z, out, o, states,
+ *    and the RMSNormGated weight w) must be 16-byte aligned and their row
+ *    strides multiples of 16 bytes; g, beta, cu_seqlens and the mixer's
+ *    norm_w need 4-byte alignment (GDR_ERR_MISALIGNED otherwise).
  *  - Threads.  Calls are independent and may be made from several host
  *    threads at once.
  */
@@ -86,7 +88,23 @@ typedef struct CUstream_st *gdr_stream_t;
  *   `scale` still multiplies q.  g = -inf is allowed (state reset).
  *   Supported: d_k == d_v in {16, 32, 64, 128}, H_v a multiple of H_k.
  *   batch == 0 is a no-op.  state_stride must be >= H_v*d_v*d_k (0 = that).
+ *   flags: 0 or GDR_DECODE_OVERLAP_STATE_LOAD (below); other bits are
+ *   rejected with GDR_ERR_INVALID_ARG.
  * ------------------------------------------------------------------------ */
+/* gdr_decode_args.flags
+ *
+ * GDR_DECODE_OVERLAP_STATE_LOAD: the decode kernel is launched as a
+ * programmatic dependent of the kernel queued just before it on the stream and
+ * may start reading the state while that kernel is still finishing (q, k, v,
+ * z, g, beta are always read after it has finished).  Set it only when that
+ * preceding kernel does not write this call's state -- e.g. consecutive
+ * decode calls of different layers.  Kernels of this library let their own
+ * dependents start only after everything queued before them has finished, so
+ * a chain of such calls is safe as long as each call's immediate predecessor
+ * leaves its state alone.  Without the flag the state is read only after
+ * the preceding kernel has finished. */
+#define GDR_DECODE_OVERLAP_STATE_LOAD 1
+
 typedef struct gdr_decode_args {
     int32_t batch, H_k, H_v, d_k, d_v;
     int32_t in_dtype;  /* gdr_dtype of q, k, v, z */
@@ -95,7 +113,7 @@ typedef struct gdr_decode_args {
     float scale;       /* multiplies q_hat; 1.0 for the plain o_t = S_t q_t */
     float eps_l2;      /* under the square root of the q/k norms */
     float eps_norm;    /* added to mean(o^2) in RMSNormGated */
-    int32_t reserved;  /* must be 0 */
+    int32_t flags;     /* 0, or GDR_DECODE_OVERLAP_STATE_LOAD */
     int64_t q_stride, k_stride, v_stride, z_stride, gb_stride, out_stride;
     int64_t state_stride;
     const void *q, *k, *v, *z;

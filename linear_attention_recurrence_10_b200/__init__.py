@@ -80,13 +80,16 @@ def status_string(status: int) -> str:
 
 def decode_step(q, k, v, g, beta, state, out, *, z=None, norm_w=None, state_out=None,
                 scale: float = 1.0, eps_l2: float = 1e-6, eps_norm: float = 1e-6,
-                qk_l2norm: bool = True, stream=None) -> torch.Tensor:
+                qk_l2norm: bool = True, overlap_state_load: bool = False,
+                stream=None) -> torch.Tensor:
     """Advance every sequence of the batch by one token (gdr_decode_step).
 
     q, k [B, H_k, d]; v, z [B, H_v, d] (bf16 or fp32, same dtype); g, beta
     [B, H_v] fp32; state [B, H_v, d, d] fp32, updated in place unless
     ``state_out`` is given; out [B, H_v, d] bf16 or fp32.  Batch rows may be
     strided views (e.g. one step of a [B, T, H, d] tensor).
+    ``overlap_state_load``: GDR_DECODE_OVERLAP_STATE_LOAD -- only when the
+    kernel queued just before this call does not write this state.
     """
     B, H_k, d = q.shape
     H_v = v.shape[1]
@@ -105,6 +108,7 @@ def decode_step(q, k, v, g, beta, state, out, *, z=None, norm_w=None, state_out=
             raise TypeError(f"{name} must have the dtype of q")
     a.out_dtype = _dtype_code(out, "out")
     a.qk_l2norm = int(bool(qk_l2norm))
+    a.flags = _abi.GDR_DECODE_OVERLAP_STATE_LOAD if overlap_state_load else 0
     a.scale, a.eps_l2, a.eps_norm = float(scale), float(eps_l2), float(eps_norm)
     a.q_stride, a.k_stride = _row_stride(q, "q"), _row_stride(k, "k")
     a.v_stride = _row_stride(v, "v")

@@ -15,6 +15,7 @@ HEADER = os.path.join(os.path.dirname(PKG), "include", "gdr.h")
 
 GDR_F32 = 0
 GDR_BF16 = 1
+GDR_DECODE_OVERLAP_STATE_LOAD = 1
 
 STATUS_NAMES = {
     0: "GDR_OK", 1: "GDR_ERR_INVALID_ARG", 2: "GDR_ERR_UNSUPPORTED", 3: "GDR_ERR_MISALIGNED",
@@ -31,7 +32,7 @@ class DecodeArgs(ctypes.Structure):
     _fields_ = [
         ("batch", _i32), ("H_k", _i32), ("H_v", _i32), ("d_k", _i32), ("d_v", _i32),
         ("in_dtype", _i32), ("out_dtype", _i32), ("qk_l2norm", _i32),
-        ("scale", _f32), ("eps_l2", _f32), ("eps_norm", _f32), ("reserved", _i32),
+        ("scale", _f32), ("eps_l2", _f32), ("eps_norm", _f32), ("flags", _i32),
         ("q_stride", _i64), ("k_stride", _i64), ("v_stride", _i64), ("z_stride", _i64),
         ("gb_stride", _i64), ("out_stride", _i64), ("state_stride", _i64),
         ("q", _vp), ("k", _vp), ("v", _vp), ("z", _vp), ("g", _vp), ("beta", _vp),

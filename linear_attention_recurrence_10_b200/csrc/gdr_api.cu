@@ -13,6 +13,9 @@ cudaError_t launch_rmsnorm_gated(const NormParams &p, int d, int o_bf16, int z_b
                                  cudaStream_t s);
 cudaError_t launch_prefill_simt(const PrefillParams &p, int d, int chunk, int in_bf16,
                                 int out_bf16, cudaStream_t s);
+size_t prefill_tc_workspace_bytes(int n_seq);
+cudaError_t launch_prefill_tc(const PrefillParams &p, void *workspace, int out_bf16,
+                              cudaStream_t s);
 }  // namespace gdr
 
 namespace {
@@ -80,7 +83,8 @@ int gdr_version(void) { return 100; }
 
 gdr_status gdr_decode_step(const gdr_decode_args *a, gdr_stream_t stream) {
     if (!a) return GDR_ERR_INVALID_ARG;
-    if (a->batch < 0 || a->reserved != 0) return GDR_ERR_INVALID_ARG;
+    if (a->batch < 0 || (a->flags & ~GDR_DECODE_OVERLAP_STATE_LOAD) != 0)
+        return GDR_ERR_INVALID_ARG;
     if (!dtype_ok(a->in_dtype) || !dtype_ok(a->out_dtype)) return GDR_ERR_INVALID_ARG;
     GDR_TRY(check_heads(a->H_k, a->H_v, a->d_k, a->d_v));
     if (a->batch == 0) return GDR_OK;
@@ -113,6 +117,7 @@ gdr_status gdr_decode_step(const gdr_decode_args *a, gdr_stream_t stream) {
     p.H_v = a->H_v;
     p.hv_per_hk = a->H_v / a->H_k;
     p.qk_l2norm = a->qk_l2norm ? 1 : 0;
+    p.overlap_state_load = (a->flags & GDR_DECODE_OVERLAP_STATE_LOAD) ? 1 : 0;
     p.scale = a->scale;
     p.eps_l2 = a->eps_l2;
     p.eps_norm = a->eps_norm;
@@ -167,11 +172,20 @@ static gdr_status check_prefill(const gdr_prefill_args *a, int *chunk_out) {
     return GDR_OK;
 }
 
+// bf16 inputs with d = 128 and chunk 64 run on the tensor cores.
+static bool tensor_core_path(const gdr_prefill_args *a, int chunk) {
+    return a->in_dtype == GDR_BF16 && a->d_k == 128 && chunk == 64;
+}
+
+static size_t workspace_bytes(const gdr_prefill_args *a, int chunk) {
+    return tensor_core_path(a, chunk) ? gdr::prefill_tc_workspace_bytes(a->n_seq) : 0;
+}
+
 gdr_status gdr_prefill_workspace_size(const gdr_prefill_args *a, size_t *bytes) {
     if (!bytes) return GDR_ERR_INVALID_ARG;
     int chunk = 0;
     GDR_TRY(check_prefill(a, &chunk));
-    *bytes = 0;
+    *bytes = workspace_bytes(a, chunk);
     return GDR_OK;
 }
 
@@ -179,8 +193,6 @@ gdr_status gdr_prefill_chunked(const gdr_prefill_args *a, void *workspace, size_
                                gdr_stream_t stream) {
     int chunk = 0;
     GDR_TRY(check_prefill(a, &chunk));
-    (void)workspace;
-    (void)ws_bytes;
     if (a->n_seq == 0) return GDR_OK;
     if (!a->cu_seqlens || !a->cu_seqlens_host) return GDR_ERR_INVALID_ARG;
     // The host copy of the offsets must start at 0, never fall, and end at n_tok.
@@ -211,6 +223,11 @@ gdr_status gdr_prefill_chunked(const gdr_prefill_args *a, void *workspace, size_
         const size_t span = (size_t)a->n_seq * a->H_v * d * d * 4;
         if (ranges_overlap(a->initial_state, span, a->final_state, span)) return GDR_ERR_INVALID_ARG;
     }
+    const size_t need = workspace_bytes(a, chunk);
+    if (need > 0) {
+        if (!workspace || ws_bytes < need) return GDR_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return GDR_ERR_MISALIGNED;
+    }
     p.n_seq = a->n_seq;
     p.H_k = a->H_k;
     p.H_v = a->H_v;
@@ -226,6 +243,9 @@ gdr_status gdr_prefill_chunked(const gdr_prefill_args *a, void *workspace, size_
     p.final_state = a->final_state;
     p.norm_w = a->norm_w;
     p.out = a->out;
+    if (tensor_core_path(a, chunk))
+        return from_cuda(gdr::launch_prefill_tc(p, workspace, a->out_dtype == GDR_BF16,
+                                                (cudaStream_t)stream));
     return from_cuda(gdr::launch_prefill_simt(p, d, chunk, a->in_dtype == GDR_BF16,
                                               a->out_dtype == GDR_BF16, (cudaStream_t)stream));
 }

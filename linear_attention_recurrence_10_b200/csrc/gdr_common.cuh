@@ -16,6 +16,7 @@ constexpr unsigned kFullMask = 0xffffffffu;
 struct DecodeParams {
     int batch, H_k, H_v, hv_per_hk;
     int qk_l2norm;
+    int overlap_state_load;  // read the state before waiting on the previous kernel
     float scale, eps_l2, eps_norm;
     int64_t q_stride, k_stride, v_stride, z_stride, gb_stride, out_stride, state_stride;
     const void *q, *k, *v, *z;
@@ -98,6 +99,20 @@ __device__ __forceinline__ void st_state4(float *p, float4 v) {
     asm volatile("st.global.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y),
                  "f"(v.z), "f"(v.w)
                  : "memory");
+}
+
+// ------------------------------------------- programmatic dependent launch
+
+// Wait until the kernel queued before this one has finished and its writes
+// are visible (a no-op when this kernel was not launched as a dependent).
+__device__ __forceinline__ void wait_for_predecessor() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// Allow the next kernel on the stream to start launching.  Called only after
+// wait_for_predecessor(), so a dependent never starts while anything queued
+// before this kernel is still running.
+__device__ __forceinline__ void release_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ----------------------------------------------------------------- math

@@ -47,10 +47,15 @@ __global__ void __launch_bounds__(2 * D) decode_kernel(const DecodeParams p) {
     const float *sin = p.state_in + (size_t)b * p.state_stride + head_off;
     float *sout = p.state_out + (size_t)b * p.state_stride + head_off;
 
-    // Issue every state load first so the whole tile is in flight at once.
+    // Issue every state load first so the whole tile is in flight at once.  With
+    // overlap_state_load the caller guarantees that the kernel before this one
+    // does not write the state, so the loads may run while it finishes.
+    if (!p.overlap_state_load) wait_for_predecessor();
     float4 S[NS];
 #pragma unroll
     for (int s = 0; s < NS; ++s) S[s] = ld_state4(sin + (size_t)(row0 + s * RPP) * D + col);
+    if (p.overlap_state_load) wait_for_predecessor();
+    release_dependents();
 
     const TIN *qp = static_cast<const TIN *>(p.q) + (size_t)b * p.q_stride + hk * D;
     const TIN *kp = static_cast<const TIN *>(p.k) + (size_t)b * p.k_stride + hk * D;
@@ -134,10 +139,26 @@ __global__ void __launch_bounds__(2 * D) decode_kernel(const DecodeParams p) {
     }
 }
 
+// Launched as a programmatic dependent of the previous kernel on the stream:
+// its blocks may be scheduled while that kernel drains, and wait in
+// wait_for_predecessor() before touching anything it may have written.
 template <int D, typename TIN, typename TOUT>
 static cudaError_t launch_decode_t(const DecodeParams &p, cudaStream_t stream) {
-    const unsigned grid = (unsigned)((int64_t)p.batch * p.H_v);
-    decode_kernel<D, TIN, TOUT><<<grid, 2 * D, 0, stream>>>(p);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((int64_t)p.batch * p.H_v));
+    cfg.blockDim = dim3(2 * D);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<D, TIN, TOUT>, p);
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return e;
+    }
     return cudaGetLastError();
 }
 

@@ -66,7 +66,7 @@ DECODE_CASES = [
     ("null_state", dict(state_in=None), INVALID),
     ("null_out", dict(out=None), INVALID),
     ("negative_batch", dict(batch=-1), INVALID),
-    ("reserved_set", dict(reserved=1), INVALID),
+    ("unknown_flag", dict(flags=2), INVALID),
     ("bad_in_dtype", dict(in_dtype=7), INVALID),
     ("bad_out_dtype", dict(out_dtype=-1), INVALID),
     ("heads_not_multiple", dict(H_k=3, H_v=4), INVALID),
@@ -161,6 +161,21 @@ def test_prefill_workspace_query(lib):
     assert lib.gdr_prefill_workspace_size(ctypes.byref(a), None) == INVALID
     a, host = _prefill_args(chunk=40)
     assert lib.gdr_prefill_workspace_size(ctypes.byref(a), ctypes.byref(n)) == UNSUPPORTED
+
+
+@host_only
+def test_prefill_workspace_required(lib):
+    # bf16, d = 128, chunk 64 runs on the tensor cores and needs a workspace.
+    a, host = _prefill_args()
+    n = ctypes.c_size_t(0)
+    assert lib.gdr_prefill_workspace_size(ctypes.byref(a), ctypes.byref(n)) == OK
+    assert n.value >= 16 + 4 * a.n_seq
+    assert lib.gdr_prefill_chunked(ctypes.byref(a), None, 0, None) == WORKSPACE
+    assert lib.gdr_prefill_chunked(ctypes.byref(a), FAKE + (12 << 32), n.value - 1, None) == WORKSPACE
+    assert lib.gdr_prefill_chunked(ctypes.byref(a), FAKE + (12 << 32) + 8, n.value, None) == MISALIGNED
+    # fp32 inputs use the CUDA-core path, which needs none.
+    a, host = _prefill_args(in_dtype=0)
+    assert lib.gdr_prefill_workspace_size(ctypes.byref(a), ctypes.byref(n)) == OK and n.value == 0
 
 
 @host_only

@@ -162,7 +162,9 @@ gdr_status gdr_decode_step(const gdr_decode_args *args, gdr_stream_t stream);
  *   (chunk 64 with d = 128 needs the tensor-core path).
  *   workspace: device memory of at least gdr_prefill_workspace_size() bytes,
  *   16-byte aligned, owned by the caller, free for reuse once the queued work
- *   has finished.
+ *   has finished.  When the size is non-zero its first 4 bytes (int32) hold,
+ *   once the work has finished, 0 or GDR_ERR_TIMEOUT if a bounded device-side
+ *   wait gave up (the outputs of that call are then incomplete).
  * ------------------------------------------------------------------------ */
 typedef struct gdr_prefill_args {
     int32_t n_seq, H_k, H_v, d_k, d_v;
@@ -190,6 +192,33 @@ gdr_status gdr_prefill_workspace_size(const gdr_prefill_args *args, size_t *byte
 
 gdr_status gdr_prefill_chunked(const gdr_prefill_args *args, void *workspace,
                                size_t workspace_bytes, gdr_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * gdr_prefill_chunked without a caller-provided workspace.
+ *
+ * The pages have no counterpart of this entry point; it exists for callers
+ * that cannot allocate device memory where they run the prefill -- a runtime
+ * that hands all free device memory to its own pools at start-up, or a plain
+ * C caller embedding the library with no memory manager.  It allocates
+ * nothing: the workspace is a fixed array inside the library's own device
+ * memory (about 16 KB, held by every GPU that loads the library until the
+ * process exits), and calls no cudaMalloc or cudaFree.
+ *
+ *   Arguments, results and errors are those of gdr_prefill_chunked, plus:
+ *   n_seq > GDR_PREFILL_NOALLOC_MAX_SEQS returns GDR_ERR_WORKSPACE (nothing
+ *   is queued); GDR_ERR_CUDA if the array's device address cannot be found.
+ *   The first call on a device looks the array's address up for that device
+ *   (the device must be current); make that first call before any stream
+ *   capture.
+ *   Every call shares the one array per device: calls that may run at the
+ *   same time on the GPU (different streams, or host threads, without
+ *   ordering between them) race on it and must not be made.  Each call
+ *   rewrites everything it reads from the array before reading it, so
+ *   results never depend on an earlier call.
+ * ------------------------------------------------------------------------ */
+#define GDR_PREFILL_NOALLOC_MAX_SEQS 4096
+
+gdr_status gdr_prefill_chunked_noalloc(const gdr_prefill_args *args, gdr_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * RMSNormGated on its own (the output gate of the mixer; Qwen3.5 Chat guide,

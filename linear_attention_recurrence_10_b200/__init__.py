@@ -19,7 +19,8 @@ import torch
 from . import _abi
 from ._abi import GDR_BF16, GDR_F32
 
-__all__ = ["GdrError", "decode_step", "prefill_chunked", "prefill_workspace_size",
+__all__ = ["GdrError", "decode_step", "prefill_chunked", "prefill_chunked_noalloc",
+           "prefill_workspace_size",
            "rmsnorm_gated", "version", "status_string"]
 
 
@@ -201,6 +202,24 @@ def prefill_chunked(q, k, v, g, beta, cu_seqlens, out, *, cu_seqlens_host=None, 
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(L.gdr_prefill_chunked(ctypes.byref(a), ws_ptr, ws_bytes, _stream(stream, q.device)),
            "gdr_prefill_chunked")
+    del host
+    return out
+
+
+def prefill_chunked_noalloc(q, k, v, g, beta, cu_seqlens, out, *, cu_seqlens_host=None,
+                            z=None, norm_w=None, initial_state=None, final_state=None,
+                            chunk: int = 0, scale: float = 1.0, eps_l2: float = 1e-6,
+                            eps_norm: float = 1e-6, qk_l2norm: bool = True,
+                            stream=None) -> torch.Tensor:
+    """gdr_prefill_chunked_noalloc: the same prefill, with no workspace to pass and
+    nothing allocated -- for callers that cannot allocate device memory here.
+    At most 4096 sequences per call; calls must not overlap on the GPU (they
+    share one scratch array per device).  Arguments as prefill_chunked."""
+    a, host = _prefill_args(q, k, v, g, beta, cu_seqlens, out, cu_seqlens_host, z, norm_w,
+                            initial_state, final_state, chunk, scale, eps_l2, eps_norm,
+                            qk_l2norm)
+    _check(_abi.lib().gdr_prefill_chunked_noalloc(ctypes.byref(a), _stream(stream, q.device)),
+           "gdr_prefill_chunked_noalloc")
     del host
     return out
 

@@ -16,6 +16,7 @@ HEADER = os.path.join(os.path.dirname(PKG), "include", "gdr.h")
 GDR_F32 = 0
 GDR_BF16 = 1
 GDR_DECODE_OVERLAP_STATE_LOAD = 1
+GDR_PREFILL_NOALLOC_MAX_SEQS = 4096
 
 STATUS_NAMES = {
     0: "GDR_OK", 1: "GDR_ERR_INVALID_ARG", 2: "GDR_ERR_UNSUPPORTED", 3: "GDR_ERR_MISALIGNED",
@@ -89,6 +90,8 @@ def lib(path: str = LIB_PATH) -> ctypes.CDLL:
     h.gdr_prefill_workspace_size.restype = ctypes.c_int
     h.gdr_prefill_chunked.argtypes = [ctypes.POINTER(PrefillArgs), _vp, ctypes.c_size_t, _vp]
     h.gdr_prefill_chunked.restype = ctypes.c_int
+    h.gdr_prefill_chunked_noalloc.argtypes = [ctypes.POINTER(PrefillArgs), _vp]
+    h.gdr_prefill_chunked_noalloc.restype = ctypes.c_int
     h.gdr_rmsnorm_gated.argtypes = [ctypes.POINTER(NormArgs), _vp]
     h.gdr_rmsnorm_gated.restype = ctypes.c_int
     h.gdr_status_string.argtypes = [ctypes.c_int]

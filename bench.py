@@ -348,6 +348,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=16)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--batch", type=int, default=BATCH)
+    ap.add_argument("--slots", type=int, default=SLOTS,
+                    help="distinct per-step inputs, cycled (fewer holds less device memory)")
     ap.add_argument("--e2e-steps", type=int, default=1024)
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -372,7 +374,7 @@ def main():
     from linear_attention_recurrence_10_b200 import build
     build.build(quiet=True)
 
-    bench = DecodeBench(device, seed=1 + rank, B=args.batch)
+    bench = DecodeBench(device, seed=1 + rank, B=args.batch, slots=args.slots)
     bench.capture()
     bench.run(0, args.warmup)
     torch.cuda.synchronize()

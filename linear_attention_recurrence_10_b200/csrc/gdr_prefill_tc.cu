@@ -8,29 +8,35 @@
 // (d_v x d_k fp32), raw bf16 rows q_r, k_r, v_r, n_r = 1/|k_r|,
 // m_r = scale/|q_r| and gamma_r the running sum of g inside the chunk:
 //
-//   [KK; QK] = [K; Q] K^T                                bf16 MMA (exact products)
-//   A_rs = beta_r e^{gamma_r-gamma_s} n_r n_s KK_rs  (s<r)     on CUDA cores
-//   P_rs = e^{gamma_r-gamma_s} m_r n_s QK_rs         (s<=r)
-//   T    = (I + A)^{-1}                                 blocked, fp32, CUDA cores
-//   U^T  = V^T (T diag(beta))^T                         tf32 MMA
-//   W    = T diag(beta e^gamma n) K                     tf32 MMA
-//   Delta^T = U^T - S_bf16 W^T                          bf16 MMA into the U^T accumulator
-//   O^T  = diag-scaled S_bf16 Q^T + Delta^T P^T         bf16 + tf32 MMA
-//   S    = e^{gamma_L} S + (Delta^T diag(e^{gamma_L-gamma} n)) K   tf32 MMA into TMEM
+//   [KK; QK] = [K; Q] K^T                                     (exact bf16 products)
+//   A_rs = beta_r e^{gamma_r-gamma_s} n_r n_s KK_rs    (s<r)   on CUDA cores
+//   P_rs = e^{gamma_r-gamma_s} m_r n_s QK_rs           (s<=r)
+//   T    = (I + A)^{-1}                                       blocked, fp32, CUDA cores
+//   U^T  = V^T (T diag(beta))^T
+//   W^T  = K^T (T diag(beta e^gamma n))^T
+//   Delta^T = U^T - S W^T                                     (into the U^T accumulator)
+//   O^T  = diag-scaled S Q^T + Delta^T P^T
+//   S    = e^{gamma_L} S + (Delta^T diag(e^{gamma_L-gamma} n)) K     (into the TMEM state)
 //   y    = RMSNormGated(O) -> out
 //
 // which is the chunkwise (WY / UT transform) form of
 // S_t = e^{g_t} S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T, o_t = S_t q_t.
-// The state lives in tensor memory in fp32 for the whole sequence; the MMAs
-// that read it see a bf16 copy.  Which operands may be bf16 was decided by
-// emulating every rounding point against the fp64 recurrence: the inverse T,
-// P and Delta must stay tf32 or better; S and W may be bf16.
+//
+// Every MMA is kind::f16 with bf16 operands and fp32 accumulation in tensor
+// memory.  The fp32 state stays in tensor memory for the whole sequence; the
+// MMAs that read it see a bf16 copy (harmless: emulating every rounding point
+// against the fp64 recurrence showed S and W may be bf16).  The computed
+// operands that must keep more precision -- T diag(beta), T diag(beta e^gamma n),
+// P, Delta and the decayed Delta -- are split into hi + lo bf16 pairs
+// (x = hi + lo to ~16 bits) and multiplied term by term (for P Delta:
+// hi*hi + hi*lo + lo*hi).  q, k, v enter the MMAs as the exact bf16 inputs.
 //
 // One CTA (256 threads) owns one (sequence, value head) and walks its chunks
-// in order.  Sequences are taken longest first (the order is written to the
-// workspace by a small pre-kernel).  Every mbarrier wait is bounded by a
-// wall-clock deadline; on expiry the CTA records GDR_ERR_TIMEOUT in the
-// workspace status word, frees its tensor memory and returns.
+// in order; each chunk's inputs are fetched by cp.async one chunk ahead.
+// Sequences are taken longest first (order written to the workspace by a
+// pre-kernel).  Every mbarrier wait is bounded by a wall-clock deadline; on
+// expiry the CTA records GDR_ERR_TIMEOUT in the workspace status word, frees
+// its tensor memory and returns.
 #include "gdr_common.cuh"
 #include "gdr_tc.cuh"
 
@@ -49,58 +55,125 @@ constexpr float kGammaFloor = -64.0f;
 constexpr int kTimeoutStatus = 6;  // GDR_ERR_TIMEOUT
 
 // Shared memory map (bytes).
-constexpr uint32_t OFF_KQ = 0;          // bf16 [K;Q] K-major, 128 rows x 128 (32 KB)
-constexpr uint32_t OFF_VT = 32768;      // fp32 V^T K-major [i][s] (32 KB); later O staging [r][i]
-constexpr uint32_t OFF_KT = 65536;      // fp32 K^T K-major [j][s] (32 KB)
-constexpr uint32_t OFF_SCR = 98304;     // fp32 A, T [64][65], X [3][16][16]; later W bf16, later Dt~
-constexpr uint32_t OFF_TBW = 135168;    // fp32 TB, TW K-major [r][s] (16 KB each); later Delta^T
-constexpr uint32_t OFF_P = 167936;      // fp32 P K-major [r][s] (16 KB)
-constexpr uint32_t OFF_S = 184320;      // bf16 S K-major [i][j] (32 KB)
-constexpr uint32_t OFF_SCAL = 217088;   // per-token scalars and the mbarrier
+constexpr uint32_t OFF_KQ = 0;          // 2 x bf16 [K;Q], 128 rows x 128, row-group major (32 KB each)
+constexpr uint32_t OFF_V = 65536;       // bf16 V, MN-major over d_v (16 KB)
+constexpr uint32_t OFF_Z = 81920;       // bf16 z rows [s][i] (16 KB)
+constexpr uint32_t OFF_SCR = 98304;     // fp32 A, T [64][65], X; later W^T tile; later Dt~ hi/lo
+constexpr uint32_t OFF_TBW = 135168;    // TB hi/lo, TW hi/lo (8 KB each); later Delta hi/lo; later O
+constexpr uint32_t OFF_P = 167936;      // P hi/lo (8 KB each)
+constexpr uint32_t OFF_S = 184320;      // bf16 S [i][j] (32 KB)
+constexpr uint32_t OFF_GB = 217088;     // 2 x (g[64], beta[64]) fp32
+constexpr uint32_t OFF_SCAL = 218112;   // per-token scalars, mbarrier
 constexpr uint32_t SMEM_BYTES = OFF_SCAL + 2048;
+constexpr uint32_t KQ_BYTES = 32768;
 
 // Tensor memory columns (512 allocated).
-constexpr uint32_t TM_D1 = 0;     // [KK; QK]           M=128, 64 cols
-constexpr uint32_t TM_U = 64;     // U^T -> Delta^T     M=128, 64 cols
-constexpr uint32_t TM_W = 128;    // W [r][j]           M=64, 128 cols
-constexpr uint32_t TM_OI = 256;   // S Q^T              M=128, 64 cols
-constexpr uint32_t TM_O2 = 320;   // Delta^T P^T        M=128, 64 cols
-constexpr uint32_t TM_S = 384;    // state S [i][j]     M=128, 128 cols
+constexpr uint32_t TM_D1 = 0;     // [KK; QK]         M=128, 64 cols
+constexpr uint32_t TM_U = 64;     // U^T -> Delta^T   M=128, 64 cols
+constexpr uint32_t TM_W = 128;    // W^T [j][r]       M=128, 64 cols
+constexpr uint32_t TM_OI = 192;   // S Q^T            M=128, 64 cols
+constexpr uint32_t TM_O2 = 256;   // Delta^T P^T      M=128, 64 cols
+constexpr uint32_t TM_S = 384;    // state S [i][j]   M=128, 128 cols
 
-// Byte offset of (row, k) in a K-major tile of R rows (16-byte chunks along K).
-__device__ __forceinline__ uint32_t kmaj(int row, int k, int R, int esz) {
-    const int E = 16 / esz;
-    return (uint32_t)((k / E) * (R * 16) + (row >> 3) * 128 + (row & 7) * 16 + (k % E) * esz);
+// Tiles written from registers, K-major: 16-byte chunks along K are R*16 bytes
+// apart, 8-row groups 128 bytes apart (LBO = R*16, SBO = 128).
+__device__ __forceinline__ uint32_t kmaj(int row, int k, int R) {
+    return (uint32_t)((k >> 3) * (R * 16) + (row >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2);
+}
+// The [K;Q] tile: 8-row groups 2048 bytes apart, 16-byte chunks along d 128
+// bytes apart.  K-major over d: LBO = 128, SBO = 2048.  Read as MN-major over
+// d with the tokens as K: SBO = 128, LBO = 2048.
+__device__ __forceinline__ uint32_t kq_off(int row, int j) {
+    return (uint32_t)((row >> 3) * 2048 + (j >> 3) * 128 + (row & 7) * 16 + (j & 7) * 2);
+}
+// V tile, MN-major over d_v with the tokens as K: SBO = 1024, LBO = 128.
+__device__ __forceinline__ uint32_t v_off(int s, int i) {
+    return (uint32_t)((i >> 3) * 1024 + (s >> 3) * 128 + (s & 7) * 16 + (i & 7) * 2);
+}
+// W tile (B operand of S W^T), MN-major over the tokens r with d_k as K:
+// SBO = 2048, LBO = 128.
+__device__ __forceinline__ uint32_t w_off(int j, int r) {
+    return (uint32_t)((r >> 3) * 2048 + (j >> 3) * 128 + (j & 7) * 16 + (r & 7) * 2);
 }
 
-// D (+)= A B^T over `ksteps` instructions; both operands K-major no-swizzle.
-template <Kind KD>
-__device__ __forceinline__ void gemm(uint32_t d, uint32_t a, uint32_t a_lbo, uint32_t b,
-                                     uint32_t b_lbo, int ksteps, uint32_t idesc, bool acc) {
+// D (+)= A B, `ksteps` bf16 instructions of K = 16, advancing A and B by the
+// given byte steps.
+__device__ __forceinline__ void gemm(uint32_t d, uint32_t a, uint32_t a_lbo, uint32_t a_sbo,
+                                     uint32_t a_step, uint32_t b, uint32_t b_lbo, uint32_t b_sbo,
+                                     uint32_t b_step, int ksteps, uint32_t idesc, bool acc) {
     for (int kk = 0; kk < ksteps; ++kk)
-        mma<KD>(d, smem_desc(a + kk * 2 * a_lbo, a_lbo, 128), smem_desc(b + kk * 2 * b_lbo, b_lbo, 128),
-                idesc, (acc || kk > 0) ? 1u : 0u);
+        mma<Kind::BF16>(d, smem_desc(a + kk * a_step, a_lbo, a_sbo),
+                        smem_desc(b + kk * b_step, b_lbo, b_sbo), idesc, (acc || kk > 0) ? 1u : 0u);
 }
 
-// Eight consecutive fp32 values as eight bf16 (round to nearest even) in 16 bytes.
-__device__ __forceinline__ uint4 pack8_bf16(const float (&v)[32], int o) {
+// z * sigmoid(z) with the fast exponential (relative error ~1e-7 here).
+__device__ __forceinline__ float fast_silu(float z) { return z / (1.0f + __expf(-z)); }
+
+// Eight fp32 values as eight bf16 (round to nearest even) in 16 bytes.
+__device__ __forceinline__ uint4 pack8(const float *v) {
     uint4 pk;
-    __nv_bfloat162 b0 = __floats2bfloat162_rn(v[o + 0], v[o + 1]);
-    __nv_bfloat162 b1 = __floats2bfloat162_rn(v[o + 2], v[o + 3]);
-    __nv_bfloat162 b2 = __floats2bfloat162_rn(v[o + 4], v[o + 5]);
-    __nv_bfloat162 b3 = __floats2bfloat162_rn(v[o + 6], v[o + 7]);
+    __nv_bfloat162 b0 = __floats2bfloat162_rn(v[0], v[1]);
+    __nv_bfloat162 b1 = __floats2bfloat162_rn(v[2], v[3]);
+    __nv_bfloat162 b2 = __floats2bfloat162_rn(v[4], v[5]);
+    __nv_bfloat162 b3 = __floats2bfloat162_rn(v[6], v[7]);
     pk.x = *reinterpret_cast<uint32_t *>(&b0);
     pk.y = *reinterpret_cast<uint32_t *>(&b1);
     pk.z = *reinterpret_cast<uint32_t *>(&b2);
     pk.w = *reinterpret_cast<uint32_t *>(&b3);
     return pk;
 }
+// Split eight fp32 values into bf16 hi = rn(x) and lo = rn(x - hi).
+__device__ __forceinline__ void split8(const float *v, uint4 &hi, uint4 &lo) {
+    float h[8], l[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        h[u] = __bfloat162float(__float2bfloat16_rn(v[u]));
+        l[u] = v[u] - h[u];
+    }
+    hi = pack8(h);
+    lo = pack8(l);
+}
+
+// One distance of the blocked triangular inverse: for every pair of 16-blocks
+// (i, j) with i - j = DIST, X = A[i-rows][16j .. 16i) T[16j .. 16i)[j-cols],
+// then T_ij = -T_ii X.  Fully unrolled so the shared-memory loads overlap.
+template <int DIST>
+__device__ __forceinline__ void offdiag_stage(const float *Ascr, float *Tscr, float *Xscr, int tid) {
+    constexpr int NBLK = 4 - DIST, NOUT = NBLK * 256;
+#pragma unroll
+    for (int e0 = 0; e0 < NOUT; e0 += NT) {
+        const int e = e0 + tid;
+        if (NOUT % NT == 0 || e < NOUT) {
+            const int j = e >> 8, i = j + DIST, rr = (e >> 4) & 15, cc = e & 15;
+            const float *arow = Ascr + (16 * i + rr) * LDA + 16 * j;
+            const float *tcol = Tscr + 16 * j * LDA + 16 * j + cc;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int k = 0; k < 16 * DIST; ++k) acc[k & 3] = fmaf(arow[k], tcol[k * LDA], acc[k & 3]);
+            Xscr[e] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int e0 = 0; e0 < NOUT; e0 += NT) {
+        const int e = e0 + tid;
+        if (NOUT % NT == 0 || e < NOUT) {
+            const int j = e >> 8, i = j + DIST, rr = (e >> 4) & 15, cc = e & 15;
+            const float *trow = Tscr + (16 * i + rr) * LDA + 16 * i;
+            const float *xcol = Xscr + (j << 8) + cc;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int k = 0; k < 16; ++k) acc[k & 3] = fmaf(trow[k], xcol[k * 16], acc[k & 3]);
+            Tscr[(16 * i + rr) * LDA + 16 * j + cc] = -((acc[0] + acc[1]) + (acc[2] + acc[3]));
+        }
+    }
+    __syncthreads();
+}
 
 struct Scalars {
     float gam[C], eg[C], bet[C], nk[C], nq[C], dec[C];
     uint64_t bar;
     uint32_t tmem;
-    int abort;
 };
 
 template <typename TOUT>
@@ -127,13 +200,66 @@ __global__ void __launch_bounds__(NT, 1) prefill_tc_kernel(const PrefillParams p
     float *Ascr = reinterpret_cast<float *>(sm + OFF_SCR);
     float *Tscr = Ascr + C * LDA;
     float *Xscr = Tscr + C * LDA;
+    float *gbuf = reinterpret_cast<float *>(sm + OFF_GB);  // [2][g 64 | beta 64]
+
+    // ---- asynchronous input fetches (every thread issues its share) ----------
+    auto fetch_kq = [&](int64_t c0, int L, int buf) {
+        unsigned char *dst = sm + OFF_KQ + buf * KQ_BYTES;
+        for (int e = tid; e < 128 * 16; e += NT) {
+            // lanes take (row % 8, 16-byte chunk) so each quarter-warp fills one
+            // contiguous 128-byte core-matrix column
+            const int row = (e & 7) + 8 * ((e >> 5) & 15);
+            const int jc = ((e >> 3) & 3) + 4 * (e >> 9);
+            const int r = row & 63;
+            const bool in = r < L;
+            const int64_t t = in ? c0 + r : t0;
+            const __nv_bfloat16 *src = row < 64 ? kg + t * p.k_stride + hk * D
+                                                : qg + t * p.q_stride + hk * D;
+            cp_async16(dst + kq_off(row, 8 * jc), src + 8 * jc, in ? 16u : 0u);
+        }
+    };
+    auto fetch_v = [&](int64_t c0, int L) {
+        for (int e = tid; e < C * 16; e += NT) {
+            const int s = (e & 7) + 8 * ((e >> 5) & 7);
+            const int ic = ((e >> 3) & 3) + 4 * (e >> 8);
+            const bool in = s < L;
+            const int64_t t = in ? c0 + s : t0;
+            cp_async16(sm + OFF_V + v_off(s, 8 * ic), vg + t * p.v_stride + hv * D + 8 * ic,
+                       in ? 16u : 0u);
+        }
+    };
+    auto fetch_z = [&](int64_t c0, int L) {
+        if (!zg) return;
+        for (int e = tid; e < C * 16; e += NT) {
+            const int s = e >> 4, ic = e & 15;
+            const bool in = s < L;
+            const int64_t t = in ? c0 + s : t0;
+            cp_async16(sm + OFF_Z + s * 256 + ic * 16, zg + t * p.z_stride + hv * D + 8 * ic,
+                       in ? 16u : 0u);
+        }
+    };
+    auto fetch_gb = [&](int64_t c0, int L, int buf) {
+        if (tid < 2 * C) {
+            const int r = tid & 63;
+            const bool in = r < L;
+            const int64_t t = in ? c0 + r : t0;
+            const float *src = (tid < C ? p.g : p.beta) + t * p.gb_stride + hv;
+            cp_async4(gbuf + buf * 2 * C + tid, src, in ? 4u : 0u);
+        }
+    };
 
     if (warp == 0) tmem_alloc(&sc.tmem, 512);
     if (tid == 0) {
         mbar_init(&sc.bar, 1);
         mbar_fence_init();
-        sc.abort = 0;
     }
+    if (t1 > t0) {
+        const int L0 = (int)((t1 - t0) < C ? (t1 - t0) : C);
+        fetch_kq(t0, L0, 0);
+        fetch_gb(t0, L0, 0);
+        fetch_v(t0, L0);
+    }
+    cp_async_commit();
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
@@ -174,118 +300,100 @@ __global__ void __launch_bounds__(NT, 1) prefill_tc_kernel(const PrefillParams p
             const int j0 = 64 * half + 32 * cc;
             float v[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = s0 ? s0[j0 + j] : 0.f;
+            for (int j4 = 0; j4 < 8; ++j4) {
+                float4 x = s0 ? *reinterpret_cast<const float4 *>(s0 + j0 + 4 * j4)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+                v[4 * j4] = x.x; v[4 * j4 + 1] = x.y; v[4 * j4 + 2] = x.z; v[4 * j4 + 3] = x.w;
+            }
             tmem_st32(tm + lane_off + TM_S + j0, v);
 #pragma unroll
             for (int j8 = 0; j8 < 4; ++j8)
-                *reinterpret_cast<uint4 *>(sm + OFF_S + kmaj(i, j0 + 8 * j8, D, 2)) = pack8_bf16(v, 8 * j8);
+                *reinterpret_cast<uint4 *>(sm + OFF_S + kmaj(i, j0 + 8 * j8, D)) = pack8(v + 8 * j8);
         }
     }
 
-    const uint32_t ID_BF_64 = instr_desc<Kind::BF16>(128, 64, false, false);
-    const uint32_t ID_BF_64_NEG = instr_desc<Kind::BF16>(128, 64, false, false, true);
-    const uint32_t ID_TF_64 = instr_desc<Kind::TF32>(128, 64, false, false);
-    const uint32_t ID_TF_128 = instr_desc<Kind::TF32>(128, 128, false, false);
-    const uint32_t ID_TF_M64_128 = instr_desc<Kind::TF32>(64, 128, false, false);
+    const uint32_t ID_KK = instr_desc<Kind::BF16>(128, 64, false, false);
+    const uint32_t ID_U = instr_desc<Kind::BF16>(128, 64, true, false);     // A = V, MN-major
+    const uint32_t ID_D = instr_desc<Kind::BF16>(128, 64, false, true, true);  // -S, B = W MN-major
+    const uint32_t ID_S = instr_desc<Kind::BF16>(128, 128, false, true);    // B = K, MN-major
+    const uint32_t aKQ = sbase + OFF_KQ;
 
+    float4 w4 = make_float4(1.f, 1.f, 1.f, 1.f);  // RMSNormGated weight of this lane's 4 columns
+    if (p.norm_w)
+        w4 = make_float4(__ldg(p.norm_w + 4 * lane), __ldg(p.norm_w + 4 * lane + 1),
+                         __ldg(p.norm_w + 4 * lane + 2), __ldg(p.norm_w + 4 * lane + 3));
     bool alive = true;
-    for (int64_t c0 = t0; c0 < t1 && alive; c0 += C) {
+    int buf = 0;
+    for (int64_t c0 = t0; c0 < t1 && alive; c0 += C, buf ^= 1) {
         const int L = (int)((t1 - c0) < C ? (t1 - c0) : C);
+        const int64_t n0 = c0 + C;
+        const int Ln = (int)((t1 - n0) < C ? (t1 - n0) : C);
+        const uint32_t kq = aKQ + buf * KQ_BYTES;
+        const unsigned char *kqp = sm + OFF_KQ + buf * KQ_BYTES;
+        const float *gb = gbuf + buf * 2 * C;
 
-        // ---- P1: inputs.  [K;Q] bf16 tile: lanes take (row % 8, 16-byte chunk) so
-        // that each quarter-warp stores one contiguous 128-byte core-matrix column.
-        for (int e = tid; e < 128 * 16; e += NT) {
-            const int row = (e & 7) + 8 * ((e >> 5) & 15);
-            const int jc = ((e >> 3) & 3) + 4 * (e >> 9);
-            const int r = row & 63;
-            uint4 val = make_uint4(0, 0, 0, 0);
-            if (r < L) {
-                const __nv_bfloat16 *src = row < 64 ? kg + (c0 + r) * p.k_stride + hk * D
-                                                    : qg + (c0 + r) * p.q_stride + hk * D;
-                val = __ldg(reinterpret_cast<const uint4 *>(src + 8 * jc));
-            }
-            *reinterpret_cast<uint4 *>(sm + OFF_KQ + kmaj(row, 8 * jc, 128, 2)) = val;
+        // ---- P1: this chunk's [K;Q], V, g, beta have landed; fetch the next
+        // chunk's [K;Q] and gates and this chunk's z.
+        cp_async_wait<0>();
+        __syncthreads();
+        if (n0 < t1) {
+            fetch_kq(n0, Ln, buf ^ 1);
+            fetch_gb(n0, Ln, buf ^ 1);
         }
-        // V^T fp32 tile [i][s]: one (i, 4 tokens) chunk per step.
-        for (int e = tid; e < D * (C / 4); e += NT) {
-            const int i = e & (D - 1), sc4 = e >> 7;
-            float4 val;
-            float *pv = &val.x;
+        cp_async_commit();
+        fetch_z(c0, L);
+        cp_async_commit();
+
+        // Norms: one row of [K;Q] per thread (zero rows past L give zero).
+        if (tid < 128) {
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int s = 4 * sc4 + u;
-                pv[u] = s < L ? __bfloat162float(vg[(c0 + s) * p.v_stride + hv * D + i]) : 0.f;
+            for (int jc = 0; jc < 16; ++jc) {
+                const uint4 raw = *reinterpret_cast<const uint4 *>(kqp + kq_off(tid, 8 * jc));
+                const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float2 f = __bfloat1622float2(h2[u]);
+                    acc[u] = fmaf(f.x, f.x, fmaf(f.y, f.y, acc[u]));
+                }
             }
-            *reinterpret_cast<float4 *>(sm + OFF_VT + kmaj(i, 4 * sc4, D, 4)) = val;
-        }
-        // Per-token scalars: norms (one warp per row), gates.
-        for (int row = warp; row < 128; row += NW) {
-            const int r = row & 63;
-            float ss = 0.f;
-            if (r < L) {
-                const __nv_bfloat16 *src = row < 64 ? kg + (c0 + r) * p.k_stride + hk * D
-                                                    : qg + (c0 + r) * p.q_stride + hk * D;
-                const float4 x = Elem<__nv_bfloat16>::load4(src + 4 * lane);
-                ss = dot4(x, x);
-            }
-            ss = group_sum<32>(ss);
-            if (lane == 0) {
-                const float f = p.qk_l2norm ? rsqrtf(ss + p.eps_l2) : 1.0f;
-                if (row < 64) sc.nk[r] = r < L ? f : 0.f;
-                else sc.nq[r] = r < L ? f * p.scale : 0.f;
-            }
-        }
-        if (warp == 0) {
-            float ga = 0.f, gb = 0.f, ba = 0.f, bb = 0.f;
-            if (lane < L) {
-                ga = fmaxf(__ldg(p.g + (c0 + lane) * p.gb_stride + hv), kGammaFloor);
-                ba = __ldg(p.beta + (c0 + lane) * p.gb_stride + hv);
-            }
-            if (lane + 32 < L) {
-                gb = fmaxf(__ldg(p.g + (c0 + lane + 32) * p.gb_stride + hv), kGammaFloor);
-                bb = __ldg(p.beta + (c0 + lane + 32) * p.gb_stride + hv);
-            }
+            const float ss = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+            const int r = tid & 63;
+            const float f = p.qk_l2norm ? rsqrtf(ss + p.eps_l2) : 1.0f;
+            if (tid < 64) sc.nk[r] = r < L ? f : 0.f;
+            else sc.nq[r] = r < L ? f * p.scale : 0.f;
+        } else if (warp == 4) {
+            float ga = fmaxf(gb[lane], kGammaFloor), gbv = fmaxf(gb[lane + 32], kGammaFloor);
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const float xa = __shfl_up_sync(kFullMask, ga, o);
-                const float xb = __shfl_up_sync(kFullMask, gb, o);
-                if (lane >= o) { ga += xa; gb += xb; }
+                const float xb = __shfl_up_sync(kFullMask, gbv, o);
+                if (lane >= o) { ga += xa; gbv += xb; }
             }
-            gb += __shfl_sync(kFullMask, ga, 31);
+            gbv += __shfl_sync(kFullMask, ga, 31);
             sc.gam[lane] = ga;
-            sc.gam[lane + 32] = gb;
-            sc.bet[lane] = ba;
-            sc.bet[lane + 32] = bb;
-            sc.eg[lane] = expf(ga);
-            sc.eg[lane + 32] = expf(gb);
+            sc.gam[lane + 32] = gbv;
+            sc.bet[lane] = gb[C + lane];
+            sc.bet[lane + 32] = gb[C + lane + 32];
+            sc.eg[lane] = __expf(ga);
+            sc.eg[lane + 32] = __expf(gbv);
         }
         __syncthreads();
-        if (tid < C) sc.dec[tid] = expf(sc.gam[L - 1] - sc.gam[tid]);
-        // K^T fp32 tile [j][s] from the bf16 tile (rows 0..63 hold K).
-        for (int e = tid; e < D * (C / 4); e += NT) {
-            const int j = e & (D - 1), sc4 = e >> 7;
-            float4 val;
-            float *pv = &val.x;
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-                pv[u] = __bfloat162float(
-                    *reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_KQ + kmaj(4 * sc4 + u, j, 128, 2)));
-            *reinterpret_cast<float4 *>(sm + OFF_KT + kmaj(j, 4 * sc4, D, 4)) = val;
-        }
+        if (tid < C) sc.dec[tid] = __expf(sc.gam[L - 1] - sc.gam[tid]);
 
         // ---- P2: [KK; QK] = [K;Q] K^T and S Q^T (state entering the chunk).
         alive = issue_and_wait([&] {
-            gemm<Kind::BF16>(tm + TM_D1, sbase + OFF_KQ, 2048, sbase + OFF_KQ, 2048, D / 16, ID_BF_64,
-                             false);
-            gemm<Kind::BF16>(tm + TM_OI, sbase + OFF_S, 2048, sbase + OFF_KQ + 1024, 2048, D / 16,
-                             ID_BF_64, false);
+            gemm(tm + TM_D1, kq, 128, 2048, 256, kq, 128, 2048, 256, D / 16, ID_KK, false);
+            gemm(tm + TM_OI, sbase + OFF_S, 2048, 128, 4096, kq + 16384, 128, 2048, 256, D / 16,
+                 ID_KK, false);
         });
         if (!alive) break;
 
-        // ---- P3: A (fp32 scratch) and P (tf32 operand tile).
+        // ---- P3: A (fp32 scratch) and P (hi/lo bf16, K-major [r][s]).
         {
             const int rr = 32 * (quad & 1) + lane;  // token row
             const int s0 = 32 * half;
+            const float gr = sc.gam[rr];
             float v[32];
             tmem_ld32(tm + lane_off + TM_D1 + s0, v);
             if (quad < 2) {
@@ -293,28 +401,30 @@ __global__ void __launch_bounds__(NT, 1) prefill_tc_kernel(const PrefillParams p
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
                     const int s = s0 + c;
-                    Ascr[rr * LDA + s] = s < rr ? f * expf(sc.gam[rr] - sc.gam[s]) * sc.nk[s] * v[c] : 0.f;
+                    Ascr[rr * LDA + s] = s < rr ? f * __expf(gr - sc.gam[s]) * sc.nk[s] * v[c] : 0.f;
                 }
             } else {
                 const float f = sc.nq[rr];
 #pragma unroll
-                for (int c4 = 0; c4 < 8; ++c4) {
-                    float4 w;
-                    float *pw = &w.x;
+                for (int c = 0; c < 32; ++c) {
+                    const int s = s0 + c;
+                    v[c] = s <= rr ? f * __expf(gr - sc.gam[s]) * sc.nk[s] * v[c] : 0.f;
+                }
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int s = s0 + 4 * c4 + u;
-                        pw[u] = s <= rr ? to_tf32(f * expf(sc.gam[rr] - sc.gam[s]) * sc.nk[s] * v[4 * c4 + u])
-                                        : 0.f;
-                    }
-                    *reinterpret_cast<float4 *>(sm + OFF_P + kmaj(rr, s0 + 4 * c4, C, 4)) = w;
+                for (int c8 = 0; c8 < 4; ++c8) {
+                    uint4 hi, lo;
+                    split8(v + 8 * c8, hi, lo);
+                    *reinterpret_cast<uint4 *>(sm + OFF_P + kmaj(rr, s0 + 8 * c8, C)) = hi;
+                    *reinterpret_cast<uint4 *>(sm + OFF_P + 8192 + kmaj(rr, s0 + 8 * c8, C)) = lo;
                 }
             }
         }
         __syncthreads();
 
         // ---- P4: T = (I + A)^{-1}, blocked by 16.  Diagonal blocks first, one
-        // column per thread; then off-diagonal blocks by distance from the diagonal:
+        // column per thread, right-looking (each finished x_s is folded into all
+        // later rows at once, so the dependent chain is 16 steps, not 120); then
+        // the off-diagonal blocks by distance from the diagonal:
         // T_ij = -T_ii sum_{16j <= k < 16i} A[i-rows][k] T[k][j-cols].
         if (tid < C) {
             const int b = tid >> 4, c = tid & 15, base = 16 * b;
@@ -322,132 +432,115 @@ __global__ void __launch_bounds__(NT, 1) prefill_tc_kernel(const PrefillParams p
 #pragma unroll
             for (int r = 0; r < 16; ++r) x[r] = (r == c) ? 1.f : 0.f;
 #pragma unroll
-            for (int r = 1; r < 16; ++r) {
-                if (r > c) {
-                    float acc = 0.f;
+            for (int s = 0; s < 15; ++s) {
 #pragma unroll
-                    for (int s = 0; s < r; ++s) acc = fmaf(Ascr[(base + r) * LDA + base + s], x[s], acc);
-                    x[r] = -acc;
-                }
+                for (int r = s + 1; r < 16; ++r)
+                    x[r] = fmaf(-Ascr[(base + r) * LDA + base + s], x[s], x[r]);
             }
 #pragma unroll
             for (int r = 0; r < 16; ++r) Tscr[(base + r) * LDA + base + c] = x[r];
-        }
-        for (int e = tid; e < C * C; e += NT) {  // zero the blocks above the diagonal
-            const int r = e >> 6, s = e & 63;
-            if ((s >> 4) > (r >> 4)) Tscr[r * LDA + s] = 0.f;
+        } else {
+            for (int e = tid - C; e < C * C; e += NT - C) {  // zero the blocks above the diagonal
+                const int r = e >> 6, s = e & 63;
+                if ((s >> 4) > (r >> 4)) Tscr[r * LDA + s] = 0.f;
+            }
         }
         __syncthreads();
-        for (int dist = 1; dist < 4; ++dist) {
-            const int nblk = 4 - dist;
-            for (int e = tid; e < nblk * 256; e += NT) {
-                const int j = e >> 8, i = j + dist, rr = (e >> 4) & 15, cc = e & 15;
-                float acc = 0.f;
-                for (int k = 16 * j; k < 16 * i; ++k)
-                    acc = fmaf(Ascr[(16 * i + rr) * LDA + k], Tscr[k * LDA + 16 * j + cc], acc);
-                Xscr[e] = acc;
-            }
-            __syncthreads();
-            for (int e = tid; e < nblk * 256; e += NT) {
-                const int j = e >> 8, i = j + dist, rr = (e >> 4) & 15, cc = e & 15;
-                float acc = 0.f;
+        offdiag_stage<1>(Ascr, Tscr, Xscr, tid);
+        offdiag_stage<2>(Ascr, Tscr, Xscr, tid);
+        offdiag_stage<3>(Ascr, Tscr, Xscr, tid);
+        // TB = T diag(beta), TW = T diag(beta e^gamma n): hi/lo bf16 tiles [r][s].
+        for (int e = tid; e < C * (C / 8); e += NT) {
+            const int r = e & 63, s8 = 8 * (e >> 6);
+            float tb[8], tw[8];
 #pragma unroll
-                for (int k = 0; k < 16; ++k)
-                    acc = fmaf(Tscr[(16 * i + rr) * LDA + 16 * i + k], Xscr[(j << 8) + k * 16 + cc], acc);
-                Tscr[(16 * i + rr) * LDA + 16 * j + cc] = -acc;
-            }
-            __syncthreads();
-        }
-        // TB = T diag(beta), TW = T diag(beta e^gamma n): tf32 tiles [r][s].
-        for (int e = tid; e < C * (C / 4); e += NT) {
-            const int r = e & 63, sc4 = e >> 6;
-            float4 tb, tw;
-            float *pb = &tb.x, *pw = &tw.x;
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int s = 4 * sc4 + u;
+            for (int u = 0; u < 8; ++u) {
+                const int s = s8 + u;
                 const float t = Tscr[r * LDA + s];
-                pb[u] = to_tf32(t * sc.bet[s]);
-                pw[u] = to_tf32(t * sc.bet[s] * sc.eg[s] * sc.nk[s]);
+                tb[u] = t * sc.bet[s];
+                tw[u] = t * sc.bet[s] * sc.eg[s] * sc.nk[s];
             }
-            *reinterpret_cast<float4 *>(sm + OFF_TBW + kmaj(r, 4 * sc4, C, 4)) = tb;
-            *reinterpret_cast<float4 *>(sm + OFF_TBW + 16384 + kmaj(r, 4 * sc4, C, 4)) = tw;
+            uint4 hi, lo;
+            split8(tb, hi, lo);
+            *reinterpret_cast<uint4 *>(sm + OFF_TBW + kmaj(r, s8, C)) = hi;
+            *reinterpret_cast<uint4 *>(sm + OFF_TBW + 8192 + kmaj(r, s8, C)) = lo;
+            split8(tw, hi, lo);
+            *reinterpret_cast<uint4 *>(sm + OFF_TBW + 16384 + kmaj(r, s8, C)) = hi;
+            *reinterpret_cast<uint4 *>(sm + OFF_TBW + 24576 + kmaj(r, s8, C)) = lo;
         }
 
-        // ---- P5: U^T = V^T TB^T (M=128), W = TW K (M=64, tokens in lanes).
+        // ---- P5: U^T = V^T TB^T, W^T = K^T TW^T (hi and lo halves).
         alive = issue_and_wait([&] {
-            gemm<Kind::TF32>(tm + TM_U, sbase + OFF_VT, 2048, sbase + OFF_TBW, 1024, C / 8, ID_TF_64,
-                             false);
-            gemm<Kind::TF32>(tm + TM_W, sbase + OFF_TBW + 16384, 1024, sbase + OFF_KT, 2048, C / 8,
-                             ID_TF_M64_128, false);
+            const uint32_t tbw = sbase + OFF_TBW;
+            gemm(tm + TM_U, sbase + OFF_V, 128, 1024, 256, tbw, 1024, 128, 2048, C / 16, ID_U, false);
+            gemm(tm + TM_U, sbase + OFF_V, 128, 1024, 256, tbw + 8192, 1024, 128, 2048, C / 16, ID_U,
+                 true);
+            gemm(tm + TM_W, kq, 2048, 128, 4096, tbw + 16384, 1024, 128, 2048, C / 16, ID_U, false);
+            gemm(tm + TM_W, kq, 2048, 128, 4096, tbw + 24576, 1024, 128, 2048, C / 16, ID_U, true);
         });
         if (!alive) break;
+        // V of this chunk is consumed: fetch the next chunk's.
+        if (n0 < t1) fetch_v(n0, Ln);
+        cp_async_commit();
 
-        // ---- P6: W -> bf16 operand [r][j]; rescale the TMEM state by e^{gamma_L}.
+        // ---- P6: W^T -> bf16 B tile; rescale the TMEM state by e^{gamma_L}.
         {
-            // An M=64 accumulator occupies lanes 0..15 of each 32-lane quadrant;
-            // the warp-wide tcgen05.ld runs on every lane, lanes 16..31 discard.
-            const int r = 16 * quad + (lane & 15);
+            const int j = 32 * quad + lane;
+            const int r0 = 32 * half;
+            float v[32];
+            tmem_ld32(tm + lane_off + TM_W + r0, v);
 #pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                const int j0 = 64 * half + 32 * cc;
-                float v[32];
-                tmem_ld32(tm + lane_off + TM_W + j0, v);
-                if (lane < 16) {
-#pragma unroll
-                    for (int j8 = 0; j8 < 4; ++j8) {
-                        *reinterpret_cast<uint4 *>(sm + OFF_SCR + kmaj(r, j0 + 8 * j8, C, 2)) =
-                            pack8_bf16(v, 8 * j8);
-                    }
-                }
-            }
+            for (int r8 = 0; r8 < 4; ++r8)
+                *reinterpret_cast<uint4 *>(sm + OFF_SCR + w_off(j, r0 + 8 * r8)) = pack8(v + 8 * r8);
             const float eL = sc.eg[L - 1];
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
                 const int j0 = 64 * half + 32 * cc;
-                float v[32];
                 tmem_ld32(tm + lane_off + TM_S + j0, v);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] *= eL;
+                for (int u = 0; u < 32; ++u) v[u] *= eL;
                 tmem_st32(tm + lane_off + TM_S + j0, v);
             }
         }
 
         // ---- P7: Delta^T = U^T - S W^T (accumulates into the U^T columns).
         alive = issue_and_wait([&] {
-            gemm<Kind::BF16>(tm + TM_U, sbase + OFF_S, 2048, sbase + OFF_SCR, 1024, D / 16, ID_BF_64_NEG,
-                             true);
+            gemm(tm + TM_U, sbase + OFF_S, 2048, 128, 4096, sbase + OFF_SCR, 128, 2048, 256, D / 16,
+                 ID_D, true);
         });
         if (!alive) break;
 
-        // ---- P8: Delta^T (tf32 [i][s]) and its decayed, k-normalised copy.
+        // ---- P8: Delta^T hi/lo and its decayed, k-normalised copy, K-major [i][s].
         {
             const int i = 32 * quad + lane;
             const int s0 = 32 * half;
-            float v[32];
+            float v[32], w[32];
             tmem_ld32(tm + lane_off + TM_U + s0, v);
 #pragma unroll
-            for (int c4 = 0; c4 < 8; ++c4) {
-                float4 a, b;
-                float *pa = &a.x, *pb = &b.x;
+            for (int c = 0; c < 32; ++c) w[c] = v[c] * sc.dec[s0 + c] * sc.nk[s0 + c];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int s = s0 + 4 * c4 + u;
-                    const float dlt = v[4 * c4 + u];
-                    pa[u] = to_tf32(dlt);
-                    pb[u] = to_tf32(dlt * sc.dec[s] * sc.nk[s]);
-                }
-                *reinterpret_cast<float4 *>(sm + OFF_TBW + kmaj(i, s0 + 4 * c4, D, 4)) = a;
-                *reinterpret_cast<float4 *>(sm + OFF_SCR + kmaj(i, s0 + 4 * c4, D, 4)) = b;
+            for (int c8 = 0; c8 < 4; ++c8) {
+                uint4 hi, lo;
+                const uint32_t o = kmaj(i, s0 + 8 * c8, D);
+                split8(v + 8 * c8, hi, lo);
+                *reinterpret_cast<uint4 *>(sm + OFF_TBW + o) = hi;
+                *reinterpret_cast<uint4 *>(sm + OFF_TBW + 16384 + o) = lo;
+                split8(w + 8 * c8, hi, lo);
+                *reinterpret_cast<uint4 *>(sm + OFF_SCR + o) = hi;
+                *reinterpret_cast<uint4 *>(sm + OFF_SCR + 16384 + o) = lo;
             }
         }
 
-        // ---- P9: O_intra^T = Delta^T P^T; S += Dt~ K.
+        // ---- P9: O_intra^T = Delta^T P^T (hi*hi + hi*lo + lo*hi); S += Dt~ K.
         alive = issue_and_wait([&] {
-            gemm<Kind::TF32>(tm + TM_O2, sbase + OFF_TBW, 2048, sbase + OFF_P, 1024, C / 8, ID_TF_64,
-                             false);
-            gemm<Kind::TF32>(tm + TM_S, sbase + OFF_SCR, 2048, sbase + OFF_KT, 2048, C / 8, ID_TF_128,
-                             true);
+            const uint32_t dh = sbase + OFF_TBW, dl = dh + 16384;
+            const uint32_t ph = sbase + OFF_P, pl = ph + 8192;
+            gemm(tm + TM_O2, dh, 2048, 128, 4096, ph, 1024, 128, 2048, C / 16, ID_KK, false);
+            gemm(tm + TM_O2, dh, 2048, 128, 4096, pl, 1024, 128, 2048, C / 16, ID_KK, true);
+            gemm(tm + TM_O2, dl, 2048, 128, 4096, ph, 1024, 128, 2048, C / 16, ID_KK, true);
+            const uint32_t eh = sbase + OFF_SCR, el = eh + 16384;
+            gemm(tm + TM_S, eh, 2048, 128, 4096, kq, 2048, 128, 4096, C / 16, ID_S, true);
+            gemm(tm + TM_S, el, 2048, 128, 4096, kq, 2048, 128, 4096, C / 16, ID_S, true);
         });
         if (!alive) break;
 
@@ -459,7 +552,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_tc_kernel(const PrefillParams p
             float a[32], b[32];
             tmem_ld32(tm + lane_off + TM_OI + r0, a);
             tmem_ld32(tm + lane_off + TM_O2 + r0, b);
-            float *Os = reinterpret_cast<float *>(sm + OFF_VT);
+            float *Os = reinterpret_cast<float *>(sm + OFF_TBW);
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
                 const int r = r0 + c;
@@ -472,39 +565,36 @@ __global__ void __launch_bounds__(NT, 1) prefill_tc_kernel(const PrefillParams p
                 tmem_ld32(tm + lane_off + TM_S + j0, v);
 #pragma unroll
                 for (int j8 = 0; j8 < 4; ++j8)
-                    *reinterpret_cast<uint4 *>(sm + OFF_S + kmaj(i, j0 + 8 * j8, D, 2)) =
-                        pack8_bf16(v, 8 * j8);
+                    *reinterpret_cast<uint4 *>(sm + OFF_S + kmaj(i, j0 + 8 * j8, D)) = pack8(v + 8 * j8);
             }
         }
+        cp_async_wait<1>();  // z of this chunk (the next chunk's V may still be in flight)
         __syncthreads();
-        // RMSNormGated per token (one warp per token), store.
+        // RMSNormGated per token (one warp per token, C / NW tokens per warp,
+        // unrolled so the tokens' reductions overlap), store.
         {
-            const float *Os = reinterpret_cast<const float *>(sm + OFF_VT);
-            for (int r = warp; r < L; r += NW) {
-                const int64_t t = c0 + r;
+            const float *Os = reinterpret_cast<const float *>(sm + OFF_TBW);
+#pragma unroll
+            for (int u = 0; u < C / NW; ++u) {
+                const int r = warp + NW * u;
                 const float4 o4 = *reinterpret_cast<const float4 *>(Os + r * D + 4 * lane);
                 float4 y = o4;
                 if (zg) {
                     const float ss = group_sum<32>(dot4(o4, o4));
                     const float rstd = rsqrtf(ss * (1.0f / D) + p.eps_norm);
-                    const float4 z4 = Elem<__nv_bfloat16>::load4(zg + t * p.z_stride + hv * D + 4 * lane);
-                    float4 w4 = make_float4(1.f, 1.f, 1.f, 1.f);
-                    if (p.norm_w) {
-                        w4.x = __ldg(p.norm_w + 4 * lane + 0);
-                        w4.y = __ldg(p.norm_w + 4 * lane + 1);
-                        w4.z = __ldg(p.norm_w + 4 * lane + 2);
-                        w4.w = __ldg(p.norm_w + 4 * lane + 3);
-                    }
-                    y.x = o4.x * rstd * w4.x * silu(z4.x);
-                    y.y = o4.y * rstd * w4.y * silu(z4.y);
-                    y.z = o4.z * rstd * w4.z * silu(z4.z);
-                    y.w = o4.w * rstd * w4.w * silu(z4.w);
+                    const uint2 zr = *reinterpret_cast<const uint2 *>(sm + OFF_Z + r * 256 + 8 * lane);
+                    const float2 za = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&zr.x));
+                    const float2 zb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&zr.y));
+                    y.x = o4.x * rstd * w4.x * fast_silu(za.x);
+                    y.y = o4.y * rstd * w4.y * fast_silu(za.y);
+                    y.z = o4.z * rstd * w4.z * fast_silu(zb.x);
+                    y.w = o4.w * rstd * w4.w * fast_silu(zb.y);
                 }
-                Elem<TOUT>::store4(og + t * p.out_stride + hv * D + 4 * lane, y);
+                if (r < L) Elem<TOUT>::store4(og + (c0 + r) * p.out_stride + hv * D + 4 * lane, y);
             }
         }
-        __syncthreads();
     }
+    cp_async_wait<0>();  // nothing may land in shared memory after the CTA ends
 
     // Final state from TMEM.
     if (alive && p.final_state) {

@@ -73,6 +73,20 @@ def load_peaks():
                 "source": "fallback"}
 
 
+def captured_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu capture of `kernel`, or None if
+    there is none or the kernel's source has changed since it was taken."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)[kernel]
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+    except (OSError, KeyError, ValueError):
+        return None
+    return rec["dram_bytes_per_launch"] if digest.startswith(rec["sha256_prefix"]) else None
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle samples while the timed region runs."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -419,7 +433,8 @@ def main():
         "tokens_per_s": args.batch * world * args.steps / (ms * 1e-3),
         "hbm_frac": gbs / world / peaks["hbm_gbs"],
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
-                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": captured_traffic("decode_kernel<128, bf16, bf16>"),
                      "kernel": "decode_kernel<128, bf16, bf16>",
                      "bytes_per_launch": per_launch_bytes, "us_per_launch": per_launch_ms * 1e3,
                      "peak_source": peaks["source"] + " (hbm_gbs, of measured copy bandwidth)"},

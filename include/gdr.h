@@ -160,9 +160,15 @@ gdr_status gdr_decode_step(const gdr_decode_args *args, gdr_stream_t stream);
  *   Supported: d_k == d_v in {16, 32, 64, 128}; bf16 inputs with d = 128 and
  *   chunk 64 (or 0) run on the tensor cores, everything else on CUDA cores
  *   (chunk 64 with d = 128 needs the tensor-core path).
- *   workspace: device memory of at least gdr_prefill_workspace_size() bytes,
- *   16-byte aligned, owned by the caller, free for reuse once the queued work
- *   has finished.  When the size is non-zero its first 4 bytes (int32) hold,
+ *   workspace: device memory, 16-byte aligned, owned by the caller, free for
+ *   reuse once the queued work has finished.  gdr_prefill_workspace_size()
+ *   bytes select the fastest variant: on the tensor-core path that is two
+ *   kernels, the first computing every chunk's state-independent part at
+ *   once into the workspace (about 65 KB per chunk of 64 tokens and value
+ *   head).  A tensor-core call given less, but at least
+ *   (16 + 4 * n_seq) rounded up to 256 bytes, runs as one kernel instead
+ *   (same results up to rounding, less parallel).  Below that:
+ *   GDR_ERR_WORKSPACE.  When the size is non-zero its first 4 bytes (int32) hold,
  *   once the work has finished, 0 or GDR_ERR_TIMEOUT if a bounded device-side
  *   wait gave up (the outputs of that call are then incomplete).
  * ------------------------------------------------------------------------ */

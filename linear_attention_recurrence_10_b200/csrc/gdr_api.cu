@@ -16,6 +16,9 @@ cudaError_t launch_prefill_simt(const PrefillParams &p, int d, int chunk, int in
 size_t prefill_tc_workspace_bytes(int n_seq);
 cudaError_t launch_prefill_tc(const PrefillParams &p, void *workspace, int out_bf16,
                               cudaStream_t s);
+size_t prefill_tc2p_workspace_bytes(int n_seq, int64_t n_chunks, int H_v);
+cudaError_t launch_prefill_tc2p(const PrefillParams &p, int64_t n_chunks, void *workspace,
+                                int out_bf16, cudaStream_t s);
 }  // namespace gdr
 
 namespace {
@@ -177,8 +180,23 @@ static bool tensor_core_path(const gdr_prefill_args *a, int chunk) {
     return a->in_dtype == GDR_BF16 && a->d_k == 128 && chunk == 64;
 }
 
+// Chunks of 64 tokens over all sequences: exact from the host offsets when
+// given, otherwise an upper bound.
+static int64_t count_chunks(const gdr_prefill_args *a) {
+    if (!a->cu_seqlens_host) return a->n_tok / 64 + a->n_seq;
+    int64_t n = 0;
+    for (int s = 0; s < a->n_seq; ++s) {
+        const int64_t len = (int64_t)a->cu_seqlens_host[s + 1] - a->cu_seqlens_host[s];
+        if (len > 0) n += (len + 63) / 64;
+    }
+    return n;
+}
+
+// The tensor-core path runs as two kernels when the workspace holds the
+// per-chunk records, else as one kernel that needs only the sequence order.
 static size_t workspace_bytes(const gdr_prefill_args *a, int chunk) {
-    return tensor_core_path(a, chunk) ? gdr::prefill_tc_workspace_bytes(a->n_seq) : 0;
+    if (!tensor_core_path(a, chunk)) return 0;
+    return gdr::prefill_tc2p_workspace_bytes(a->n_seq, count_chunks(a), a->H_v);
 }
 
 gdr_status gdr_prefill_workspace_size(const gdr_prefill_args *a, size_t *bytes) {
@@ -223,9 +241,12 @@ gdr_status gdr_prefill_chunked(const gdr_prefill_args *a, void *workspace, size_
         const size_t span = (size_t)a->n_seq * a->H_v * d * d * 4;
         if (ranges_overlap(a->initial_state, span, a->final_state, span)) return GDR_ERR_INVALID_ARG;
     }
-    const size_t need = workspace_bytes(a, chunk);
-    if (need > 0) {
-        if (!workspace || ws_bytes < need) return GDR_ERR_WORKSPACE;
+    const bool tc = tensor_core_path(a, chunk);
+    const int64_t n_chunks = tc ? count_chunks(a) : 0;
+    const size_t need_one = tc ? gdr::prefill_tc_workspace_bytes(a->n_seq) : 0;
+    const size_t need_two = tc ? gdr::prefill_tc2p_workspace_bytes(a->n_seq, n_chunks, a->H_v) : 0;
+    if (tc) {
+        if (!workspace || ws_bytes < need_one) return GDR_ERR_WORKSPACE;
         if (!aligned16(workspace)) return GDR_ERR_MISALIGNED;
     }
     p.n_seq = a->n_seq;
@@ -243,7 +264,10 @@ gdr_status gdr_prefill_chunked(const gdr_prefill_args *a, void *workspace, size_
     p.final_state = a->final_state;
     p.norm_w = a->norm_w;
     p.out = a->out;
-    if (tensor_core_path(a, chunk))
+    if (tc && ws_bytes >= need_two)
+        return from_cuda(gdr::launch_prefill_tc2p(p, n_chunks, workspace, a->out_dtype == GDR_BF16,
+                                                  (cudaStream_t)stream));
+    if (tc)
         return from_cuda(gdr::launch_prefill_tc(p, workspace, a->out_dtype == GDR_BF16,
                                                 (cudaStream_t)stream));
     return from_cuda(gdr::launch_prefill_simt(p, d, chunk, a->in_dtype == GDR_BF16,

@@ -1,0 +1,670 @@
+// gdr_prefill_2p.cu -- the tensor-core chunked prefill (bf16, d = 128, chunk 64)
+// as two kernels, for calls whose workspace has room for per-chunk results.
+//
+// Most of a chunk's work does not depend on the state entering it: the gates,
+// the q/k norms, A and P, the inverse T = (I + A)^{-1}, U = T diag(beta) V and
+// W = T diag(beta e^gamma n) K (the chunkwise WY / UT form of the gated delta
+// rule named in the Qwen3.5 Chat guide, section "Architektur").  So:
+//
+//   prep kernel:  one CTA per (chunk, value head), every chunk at once, over
+//                 the whole GPU.  Writes, per unit, a 65 KB record to the
+//                 workspace: W (bf16, already in the MMA operand layout),
+//                 P (hi + lo bf16), U (fp32) and the per-token scalars.
+//   recur kernel: one CTA per (sequence, value head), chunks in order, only
+//                 the state-dependent part:
+//                   Delta^T = U^T - S W^T
+//                   O^T     = diag-scaled S Q^T + Delta^T P^T
+//                   S       = e^{gamma_L} S + (Delta^T diag(e^{gamma_L-gamma} n)) K
+//                   y       = RMSNormGated(O)
+//
+// Arithmetic, operand precisions (bf16 MMAs, hi + lo pairs for T, P, Delta)
+// and layouts are those of the one-kernel version in gdr_prefill_tc.cu.
+#include "gdr_prefill_common.cuh"
+
+namespace gdr {
+namespace tcp2 {
+
+using namespace gdr::tcp;
+
+constexpr int NT = 512;  // threads (16 warps) in both kernels
+constexpr int NW = NT / 32;
+
+// Per-(chunk, value head) record in the workspace.
+// The first REC_STAGED bytes (W, P, scalars) are staged in shared memory by the
+// recurrence; U is read from here straight into registers.
+constexpr uint32_t REC_W = 0;        // bf16 W, MN-major B tile (w_off), 16 KB
+constexpr uint32_t REC_P = 16384;    // P hi, then lo, K-major [r][s] (kmaj R=64), 8 KB each
+constexpr uint32_t REC_SCAL = 32768; // fp32 eg[64] | nqe[64] | dn[64] | eL | pad
+constexpr uint32_t REC_STAGED = 33792;
+constexpr uint32_t REC_U = 33792;    // fp32 U: byte (s/4)*2048 + i*16 + (s%4)*4, 32 KB
+constexpr uint32_t REC_BYTES = 66560;
+__host__ __device__ constexpr uint32_t u_off(int s, int i) {
+    return (uint32_t)((s >> 2) * 2048 + i * 16 + (s & 3) * 4);
+}
+
+// Workspace: status word, longest-first order, chunk offsets, then records.
+struct WsLayout {
+    size_t order, chunk_off, rec, total;
+};
+__host__ __device__ inline WsLayout ws_layout(int n_seq, int64_t n_chunks, int H_v) {
+    WsLayout w;
+    w.order = 16;
+    w.chunk_off = (w.order + 4 * (size_t)n_seq + 15) & ~(size_t)15;
+    w.rec = (w.chunk_off + 4 * ((size_t)n_seq + 1) + 255) & ~(size_t)255;
+    w.total = w.rec + (size_t)n_chunks * H_v * REC_BYTES;
+    return w;
+}
+
+// ------------------------------------------------------------- pre-kernel
+// Longest-first order (as the one-kernel path), the status word, and the
+// running count of chunks before each sequence.  One block of 1024 threads.
+__global__ void __launch_bounds__(1024) plan_kernel(const int32_t *cu, int n_seq, int *status,
+                                                    int *order, int *chunk_off) {
+    __shared__ int part[1024];
+    const int tid = threadIdx.x;
+    if (tid == 0) *status = 0;
+    for (int s = tid; s < n_seq; s += 1024) {
+        const int ls = cu[s + 1] - cu[s];
+        int rank = 0;
+        for (int t = 0; t < n_seq; ++t) {
+            const int lt = cu[t + 1] - cu[t];
+            rank += (lt > ls) || (lt == ls && t < s);
+        }
+        order[rank] = s;
+    }
+    // Exclusive scan of ceil(len / C) over sequences: each thread a contiguous range.
+    const int per = (n_seq + 1023) / 1024;
+    const int lo = tid * per, hi = min(n_seq, lo + per);
+    int sum = 0;
+    for (int s = lo; s < hi; ++s) sum += (cu[s + 1] - cu[s] + C - 1) / C;
+    part[tid] = sum;
+    __syncthreads();
+    for (int o = 1; o < 1024; o <<= 1) {
+        const int add = tid >= o ? part[tid - o] : 0;
+        __syncthreads();
+        part[tid] += add;
+        __syncthreads();
+    }
+    int run = tid ? part[tid - 1] : 0;
+    for (int s = lo; s < hi; ++s) {
+        chunk_off[s] = run;
+        run += (cu[s + 1] - cu[s] + C - 1) / C;
+    }
+    if (tid == 1023) chunk_off[n_seq] = part[1023];
+}
+
+// ------------------------------------------------------------ prep kernel
+
+// 256 threads and ~99 KB of shared memory, so two prep CTAs share an SM and
+// hide each other's latencies.
+constexpr int PNT = 256;
+constexpr int PSL = 512 / PNT;      // 16-column slices of a 64-column accumulator per thread
+constexpr uint32_t A_KQ = 0;        // bf16 [K;Q] (32 KB)
+constexpr uint32_t A_V = 32768;     // bf16 V (16 KB)
+constexpr uint32_t A_T = 49152;     // fp32 T [64][65]
+constexpr uint32_t A_AX = 65792;    // fp32 A [64][65] and X; once T is built, TB/TW (32 KB) over them
+constexpr uint32_t A_TBW = A_AX;
+constexpr uint32_t A_GB = 98560;    // g[64], beta[64]
+constexpr uint32_t A_SCAL = 99072;  // scalars, mbarrier
+constexpr uint32_t A_SMEM = A_SCAL + 2048;
+
+struct PrepScalars {
+    float gam[C], eg[C], bet[C], nk[C], nq[C], dec[C];
+    uint64_t bar;
+    uint32_t tmem;
+};
+
+__global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p, const int *chunk_off,
+                                                     unsigned char *records, int *status) {
+    extern __shared__ __align__(1024) unsigned char sm[];
+    PrepScalars &sc = *reinterpret_cast<PrepScalars *>(sm + A_SCAL);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int quad = warp & 3, part = warp >> 2;
+    const int gchunk = blockIdx.x / p.H_v, hv = blockIdx.x % p.H_v;
+    const int hk = hv / p.hv_per_hk;
+    // The sequence holding this chunk: the last s with chunk_off[s] <= gchunk.
+    int lo = 0, hi = p.n_seq - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (chunk_off[mid] <= gchunk) lo = mid; else hi = mid - 1;
+    }
+    const int seq = lo;
+    const int64_t t0 = p.cu_seqlens[seq], t1 = p.cu_seqlens[seq + 1];
+    const int64_t c0 = t0 + (int64_t)(gchunk - chunk_off[seq]) * C;
+    const int L = (int)((t1 - c0) < C ? (t1 - c0) : C);
+    unsigned char *rec = records + ((size_t)gchunk * p.H_v + hv) * REC_BYTES;
+
+    const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(p.q);
+    const __nv_bfloat16 *kg = static_cast<const __nv_bfloat16 *>(p.k);
+    const __nv_bfloat16 *vg = static_cast<const __nv_bfloat16 *>(p.v);
+    const uint32_t sbase = smem_u32(sm);
+    float *Ascr = reinterpret_cast<float *>(sm + A_AX);
+    float *Xscr = Ascr + C * LDA;
+    float *Tscr = reinterpret_cast<float *>(sm + A_T);
+    float *gbuf = reinterpret_cast<float *>(sm + A_GB);
+
+    if (warp == 0) tmem_alloc(&sc.tmem, 256);
+    if (tid == 0) {
+        mbar_init(&sc.bar, 1);
+        mbar_fence_init();
+    }
+    for (int e = tid; e < 128 * 16; e += PNT) {
+        const int row = (e & 7) + 8 * ((e >> 5) & 15);
+        const int jc = ((e >> 3) & 3) + 4 * (e >> 9);
+        const int r = row & 63;
+        const bool in = r < L;
+        const int64_t t = in ? c0 + r : c0;
+        const __nv_bfloat16 *src = row < 64 ? kg + t * p.k_stride + hk * D : qg + t * p.q_stride + hk * D;
+        cp_async16(sm + A_KQ + kq_off(row, 8 * jc), src + 8 * jc, in ? 16u : 0u);
+    }
+    for (int e = tid; e < C * 16; e += PNT) {
+        const int s = (e & 7) + 8 * ((e >> 5) & 7);
+        const int ic = ((e >> 3) & 3) + 4 * (e >> 8);
+        const bool in = s < L;
+        const int64_t t = in ? c0 + s : c0;
+        cp_async16(sm + A_V + v_off(s, 8 * ic), vg + t * p.v_stride + hv * D + 8 * ic, in ? 16u : 0u);
+    }
+    if (tid < 2 * C) {
+        const int r = tid & 63;
+        const bool in = r < L;
+        const int64_t t = in ? c0 + r : c0;
+        cp_async4(gbuf + tid, (tid < C ? p.g : p.beta) + t * p.gb_stride + hv, in ? 4u : 0u);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tm = sc.tmem;
+    const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
+    constexpr uint32_t TM_D1 = 0, TM_U = 64, TM_W = 128;
+
+    // Norms (one row of [K;Q] per thread) and the running sums of g.
+    if (tid < 128) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int jc = 0; jc < 16; ++jc) {
+            const uint4 raw = *reinterpret_cast<const uint4 *>(sm + A_KQ + kq_off(tid, 8 * jc));
+            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float2 f = __bfloat1622float2(h2[u]);
+                acc[u] = fmaf(f.x, f.x, fmaf(f.y, f.y, acc[u]));
+            }
+        }
+        const float ss = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        const int r = tid & 63;
+        const float f = p.qk_l2norm ? rsqrtf(ss + p.eps_l2) : 1.0f;
+        if (tid < 64) sc.nk[r] = r < L ? f : 0.f;
+        else sc.nq[r] = r < L ? f * p.scale : 0.f;
+    } else if (warp == 4) {
+        float ga = fmaxf(gbuf[lane], kGammaFloor), gb = fmaxf(gbuf[lane + 32], kGammaFloor);
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float xa = __shfl_up_sync(kFullMask, ga, o);
+            const float xb = __shfl_up_sync(kFullMask, gb, o);
+            if (lane >= o) { ga += xa; gb += xb; }
+        }
+        gb += __shfl_sync(kFullMask, ga, 31);
+        sc.gam[lane] = ga;
+        sc.gam[lane + 32] = gb;
+        sc.bet[lane] = gbuf[C + lane];
+        sc.bet[lane + 32] = gbuf[C + lane + 32];
+        sc.eg[lane] = __expf(ga);
+        sc.eg[lane + 32] = __expf(gb);
+    }
+    __syncthreads();
+    if (tid < C) sc.dec[tid] = __expf(sc.gam[L - 1] - sc.gam[tid]);
+
+    uint32_t phase = 0;
+    auto issue_and_wait = [&](auto issue) -> bool {
+        fence_smem_to_async();
+        fence_before_sync();
+        __syncthreads();
+        if (tid == 0) {
+            fence_after_sync();
+            issue();
+            commit(smem_u32(&sc.bar));
+        }
+        const bool ok = mbar_wait(&sc.bar, phase, kWaitNs);
+        phase ^= 1;
+        const int bad = __syncthreads_or(!ok);
+        fence_after_sync();
+        if (bad && tid == 0) atomicExch(status, kTimeoutStatus);
+        return !bad;
+    };
+    const uint32_t ID_KK = instr_desc<Kind::BF16>(128, 64, false, false);
+    const uint32_t ID_U = instr_desc<Kind::BF16>(128, 64, true, false);
+    const uint32_t kq = sbase + A_KQ;
+
+    bool alive = issue_and_wait([&] {
+        gemm(tm + TM_D1, kq, 128, 2048, 256, kq, 128, 2048, 256, D / 16, ID_KK, false);
+    });
+    if (alive) {
+        // A (fp32 scratch) and P (hi/lo bf16 straight into the record).
+        const int rr = 32 * (quad & 1) + lane;
+        const float gr = sc.gam[rr];
+#pragma unroll
+        for (int sl = 0; sl < PSL; ++sl) {
+        const int s0 = 16 * (part * PSL + sl);
+        float v[16];
+        tmem_ld16(tm + lane_off + TM_D1 + s0, v);
+        if (quad < 2) {
+            const float f = sc.bet[rr] * sc.nk[rr];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const int s = s0 + c;
+                Ascr[rr * LDA + s] = s < rr ? f * __expf(gr - sc.gam[s]) * sc.nk[s] * v[c] : 0.f;
+            }
+        } else {
+            const float f = sc.nq[rr];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const int s = s0 + c;
+                v[c] = s <= rr ? f * __expf(gr - sc.gam[s]) * sc.nk[s] * v[c] : 0.f;
+            }
+#pragma unroll
+            for (int c8 = 0; c8 < 2; ++c8) {
+                uint4 h, l;
+                split8(v + 8 * c8, h, l);
+                *reinterpret_cast<uint4 *>(rec + REC_P + kmaj(rr, s0 + 8 * c8, C)) = h;
+                *reinterpret_cast<uint4 *>(rec + REC_P + 8192 + kmaj(rr, s0 + 8 * c8, C)) = l;
+            }
+        }
+        }
+        __syncthreads();
+        invert_unit_lower<PNT>(Ascr, Tscr, Xscr, tid);
+        for (int e = tid; e < C * (C / 8); e += PNT) {
+            const int r = e & 63, s8 = 8 * (e >> 6);
+            float tb[8], tw[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int s = s8 + u;
+                const float t = Tscr[r * LDA + s];
+                tb[u] = t * sc.bet[s];
+                tw[u] = t * sc.bet[s] * sc.eg[s] * sc.nk[s];
+            }
+            uint4 h, l;
+            split8(tb, h, l);
+            *reinterpret_cast<uint4 *>(sm + A_TBW + kmaj(r, s8, C)) = h;
+            *reinterpret_cast<uint4 *>(sm + A_TBW + 8192 + kmaj(r, s8, C)) = l;
+            split8(tw, h, l);
+            *reinterpret_cast<uint4 *>(sm + A_TBW + 16384 + kmaj(r, s8, C)) = h;
+            *reinterpret_cast<uint4 *>(sm + A_TBW + 24576 + kmaj(r, s8, C)) = l;
+        }
+        alive = issue_and_wait([&] {
+            const uint32_t tbw = sbase + A_TBW;
+            gemm(tm + TM_U, sbase + A_V, 128, 1024, 256, tbw, 1024, 128, 2048, C / 16, ID_U, false);
+            gemm(tm + TM_U, sbase + A_V, 128, 1024, 256, tbw + 8192, 1024, 128, 2048, C / 16, ID_U, true);
+            gemm(tm + TM_W, kq, 2048, 128, 4096, tbw + 16384, 1024, 128, 2048, C / 16, ID_U, false);
+            gemm(tm + TM_W, kq, 2048, 128, 4096, tbw + 24576, 1024, 128, 2048, C / 16, ID_U, true);
+        });
+    }
+    if (alive) {
+        // W^T [j][r] -> bf16 MN-major B tile; U^T [i][s] -> fp32 record; scalars.
+        const int x = 32 * quad + lane;  // j for W, i for U
+#pragma unroll
+        for (int sl = 0; sl < PSL; ++sl) {
+        const int c0l = 16 * (part * PSL + sl);
+        float w[16], u[16];
+        tmem_ld16(tm + lane_off + TM_W + c0l, w);
+        tmem_ld16(tm + lane_off + TM_U + c0l, u);
+#pragma unroll
+        for (int r8 = 0; r8 < 2; ++r8)
+            *reinterpret_cast<uint4 *>(rec + REC_W + w_off(x, c0l + 8 * r8)) = pack8(w + 8 * r8);
+#pragma unroll
+        for (int s4 = 0; s4 < 4; ++s4)
+            *reinterpret_cast<float4 *>(rec + REC_U + u_off(c0l + 4 * s4, x)) =
+                make_float4(u[4 * s4], u[4 * s4 + 1], u[4 * s4 + 2], u[4 * s4 + 3]);
+        }
+        float *scal = reinterpret_cast<float *>(rec + REC_SCAL);
+        if (tid < C) {
+            scal[tid] = sc.eg[tid];
+            scal[C + tid] = sc.nq[tid] * sc.eg[tid];
+            scal[2 * C + tid] = sc.dec[tid] * sc.nk[tid];
+        } else if (tid == C) {
+            scal[3 * C] = sc.eg[L - 1];
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        fence_after_sync();
+        tmem_free(tm, 256);
+    }
+}
+
+// ----------------------------------------------------------- recur kernel
+
+constexpr uint32_t B_KQ = 0;          // bf16 [K;Q] (32 KB)
+constexpr uint32_t B_REC = 32768;     // 2 x staged record (W, P, scalars: 33 KB each)
+constexpr uint32_t B_Z = 100352;      // 2 x bf16 z [s][i] (16 KB each)
+constexpr uint32_t B_S = 133120;      // bf16 S [i][j] (32 KB)
+constexpr uint32_t B_DL = 165888;     // Delta hi/lo (32 KB); later O [r][i] fp32
+constexpr uint32_t B_DT = 198656;     // decayed Delta hi/lo (32 KB)
+constexpr uint32_t B_BAR = 231424;    // mbarriers (MMA, 2 records, 2 z), TMEM address
+constexpr uint32_t B_SMEM = B_BAR + 64;
+
+template <typename TOUT>
+__global__ void __launch_bounds__(NT, 1) recur_kernel(const PrefillParams p, const int *order,
+                                                      const int *chunk_off,
+                                                      const unsigned char *records, int *status) {
+    extern __shared__ __align__(1024) unsigned char sm[];
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + B_BAR);
+    uint64_t *rbar = bar + 1;  // [2]: a staged record landed
+    uint64_t *zbar = bar + 3;  // [2]: a chunk's z rows landed
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + B_BAR + 40);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int quad = warp & 3, part = warp >> 2;
+    const int seq = order[blockIdx.x / p.H_v];
+    const int hv = blockIdx.x % p.H_v;
+    const int hk = hv / p.hv_per_hk;
+    const int64_t t0 = p.cu_seqlens[seq], t1 = p.cu_seqlens[seq + 1];
+    const unsigned char *rec0 = records + ((size_t)chunk_off[seq] * p.H_v + hv) * REC_BYTES;
+    const size_t rec_step = (size_t)p.H_v * REC_BYTES;
+
+    const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(p.q);
+    const __nv_bfloat16 *kg = static_cast<const __nv_bfloat16 *>(p.k);
+    const __nv_bfloat16 *zg = static_cast<const __nv_bfloat16 *>(p.z);
+    TOUT *og = static_cast<TOUT *>(p.out);
+    const uint32_t sbase = smem_u32(sm);
+
+    // Half of the [K;Q] tile: K (rows 0..63) is read only by the last MMA of a
+    // chunk and Q (rows 64..127) only by the first, so each is fetched as soon
+    // as the current chunk is done with it.
+    auto fetch_half = [&](int64_t c0, int L, bool q_half) {
+        const __nv_bfloat16 *base = q_half ? qg + hk * D : kg + hk * D;
+        const int64_t stride = q_half ? p.q_stride : p.k_stride;
+        for (int e = tid; e < 64 * 16; e += NT) {
+            const int r = (e & 7) + 8 * ((e >> 5) & 7);
+            const int jc = ((e >> 3) & 3) + 4 * (e >> 8);
+            const bool in = r < L;
+            const int64_t t = in ? c0 + r : t0;
+            cp_async16(sm + B_KQ + kq_off(r + (q_half ? 64 : 0), 8 * jc), base + t * stride + 8 * jc,
+                       in ? 16u : 0u);
+        }
+    };
+    // The staged part of a record is one contiguous block: one bulk copy.
+    auto fetch_rec = [&](const unsigned char *rec, int buf) {
+        if (tid == 0) {
+            bulk_expect(rbar + buf, REC_STAGED);
+            bulk_copy(sm + B_REC + buf * REC_STAGED, rec, REC_STAGED, rbar + buf);
+        }
+    };
+    // z: one bulk copy per token row (256 contiguous bytes of this head).
+    auto fetch_z = [&](int64_t c0, int L, int buf) {
+        if (!zg || warp != 0) return;
+        if (lane == 0) bulk_expect(zbar + buf, (uint32_t)L * 256u);
+        __syncwarp();
+        for (int s = lane; s < L; s += 32)
+            bulk_copy(sm + B_Z + buf * 16384 + s * 256, zg + (c0 + s) * p.z_stride + hv * D, 256u,
+                      zbar + buf);
+    };
+
+    if (warp == 0) tmem_alloc(tmem_slot, 512);
+    if (tid == 0) {
+        for (int i = 0; i < 5; ++i) mbar_init(bar + i, 1);
+        mbar_fence_init();
+    }
+    __syncthreads();
+    if (t1 > t0) {
+        const int L0 = (int)((t1 - t0) < C ? (t1 - t0) : C);
+        fetch_half(t0, L0, true);
+        cp_async_commit();
+        fetch_half(t0, L0, false);
+        fetch_rec(rec0, 0);
+        fetch_z(t0, L0, 0);
+    } else {
+        cp_async_commit();
+    }
+    cp_async_commit();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tm = *tmem_slot;
+    const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
+    constexpr uint32_t TM_OI = 0, TM_D = 64, TM_O2 = 128, TM_S = 256;
+    uint32_t phase = 0;
+    auto issue = [&](auto body) {
+        fence_smem_to_async();
+        fence_before_sync();
+        __syncthreads();
+        if (tid == 0) {
+            fence_after_sync();
+            body();
+            commit(smem_u32(bar));
+        }
+    };
+    auto wait_mma = [&]() -> bool {
+        const bool ok = mbar_wait(bar, phase, kWaitNs);
+        phase ^= 1;
+        const int bad = __syncthreads_or(!ok);
+        fence_after_sync();
+        if (bad && tid == 0) atomicExch(status, kTimeoutStatus);
+        return !bad;
+    };
+
+    // Initial state into TMEM (fp32) and its bf16 copy into smem.
+    {
+        const int i = 32 * quad + lane, j0 = 32 * part;
+        const float *s0 = p.initial_state
+                              ? p.initial_state + ((size_t)seq * p.H_v + hv) * D * D + (size_t)i * D + j0
+                              : nullptr;
+        float v[32];
+#pragma unroll
+        for (int j4 = 0; j4 < 8; ++j4) {
+            const float4 x = s0 ? *reinterpret_cast<const float4 *>(s0 + 4 * j4) : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[4 * j4] = x.x; v[4 * j4 + 1] = x.y; v[4 * j4 + 2] = x.z; v[4 * j4 + 3] = x.w;
+        }
+        tmem_st32(tm + lane_off + TM_S + j0, v);
+#pragma unroll
+        for (int j8 = 0; j8 < 4; ++j8)
+            *reinterpret_cast<uint4 *>(sm + B_S + kmaj(i, j0 + 8 * j8, D)) = pack8(v + 8 * j8);
+    }
+
+    float4 w4 = make_float4(1.f, 1.f, 1.f, 1.f);
+    if (p.norm_w)
+        w4 = make_float4(__ldg(p.norm_w + 4 * lane), __ldg(p.norm_w + 4 * lane + 1),
+                         __ldg(p.norm_w + 4 * lane + 2), __ldg(p.norm_w + 4 * lane + 3));
+    const uint32_t ID_KK = instr_desc<Kind::BF16>(128, 64, false, false);
+    const uint32_t ID_D = instr_desc<Kind::BF16>(128, 64, false, true, true);  // -S, B = W MN-major
+    const uint32_t ID_S = instr_desc<Kind::BF16>(128, 128, false, true);       // B = K, MN-major
+    const uint32_t kq = sbase + B_KQ;
+
+    bool alive = true;
+    const unsigned char *rec = rec0;
+    int it = 0;
+    for (int64_t c0 = t0; c0 < t1 && alive; c0 += C, rec += rec_step, ++it) {
+        const int buf = it & 1;
+        const uint32_t in_phase = (uint32_t)(it >> 1) & 1u;  // use count of this buffer
+        const uint32_t rec_s = sbase + B_REC + buf * REC_STAGED;
+        const float *rscal = reinterpret_cast<const float *>(sm + B_REC + buf * REC_STAGED + REC_SCAL);
+        const unsigned char *zbuf = sm + B_Z + buf * 16384;
+        const int L = (int)((t1 - c0) < C ? (t1 - c0) : C);
+        const int64_t n0 = c0 + C;
+        const int Ln = (int)((t1 - n0) < C ? (t1 - n0) : C);
+
+        // cp.async groups, oldest first: Q(c), K(c) -- Q(c) is needed now.
+        cp_async_wait<1>();  // this chunk's Q
+        {
+            bool ok = mbar_wait(rbar + buf, in_phase, kWaitNs);  // its record
+            if (zg) ok = mbar_wait(zbar + buf, in_phase, kWaitNs) && ok;  // its z rows
+            if (__syncthreads_or(!ok)) {
+                if (tid == 0) atomicExch(status, kTimeoutStatus);
+                alive = false;
+                break;
+            }
+        }
+        // The other buffers were last used by the previous chunk, which is done:
+        // fetch the next chunk's staged record and z a whole chunk ahead.
+        if (n0 < t1) {
+            fetch_rec(rec + rec_step, buf ^ 1);
+            fetch_z(n0, Ln, buf ^ 1);
+        }
+        // U of this chunk, straight into registers for the Delta epilogue.
+        float4 uu[4];
+        {
+            const int i = 32 * quad + lane, s0 = 16 * part;
+#pragma unroll
+            for (int s4 = 0; s4 < 4; ++s4)
+                uu[s4] = __ldg(reinterpret_cast<const float4 *>(rec + REC_U + u_off(s0 + 4 * s4, i)));
+        }
+
+        // O_inter^T = S Q^T and -S W^T, with the state entering the chunk.
+        issue([&] {
+            gemm(tm + TM_OI, sbase + B_S, 2048, 128, 4096, kq + 16384, 128, 2048, 256, D / 16, ID_KK, false);
+            gemm(tm + TM_D, sbase + B_S, 2048, 128, 4096, rec_s + REC_W, 128, 2048, 256, D / 16, ID_D, false);
+        });
+        // Meanwhile: S <- e^{gamma_L} S in TMEM (columns the MMAs do not touch).
+        {
+            const int j0 = 32 * part;
+            const float eL = rscal[3 * C];
+            float v[32];
+            tmem_ld32(tm + lane_off + TM_S + j0, v);
+#pragma unroll
+            for (int u = 0; u < 32; ++u) v[u] *= eL;
+            tmem_st32(tm + lane_off + TM_S + j0, v);
+        }
+        alive = wait_mma();
+        if (!alive) break;
+        if (n0 < t1) fetch_half(n0, Ln, true);  // Q of the next chunk
+        cp_async_commit();
+
+        // Delta^T = U^T - S W^T, as hi/lo tiles, and its decayed, k-normalised copy.
+        {
+            const int i = 32 * quad + lane, s0 = 16 * part;
+            float v[16], w[16];
+            tmem_ld16(tm + lane_off + TM_D + s0, v);
+#pragma unroll
+            for (int s4 = 0; s4 < 4; ++s4) {
+                v[4 * s4] += uu[s4].x; v[4 * s4 + 1] += uu[s4].y;
+                v[4 * s4 + 2] += uu[s4].z; v[4 * s4 + 3] += uu[s4].w;
+            }
+#pragma unroll
+            for (int c = 0; c < 16; ++c) w[c] = v[c] * rscal[2 * C + s0 + c];
+#pragma unroll
+            for (int c8 = 0; c8 < 2; ++c8) {
+                uint4 h, l;
+                const uint32_t o = kmaj(i, s0 + 8 * c8, D);
+                split8(v + 8 * c8, h, l);
+                *reinterpret_cast<uint4 *>(sm + B_DL + o) = h;
+                *reinterpret_cast<uint4 *>(sm + B_DL + 16384 + o) = l;
+                split8(w + 8 * c8, h, l);
+                *reinterpret_cast<uint4 *>(sm + B_DT + o) = h;
+                *reinterpret_cast<uint4 *>(sm + B_DT + 16384 + o) = l;
+            }
+        }
+        // O_intra^T = Delta^T P^T (hi*hi + hi*lo + lo*hi); S += Dt~ K.
+        cp_async_wait<1>();  // this chunk's K (the next chunk's Q may be in flight)
+        issue([&] {
+            const uint32_t dh = sbase + B_DL, dl = dh + 16384, ph = rec_s + REC_P, pl = ph + 8192;
+            gemm(tm + TM_O2, dh, 2048, 128, 4096, ph, 1024, 128, 2048, C / 16, ID_KK, false);
+            gemm(tm + TM_O2, dh, 2048, 128, 4096, pl, 1024, 128, 2048, C / 16, ID_KK, true);
+            gemm(tm + TM_O2, dl, 2048, 128, 4096, ph, 1024, 128, 2048, C / 16, ID_KK, true);
+            const uint32_t eh = sbase + B_DT, el = eh + 16384;
+            gemm(tm + TM_S, eh, 2048, 128, 4096, kq, 2048, 128, 4096, C / 16, ID_S, true);
+            gemm(tm + TM_S, el, 2048, 128, 4096, kq, 2048, 128, 4096, C / 16, ID_S, true);
+        });
+        alive = wait_mma();
+        if (!alive) break;
+
+        // This chunk's K is consumed: fetch the next chunk's.
+        const int r0 = 16 * part;
+        if (n0 < t1) fetch_half(n0, Ln, false);
+        cp_async_commit();
+
+        // O = (m e^gamma)(S Q^T) + Delta P^T staged as [r][i]; the new state's bf16 copy.
+        {
+            const int i = 32 * quad + lane;
+            float a[16], b[16];
+            tmem_ld16(tm + lane_off + TM_OI + r0, a);
+            tmem_ld16(tm + lane_off + TM_O2 + r0, b);
+            float *Os = reinterpret_cast<float *>(sm + B_DL);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) Os[(r0 + c) * D + i] = fmaf(rscal[C + r0 + c], a[c], b[c]);
+            const int j0 = 32 * part;
+            float v[32];
+            tmem_ld32(tm + lane_off + TM_S + j0, v);
+#pragma unroll
+            for (int j8 = 0; j8 < 4; ++j8)
+                *reinterpret_cast<uint4 *>(sm + B_S + kmaj(i, j0 + 8 * j8, D)) = pack8(v + 8 * j8);
+        }
+        __syncthreads();
+        // RMSNormGated per token (one warp per C / NW tokens, unrolled), store.
+        {
+            const float *Os = reinterpret_cast<const float *>(sm + B_DL);
+#pragma unroll
+            for (int u = 0; u < C / NW; ++u) {
+                const int r = warp + NW * u;
+                const float4 o4 = *reinterpret_cast<const float4 *>(Os + r * D + 4 * lane);
+                float4 y = o4;
+                if (zg) {
+                    const float ss = group_sum<32>(dot4(o4, o4));
+                    const float rstd = rsqrtf(ss * (1.0f / D) + p.eps_norm);
+                    const uint2 zr = *reinterpret_cast<const uint2 *>(zbuf + r * 256 + 8 * lane);
+                    const float2 za = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&zr.x));
+                    const float2 zb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&zr.y));
+                    y.x = o4.x * rstd * w4.x * fast_silu(za.x);
+                    y.y = o4.y * rstd * w4.y * fast_silu(za.y);
+                    y.z = o4.z * rstd * w4.z * fast_silu(zb.x);
+                    y.w = o4.w * rstd * w4.w * fast_silu(zb.y);
+                }
+                if (r < L) Elem<TOUT>::store4(og + (c0 + r) * p.out_stride + hv * D + 4 * lane, y);
+            }
+        }
+        __syncthreads();
+    }
+    cp_async_wait<0>();  // nothing may land in shared memory after the CTA ends
+
+    if (alive && p.final_state) {
+        const int i = 32 * quad + lane, j0 = 32 * part;
+        float *dst = p.final_state + ((size_t)seq * p.H_v + hv) * D * D + (size_t)i * D + j0;
+        float v[32];
+        tmem_ld32(tm + lane_off + TM_S + j0, v);
+#pragma unroll
+        for (int j4 = 0; j4 < 8; ++j4)
+            *reinterpret_cast<float4 *>(dst + 4 * j4) = make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        fence_after_sync();
+        tmem_free(tm, 512);
+    }
+}
+
+}  // namespace tcp2
+
+size_t prefill_tc2p_workspace_bytes(int n_seq, int64_t n_chunks, int H_v) {
+    return tcp2::ws_layout(n_seq, n_chunks, H_v).total;
+}
+
+cudaError_t launch_prefill_tc2p(const PrefillParams &p, int64_t n_chunks, void *workspace,
+                                int out_bf16, cudaStream_t s) {
+    const tcp2::WsLayout w = tcp2::ws_layout(p.n_seq, n_chunks, p.H_v);
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    int *status = reinterpret_cast<int *>(ws);
+    int *order = reinterpret_cast<int *>(ws + w.order);
+    int *chunk_off = reinterpret_cast<int *>(ws + w.chunk_off);
+    unsigned char *records = ws + w.rec;
+    tcp2::plan_kernel<<<1, 1024, 0, s>>>(p.cu_seqlens, p.n_seq, status, order, chunk_off);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (n_chunks > 0) {
+        e = cudaFuncSetAttribute(tcp2::prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)tcp2::A_SMEM);
+        if (e != cudaSuccess) return e;
+        tcp2::prep_kernel<<<(unsigned)(n_chunks * p.H_v), tcp2::PNT, tcp2::A_SMEM, s>>>(p, chunk_off,
+                                                                                     records, status);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    auto kern = out_bf16 ? tcp2::recur_kernel<__nv_bfloat16> : tcp2::recur_kernel<float>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcp2::B_SMEM);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)((int64_t)p.n_seq * p.H_v), tcp2::NT, tcp2::B_SMEM, s>>>(p, order, chunk_off,
+                                                                              records, status);
+    return cudaGetLastError();
+}
+
+}  // namespace gdr

@@ -1,0 +1,150 @@
+// gdr_prefill_common.cuh -- pieces shared by the tensor-core prefill kernels:
+// sizes, shared-memory operand layouts, the MMA loop, bf16 hi/lo splitting and
+// the blocked fp32 inverse of the chunk's unit lower-triangular matrix.
+#pragma once
+
+#include "gdr_common.cuh"
+#include "gdr_tc.cuh"
+
+namespace gdr {
+namespace tcp {
+
+using namespace gdr::tc;
+
+constexpr int D = 128;       // d_k = d_v
+constexpr int C = 64;        // chunk
+constexpr int LDA = C + 1;   // padded row stride of the fp32 scratch matrices
+constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s: far beyond any chunk's work
+constexpr float kGammaFloor = -64.0f;
+constexpr int kTimeoutStatus = 6;  // GDR_ERR_TIMEOUT
+
+// Tiles written from registers, K-major: 16-byte chunks along K are R*16 bytes
+// apart, 8-row groups 128 bytes apart (LBO = R*16, SBO = 128).
+__device__ __forceinline__ uint32_t kmaj(int row, int k, int R) {
+    return (uint32_t)((k >> 3) * (R * 16) + (row >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2);
+}
+// The [K;Q] tile: 8-row groups 2048 bytes apart, 16-byte chunks along d 128
+// bytes apart.  K-major over d: LBO = 128, SBO = 2048.  Read as MN-major over
+// d with the tokens as K: SBO = 128, LBO = 2048.
+__device__ __forceinline__ uint32_t kq_off(int row, int j) {
+    return (uint32_t)((row >> 3) * 2048 + (j >> 3) * 128 + (row & 7) * 16 + (j & 7) * 2);
+}
+// V tile, MN-major over d_v with the tokens as K: SBO = 1024, LBO = 128.
+__device__ __forceinline__ uint32_t v_off(int s, int i) {
+    return (uint32_t)((i >> 3) * 1024 + (s >> 3) * 128 + (s & 7) * 16 + (i & 7) * 2);
+}
+// W tile (B operand of S W^T), MN-major over the tokens r with d_k as K:
+// SBO = 2048, LBO = 128.
+__device__ __forceinline__ uint32_t w_off(int j, int r) {
+    return (uint32_t)((r >> 3) * 2048 + (j >> 3) * 128 + (j & 7) * 16 + (r & 7) * 2);
+}
+
+// D (+)= A B, `ksteps` bf16 instructions of K = 16, advancing A and B by the
+// given byte steps.
+__device__ __forceinline__ void gemm(uint32_t d, uint32_t a, uint32_t a_lbo, uint32_t a_sbo,
+                                     uint32_t a_step, uint32_t b, uint32_t b_lbo, uint32_t b_sbo,
+                                     uint32_t b_step, int ksteps, uint32_t idesc, bool acc) {
+    for (int kk = 0; kk < ksteps; ++kk)
+        mma<Kind::BF16>(d, smem_desc(a + kk * a_step, a_lbo, a_sbo),
+                        smem_desc(b + kk * b_step, b_lbo, b_sbo), idesc, (acc || kk > 0) ? 1u : 0u);
+}
+
+// z * sigmoid(z) with the fast exponential (relative error ~1e-7 here).
+__device__ __forceinline__ float fast_silu(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
+
+// Eight fp32 values as eight bf16 (round to nearest even) in 16 bytes.
+__device__ __forceinline__ uint4 pack8(const float *v) {
+    uint4 pk;
+    __nv_bfloat162 b0 = __floats2bfloat162_rn(v[0], v[1]);
+    __nv_bfloat162 b1 = __floats2bfloat162_rn(v[2], v[3]);
+    __nv_bfloat162 b2 = __floats2bfloat162_rn(v[4], v[5]);
+    __nv_bfloat162 b3 = __floats2bfloat162_rn(v[6], v[7]);
+    pk.x = *reinterpret_cast<uint32_t *>(&b0);
+    pk.y = *reinterpret_cast<uint32_t *>(&b1);
+    pk.z = *reinterpret_cast<uint32_t *>(&b2);
+    pk.w = *reinterpret_cast<uint32_t *>(&b3);
+    return pk;
+}
+// Split eight fp32 values into bf16 hi = rn(x) and lo = rn(x - hi).
+__device__ __forceinline__ void split8(const float *v, uint4 &hi, uint4 &lo) {
+    float h[8], l[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        h[u] = __bfloat162float(__float2bfloat16_rn(v[u]));
+        l[u] = v[u] - h[u];
+    }
+    hi = pack8(h);
+    lo = pack8(l);
+}
+
+// One distance of the blocked triangular inverse: for every pair of 16-blocks
+// (i, j) with i - j = DIST, X = A[i-rows][16j .. 16i) T[16j .. 16i)[j-cols],
+// then T_ij = -T_ii X.  Fully unrolled so the shared-memory loads overlap.
+template <int DIST, int NT>
+__device__ __forceinline__ void offdiag_stage(const float *Ascr, float *Tscr, float *Xscr, int tid) {
+    constexpr int NBLK = 4 - DIST, NOUT = NBLK * 256;
+#pragma unroll
+    for (int e0 = 0; e0 < NOUT; e0 += NT) {
+        const int e = e0 + tid;
+        if (NOUT % NT == 0 || e < NOUT) {
+            const int j = e >> 8, i = j + DIST, rr = (e >> 4) & 15, cc = e & 15;
+            const float *arow = Ascr + (16 * i + rr) * LDA + 16 * j;
+            const float *tcol = Tscr + 16 * j * LDA + 16 * j + cc;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int k = 0; k < 16 * DIST; ++k) acc[k & 3] = fmaf(arow[k], tcol[k * LDA], acc[k & 3]);
+            Xscr[e] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int e0 = 0; e0 < NOUT; e0 += NT) {
+        const int e = e0 + tid;
+        if (NOUT % NT == 0 || e < NOUT) {
+            const int j = e >> 8, i = j + DIST, rr = (e >> 4) & 15, cc = e & 15;
+            const float *trow = Tscr + (16 * i + rr) * LDA + 16 * i;
+            const float *xcol = Xscr + (j << 8) + cc;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int k = 0; k < 16; ++k) acc[k & 3] = fmaf(trow[k], xcol[k * 16], acc[k & 3]);
+            Tscr[(16 * i + rr) * LDA + 16 * j + cc] = -((acc[0] + acc[1]) + (acc[2] + acc[3]));
+        }
+    }
+    __syncthreads();
+}
+
+
+// T = (I + A)^{-1} for the strictly lower-triangular 64 x 64 A in Ascr (fp32,
+// row stride LDA), blocked by 16.  Diagonal blocks first, one column per
+// thread, right-looking (each finished x_s is folded into all later rows at
+// once, so the dependent chain is 16 steps); then the off-diagonal blocks by
+// distance from the diagonal: T_ij = -T_ii sum_{16j <= k < 16i} A[i-rows][k] T[k][j-cols].
+// Every thread of the block calls it; it ends with the block synchronised.
+template <int NT>
+__device__ __forceinline__ void invert_unit_lower(const float *Ascr, float *Tscr, float *Xscr, int tid) {
+    if (tid < C) {
+        const int b = tid >> 4, c = tid & 15, base = 16 * b;
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) x[r] = (r == c) ? 1.f : 0.f;
+#pragma unroll
+        for (int s = 0; s < 15; ++s) {
+#pragma unroll
+            for (int r = s + 1; r < 16; ++r) x[r] = fmaf(-Ascr[(base + r) * LDA + base + s], x[s], x[r]);
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Tscr[(base + r) * LDA + base + c] = x[r];
+    } else {
+        for (int e = tid - C; e < C * C; e += NT - C) {  // zero the blocks above the diagonal
+            const int r = e >> 6, s = e & 63;
+            if ((s >> 4) > (r >> 4)) Tscr[r * LDA + s] = 0.f;
+        }
+    }
+    __syncthreads();
+    offdiag_stage<1, NT>(Ascr, Tscr, Xscr, tid);
+    offdiag_stage<2, NT>(Ascr, Tscr, Xscr, tid);
+    offdiag_stage<3, NT>(Ascr, Tscr, Xscr, tid);
+}
+
+}  // namespace tcp
+}  // namespace gdr

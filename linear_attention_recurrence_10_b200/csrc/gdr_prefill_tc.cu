@@ -31,28 +31,19 @@
 // (x = hi + lo to ~16 bits) and multiplied term by term (for P Delta:
 // hi*hi + hi*lo + lo*hi).  q, k, v enter the MMAs as the exact bf16 inputs.
 //
-// One CTA (256 threads) owns one (sequence, value head) and walks its chunks
+// One CTA (512 threads) owns one (sequence, value head) and walks its chunks
 // in order; each chunk's inputs are fetched by cp.async one chunk ahead.
 // Sequences are taken longest first (order written to the workspace by a
 // pre-kernel).  Every mbarrier wait is bounded by a wall-clock deadline; on
 // expiry the CTA records GDR_ERR_TIMEOUT in the workspace status word, frees
 // its tensor memory and returns.
-#include "gdr_common.cuh"
-#include "gdr_tc.cuh"
+#include "gdr_prefill_common.cuh"
 
 namespace gdr {
 namespace tcp {
 
-using namespace gdr::tc;
-
-constexpr int D = 128;       // d_k = d_v
-constexpr int C = 64;        // chunk
-constexpr int NT = 256;      // threads
+constexpr int NT = 512;      // threads (16 warps)
 constexpr int NW = NT / 32;
-constexpr int LDA = C + 1;   // padded row stride of the fp32 scratch matrices
-constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s: far beyond any chunk's work
-constexpr float kGammaFloor = -64.0f;
-constexpr int kTimeoutStatus = 6;  // GDR_ERR_TIMEOUT
 
 // Shared memory map (bytes).
 constexpr uint32_t OFF_KQ = 0;          // 2 x bf16 [K;Q], 128 rows x 128, row-group major (32 KB each)
@@ -75,101 +66,6 @@ constexpr uint32_t TM_OI = 192;   // S Q^T            M=128, 64 cols
 constexpr uint32_t TM_O2 = 256;   // Delta^T P^T      M=128, 64 cols
 constexpr uint32_t TM_S = 384;    // state S [i][j]   M=128, 128 cols
 
-// Tiles written from registers, K-major: 16-byte chunks along K are R*16 bytes
-// apart, 8-row groups 128 bytes apart (LBO = R*16, SBO = 128).
-__device__ __forceinline__ uint32_t kmaj(int row, int k, int R) {
-    return (uint32_t)((k >> 3) * (R * 16) + (row >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2);
-}
-// The [K;Q] tile: 8-row groups 2048 bytes apart, 16-byte chunks along d 128
-// bytes apart.  K-major over d: LBO = 128, SBO = 2048.  Read as MN-major over
-// d with the tokens as K: SBO = 128, LBO = 2048.
-__device__ __forceinline__ uint32_t kq_off(int row, int j) {
-    return (uint32_t)((row >> 3) * 2048 + (j >> 3) * 128 + (row & 7) * 16 + (j & 7) * 2);
-}
-// V tile, MN-major over d_v with the tokens as K: SBO = 1024, LBO = 128.
-__device__ __forceinline__ uint32_t v_off(int s, int i) {
-    return (uint32_t)((i >> 3) * 1024 + (s >> 3) * 128 + (s & 7) * 16 + (i & 7) * 2);
-}
-// W tile (B operand of S W^T), MN-major over the tokens r with d_k as K:
-// SBO = 2048, LBO = 128.
-__device__ __forceinline__ uint32_t w_off(int j, int r) {
-    return (uint32_t)((r >> 3) * 2048 + (j >> 3) * 128 + (j & 7) * 16 + (r & 7) * 2);
-}
-
-// D (+)= A B, `ksteps` bf16 instructions of K = 16, advancing A and B by the
-// given byte steps.
-__device__ __forceinline__ void gemm(uint32_t d, uint32_t a, uint32_t a_lbo, uint32_t a_sbo,
-                                     uint32_t a_step, uint32_t b, uint32_t b_lbo, uint32_t b_sbo,
-                                     uint32_t b_step, int ksteps, uint32_t idesc, bool acc) {
-    for (int kk = 0; kk < ksteps; ++kk)
-        mma<Kind::BF16>(d, smem_desc(a + kk * a_step, a_lbo, a_sbo),
-                        smem_desc(b + kk * b_step, b_lbo, b_sbo), idesc, (acc || kk > 0) ? 1u : 0u);
-}
-
-// z * sigmoid(z) with the fast exponential (relative error ~1e-7 here).
-__device__ __forceinline__ float fast_silu(float z) { return z / (1.0f + __expf(-z)); }
-
-// Eight fp32 values as eight bf16 (round to nearest even) in 16 bytes.
-__device__ __forceinline__ uint4 pack8(const float *v) {
-    uint4 pk;
-    __nv_bfloat162 b0 = __floats2bfloat162_rn(v[0], v[1]);
-    __nv_bfloat162 b1 = __floats2bfloat162_rn(v[2], v[3]);
-    __nv_bfloat162 b2 = __floats2bfloat162_rn(v[4], v[5]);
-    __nv_bfloat162 b3 = __floats2bfloat162_rn(v[6], v[7]);
-    pk.x = *reinterpret_cast<uint32_t *>(&b0);
-    pk.y = *reinterpret_cast<uint32_t *>(&b1);
-    pk.z = *reinterpret_cast<uint32_t *>(&b2);
-    pk.w = *reinterpret_cast<uint32_t *>(&b3);
-    return pk;
-}
-// Split eight fp32 values into bf16 hi = rn(x) and lo = rn(x - hi).
-__device__ __forceinline__ void split8(const float *v, uint4 &hi, uint4 &lo) {
-    float h[8], l[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-        h[u] = __bfloat162float(__float2bfloat16_rn(v[u]));
-        l[u] = v[u] - h[u];
-    }
-    hi = pack8(h);
-    lo = pack8(l);
-}
-
-// One distance of the blocked triangular inverse: for every pair of 16-blocks
-// (i, j) with i - j = DIST, X = A[i-rows][16j .. 16i) T[16j .. 16i)[j-cols],
-// then T_ij = -T_ii X.  Fully unrolled so the shared-memory loads overlap.
-template <int DIST>
-__device__ __forceinline__ void offdiag_stage(const float *Ascr, float *Tscr, float *Xscr, int tid) {
-    constexpr int NBLK = 4 - DIST, NOUT = NBLK * 256;
-#pragma unroll
-    for (int e0 = 0; e0 < NOUT; e0 += NT) {
-        const int e = e0 + tid;
-        if (NOUT % NT == 0 || e < NOUT) {
-            const int j = e >> 8, i = j + DIST, rr = (e >> 4) & 15, cc = e & 15;
-            const float *arow = Ascr + (16 * i + rr) * LDA + 16 * j;
-            const float *tcol = Tscr + 16 * j * LDA + 16 * j + cc;
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int k = 0; k < 16 * DIST; ++k) acc[k & 3] = fmaf(arow[k], tcol[k * LDA], acc[k & 3]);
-            Xscr[e] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-        }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int e0 = 0; e0 < NOUT; e0 += NT) {
-        const int e = e0 + tid;
-        if (NOUT % NT == 0 || e < NOUT) {
-            const int j = e >> 8, i = j + DIST, rr = (e >> 4) & 15, cc = e & 15;
-            const float *trow = Tscr + (16 * i + rr) * LDA + 16 * i;
-            const float *xcol = Xscr + (j << 8) + cc;
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int k = 0; k < 16; ++k) acc[k & 3] = fmaf(trow[k], xcol[k * 16], acc[k & 3]);
-            Tscr[(16 * i + rr) * LDA + 16 * j + cc] = -((acc[0] + acc[1]) + (acc[2] + acc[3]));
-        }
-    }
-    __syncthreads();
-}
-
 struct Scalars {
     float gam[C], eg[C], bet[C], nk[C], nq[C], dec[C];
     uint64_t bar;
@@ -182,7 +78,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_tc_kernel(const PrefillParams p
     extern __shared__ __align__(1024) unsigned char sm[];
     Scalars &sc = *reinterpret_cast<Scalars *>(sm + OFF_SCAL);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int quad = warp & 3, half = warp >> 2;  // TMEM lane quadrant, column half
+    const int quad = warp & 3, part = warp >> 2;  // TMEM lane quadrant, column quarter
 
     const int unit = blockIdx.x;
     const int seq = order[unit / p.H_v];
@@ -296,8 +192,8 @@ __global__ void __launch_bounds__(NT, 1) prefill_tc_kernel(const PrefillParams p
                               ? p.initial_state + ((size_t)seq * p.H_v + hv) * D * D + (size_t)i * D
                               : nullptr;
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-            const int j0 = 64 * half + 32 * cc;
+        for (int cc = 0; cc < 1; ++cc) {
+            const int j0 = 32 * part;
             float v[32];
 #pragma unroll
             for (int j4 = 0; j4 < 8; ++j4) {
@@ -392,26 +288,26 @@ __global__ void __launch_bounds__(NT, 1) prefill_tc_kernel(const PrefillParams p
         // ---- P3: A (fp32 scratch) and P (hi/lo bf16, K-major [r][s]).
         {
             const int rr = 32 * (quad & 1) + lane;  // token row
-            const int s0 = 32 * half;
+            const int s0 = 16 * part;
             const float gr = sc.gam[rr];
-            float v[32];
-            tmem_ld32(tm + lane_off + TM_D1 + s0, v);
+            float v[16];
+            tmem_ld16(tm + lane_off + TM_D1 + s0, v);
             if (quad < 2) {
                 const float f = sc.bet[rr] * sc.nk[rr];
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
+                for (int c = 0; c < 16; ++c) {
                     const int s = s0 + c;
                     Ascr[rr * LDA + s] = s < rr ? f * __expf(gr - sc.gam[s]) * sc.nk[s] * v[c] : 0.f;
                 }
             } else {
                 const float f = sc.nq[rr];
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
+                for (int c = 0; c < 16; ++c) {
                     const int s = s0 + c;
                     v[c] = s <= rr ? f * __expf(gr - sc.gam[s]) * sc.nk[s] * v[c] : 0.f;
                 }
 #pragma unroll
-                for (int c8 = 0; c8 < 4; ++c8) {
+                for (int c8 = 0; c8 < 2; ++c8) {
                     uint4 hi, lo;
                     split8(v + 8 * c8, hi, lo);
                     *reinterpret_cast<uint4 *>(sm + OFF_P + kmaj(rr, s0 + 8 * c8, C)) = hi;
@@ -421,34 +317,8 @@ __global__ void __launch_bounds__(NT, 1) prefill_tc_kernel(const PrefillParams p
         }
         __syncthreads();
 
-        // ---- P4: T = (I + A)^{-1}, blocked by 16.  Diagonal blocks first, one
-        // column per thread, right-looking (each finished x_s is folded into all
-        // later rows at once, so the dependent chain is 16 steps, not 120); then
-        // the off-diagonal blocks by distance from the diagonal:
-        // T_ij = -T_ii sum_{16j <= k < 16i} A[i-rows][k] T[k][j-cols].
-        if (tid < C) {
-            const int b = tid >> 4, c = tid & 15, base = 16 * b;
-            float x[16];
-#pragma unroll
-            for (int r = 0; r < 16; ++r) x[r] = (r == c) ? 1.f : 0.f;
-#pragma unroll
-            for (int s = 0; s < 15; ++s) {
-#pragma unroll
-                for (int r = s + 1; r < 16; ++r)
-                    x[r] = fmaf(-Ascr[(base + r) * LDA + base + s], x[s], x[r]);
-            }
-#pragma unroll
-            for (int r = 0; r < 16; ++r) Tscr[(base + r) * LDA + base + c] = x[r];
-        } else {
-            for (int e = tid - C; e < C * C; e += NT - C) {  // zero the blocks above the diagonal
-                const int r = e >> 6, s = e & 63;
-                if ((s >> 4) > (r >> 4)) Tscr[r * LDA + s] = 0.f;
-            }
-        }
-        __syncthreads();
-        offdiag_stage<1>(Ascr, Tscr, Xscr, tid);
-        offdiag_stage<2>(Ascr, Tscr, Xscr, tid);
-        offdiag_stage<3>(Ascr, Tscr, Xscr, tid);
+        // ---- P4: T = (I + A)^{-1} (blocked fp32 inverse).
+        invert_unit_lower<NT>(Ascr, Tscr, Xscr, tid);
         // TB = T diag(beta), TW = T diag(beta e^gamma n): hi/lo bf16 tiles [r][s].
         for (int e = tid; e < C * (C / 8); e += NT) {
             const int r = e & 63, s8 = 8 * (e >> 6);
@@ -486,16 +356,17 @@ __global__ void __launch_bounds__(NT, 1) prefill_tc_kernel(const PrefillParams p
         // ---- P6: W^T -> bf16 B tile; rescale the TMEM state by e^{gamma_L}.
         {
             const int j = 32 * quad + lane;
-            const int r0 = 32 * half;
-            float v[32];
-            tmem_ld32(tm + lane_off + TM_W + r0, v);
+            const int r0 = 16 * part;
+            float wv[16];
+            tmem_ld16(tm + lane_off + TM_W + r0, wv);
 #pragma unroll
-            for (int r8 = 0; r8 < 4; ++r8)
-                *reinterpret_cast<uint4 *>(sm + OFF_SCR + w_off(j, r0 + 8 * r8)) = pack8(v + 8 * r8);
+            for (int r8 = 0; r8 < 2; ++r8)
+                *reinterpret_cast<uint4 *>(sm + OFF_SCR + w_off(j, r0 + 8 * r8)) = pack8(wv + 8 * r8);
+            float v[32];
             const float eL = sc.eg[L - 1];
 #pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                const int j0 = 64 * half + 32 * cc;
+            for (int cc = 0; cc < 1; ++cc) {
+                const int j0 = 32 * part;
                 tmem_ld32(tm + lane_off + TM_S + j0, v);
 #pragma unroll
                 for (int u = 0; u < 32; ++u) v[u] *= eL;
@@ -513,13 +384,13 @@ __global__ void __launch_bounds__(NT, 1) prefill_tc_kernel(const PrefillParams p
         // ---- P8: Delta^T hi/lo and its decayed, k-normalised copy, K-major [i][s].
         {
             const int i = 32 * quad + lane;
-            const int s0 = 32 * half;
-            float v[32], w[32];
-            tmem_ld32(tm + lane_off + TM_U + s0, v);
+            const int s0 = 16 * part;
+            float v[16], w[16];
+            tmem_ld16(tm + lane_off + TM_U + s0, v);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) w[c] = v[c] * sc.dec[s0 + c] * sc.nk[s0 + c];
+            for (int c = 0; c < 16; ++c) w[c] = v[c] * sc.dec[s0 + c] * sc.nk[s0 + c];
 #pragma unroll
-            for (int c8 = 0; c8 < 4; ++c8) {
+            for (int c8 = 0; c8 < 2; ++c8) {
                 uint4 hi, lo;
                 const uint32_t o = kmaj(i, s0 + 8 * c8, D);
                 split8(v + 8 * c8, hi, lo);
@@ -548,19 +419,19 @@ __global__ void __launch_bounds__(NT, 1) prefill_tc_kernel(const PrefillParams p
         // state's bf16 copy for the next chunk.
         {
             const int i = 32 * quad + lane;
-            const int r0 = 32 * half;
-            float a[32], b[32];
-            tmem_ld32(tm + lane_off + TM_OI + r0, a);
-            tmem_ld32(tm + lane_off + TM_O2 + r0, b);
+            const int r0 = 16 * part;
+            float a[16], b[16];
+            tmem_ld16(tm + lane_off + TM_OI + r0, a);
+            tmem_ld16(tm + lane_off + TM_O2 + r0, b);
             float *Os = reinterpret_cast<float *>(sm + OFF_TBW);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
+            for (int c = 0; c < 16; ++c) {
                 const int r = r0 + c;
                 Os[r * D + i] = fmaf(sc.nq[r] * sc.eg[r], a[c], b[c]);
             }
 #pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                const int j0 = 64 * half + 32 * cc;
+            for (int cc = 0; cc < 1; ++cc) {
+                const int j0 = 32 * part;
                 float v[32];
                 tmem_ld32(tm + lane_off + TM_S + j0, v);
 #pragma unroll
@@ -601,8 +472,8 @@ __global__ void __launch_bounds__(NT, 1) prefill_tc_kernel(const PrefillParams p
         const int i = 32 * quad + lane;
         float *dst = p.final_state + ((size_t)seq * p.H_v + hv) * D * D + (size_t)i * D;
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-            const int j0 = 64 * half + 32 * cc;
+        for (int cc = 0; cc < 1; ++cc) {
+            const int j0 = 32 * part;
             float v[32];
             tmem_ld32(tm + lane_off + TM_S + j0, v);
 #pragma unroll

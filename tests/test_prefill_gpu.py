@@ -219,3 +219,15 @@ def test_long_context_gva_prefill_full():
         t0, t1 = inp.cu_seqlens[s], inp.cu_seqlens[s + 1]
         assert rel_l2(f64(out[t0:t1, h]), ref.y[:, 0]) <= 2e-3, (s, h)
         assert rel_l2(f64(final[s, h]), ref.state[0, 0]) <= 1e-3, (s, h)
+
+
+@pytest.mark.parametrize("lens", [[64], [63, 65, 0, 128, 200], [257, 3, 64 * 5 + 17]])
+def test_tc_one_kernel_variant(lens):
+    """A workspace too small for the per-chunk records (but holding the sequence
+    order) runs the tensor-core prefill as one kernel; same bars."""
+    inp = synth.make_inputs(lens, 2, 4, 128, seed=500 + sum(lens), dtype=torch.bfloat16,
+                            s0_std=0.02)
+    small = (16 + 4 * len(lens) + 255) // 256 * 256
+    ws = torch.empty(small, dtype=torch.uint8, device="cuda")
+    out, final = run_prefill(inp, chunk=64, workspace=ws)
+    _check(inp, out, final, torch.bfloat16)

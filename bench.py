@@ -228,17 +228,13 @@ def time_region(fn, n, ranks):
     torch.cuda.synchronize()
     if ranks > 1:
         torch.distributed.barrier()
-    ms = e0.elapsed_time(e1)
-    if ranks > 1:
-        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    return ms
+    from linear_attention_recurrence_10_b200.ranks import max_over_ranks
+    return max_over_ranks(e0.elapsed_time(e1), ranks, device="cuda")
 
 
 # ---------------------------------------------------------------- prefill
 
-def prefill_measure(device, reps=5):
+def prefill_measure(device, reps=5, world=1):
     import linear_attention_recurrence_10_b200 as gdr
     from linear_attention_recurrence_10_b200 import synth
     inp = synth.make_inputs([P_LEN] * P_SEQS, P_H, P_H, D, seed=2, device=device)
@@ -261,21 +257,18 @@ def prefill_measure(device, reps=5):
     times = []
     for _ in range(reps):
         flush.zero_()  # evict L2 between repetitions
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        call()
-        e1.record()
-        torch.cuda.synchronize()
-        times.append(e0.elapsed_time(e1))
+        times.append(time_region(call, 1, world))  # max over ranks
     ms = statistics.median(times)
-    n_tok = inp.n_tok
+    n_tok = inp.n_tok * world
     flops = n_tok * P_H * prefill_flops_per_token_head(P_CHUNK, D, gva=False)
+    per_gpu_tflops = flops / world / (ms * 1e-3) / 1e12
     peaks = load_peaks()
     tflops = flops / (ms * 1e-3) / 1e12
     return {"metric": "chunked-prefill tokens/s", "value": n_tok / (ms * 1e-3), "unit": "tokens/s",
             "ms": ms, "workload": f"Qwen3.5-0.8B-shaped prefill: {P_SEQS} x {P_LEN} tokens, "
                                   f"{P_H}/{P_H} heads, d={D}, bf16, chunk {P_CHUNK}, S_0=0",
-            "tflops": tflops, "tc_frac": tflops / peaks["bf16_tflops"],
+            "n_gpus": world, "scaling": "weak",
+            "tflops": tflops, "tc_frac": per_gpu_tflops / peaks["bf16_tflops"],
             "tc_peak_tflops": peaks["bf16_tflops"], "flops_per_token_head":
                 prefill_flops_per_token_head(P_CHUNK, D, gva=False),
             "l2": "flushed (256 MB write) before each repetition", "reps": reps}
@@ -371,9 +364,9 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from linear_attention_recurrence_10_b200.ranks import rank_env, weak_scaling_rate
+    env = rank_env()
+    world, rank, local = env.world, env.rank, env.local
     if args.impl == "reference":
         run_reference(args, rank, world)
         return
@@ -399,8 +392,7 @@ def main():
     clock_info = clocks.summary()
 
     peaks = load_peaks()
-    bytes_total = bench.bytes_per_step * args.steps * world
-    gbs = bytes_total / (ms * 1e-3) / 1e9
+    gbs = weak_scaling_rate(bench.bytes_per_step * args.steps, world, ms) / 1e9
     per_launch_ms = ms / (args.steps * bench.launches_per_step)
     per_launch_bytes = decode_bytes_per_layer_step(args.batch, H_K, H_V, D)
     achieved = per_launch_bytes / (per_launch_ms * 1e-3) / 1e9
@@ -411,9 +403,9 @@ def main():
         e2e.step(s)
     ms_e2e = time_region(lambda: [e2e.step(s) for s in range(args.e2e_steps)], args.e2e_steps,
                          world)
-    e2e_gbs = bench.bytes_per_step * args.e2e_steps * world / (ms_e2e * 1e-3) / 1e9
+    e2e_gbs = weak_scaling_rate(bench.bytes_per_step * args.e2e_steps, world, ms_e2e) / 1e9
 
-    prefill = None if args.no_prefill else prefill_measure(device)
+    prefill = None if args.no_prefill else prefill_measure(device, world=world)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_sample()
@@ -430,7 +422,7 @@ def main():
             "l2": f"inputs larger than L2: {LAYERS} layer states "
                   f"({LAYERS * args.batch * H_V * D * D * 4 / 1e6:.0f} MB) rotate every step",
             "launch": "one CUDA graph per step (one decode launch per layer)"},
-        "tokens_per_s": args.batch * world * args.steps / (ms * 1e-3),
+        "tokens_per_s": weak_scaling_rate(args.batch * args.steps, world, ms),
         "hbm_frac": gbs / world / peaks["hbm_gbs"],
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],

@@ -342,7 +342,7 @@ constexpr uint32_t B_Z = 100352;      // 2 x bf16 z [s][i] (16 KB each)
 constexpr uint32_t B_S = 133120;      // bf16 S [i][j] (32 KB)
 constexpr uint32_t B_DL = 165888;     // Delta hi/lo (32 KB); later O [r][i] fp32
 constexpr uint32_t B_DT = 198656;     // decayed Delta hi/lo (32 KB)
-constexpr uint32_t B_BAR = 231424;    // mbarriers (MMA, 2 records, 2 z), TMEM address
+constexpr uint32_t B_BAR = 231424;    // mbarriers (MMA, 2 records), TMEM address
 constexpr uint32_t B_SMEM = B_BAR + 64;
 
 template <typename TOUT>
@@ -352,7 +352,6 @@ __global__ void __launch_bounds__(NT, 1) recur_kernel(const PrefillParams p, con
     extern __shared__ __align__(1024) unsigned char sm[];
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + B_BAR);
     uint64_t *rbar = bar + 1;  // [2]: a staged record landed
-    uint64_t *zbar = bar + 3;  // [2]: a chunk's z rows landed
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + B_BAR + 40);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int quad = warp & 3, part = warp >> 2;
@@ -391,19 +390,21 @@ __global__ void __launch_bounds__(NT, 1) recur_kernel(const PrefillParams p, con
             bulk_copy(sm + B_REC + buf * REC_STAGED, rec, REC_STAGED, rbar + buf);
         }
     };
-    // z: one bulk copy per token row (256 contiguous bytes of this head).
+    // z rows (256 contiguous bytes of this head per token), spread over all
+    // threads as 16-byte cp.async copies; they join the K group of the chunk.
     auto fetch_z = [&](int64_t c0, int L, int buf) {
-        if (!zg || warp != 0) return;
-        if (lane == 0) bulk_expect(zbar + buf, (uint32_t)L * 256u);
-        __syncwarp();
-        for (int s = lane; s < L; s += 32)
-            bulk_copy(sm + B_Z + buf * 16384 + s * 256, zg + (c0 + s) * p.z_stride + hv * D, 256u,
-                      zbar + buf);
+        if (!zg) return;
+        for (int e = tid; e < C * 16; e += NT) {
+            const int r = e >> 4, c16 = e & 15;
+            if (r < L)
+                cp_async16(sm + B_Z + buf * 16384 + r * 256 + c16 * 16,
+                           zg + (c0 + r) * p.z_stride + hv * D + 8 * c16, 16u);
+        }
     };
 
     if (warp == 0) tmem_alloc(tmem_slot, 512);
     if (tid == 0) {
-        for (int i = 0; i < 5; ++i) mbar_init(bar + i, 1);
+        for (int i = 0; i < 3; ++i) mbar_init(bar + i, 1);
         mbar_fence_init();
     }
     __syncthreads();
@@ -488,7 +489,6 @@ __global__ void __launch_bounds__(NT, 1) recur_kernel(const PrefillParams p, con
         cp_async_wait<1>();  // this chunk's Q
         {
             bool ok = mbar_wait(rbar + buf, in_phase, kWaitNs);  // its record
-            if (zg) ok = mbar_wait(zbar + buf, in_phase, kWaitNs) && ok;  // its z rows
             if (__syncthreads_or(!ok)) {
                 if (tid == 0) atomicExch(status, kTimeoutStatus);
                 alive = false;
@@ -499,7 +499,6 @@ __global__ void __launch_bounds__(NT, 1) recur_kernel(const PrefillParams p, con
         // fetch the next chunk's staged record and z a whole chunk ahead.
         if (n0 < t1) {
             fetch_rec(rec + rec_step, buf ^ 1);
-            fetch_z(n0, Ln, buf ^ 1);
         }
         // U of this chunk, straight into registers for the Delta epilogue.
         float4 uu[4];
@@ -570,7 +569,10 @@ __global__ void __launch_bounds__(NT, 1) recur_kernel(const PrefillParams p, con
 
         // This chunk's K is consumed: fetch the next chunk's.
         const int r0 = 16 * part;
-        if (n0 < t1) fetch_half(n0, Ln, false);
+        if (n0 < t1) {
+            fetch_half(n0, Ln, false);
+            fetch_z(n0, Ln, buf ^ 1);  // read by the next chunk's norm, after its K wait
+        }
         cp_async_commit();
 
         // O = (m e^gamma)(S Q^T) + Delta P^T staged as [r][i]; the new state's bf16 copy.

@@ -24,9 +24,6 @@ from dataclasses import dataclass, field
 
 import torch
 
-_NAMES = ("q", "k", "v", "z", "g", "beta", "s0", "w", "len")
-
-
 def _seed_for(seed: int, name: str) -> int:
     return (int(seed) * 1_000_003 + zlib.crc32(name.encode())) & ((1 << 62) - 1)
 

@@ -26,8 +26,6 @@ namespace tcp2 {
 
 using namespace gdr::tcp;
 
-constexpr int NT = 512;  // threads (16 warps) in both kernels
-constexpr int NW = NT / 32;
 
 // Per-(chunk, value head) record in the workspace.
 // The first REC_STAGED bytes (W, P, scalars) are staged in shared memory by the
@@ -335,297 +333,406 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p, con
 }
 
 // ----------------------------------------------------------- recur kernel
+//
+// One CTA per (sequence, value head) walks the chunks in order.  Only the
+// state path is serial: Delta = U - W S^T needs the state entering the chunk,
+// and the next state needs Delta.  The output of a chunk (O = (m e^gamma) Q S^T
+// + P Delta, then RMSNormGated) feeds nothing later, so the CTA is split into
+// four roles that run concurrently and hand work over on mbarriers:
+//   warps 0-7   state group: the Delta epilogue (hi/lo tiles of Delta and of
+//               its decayed, k-normalised copy) and, once the state update is
+//               done, the bf16 copy of S for the next chunk's products, with
+//               the next chunk's e^{gamma_L} folded into the same pass;
+//   warps 8-15  output group, one chunk behind: S Q^T and P Delta out of
+//               double-buffered TMEM, staged through shared memory so that
+//               one warp normalises, gates and stores whole tokens;
+//   warp 16     producer: K and Q tiles (cp.async with zero fill past the
+//               sequence end, counted on an mbarrier), the staged records
+//               (one bulk copy each, double-buffered) and an L2 prefetch of
+//               the next chunk's U;
+//   warp 17     MMA issue, state path first (-S W^T before S Q^T, the state
+//               update before P Delta), each group committed on its own
+//               barrier so the state group never waits for output products.
 
-constexpr uint32_t B_KQ = 0;          // bf16 [K;Q] (32 KB)
-constexpr uint32_t B_REC = 32768;     // 2 x staged record (W, P, scalars: 33 KB each)
-constexpr uint32_t B_Z = 100352;      // 2 x bf16 z [s][i] (16 KB each)
-constexpr uint32_t B_S = 133120;      // bf16 S [i][j] (32 KB)
-constexpr uint32_t B_DL = 165888;     // Delta hi/lo (32 KB); later O [r][i] fp32
-constexpr uint32_t B_DT = 198656;     // decayed Delta hi/lo (32 KB)
-constexpr uint32_t B_BAR = 231424;    // mbarriers (MMA, 2 records), TMEM address
-constexpr uint32_t B_SMEM = B_BAR + 64;
+constexpr int RNT = 576;                       // 18 warps
+constexpr int OG_BAR = 1, OG_N = 256;
+constexpr uint32_t B_KQ = 0;                   // bf16 [K;Q] (32 KB)
+constexpr uint32_t B_REC = 32768;              // 2 x staged record (W, P, scalars: 33 KB each)
+constexpr uint32_t B_S = 100352;               // bf16 S [i][j] (32 KB)
+constexpr uint32_t B_DL = 133120;              // Delta hi/lo (32 KB)
+constexpr uint32_t B_DT = 165888;              // decayed Delta hi/lo (32 KB)
+constexpr uint32_t B_OS = 198656;              // fp32 O [r][i] of the chunk being output (32 KB)
+constexpr uint32_t B_BAR = 231424;             // 13 mbarriers, then the TMEM address
+constexpr uint32_t B_SMEM = B_BAR + 128;
+// TMEM columns: the fp32 state, -S W^T, and two buffers each of S Q^T and P Delta.
+constexpr uint32_t TM_S = 0, TM_D = 128, TM_OI = 192, TM_O2 = 320;
 
 template <typename TOUT>
-__global__ void __launch_bounds__(NT, 1) recur_kernel(const PrefillParams p, const int *order,
-                                                      const int *chunk_off,
-                                                      const unsigned char *records, int *status) {
+__global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, const int *order,
+                                                       const int *chunk_off,
+                                                       const unsigned char *records, int *status) {
     extern __shared__ __align__(1024) unsigned char sm[];
-    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + B_BAR);
-    uint64_t *rbar = bar + 1;  // [2]: a staged record landed
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + B_BAR + 40);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + B_BAR);
+    uint64_t *bar_q = bars, *bar_k = bars + 1;   // tiles landed (32 producer lanes each)
+    uint64_t *bar_rec = bars + 2;                // [2] staged record landed
+    uint64_t *bar_gd = bars + 4;                 // -S W^T done
+    uint64_t *bar_qfree = bars + 5;              // S Q^T done: the Q tile may be refilled
+    uint64_t *bar_gs = bars + 6;                 // state update done: the K tile may be refilled
+    uint64_t *bar_oready = bars + 7;             // [2] P Delta (and S Q^T) of a chunk done
+    uint64_t *bar_ofree = bars + 9;              // [2] output group done with a chunk's buffers
+    uint64_t *bar_sready = bars + 11;            // state group: bf16 S staged (8 warps)
+    uint64_t *bar_dready = bars + 12;            // state group: Delta tiles staged (8 warps)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + B_BAR + 112);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int quad = warp & 3, part = warp >> 2;
     const int seq = order[blockIdx.x / p.H_v];
     const int hv = blockIdx.x % p.H_v;
     const int hk = hv / p.hv_per_hk;
     const int64_t t0 = p.cu_seqlens[seq], t1 = p.cu_seqlens[seq + 1];
+    const int n_chunks = (int)((t1 - t0 + C - 1) / C);
     const unsigned char *rec0 = records + ((size_t)chunk_off[seq] * p.H_v + hv) * REC_BYTES;
     const size_t rec_step = (size_t)p.H_v * REC_BYTES;
-
-    const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(p.q);
-    const __nv_bfloat16 *kg = static_cast<const __nv_bfloat16 *>(p.k);
-    const __nv_bfloat16 *zg = static_cast<const __nv_bfloat16 *>(p.z);
-    TOUT *og = static_cast<TOUT *>(p.out);
     const uint32_t sbase = smem_u32(sm);
-
-    // Half of the [K;Q] tile: K (rows 0..63) is read only by the last MMA of a
-    // chunk and Q (rows 64..127) only by the first, so each is fetched as soon
-    // as the current chunk is done with it.
-    auto fetch_half = [&](int64_t c0, int L, bool q_half) {
-        const __nv_bfloat16 *base = q_half ? qg + hk * D : kg + hk * D;
-        const int64_t stride = q_half ? p.q_stride : p.k_stride;
-        for (int e = tid; e < 64 * 16; e += NT) {
-            const int r = (e & 7) + 8 * ((e >> 5) & 7);
-            const int jc = ((e >> 3) & 3) + 4 * (e >> 8);
-            const bool in = r < L;
-            const int64_t t = in ? c0 + r : t0;
-            cp_async16(sm + B_KQ + kq_off(r + (q_half ? 64 : 0), 8 * jc), base + t * stride + 8 * jc,
-                       in ? 16u : 0u);
-        }
+    auto chunk_len = [&](int c) {
+        const int64_t left = t1 - t0 - (int64_t)c * C;
+        return (int)(left < C ? left : C);
     };
-    // The staged part of a record is one contiguous block: one bulk copy.
-    auto fetch_rec = [&](const unsigned char *rec, int buf) {
-        if (tid == 0) {
-            bulk_expect(rbar + buf, REC_STAGED);
-            bulk_copy(sm + B_REC + buf * REC_STAGED, rec, REC_STAGED, rbar + buf);
-        }
-    };
-    // z rows (256 contiguous bytes of this head per token), spread over all
-    // threads as 16-byte cp.async copies; they join the K group of the chunk.
-    auto fetch_z = [&](int64_t c0, int L, int buf) {
-        if (!zg) return;
-        for (int e = tid; e < C * 16; e += NT) {
-            const int r = e >> 4, c16 = e & 15;
-            if (r < L)
-                cp_async16(sm + B_Z + buf * 16384 + r * 256 + c16 * 16,
-                           zg + (c0 + r) * p.z_stride + hv * D + 8 * c16, 16u);
-        }
+    auto fail = [&]() { atomicExch(status, kTimeoutStatus); };
+    auto rscal = [&](int c) {
+        return reinterpret_cast<const float *>(sm + B_REC + (c & 1) * REC_STAGED + REC_SCAL);
     };
 
     if (warp == 0) tmem_alloc(tmem_slot, 512);
     if (tid == 0) {
-        for (int i = 0; i < 3; ++i) mbar_init(bar + i, 1);
+        mbar_init(bar_q, 32);
+        mbar_init(bar_k, 32);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_rec + b, 1);
+            mbar_init(bar_oready + b, 1);
+            mbar_init(bar_ofree + b, 8);
+        }
+        mbar_init(bar_gd, 1);
+        mbar_init(bar_qfree, 1);
+        mbar_init(bar_gs, 1);
+        mbar_init(bar_sready, 8);
+        mbar_init(bar_dready, 8);
         mbar_fence_init();
     }
-    __syncthreads();
-    if (t1 > t0) {
-        const int L0 = (int)((t1 - t0) < C ? (t1 - t0) : C);
-        fetch_half(t0, L0, true);
-        cp_async_commit();
-        fetch_half(t0, L0, false);
-        fetch_rec(rec0, 0);
-        fetch_z(t0, L0, 0);
-    } else {
-        cp_async_commit();
-    }
-    cp_async_commit();
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
     const uint32_t tm = *tmem_slot;
-    const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
-    constexpr uint32_t TM_OI = 0, TM_D = 64, TM_O2 = 128, TM_S = 256;
-    uint32_t phase = 0;
-    auto issue = [&](auto body) {
-        fence_smem_to_async();
-        fence_before_sync();
-        __syncthreads();
-        if (tid == 0) {
-            fence_after_sync();
-            body();
-            commit(smem_u32(bar));
+    bool state_ok = false;
+
+    if (warp == 17) {
+        // ------------------------------------------------------ MMA issue
+        if (lane == 0 && n_chunks > 0) {
+            const uint32_t ID_KK = instr_desc<Kind::BF16>(128, 64, false, false);
+            const uint32_t ID_D = instr_desc<Kind::BF16>(128, 64, false, true, true);  // -S, B = W MN-major
+            const uint32_t ID_S = instr_desc<Kind::BF16>(128, 128, false, true);       // B = K, MN-major
+            const uint32_t kq = sbase + B_KQ;
+            bool ok = true;
+            for (int c = 0; c < n_chunks && ok; ++c) {
+                const int b = c & 1;
+                const uint32_t rec_s = sbase + B_REC + b * REC_STAGED;
+                ok = mbar_wait(bar_sready, (uint32_t)c & 1u, kWaitNs) &&
+                     mbar_wait(bar_rec + b, (uint32_t)(c >> 1) & 1u, kWaitNs) &&
+                     mbar_wait(bar_q, (uint32_t)c & 1u, kWaitNs) &&
+                     (c < 2 || mbar_wait(bar_ofree + b, (uint32_t)((c >> 1) - 1) & 1u, kWaitNs));
+                if (!ok) break;
+                fence_after_sync();
+                fence_smem_to_async();
+                gemm(tm + TM_D, sbase + B_S, 2048, 128, 4096, rec_s + REC_W, 128, 2048, 256, D / 16, ID_D, false);
+                commit(smem_u32(bar_gd));
+                gemm(tm + TM_OI + 64 * b, sbase + B_S, 2048, 128, 4096, kq + 16384, 128, 2048, 256, D / 16, ID_KK, false);
+                commit(smem_u32(bar_qfree));
+                ok = mbar_wait(bar_dready, (uint32_t)c & 1u, kWaitNs) &&
+                     mbar_wait(bar_k, (uint32_t)c & 1u, kWaitNs);
+                if (!ok) break;
+                fence_after_sync();
+                fence_smem_to_async();
+                // S <- e^{gamma_L} S + Dt~^T K (hi + lo); then O_intra^T = Delta^T P^T
+                // (hi*hi + hi*lo + lo*hi) into this chunk's output buffer.
+                const uint32_t eh = sbase + B_DT, el = eh + 16384;
+                gemm(tm + TM_S, eh, 2048, 128, 4096, kq, 2048, 128, 4096, C / 16, ID_S, true);
+                gemm(tm + TM_S, el, 2048, 128, 4096, kq, 2048, 128, 4096, C / 16, ID_S, true);
+                commit(smem_u32(bar_gs));
+                const uint32_t dh = sbase + B_DL, dl = dh + 16384, ph = rec_s + REC_P, pl = ph + 8192;
+                const uint32_t o2 = tm + TM_O2 + 64 * b;
+                gemm(o2, dh, 2048, 128, 4096, ph, 1024, 128, 2048, C / 16, ID_KK, false);
+                gemm(o2, dh, 2048, 128, 4096, pl, 1024, 128, 2048, C / 16, ID_KK, true);
+                gemm(o2, dl, 2048, 128, 4096, ph, 1024, 128, 2048, C / 16, ID_KK, true);
+                commit(smem_u32(bar_oready + b));
+            }
+            if (!ok) fail();
         }
-    };
-    auto wait_mma = [&]() -> bool {
-        const bool ok = mbar_wait(bar, phase, kWaitNs);
-        phase ^= 1;
-        const int bad = __syncthreads_or(!ok);
-        fence_after_sync();
-        if (bad && tid == 0) atomicExch(status, kTimeoutStatus);
-        return !bad;
-    };
-
-    // Initial state into TMEM (fp32) and its bf16 copy into smem.
-    {
-        const int i = 32 * quad + lane, j0 = 32 * part;
-        const float *s0 = p.initial_state
-                              ? p.initial_state + ((size_t)seq * p.H_v + hv) * D * D + (size_t)i * D + j0
-                              : nullptr;
-        float v[32];
-#pragma unroll
-        for (int j4 = 0; j4 < 8; ++j4) {
-            const float4 x = s0 ? *reinterpret_cast<const float4 *>(s0 + 4 * j4) : make_float4(0.f, 0.f, 0.f, 0.f);
-            v[4 * j4] = x.x; v[4 * j4 + 1] = x.y; v[4 * j4 + 2] = x.z; v[4 * j4 + 3] = x.w;
-        }
-        tmem_st32(tm + lane_off + TM_S + j0, v);
-#pragma unroll
-        for (int j8 = 0; j8 < 4; ++j8)
-            *reinterpret_cast<uint4 *>(sm + B_S + kmaj(i, j0 + 8 * j8, D)) = pack8(v + 8 * j8);
-    }
-
-    float4 w4 = make_float4(1.f, 1.f, 1.f, 1.f);
-    if (p.norm_w)
-        w4 = make_float4(__ldg(p.norm_w + 4 * lane), __ldg(p.norm_w + 4 * lane + 1),
-                         __ldg(p.norm_w + 4 * lane + 2), __ldg(p.norm_w + 4 * lane + 3));
-    const uint32_t ID_KK = instr_desc<Kind::BF16>(128, 64, false, false);
-    const uint32_t ID_D = instr_desc<Kind::BF16>(128, 64, false, true, true);  // -S, B = W MN-major
-    const uint32_t ID_S = instr_desc<Kind::BF16>(128, 128, false, true);       // B = K, MN-major
-    const uint32_t kq = sbase + B_KQ;
-
-    bool alive = true;
-    const unsigned char *rec = rec0;
-    int it = 0;
-    for (int64_t c0 = t0; c0 < t1 && alive; c0 += C, rec += rec_step, ++it) {
-        const int buf = it & 1;
-        const uint32_t in_phase = (uint32_t)(it >> 1) & 1u;  // use count of this buffer
-        const uint32_t rec_s = sbase + B_REC + buf * REC_STAGED;
-        const float *rscal = reinterpret_cast<const float *>(sm + B_REC + buf * REC_STAGED + REC_SCAL);
-        const unsigned char *zbuf = sm + B_Z + buf * 16384;
-        const int L = (int)((t1 - c0) < C ? (t1 - c0) : C);
-        const int64_t n0 = c0 + C;
-        const int Ln = (int)((t1 - n0) < C ? (t1 - n0) : C);
-
-        // cp.async groups, oldest first: Q(c), K(c) -- Q(c) is needed now.
-        cp_async_wait<1>();  // this chunk's Q
-        {
-            bool ok = mbar_wait(rbar + buf, in_phase, kWaitNs);  // its record
-            if (__syncthreads_or(!ok)) {
-                if (tid == 0) atomicExch(status, kTimeoutStatus);
-                alive = false;
-                break;
+        __syncwarp();
+    } else if (warp == 16) {
+        // ------------------------------------------------------ producer
+        const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(p.q) + hk * D;
+        const __nv_bfloat16 *kg = static_cast<const __nv_bfloat16 *>(p.k) + hk * D;
+        // 64 rows x 256 bytes; lanes cover 8 rows x 4 column chunks (512
+        // contiguous bytes of shared memory) per step.
+        auto fetch = [&](int64_t c0, int L, bool q_half) {
+            const __nv_bfloat16 *base = q_half ? qg : kg;
+            const int64_t stride = q_half ? p.q_stride : p.k_stride;
+#pragma unroll 8
+            for (int e = lane; e < 64 * 16; e += 32) {
+                const int r = (e & 7) + 8 * ((e >> 5) & 7);
+                const int jc = ((e >> 3) & 3) + 4 * (e >> 8);
+                const bool in = r < L;
+                const int64_t t = in ? c0 + r : t0;
+                cp_async16(sm + B_KQ + kq_off(r + (q_half ? 64 : 0), 8 * jc),
+                           base + t * stride + 8 * jc, in ? 16u : 0u);
+            }
+            cp_async_arrive(q_half ? bar_q : bar_k);
+        };
+        int issued[2] = {0, 0};
+        auto fetch_rec = [&](int c) {
+            const int b = c & 1;
+            ++issued[b];
+            if (lane == 0) {
+                const unsigned char *rec = rec0 + (size_t)c * rec_step;
+                bulk_expect(bar_rec + b, REC_STAGED);
+                bulk_copy(sm + B_REC + b * REC_STAGED, rec, REC_STAGED, bar_rec + b);
+                bulk_prefetch_l2(rec + REC_U, REC_BYTES - REC_U);  // read by the state group
+            }
+        };
+        bool ok = true;
+        for (int c = 0; c < n_chunks && c < 2; ++c) fetch_rec(c);
+        for (int c = 0; c < n_chunks && ok; ++c) {
+            const int64_t c0 = t0 + (int64_t)c * C;
+            const int L = chunk_len(c);
+            if (c > 0) ok = mbar_wait(bar_qfree, (c - 1) & 1, kWaitNs);
+            if (!ok) break;
+            fetch(c0, L, true);
+            if (c > 0) ok = mbar_wait(bar_gs, (c - 1) & 1, kWaitNs);
+            if (!ok) break;
+            fetch(c0, L, false);
+            // Record c+1 replaces record c-1 once the output group is done with it.
+            if (c >= 1 && c + 1 < n_chunks) {
+                ok = mbar_wait(bar_ofree + ((c + 1) & 1), ((c - 1) >> 1) & 1, kWaitNs);
+                if (!ok) break;
+                fetch_rec(c + 1);
             }
         }
-        // The other buffers were last used by the previous chunk, which is done:
-        // fetch the next chunk's staged record and z a whole chunk ahead.
-        if (n0 < t1) {
-            fetch_rec(rec + rec_step, buf ^ 1);
+        cp_async_wait_all();
+        if (!ok) {
+            if (lane == 0) fail();
+            // No bulk copy may land after the CTA ends.
+            for (int b = 0; b < 2; ++b)
+                if (issued[b] > 0) mbar_wait(bar_rec + b, (uint32_t)(issued[b] - 1) & 1u, kWaitNs);
         }
-        // U of this chunk, straight into registers for the Delta epilogue.
-        float4 uu[4];
-        {
-            const int i = 32 * quad + lane, s0 = 16 * part;
-#pragma unroll
-            for (int s4 = 0; s4 < 4; ++s4)
-                uu[s4] = __ldg(reinterpret_cast<const float4 *>(rec + REC_U + u_off(s0 + 4 * s4, i)));
-        }
-
-        // O_inter^T = S Q^T and -S W^T, with the state entering the chunk.
-        issue([&] {
-            gemm(tm + TM_OI, sbase + B_S, 2048, 128, 4096, kq + 16384, 128, 2048, 256, D / 16, ID_KK, false);
-            gemm(tm + TM_D, sbase + B_S, 2048, 128, 4096, rec_s + REC_W, 128, 2048, 256, D / 16, ID_D, false);
-        });
-        // Meanwhile: S <- e^{gamma_L} S in TMEM (columns the MMAs do not touch).
-        {
-            const int j0 = 32 * part;
-            const float eL = rscal[3 * C];
-            float v[32];
-            tmem_ld32(tm + lane_off + TM_S + j0, v);
-#pragma unroll
-            for (int u = 0; u < 32; ++u) v[u] *= eL;
-            tmem_st32(tm + lane_off + TM_S + j0, v);
-        }
-        alive = wait_mma();
-        if (!alive) break;
-        if (n0 < t1) fetch_half(n0, Ln, true);  // Q of the next chunk
-        cp_async_commit();
-
-        // Delta^T = U^T - S W^T, as hi/lo tiles, and its decayed, k-normalised copy.
-        {
-            const int i = 32 * quad + lane, s0 = 16 * part;
-            float v[16], w[16];
-            tmem_ld16(tm + lane_off + TM_D + s0, v);
-#pragma unroll
-            for (int s4 = 0; s4 < 4; ++s4) {
-                v[4 * s4] += uu[s4].x; v[4 * s4 + 1] += uu[s4].y;
-                v[4 * s4 + 2] += uu[s4].z; v[4 * s4 + 3] += uu[s4].w;
-            }
-#pragma unroll
-            for (int c = 0; c < 16; ++c) w[c] = v[c] * rscal[2 * C + s0 + c];
-#pragma unroll
-            for (int c8 = 0; c8 < 2; ++c8) {
-                uint4 h, l;
-                const uint32_t o = kmaj(i, s0 + 8 * c8, D);
-                split8(v + 8 * c8, h, l);
-                *reinterpret_cast<uint4 *>(sm + B_DL + o) = h;
-                *reinterpret_cast<uint4 *>(sm + B_DL + 16384 + o) = l;
-                split8(w + 8 * c8, h, l);
-                *reinterpret_cast<uint4 *>(sm + B_DT + o) = h;
-                *reinterpret_cast<uint4 *>(sm + B_DT + 16384 + o) = l;
-            }
-        }
-        // O_intra^T = Delta^T P^T (hi*hi + hi*lo + lo*hi); S += Dt~ K.
-        cp_async_wait<1>();  // this chunk's K (the next chunk's Q may be in flight)
-        issue([&] {
-            const uint32_t dh = sbase + B_DL, dl = dh + 16384, ph = rec_s + REC_P, pl = ph + 8192;
-            gemm(tm + TM_O2, dh, 2048, 128, 4096, ph, 1024, 128, 2048, C / 16, ID_KK, false);
-            gemm(tm + TM_O2, dh, 2048, 128, 4096, pl, 1024, 128, 2048, C / 16, ID_KK, true);
-            gemm(tm + TM_O2, dl, 2048, 128, 4096, ph, 1024, 128, 2048, C / 16, ID_KK, true);
-            const uint32_t eh = sbase + B_DT, el = eh + 16384;
-            gemm(tm + TM_S, eh, 2048, 128, 4096, kq, 2048, 128, 4096, C / 16, ID_S, true);
-            gemm(tm + TM_S, el, 2048, 128, 4096, kq, 2048, 128, 4096, C / 16, ID_S, true);
-        });
-        alive = wait_mma();
-        if (!alive) break;
-
-        // This chunk's K is consumed: fetch the next chunk's.
-        const int r0 = 16 * part;
-        if (n0 < t1) {
-            fetch_half(n0, Ln, false);
-            fetch_z(n0, Ln, buf ^ 1);  // read by the next chunk's norm, after its K wait
-        }
-        cp_async_commit();
-
-        // O = (m e^gamma)(S Q^T) + Delta P^T staged as [r][i]; the new state's bf16 copy.
-        {
-            const int i = 32 * quad + lane;
-            float a[16], b[16];
-            tmem_ld16(tm + lane_off + TM_OI + r0, a);
-            tmem_ld16(tm + lane_off + TM_O2 + r0, b);
-            float *Os = reinterpret_cast<float *>(sm + B_DL);
-#pragma unroll
-            for (int c = 0; c < 16; ++c) Os[(r0 + c) * D + i] = fmaf(rscal[C + r0 + c], a[c], b[c]);
-            const int j0 = 32 * part;
-            float v[32];
-            tmem_ld32(tm + lane_off + TM_S + j0, v);
+        __syncwarp();
+    } else if (warp < 8) {
+        // --------------------------------------------------- state group
+        const int quad = warp & 3, half = warp >> 2;
+        const int i = 32 * quad + lane;
+        const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
+        // Every wait's outcome is made warp-uniform, so a warp stops as a whole.
+        auto wait_all = [&](uint64_t *bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, kWaitNs)) != 0;
+        };
+        // Hand the staged tiles and TMEM to the MMA warp: one arrival per warp.
+        auto publish = [&](uint64_t *bar) {
+            fence_smem_to_async();
+            fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar);
+        };
+        // Row i of S (32 columns from j0): bf16 copy for the MMAs and, scaled by
+        // e^{gamma_L} of the coming chunk, back into TMEM for its update.
+        auto stage_state = [&](float (&v)[32], int j0, float eL) {
 #pragma unroll
             for (int j8 = 0; j8 < 4; ++j8)
                 *reinterpret_cast<uint4 *>(sm + B_S + kmaj(i, j0 + 8 * j8, D)) = pack8(v + 8 * j8);
-        }
-        __syncthreads();
-        // RMSNormGated per token (one warp per C / NW tokens, unrolled), store.
-        {
-            const float *Os = reinterpret_cast<const float *>(sm + B_DL);
 #pragma unroll
-            for (int u = 0; u < C / NW; ++u) {
-                const int r = warp + NW * u;
+            for (int u = 0; u < 32; ++u) v[u] *= eL;
+            tmem_st32(tm + lane_off + TM_S + j0, v);
+        };
+
+        if (n_chunks == 0) {
+            // An empty sequence leaves its state as it came in.
+            if (p.final_state) {
+                const size_t off = ((size_t)seq * p.H_v + hv) * D * D + (size_t)i * D + 64 * half;
+#pragma unroll 4
+                for (int j4 = 0; j4 < 16; ++j4)
+                    *reinterpret_cast<float4 *>(p.final_state + off + 4 * j4) =
+                        p.initial_state ? __ldg(reinterpret_cast<const float4 *>(p.initial_state + off + 4 * j4))
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+        bool ok = n_chunks > 0 && wait_all(bar_rec, 0);
+        if (ok) {
+            const float eL = rscal(0)[3 * C];
+            const float *s0 = p.initial_state
+                                  ? p.initial_state + ((size_t)seq * p.H_v + hv) * D * D + (size_t)i * D
+                                  : nullptr;
+#pragma unroll 1
+            for (int jj = 0; jj < 2; ++jj) {
+                const int j0 = 64 * half + 32 * jj;
+                float v[32];
+#pragma unroll
+                for (int j4 = 0; j4 < 8; ++j4) {
+                    const float4 x = s0 ? __ldg(reinterpret_cast<const float4 *>(s0 + j0 + 4 * j4))
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                    v[4 * j4] = x.x; v[4 * j4 + 1] = x.y; v[4 * j4 + 2] = x.z; v[4 * j4 + 3] = x.w;
+                }
+                stage_state(v, j0, eL);
+            }
+            publish(bar_sready);
+        }
+        int c = 0;
+        for (; c < n_chunks && ok; ++c) {
+            const unsigned char *rec = rec0 + (size_t)c * rec_step;
+            const float *sc = rscal(c);
+            // U (rows s = 32*half ..) for the Delta epilogue (prefetched into L2).
+            float4 uu[8];
+#pragma unroll
+            for (int s4 = 0; s4 < 8; ++s4)
+                uu[s4] = __ldg(reinterpret_cast<const float4 *>(rec + REC_U + u_off(32 * half + 4 * s4, i)));
+
+            // Delta^T = U^T - S W^T as hi/lo tiles, and its decayed, k-normalised copy.
+            ok = wait_all(bar_gd, (uint32_t)c & 1u);
+            if (!ok) break;
+            fence_after_sync();
+#pragma unroll
+            for (int h16 = 0; h16 < 2; ++h16) {
+                const int s0 = 32 * half + 16 * h16;
+                float v[16], w[16];
+                tmem_ld16(tm + lane_off + TM_D + s0, v);
+#pragma unroll
+                for (int s4 = 0; s4 < 4; ++s4) {
+                    const float4 u = uu[4 * h16 + s4];
+                    v[4 * s4] += u.x; v[4 * s4 + 1] += u.y; v[4 * s4 + 2] += u.z; v[4 * s4 + 3] += u.w;
+                }
+#pragma unroll
+                for (int s = 0; s < 16; ++s) w[s] = v[s] * sc[2 * C + s0 + s];
+#pragma unroll
+                for (int c8 = 0; c8 < 2; ++c8) {
+                    uint4 hi, lo;
+                    const uint32_t o = kmaj(i, s0 + 8 * c8, D);
+                    split8(v + 8 * c8, hi, lo);
+                    *reinterpret_cast<uint4 *>(sm + B_DL + o) = hi;
+                    *reinterpret_cast<uint4 *>(sm + B_DL + 16384 + o) = lo;
+                    split8(w + 8 * c8, hi, lo);
+                    *reinterpret_cast<uint4 *>(sm + B_DT + o) = hi;
+                    *reinterpret_cast<uint4 *>(sm + B_DT + 16384 + o) = lo;
+                }
+            }
+            publish(bar_dready);
+
+            // Once the state update is done: the next chunk's bf16 S and scaled S.
+            ok = wait_all(bar_gs, (uint32_t)c & 1u);
+            if (!ok || c + 1 == n_chunks) continue;
+            ok = wait_all(bar_rec + ((c + 1) & 1), (uint32_t)((c + 1) >> 1) & 1u);
+            if (!ok) continue;
+            fence_after_sync();
+            const float eL = rscal(c + 1)[3 * C];
+#pragma unroll 1
+            for (int jj = 0; jj < 2; ++jj) {
+                const int j0 = 64 * half + 32 * jj;
+                float v[32];
+                tmem_ld32(tm + lane_off + TM_S + j0, v);
+                stage_state(v, j0, eL);
+            }
+            publish(bar_sready);
+        }
+        state_ok = ok && n_chunks > 0 && c == n_chunks;
+        if (n_chunks > 0 && !state_ok && lane == 0) fail();
+    } else {
+        // -------------------------------------------------- output group
+        const int quad = warp & 3, half = (warp >> 2) & 1;
+        const int og = warp - 8;                // 0..7: tokens 8*og .. 8*og+7 in the norm
+        const int i = 32 * quad + lane;
+        const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
+        const __nv_bfloat16 *zg = static_cast<const __nv_bfloat16 *>(p.z);
+        TOUT *out = static_cast<TOUT *>(p.out);
+        float *Os = reinterpret_cast<float *>(sm + B_OS);
+        float4 w4 = make_float4(1.f, 1.f, 1.f, 1.f);
+        if (zg && p.norm_w)
+            w4 = make_float4(__ldg(p.norm_w + 4 * lane), __ldg(p.norm_w + 4 * lane + 1),
+                             __ldg(p.norm_w + 4 * lane + 2), __ldg(p.norm_w + 4 * lane + 3));
+        bool dead = false;
+        for (int c = 0; c < n_chunks && !dead; ++c) {
+            const int b = c & 1;
+            const int64_t c0 = t0 + (int64_t)c * C;
+            const int L = chunk_len(c);
+            // z of this warp's 8 tokens (4 values per lane), loaded before the wait.
+            uint2 zr[8];
+            if (zg) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int r = 8 * og + u;
+                    zr[u] = r < L ? __ldg(reinterpret_cast<const uint2 *>(zg + (c0 + r) * p.z_stride + hv * D + 4 * lane))
+                                  : make_uint2(0u, 0u);
+                }
+            }
+            bool ok = mbar_wait(bar_oready + b, (uint32_t)(c >> 1) & 1u, kWaitNs);
+            if (ok) {
+                // O^T [i][r] = (m e^gamma)_r (S Q^T) + (P Delta)^T, staged as O [r][i].
+                fence_after_sync();
+                const float *sc = rscal(c);
+                const int r0 = 32 * half;
+#pragma unroll
+                for (int h16 = 0; h16 < 2; ++h16) {
+                    float a[16], d[16];
+                    tmem_ld16(tm + lane_off + TM_OI + 64 * b + r0 + 16 * h16, a);
+                    tmem_ld16(tm + lane_off + TM_O2 + 64 * b + r0 + 16 * h16, d);
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        const int r = r0 + 16 * h16 + k;
+                        Os[r * D + i] = fmaf(sc[C + r], a[k], d[k]);
+                    }
+                }
+            }
+            // TMEM buffers and the record's scalars go back to the MMA warp and producer.
+            fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_ofree + b);
+            dead = group_sync_or(OG_BAR, OG_N, !ok);
+            if (dead) break;
+            // RMSNormGated: one warp per token, 4 values per lane.
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int r = 8 * og + u;
                 const float4 o4 = *reinterpret_cast<const float4 *>(Os + r * D + 4 * lane);
                 float4 y = o4;
                 if (zg) {
                     const float ss = group_sum<32>(dot4(o4, o4));
                     const float rstd = rsqrtf(ss * (1.0f / D) + p.eps_norm);
-                    const uint2 zr = *reinterpret_cast<const uint2 *>(zbuf + r * 256 + 8 * lane);
-                    const float2 za = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&zr.x));
-                    const float2 zb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&zr.y));
+                    const float2 za = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&zr[u].x));
+                    const float2 zb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&zr[u].y));
                     y.x = o4.x * rstd * w4.x * fast_silu(za.x);
                     y.y = o4.y * rstd * w4.y * fast_silu(za.y);
                     y.z = o4.z * rstd * w4.z * fast_silu(zb.x);
                     y.w = o4.w * rstd * w4.w * fast_silu(zb.y);
                 }
-                if (r < L) Elem<TOUT>::store4(og + (c0 + r) * p.out_stride + hv * D + 4 * lane, y);
+                if (r < L) Elem<TOUT>::store4(out + (c0 + r) * p.out_stride + hv * D + 4 * lane, y);
             }
+            // The stage is rewritten by the next chunk.
+            group_sync_or(OG_BAR, OG_N, false);
         }
-        __syncthreads();
+        if (dead && tid == 256) fail();
     }
-    cp_async_wait<0>();  // nothing may land in shared memory after the CTA ends
 
-    if (alive && p.final_state) {
-        const int i = 32 * quad + lane, j0 = 32 * part;
-        float *dst = p.final_state + ((size_t)seq * p.H_v + hv) * D * D + (size_t)i * D + j0;
-        float v[32];
-        tmem_ld32(tm + lane_off + TM_S + j0, v);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (warp < 8 && state_ok && p.final_state) {
+        const int quad = warp & 3, half = warp >> 2;
+        const int i = 32 * quad + lane;
+        const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
+        float *dst = p.final_state + ((size_t)seq * p.H_v + hv) * D * D + (size_t)i * D;
+#pragma unroll 1
+        for (int jj = 0; jj < 2; ++jj) {
+            const int j0 = 64 * half + 32 * jj;
+            float v[32];
+            tmem_ld32(tm + lane_off + TM_S + j0, v);
 #pragma unroll
-        for (int j4 = 0; j4 < 8; ++j4)
-            *reinterpret_cast<float4 *>(dst + 4 * j4) = make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
+            for (int j4 = 0; j4 < 8; ++j4)
+                *reinterpret_cast<float4 *>(dst + j0 + 4 * j4) =
+                    make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
+        }
     }
     fence_before_sync();
     __syncthreads();
@@ -664,7 +771,7 @@ cudaError_t launch_prefill_tc2p(const PrefillParams &p, int64_t n_chunks, void *
     auto kern = out_bf16 ? tcp2::recur_kernel<__nv_bfloat16> : tcp2::recur_kernel<float>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcp2::B_SMEM);
     if (e != cudaSuccess) return e;
-    kern<<<(unsigned)((int64_t)p.n_seq * p.H_v), tcp2::NT, tcp2::B_SMEM, s>>>(p, order, chunk_off,
+    kern<<<(unsigned)((int64_t)p.n_seq * p.H_v), tcp2::RNT, tcp2::B_SMEM, s>>>(p, order, chunk_off,
                                                                               records, status);
     return cudaGetLastError();
 }

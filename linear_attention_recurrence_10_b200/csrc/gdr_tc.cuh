@@ -181,18 +181,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64
     const uint32_t a = smem_u32(bar);
     uint64_t start = 0;
     for (uint32_t i = 0;; ++i) {
+        // try_wait may suspend the thread (for a bounded, hardware-chosen time)
+        // instead of spinning, leaving issue slots to the warps doing work.
         uint32_t done;
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
-            "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
             "selp.b32 %0, 1, 0, p;\n\t}\n"
             : "=r"(done)
             : "r"(a), "r"(parity)
             : "memory");
         if (done) return true;
         if (i == 0) start = global_ns();
-        else if ((i & 63) == 0 && global_ns() - start > timeout_ns) return false;
-        if (i > 256) __nanosleep(64);
+        else if (global_ns() - start > timeout_ns) return false;
     }
 }
 
@@ -237,6 +238,45 @@ __device__ __forceinline__ void bulk_copy(void *smem_dst, const void *gmem_src, 
             smem_u32(smem_dst)),
         "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
+}
+
+// Start moving `bytes` (a multiple of 16, 16-byte aligned) of global memory
+// into L2; nothing is written anywhere and nothing needs to be waited for.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *gmem_src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gmem_src), "r"(bytes)
+                 : "memory");
+}
+
+// A plain arrival (release semantics) on the barrier.
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// One arrival on the barrier once every cp.async this thread has issued so far
+// has landed.  The arrival is not pre-counted (.noinc): the barrier's expected
+// count must include one per calling thread.
+__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// ------------------------------------------------------ named barriers
+
+// Barrier `id` (1..15) over `n` threads (a multiple of 32) that also returns
+// whether `pred` held in any of them -- lets a group agree to stop together.
+__device__ __forceinline__ bool group_sync_or(int id, int n, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.cta.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}\n"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
 }
 
 // fp32 -> tf32 (round to nearest, ties away), kept in a 32-bit container.

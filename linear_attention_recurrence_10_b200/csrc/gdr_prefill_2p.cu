@@ -31,7 +31,7 @@ using namespace gdr::tcp;
 // The first REC_STAGED bytes (W, P, scalars) are staged in shared memory by the
 // recurrence; U is read from here straight into registers.
 constexpr uint32_t REC_W = 0;        // bf16 W, MN-major B tile (w_off), 16 KB
-constexpr uint32_t REC_P = 16384;    // P hi, then lo, K-major [r][s] (kmaj R=64), 8 KB each
+constexpr uint32_t REC_P = 16384;    // P~ = P diag(1/dn) hi, then lo, K-major [r][s] (kmaj R=64), 8 KB each
 constexpr uint32_t REC_SCAL = 32768; // fp32 eg[64] | nqe[64] | dn[64] | eL | pad
 constexpr uint32_t REC_STAGED = 33792;
 constexpr uint32_t REC_U = 33792;    // fp32 U: byte (s/4)*2048 + i*16 + (s%4)*4, 32 KB
@@ -255,11 +255,14 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p, con
                 Ascr[rr * LDA + s] = s < rr ? f * __expf(gr - sc.gam[s]) * sc.nk[s] * v[c] : 0.f;
             }
         } else {
-            const float f = sc.nq[rr];
+            // P~ = P diag(1/dn): P_rs = nq_r e^{gamma_r - gamma_s} n_s QK_rs over
+            // dn_s = e^{gamma_L - gamma_s} n_s leaves nq_r e^{gamma_r - gamma_L} QK_rs,
+            // so that P Delta = P~ (diag(dn) Delta) reuses the decayed Delta tiles.
+            const float f = sc.nq[rr] * __expf(gr - sc.gam[L - 1]);
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
                 const int s = s0 + c;
-                v[c] = s <= rr ? f * __expf(gr - sc.gam[s]) * sc.nk[s] * v[c] : 0.f;
+                v[c] = (s <= rr && sc.nk[s] != 0.f) ? f * v[c] : 0.f;
             }
 #pragma unroll
             for (int c8 = 0; c8 < 2; ++c8) {
@@ -339,17 +342,19 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p, con
 // and the next state needs Delta.  The output of a chunk (O = (m e^gamma) Q S^T
 // + P Delta, then RMSNormGated) feeds nothing later, so the CTA is split into
 // four roles that run concurrently and hand work over on mbarriers:
-//   warps 0-7   state group: the Delta epilogue (hi/lo tiles of Delta and of
-//               its decayed, k-normalised copy) and, once the state update is
-//               done, the bf16 copy of S for the next chunk's products, with
-//               the next chunk's e^{gamma_L} folded into the same pass;
-//   warps 8-15  output group, one chunk behind: S Q^T and P Delta out of
+//   warps 0-7   state group: the Delta epilogue (hi/lo tiles of Delta scaled
+//               by dn = e^{gamma_L - gamma} n, which feed both the state
+//               update and, with P~ = P diag(1/dn), the intra-chunk output)
+//               and, once the state update is done, the bf16 copy of S for
+//               the next chunk's products, with the next chunk's e^{gamma_L}
+//               folded into the same pass;
+//   warps 8-15  output group, one chunk behind: S Q^T and P~ Dt~ out of
 //               double-buffered TMEM, staged through shared memory so that
 //               one warp normalises, gates and stores whole tokens;
 //   warp 16     producer: K and Q tiles (cp.async with zero fill past the
 //               sequence end, counted on an mbarrier), the staged records
-//               (one bulk copy each, double-buffered) and an L2 prefetch of
-//               the next chunk's U;
+//               (one bulk copy each, double-buffered, with an L2 prefetch of
+//               their U) and each chunk's U into a stage of its own;
 //   warp 17     MMA issue, state path first (-S W^T before S Q^T, the state
 //               update before P Delta), each group committed on its own
 //               barrier so the state group never waits for output products.
@@ -359,7 +364,7 @@ constexpr int OG_BAR = 1, OG_N = 256;
 constexpr uint32_t B_KQ = 0;                   // bf16 [K;Q] (32 KB)
 constexpr uint32_t B_REC = 32768;              // 2 x staged record (W, P, scalars: 33 KB each)
 constexpr uint32_t B_S = 100352;               // bf16 S [i][j] (32 KB)
-constexpr uint32_t B_DL = 133120;              // Delta hi/lo (32 KB)
+constexpr uint32_t B_U = 133120;               // fp32 U of the current chunk (32 KB, record layout)
 constexpr uint32_t B_DT = 165888;              // decayed Delta hi/lo (32 KB)
 constexpr uint32_t B_OS = 198656;              // fp32 O [r][i] of the chunk being output (32 KB)
 constexpr uint32_t B_BAR = 231424;             // 13 mbarriers, then the TMEM address
@@ -382,7 +387,8 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
     uint64_t *bar_ofree = bars + 9;              // [2] output group done with a chunk's buffers
     uint64_t *bar_sready = bars + 11;            // state group: bf16 S staged (8 warps)
     uint64_t *bar_dready = bars + 12;            // state group: Delta tiles staged (8 warps)
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + B_BAR + 112);
+    uint64_t *bar_u = bars + 13;                 // U of the current chunk landed
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + B_BAR + 120);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int seq = order[blockIdx.x / p.H_v];
     const int hv = blockIdx.x % p.H_v;
@@ -415,6 +421,7 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
         mbar_init(bar_gs, 1);
         mbar_init(bar_sready, 8);
         mbar_init(bar_dready, 8);
+        mbar_init(bar_u, 1);
         mbar_fence_init();
     }
     fence_before_sync();
@@ -450,13 +457,13 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
                 if (!ok) break;
                 fence_after_sync();
                 fence_smem_to_async();
-                // S <- e^{gamma_L} S + Dt~^T K (hi + lo); then O_intra^T = Delta^T P^T
+                // S <- e^{gamma_L} S + Dt~^T K (hi + lo); then O_intra^T = Dt~^T P~^T
                 // (hi*hi + hi*lo + lo*hi) into this chunk's output buffer.
                 const uint32_t eh = sbase + B_DT, el = eh + 16384;
                 gemm(tm + TM_S, eh, 2048, 128, 4096, kq, 2048, 128, 4096, C / 16, ID_S, true);
                 gemm(tm + TM_S, el, 2048, 128, 4096, kq, 2048, 128, 4096, C / 16, ID_S, true);
                 commit(smem_u32(bar_gs));
-                const uint32_t dh = sbase + B_DL, dl = dh + 16384, ph = rec_s + REC_P, pl = ph + 8192;
+                const uint32_t dh = eh, dl = el, ph = rec_s + REC_P, pl = ph + 8192;
                 const uint32_t o2 = tm + TM_O2 + 64 * b;
                 gemm(o2, dh, 2048, 128, 4096, ph, 1024, 128, 2048, C / 16, ID_KK, false);
                 gemm(o2, dh, 2048, 128, 4096, pl, 1024, 128, 2048, C / 16, ID_KK, true);
@@ -486,7 +493,7 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
             }
             cp_async_arrive(q_half ? bar_q : bar_k);
         };
-        int issued[2] = {0, 0};
+        int issued[2] = {0, 0}, u_issued = 0;
         auto fetch_rec = [&](int c) {
             const int b = c & 1;
             ++issued[b];
@@ -505,6 +512,14 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
             if (c > 0) ok = mbar_wait(bar_qfree, (c - 1) & 1, kWaitNs);
             if (!ok) break;
             fetch(c0, L, true);
+            // U of chunk c once the Delta epilogue of chunk c-1 is done with the stage.
+            if (c > 0) ok = mbar_wait(bar_dready, (c - 1) & 1, kWaitNs);
+            if (!ok) break;
+            ++u_issued;
+            if (lane == 0) {
+                bulk_expect(bar_u, REC_BYTES - REC_U);
+                bulk_copy(sm + B_U, rec0 + (size_t)c * rec_step + REC_U, REC_BYTES - REC_U, bar_u);
+            }
             if (c > 0) ok = mbar_wait(bar_gs, (c - 1) & 1, kWaitNs);
             if (!ok) break;
             fetch(c0, L, false);
@@ -521,6 +536,7 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
             // No bulk copy may land after the CTA ends.
             for (int b = 0; b < 2; ++b)
                 if (issued[b] > 0) mbar_wait(bar_rec + b, (uint32_t)(issued[b] - 1) & 1u, kWaitNs);
+            if (u_issued > 0) mbar_wait(bar_u, (uint32_t)(u_issued - 1) & 1u, kWaitNs);
         }
         __syncwarp();
     } else if (warp < 8) {
@@ -583,38 +599,30 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
         }
         int c = 0;
         for (; c < n_chunks && ok; ++c) {
-            const unsigned char *rec = rec0 + (size_t)c * rec_step;
             const float *sc = rscal(c);
-            // U (rows s = 32*half ..) for the Delta epilogue (prefetched into L2).
-            float4 uu[8];
-#pragma unroll
-            for (int s4 = 0; s4 < 8; ++s4)
-                uu[s4] = __ldg(reinterpret_cast<const float4 *>(rec + REC_U + u_off(32 * half + 4 * s4, i)));
-
-            // Delta^T = U^T - S W^T as hi/lo tiles, and its decayed, k-normalised copy.
-            ok = wait_all(bar_gd, (uint32_t)c & 1u);
+            // Dt~^T = (U^T - S W^T) diag(dn) as hi/lo tiles.
+            ok = wait_all(bar_gd, (uint32_t)c & 1u) && wait_all(bar_u, (uint32_t)c & 1u);
             if (!ok) break;
             fence_after_sync();
 #pragma unroll
             for (int h16 = 0; h16 < 2; ++h16) {
                 const int s0 = 32 * half + 16 * h16;
-                float v[16], w[16];
+                float v[16];
                 tmem_ld16(tm + lane_off + TM_D + s0, v);
 #pragma unroll
                 for (int s4 = 0; s4 < 4; ++s4) {
-                    const float4 u = uu[4 * h16 + s4];
-                    v[4 * s4] += u.x; v[4 * s4 + 1] += u.y; v[4 * s4 + 2] += u.z; v[4 * s4 + 3] += u.w;
+                    const float4 u = *reinterpret_cast<const float4 *>(sm + B_U + u_off(s0 + 4 * s4, i));
+                    const float4 dn = *reinterpret_cast<const float4 *>(sc + 2 * C + s0 + 4 * s4);
+                    v[4 * s4] = (v[4 * s4] + u.x) * dn.x;
+                    v[4 * s4 + 1] = (v[4 * s4 + 1] + u.y) * dn.y;
+                    v[4 * s4 + 2] = (v[4 * s4 + 2] + u.z) * dn.z;
+                    v[4 * s4 + 3] = (v[4 * s4 + 3] + u.w) * dn.w;
                 }
-#pragma unroll
-                for (int s = 0; s < 16; ++s) w[s] = v[s] * sc[2 * C + s0 + s];
 #pragma unroll
                 for (int c8 = 0; c8 < 2; ++c8) {
                     uint4 hi, lo;
                     const uint32_t o = kmaj(i, s0 + 8 * c8, D);
                     split8(v + 8 * c8, hi, lo);
-                    *reinterpret_cast<uint4 *>(sm + B_DL + o) = hi;
-                    *reinterpret_cast<uint4 *>(sm + B_DL + 16384 + o) = lo;
-                    split8(w + 8 * c8, hi, lo);
                     *reinterpret_cast<uint4 *>(sm + B_DT + o) = hi;
                     *reinterpret_cast<uint4 *>(sm + B_DT + 16384 + o) = lo;
                 }
@@ -679,9 +687,13 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
                     tmem_ld16(tm + lane_off + TM_OI + 64 * b + r0 + 16 * h16, a);
                     tmem_ld16(tm + lane_off + TM_O2 + 64 * b + r0 + 16 * h16, d);
 #pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        const int r = r0 + 16 * h16 + k;
-                        Os[r * D + i] = fmaf(sc[C + r], a[k], d[k]);
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const int r = r0 + 16 * h16 + 4 * k4;
+                        const float4 m = *reinterpret_cast<const float4 *>(sc + C + r);
+                        Os[r * D + i] = fmaf(m.x, a[4 * k4], d[4 * k4]);
+                        Os[(r + 1) * D + i] = fmaf(m.y, a[4 * k4 + 1], d[4 * k4 + 1]);
+                        Os[(r + 2) * D + i] = fmaf(m.z, a[4 * k4 + 2], d[4 * k4 + 2]);
+                        Os[(r + 3) * D + i] = fmaf(m.w, a[4 * k4 + 3], d[4 * k4 + 3]);
                     }
                 }
             }
@@ -691,21 +703,45 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
             if (lane == 0) mbar_arrive(bar_ofree + b);
             dead = group_sync_or(OG_BAR, OG_N, !ok);
             if (dead) break;
-            // RMSNormGated: one warp per token, 4 values per lane.
+            // RMSNormGated: a warp holds 8 whole tokens, 4 values per lane.
+            float4 o4[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) o4[u] = *reinterpret_cast<const float4 *>(Os + (8 * og + u) * D + 4 * lane);
+            float rstd_l = 0.f;
+            if (zg) {
+                // Sums of squares of the 8 tokens by a transposing butterfly: after
+                // the xor-4/2/1 stages lane l holds token (l & 7) summed over 8
+                // lanes; xor 8 and 16 finish the sum (9 shuffles for 8 tokens).
+                float ps[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) ps[u] = dot4(o4[u], o4[u]);
+#pragma unroll
+                for (int st = 4; st >= 1; st >>= 1) {
+                    const bool upper = (lane & st) != 0;
+#pragma unroll
+                    for (int j = 0; j < st; ++j) {
+                        const float send = upper ? ps[j] : ps[j + st];
+                        const float keep = upper ? ps[j + st] : ps[j];
+                        ps[j] = keep + __shfl_xor_sync(0xffffffffu, send, st);
+                    }
+                }
+                float t = ps[0];
+                t += __shfl_xor_sync(0xffffffffu, t, 8);
+                t += __shfl_xor_sync(0xffffffffu, t, 16);
+                rstd_l = rsqrtf(t * (1.0f / D) + p.eps_norm);
+            }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int r = 8 * og + u;
-                const float4 o4 = *reinterpret_cast<const float4 *>(Os + r * D + 4 * lane);
-                float4 y = o4;
+                float4 y = o4[u];
                 if (zg) {
-                    const float ss = group_sum<32>(dot4(o4, o4));
-                    const float rstd = rsqrtf(ss * (1.0f / D) + p.eps_norm);
+                    const float rstd = __shfl_sync(0xffffffffu, rstd_l, u);
                     const float2 za = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&zr[u].x));
                     const float2 zb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&zr[u].y));
-                    y.x = o4.x * rstd * w4.x * fast_silu(za.x);
-                    y.y = o4.y * rstd * w4.y * fast_silu(za.y);
-                    y.z = o4.z * rstd * w4.z * fast_silu(zb.x);
-                    y.w = o4.w * rstd * w4.w * fast_silu(zb.y);
+                    y.x *= rstd * w4.x * fast_silu(za.x);
+                    y.y *= rstd * w4.y * fast_silu(za.y);
+                    y.z *= rstd * w4.z * fast_silu(zb.x);
+                    y.w *= rstd * w4.w * fast_silu(zb.y);
                 }
                 if (r < L) Elem<TOUT>::store4(out + (c0 + r) * p.out_stride + hv * D + 4 * lane, y);
             }

@@ -67,14 +67,17 @@ __device__ __forceinline__ uint4 pack8(const float *v) {
 }
 // Split eight fp32 values into bf16 hi = rn(x) and lo = rn(x - hi).
 __device__ __forceinline__ void split8(const float *v, uint4 &hi, uint4 &lo) {
-    float h[8], l[8];
+    uint32_t h[4], l[4];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-        h[u] = __bfloat162float(__float2bfloat16_rn(v[u]));
-        l[u] = v[u] - h[u];
+    for (int u = 0; u < 4; ++u) {
+        const __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * u], v[2 * u + 1]);
+        const float2 f = __bfloat1622float2(b);
+        const __nv_bfloat162 r = __floats2bfloat162_rn(v[2 * u] - f.x, v[2 * u + 1] - f.y);
+        h[u] = *reinterpret_cast<const uint32_t *>(&b);
+        l[u] = *reinterpret_cast<const uint32_t *>(&r);
     }
-    hi = pack8(h);
-    lo = pack8(l);
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
 // One distance of the blocked triangular inverse: for every pair of 16-blocks

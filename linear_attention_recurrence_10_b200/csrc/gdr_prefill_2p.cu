@@ -31,7 +31,7 @@ using namespace gdr::tcp;
 // The first REC_STAGED bytes (W, P, scalars) are staged in shared memory by the
 // recurrence; U is read from here straight into registers.
 constexpr uint32_t REC_W = 0;        // bf16 W, MN-major B tile (w_off), 16 KB
-constexpr uint32_t REC_P = 16384;    // P~ = P diag(1/dn) hi, then lo, K-major [r][s] (kmaj R=64), 8 KB each
+constexpr uint32_t REC_P = 16384;    // P hi, then lo, K-major [r][s] (kmaj R=64), 8 KB each
 constexpr uint32_t REC_SCAL = 32768; // fp32 eg[64] | nqe[64] | dn[64] | eL | pad
 constexpr uint32_t REC_STAGED = 33792;
 constexpr uint32_t REC_U = 33792;    // fp32 U: byte (s/4)*2048 + i*16 + (s%4)*4, 32 KB
@@ -255,14 +255,14 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p, con
                 Ascr[rr * LDA + s] = s < rr ? f * __expf(gr - sc.gam[s]) * sc.nk[s] * v[c] : 0.f;
             }
         } else {
-            // P~ = P diag(1/dn): P_rs = nq_r e^{gamma_r - gamma_s} n_s QK_rs over
-            // dn_s = e^{gamma_L - gamma_s} n_s leaves nq_r e^{gamma_r - gamma_L} QK_rs,
-            // so that P Delta = P~ (diag(dn) Delta) reuses the decayed Delta tiles.
-            const float f = sc.nq[rr] * __expf(gr - sc.gam[L - 1]);
+            // P_rs = nq_r e^{gamma_r - gamma_s} n_s QK_rs (s <= r): every factor is
+            // at most one in size whatever the decay, which a rescaled form
+            // (say P diag(1/dn)) would not be.
+            const float f = sc.nq[rr];
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
                 const int s = s0 + c;
-                v[c] = (s <= rr && sc.nk[s] != 0.f) ? f * v[c] : 0.f;
+                v[c] = s <= rr ? f * __expf(gr - sc.gam[s]) * sc.nk[s] * v[c] : 0.f;
             }
 #pragma unroll
             for (int c8 = 0; c8 < 2; ++c8) {
@@ -342,19 +342,18 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p, con
 // and the next state needs Delta.  The output of a chunk (O = (m e^gamma) Q S^T
 // + P Delta, then RMSNormGated) feeds nothing later, so the CTA is split into
 // four roles that run concurrently and hand work over on mbarriers:
-//   warps 0-7   state group: the Delta epilogue (hi/lo tiles of Delta scaled
-//               by dn = e^{gamma_L - gamma} n, which feed both the state
-//               update and, with P~ = P diag(1/dn), the intra-chunk output)
-//               and, once the state update is done, the bf16 copy of S for
-//               the next chunk's products, with the next chunk's e^{gamma_L}
-//               folded into the same pass;
-//   warps 8-15  output group, one chunk behind: S Q^T and P~ Dt~ out of
+//   warps 0-7   state group: the Delta epilogue (hi/lo tiles of Delta and of
+//               its decayed, k-normalised copy) and, once the state update is
+//               done, the bf16 copy of S for the next chunk's products, with
+//               the next chunk's e^{gamma_L} folded into the same pass;
+//   warps 8-15  output group, one chunk behind: S Q^T and P Delta out of
 //               double-buffered TMEM, staged through shared memory so that
 //               one warp normalises, gates and stores whole tokens;
 //   warp 16     producer: K and Q tiles (cp.async with zero fill past the
-//               sequence end, counted on an mbarrier), the staged records
-//               (one bulk copy each, double-buffered, with an L2 prefetch of
-//               their U) and each chunk's U into a stage of its own;
+//               sequence end, counted on an mbarrier), and by bulk copy each
+//               chunk's W, P, U and scalars, every one into its stage as soon
+//               as the previous chunk is done with it (the record is first
+//               prefetched into L2 a chunk ahead);
 //   warp 17     MMA issue, state path first (-S W^T before S Q^T, the state
 //               update before P Delta), each group committed on its own
 //               barrier so the state group never waits for output products.
@@ -362,13 +361,17 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p, con
 constexpr int RNT = 576;                       // 18 warps
 constexpr int OG_BAR = 1, OG_N = 256;
 constexpr uint32_t B_KQ = 0;                   // bf16 [K;Q] (32 KB)
-constexpr uint32_t B_REC = 32768;              // 2 x staged record (W, P, scalars: 33 KB each)
-constexpr uint32_t B_S = 100352;               // bf16 S [i][j] (32 KB)
-constexpr uint32_t B_U = 133120;               // fp32 U of the current chunk (32 KB, record layout)
-constexpr uint32_t B_DT = 165888;              // decayed Delta hi/lo (32 KB)
+constexpr uint32_t B_W = 32768;                // bf16 W of the current chunk (16 KB)
+constexpr uint32_t B_P = 49152;                // bf16 P hi/lo of the current chunk (16 KB)
+constexpr uint32_t B_SC = 65536;               // 2 x scalars (eg, nqe, dn, eL: 1 KB each)
+constexpr uint32_t B_S = 67584;                // bf16 S [i][j] (32 KB)
+constexpr uint32_t B_DL = 100352;              // Delta hi/lo (32 KB)
+constexpr uint32_t B_DT = 133120;              // decayed Delta hi/lo (32 KB)
+constexpr uint32_t B_U = 165888;               // fp32 U of the current chunk (32 KB, record layout)
 constexpr uint32_t B_OS = 198656;              // fp32 O [r][i] of the chunk being output (32 KB)
-constexpr uint32_t B_BAR = 231424;             // 13 mbarriers, then the TMEM address
-constexpr uint32_t B_SMEM = B_BAR + 128;
+constexpr uint32_t B_BAR = 231424;             // 16 mbarriers, then the TMEM address
+constexpr uint32_t B_SMEM = B_BAR + 144;
+constexpr uint32_t SC_BYTES = REC_STAGED - REC_SCAL;
 // TMEM columns: the fp32 state, -S W^T, and two buffers each of S Q^T and P Delta.
 constexpr uint32_t TM_S = 0, TM_D = 128, TM_OI = 192, TM_O2 = 320;
 
@@ -379,16 +382,18 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
     extern __shared__ __align__(1024) unsigned char sm[];
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + B_BAR);
     uint64_t *bar_q = bars, *bar_k = bars + 1;   // tiles landed (32 producer lanes each)
-    uint64_t *bar_rec = bars + 2;                // [2] staged record landed
-    uint64_t *bar_gd = bars + 4;                 // -S W^T done
-    uint64_t *bar_qfree = bars + 5;              // S Q^T done: the Q tile may be refilled
-    uint64_t *bar_gs = bars + 6;                 // state update done: the K tile may be refilled
-    uint64_t *bar_oready = bars + 7;             // [2] P Delta (and S Q^T) of a chunk done
-    uint64_t *bar_ofree = bars + 9;              // [2] output group done with a chunk's buffers
-    uint64_t *bar_sready = bars + 11;            // state group: bf16 S staged (8 warps)
-    uint64_t *bar_dready = bars + 12;            // state group: Delta tiles staged (8 warps)
-    uint64_t *bar_u = bars + 13;                 // U of the current chunk landed
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + B_BAR + 120);
+    uint64_t *bar_w = bars + 2;                  // W landed
+    uint64_t *bar_p = bars + 3;                  // P landed
+    uint64_t *bar_sc = bars + 4;                 // [2] scalars landed
+    uint64_t *bar_u = bars + 6;                  // U landed
+    uint64_t *bar_gd = bars + 7;                 // -S W^T done (W may be refilled)
+    uint64_t *bar_qfree = bars + 8;              // S Q^T done (Q may be refilled)
+    uint64_t *bar_gs = bars + 9;                 // state update done (K may be refilled)
+    uint64_t *bar_oready = bars + 10;            // [2] P Delta (and S Q^T) of a chunk done
+    uint64_t *bar_ofree = bars + 12;             // [2] output group done with a chunk's buffers
+    uint64_t *bar_sready = bars + 14;            // state group: bf16 S staged (8 warps)
+    uint64_t *bar_dready = bars + 15;            // state group: Delta tiles staged (8 warps)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + B_BAR + 128);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int seq = order[blockIdx.x / p.H_v];
     const int hv = blockIdx.x % p.H_v;
@@ -403,25 +408,25 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
         return (int)(left < C ? left : C);
     };
     auto fail = [&]() { atomicExch(status, kTimeoutStatus); };
-    auto rscal = [&](int c) {
-        return reinterpret_cast<const float *>(sm + B_REC + (c & 1) * REC_STAGED + REC_SCAL);
-    };
+    auto scal = [&](int c) { return reinterpret_cast<const float *>(sm + B_SC + (c & 1) * SC_BYTES); };
 
     if (warp == 0) tmem_alloc(tmem_slot, 512);
     if (tid == 0) {
         mbar_init(bar_q, 32);
         mbar_init(bar_k, 32);
         for (int b = 0; b < 2; ++b) {
-            mbar_init(bar_rec + b, 1);
+            mbar_init(bar_sc + b, 1);
             mbar_init(bar_oready + b, 1);
             mbar_init(bar_ofree + b, 8);
         }
+        mbar_init(bar_w, 1);
+        mbar_init(bar_p, 1);
+        mbar_init(bar_u, 1);
         mbar_init(bar_gd, 1);
         mbar_init(bar_qfree, 1);
         mbar_init(bar_gs, 1);
         mbar_init(bar_sready, 8);
         mbar_init(bar_dready, 8);
-        mbar_init(bar_u, 1);
         mbar_fence_init();
     }
     fence_before_sync();
@@ -440,34 +445,35 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
             bool ok = true;
             for (int c = 0; c < n_chunks && ok; ++c) {
                 const int b = c & 1;
-                const uint32_t rec_s = sbase + B_REC + b * REC_STAGED;
-                ok = mbar_wait(bar_sready, (uint32_t)c & 1u, kWaitNs) &&
-                     mbar_wait(bar_rec + b, (uint32_t)(c >> 1) & 1u, kWaitNs) &&
-                     mbar_wait(bar_q, (uint32_t)c & 1u, kWaitNs) &&
+                const uint32_t ph = (uint32_t)c & 1u;
+                ok = mbar_wait(bar_sready, ph, kWaitNs) && mbar_wait(bar_w, ph, kWaitNs) &&
+                     mbar_wait(bar_q, ph, kWaitNs) &&
                      (c < 2 || mbar_wait(bar_ofree + b, (uint32_t)((c >> 1) - 1) & 1u, kWaitNs));
                 if (!ok) break;
                 fence_after_sync();
                 fence_smem_to_async();
-                gemm(tm + TM_D, sbase + B_S, 2048, 128, 4096, rec_s + REC_W, 128, 2048, 256, D / 16, ID_D, false);
+                gemm(tm + TM_D, sbase + B_S, 2048, 128, 4096, sbase + B_W, 128, 2048, 256, D / 16, ID_D, false);
                 commit(smem_u32(bar_gd));
                 gemm(tm + TM_OI + 64 * b, sbase + B_S, 2048, 128, 4096, kq + 16384, 128, 2048, 256, D / 16, ID_KK, false);
                 commit(smem_u32(bar_qfree));
-                ok = mbar_wait(bar_dready, (uint32_t)c & 1u, kWaitNs) &&
-                     mbar_wait(bar_k, (uint32_t)c & 1u, kWaitNs);
+                ok = mbar_wait(bar_dready, ph, kWaitNs) && mbar_wait(bar_k, ph, kWaitNs);
                 if (!ok) break;
                 fence_after_sync();
                 fence_smem_to_async();
-                // S <- e^{gamma_L} S + Dt~^T K (hi + lo); then O_intra^T = Dt~^T P~^T
+                // S <- e^{gamma_L} S + Dt~^T K (hi + lo); then O_intra^T = Delta^T P^T
                 // (hi*hi + hi*lo + lo*hi) into this chunk's output buffer.
                 const uint32_t eh = sbase + B_DT, el = eh + 16384;
                 gemm(tm + TM_S, eh, 2048, 128, 4096, kq, 2048, 128, 4096, C / 16, ID_S, true);
                 gemm(tm + TM_S, el, 2048, 128, 4096, kq, 2048, 128, 4096, C / 16, ID_S, true);
                 commit(smem_u32(bar_gs));
-                const uint32_t dh = eh, dl = el, ph = rec_s + REC_P, pl = ph + 8192;
+                ok = mbar_wait(bar_p, ph, kWaitNs);
+                if (!ok) break;
+                fence_smem_to_async();
+                const uint32_t dh = sbase + B_DL, dl = dh + 16384, pb = sbase + B_P, pl = pb + 8192;
                 const uint32_t o2 = tm + TM_O2 + 64 * b;
-                gemm(o2, dh, 2048, 128, 4096, ph, 1024, 128, 2048, C / 16, ID_KK, false);
+                gemm(o2, dh, 2048, 128, 4096, pb, 1024, 128, 2048, C / 16, ID_KK, false);
                 gemm(o2, dh, 2048, 128, 4096, pl, 1024, 128, 2048, C / 16, ID_KK, true);
-                gemm(o2, dl, 2048, 128, 4096, ph, 1024, 128, 2048, C / 16, ID_KK, true);
+                gemm(o2, dl, 2048, 128, 4096, pb, 1024, 128, 2048, C / 16, ID_KK, true);
                 commit(smem_u32(bar_oready + b));
             }
             if (!ok) fail();
@@ -493,50 +499,67 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
             }
             cp_async_arrive(q_half ? bar_q : bar_k);
         };
-        int issued[2] = {0, 0}, u_issued = 0;
-        auto fetch_rec = [&](int c) {
-            const int b = c & 1;
-            ++issued[b];
+        // Bulk copies, each counted so that an early exit can wait for them.
+        int n_w = 0, n_p = 0, n_u = 0, n_sc[2] = {0, 0};
+        auto bulk = [&](uint32_t dst, uint32_t src_off, uint32_t bytes, uint64_t *bar, int c) {
             if (lane == 0) {
-                const unsigned char *rec = rec0 + (size_t)c * rec_step;
-                bulk_expect(bar_rec + b, REC_STAGED);
-                bulk_copy(sm + B_REC + b * REC_STAGED, rec, REC_STAGED, bar_rec + b);
-                bulk_prefetch_l2(rec + REC_U, REC_BYTES - REC_U);  // read by the state group
+                bulk_expect(bar, bytes);
+                bulk_copy(sm + dst, rec0 + (size_t)c * rec_step + src_off, bytes, bar);
             }
         };
+        auto prefetch = [&](int c) {
+            if (lane == 0 && c < n_chunks) bulk_prefetch_l2(rec0 + (size_t)c * rec_step, REC_BYTES);
+        };
         bool ok = true;
-        for (int c = 0; c < n_chunks && c < 2; ++c) fetch_rec(c);
+        prefetch(0);
+        prefetch(1);
+        for (int c = 0; c < n_chunks && c < 2; ++c) {
+            bulk(B_SC + (c & 1) * SC_BYTES, REC_SCAL, SC_BYTES, bar_sc + (c & 1), c);
+            ++n_sc[c & 1];
+        }
         for (int c = 0; c < n_chunks && ok; ++c) {
             const int64_t c0 = t0 + (int64_t)c * C;
             const int L = chunk_len(c);
-            if (c > 0) ok = mbar_wait(bar_qfree, (c - 1) & 1, kWaitNs);
+            const uint32_t pp = (uint32_t)(c - 1) & 1u;  // phase of chunk c-1's events
+            // Q and W of chunk c once chunk c-1's S Q^T (issued after -S W^T) is done.
+            if (c > 0) ok = mbar_wait(bar_qfree, pp, kWaitNs);
             if (!ok) break;
             fetch(c0, L, true);
-            // U of chunk c once the Delta epilogue of chunk c-1 is done with the stage.
-            if (c > 0) ok = mbar_wait(bar_dready, (c - 1) & 1, kWaitNs);
+            bulk(B_W, REC_W, REC_P - REC_W, bar_w, c);
+            ++n_w;
+            // U once chunk c-1's Delta epilogue is done with the stage.
+            if (c > 0) ok = mbar_wait(bar_dready, pp, kWaitNs);
             if (!ok) break;
-            ++u_issued;
-            if (lane == 0) {
-                bulk_expect(bar_u, REC_BYTES - REC_U);
-                bulk_copy(sm + B_U, rec0 + (size_t)c * rec_step + REC_U, REC_BYTES - REC_U, bar_u);
-            }
-            if (c > 0) ok = mbar_wait(bar_gs, (c - 1) & 1, kWaitNs);
+            bulk(B_U, REC_U, REC_BYTES - REC_U, bar_u, c);
+            ++n_u;
+            // K once chunk c-1's state update is done.
+            if (c > 0) ok = mbar_wait(bar_gs, pp, kWaitNs);
             if (!ok) break;
             fetch(c0, L, false);
-            // Record c+1 replaces record c-1 once the output group is done with it.
+            // P once chunk c-1's P Delta is done.
+            if (c > 0) ok = mbar_wait(bar_oready + ((c - 1) & 1), (uint32_t)((c - 1) >> 1) & 1u, kWaitNs);
+            if (!ok) break;
+            bulk(B_P, REC_P, REC_SCAL - REC_P, bar_p, c);
+            ++n_p;
+            // Scalars of chunk c+1 replace chunk c-1's once the output group is
+            // done with them; the record after that goes to L2.
             if (c >= 1 && c + 1 < n_chunks) {
-                ok = mbar_wait(bar_ofree + ((c + 1) & 1), ((c - 1) >> 1) & 1, kWaitNs);
+                ok = mbar_wait(bar_ofree + ((c + 1) & 1), (uint32_t)((c - 1) >> 1) & 1u, kWaitNs);
                 if (!ok) break;
-                fetch_rec(c + 1);
+                bulk(B_SC + ((c + 1) & 1) * SC_BYTES, REC_SCAL, SC_BYTES, bar_sc + ((c + 1) & 1), c + 1);
+                ++n_sc[(c + 1) & 1];
             }
+            prefetch(c + 2);
         }
         cp_async_wait_all();
         if (!ok) {
             if (lane == 0) fail();
             // No bulk copy may land after the CTA ends.
+            if (n_w) mbar_wait(bar_w, (uint32_t)(n_w - 1) & 1u, kWaitNs);
+            if (n_p) mbar_wait(bar_p, (uint32_t)(n_p - 1) & 1u, kWaitNs);
+            if (n_u) mbar_wait(bar_u, (uint32_t)(n_u - 1) & 1u, kWaitNs);
             for (int b = 0; b < 2; ++b)
-                if (issued[b] > 0) mbar_wait(bar_rec + b, (uint32_t)(issued[b] - 1) & 1u, kWaitNs);
-            if (u_issued > 0) mbar_wait(bar_u, (uint32_t)(u_issued - 1) & 1u, kWaitNs);
+                if (n_sc[b]) mbar_wait(bar_sc + b, (uint32_t)(n_sc[b] - 1) & 1u, kWaitNs);
         }
         __syncwarp();
     } else if (warp < 8) {
@@ -577,9 +600,9 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
                                         : make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
-        bool ok = n_chunks > 0 && wait_all(bar_rec, 0);
+        bool ok = n_chunks > 0 && wait_all(bar_sc, 0);
         if (ok) {
-            const float eL = rscal(0)[3 * C];
+            const float eL = scal(0)[3 * C];
             const float *s0 = p.initial_state
                                   ? p.initial_state + ((size_t)seq * p.H_v + hv) * D * D + (size_t)i * D
                                   : nullptr;
@@ -599,30 +622,32 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
         }
         int c = 0;
         for (; c < n_chunks && ok; ++c) {
-            const float *sc = rscal(c);
-            // Dt~^T = (U^T - S W^T) diag(dn) as hi/lo tiles.
+            const float *sc = scal(c);  // landed: it gave this chunk's e^{gamma_L}
+            // Delta^T = U^T - S W^T as hi/lo tiles, and its decayed, k-normalised copy.
             ok = wait_all(bar_gd, (uint32_t)c & 1u) && wait_all(bar_u, (uint32_t)c & 1u);
             if (!ok) break;
             fence_after_sync();
 #pragma unroll
             for (int h16 = 0; h16 < 2; ++h16) {
                 const int s0 = 32 * half + 16 * h16;
-                float v[16];
+                float v[16], w[16];
                 tmem_ld16(tm + lane_off + TM_D + s0, v);
 #pragma unroll
                 for (int s4 = 0; s4 < 4; ++s4) {
                     const float4 u = *reinterpret_cast<const float4 *>(sm + B_U + u_off(s0 + 4 * s4, i));
                     const float4 dn = *reinterpret_cast<const float4 *>(sc + 2 * C + s0 + 4 * s4);
-                    v[4 * s4] = (v[4 * s4] + u.x) * dn.x;
-                    v[4 * s4 + 1] = (v[4 * s4 + 1] + u.y) * dn.y;
-                    v[4 * s4 + 2] = (v[4 * s4 + 2] + u.z) * dn.z;
-                    v[4 * s4 + 3] = (v[4 * s4 + 3] + u.w) * dn.w;
+                    v[4 * s4] += u.x; v[4 * s4 + 1] += u.y; v[4 * s4 + 2] += u.z; v[4 * s4 + 3] += u.w;
+                    w[4 * s4] = v[4 * s4] * dn.x; w[4 * s4 + 1] = v[4 * s4 + 1] * dn.y;
+                    w[4 * s4 + 2] = v[4 * s4 + 2] * dn.z; w[4 * s4 + 3] = v[4 * s4 + 3] * dn.w;
                 }
 #pragma unroll
                 for (int c8 = 0; c8 < 2; ++c8) {
                     uint4 hi, lo;
                     const uint32_t o = kmaj(i, s0 + 8 * c8, D);
                     split8(v + 8 * c8, hi, lo);
+                    *reinterpret_cast<uint4 *>(sm + B_DL + o) = hi;
+                    *reinterpret_cast<uint4 *>(sm + B_DL + 16384 + o) = lo;
+                    split8(w + 8 * c8, hi, lo);
                     *reinterpret_cast<uint4 *>(sm + B_DT + o) = hi;
                     *reinterpret_cast<uint4 *>(sm + B_DT + 16384 + o) = lo;
                 }
@@ -632,10 +657,10 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
             // Once the state update is done: the next chunk's bf16 S and scaled S.
             ok = wait_all(bar_gs, (uint32_t)c & 1u);
             if (!ok || c + 1 == n_chunks) continue;
-            ok = wait_all(bar_rec + ((c + 1) & 1), (uint32_t)((c + 1) >> 1) & 1u);
+            ok = wait_all(bar_sc + ((c + 1) & 1), (uint32_t)((c + 1) >> 1) & 1u);
             if (!ok) continue;
             fence_after_sync();
-            const float eL = rscal(c + 1)[3 * C];
+            const float eL = scal(c + 1)[3 * C];
 #pragma unroll 1
             for (int jj = 0; jj < 2; ++jj) {
                 const int j0 = 64 * half + 32 * jj;
@@ -660,26 +685,33 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
         if (zg && p.norm_w)
             w4 = make_float4(__ldg(p.norm_w + 4 * lane), __ldg(p.norm_w + 4 * lane + 1),
                              __ldg(p.norm_w + 4 * lane + 2), __ldg(p.norm_w + 4 * lane + 3));
+        // z of this warp's 8 tokens of chunk c (4 values per lane), loaded a
+        // whole chunk before it is used.
+        auto load_z = [&](int c, uint2 (&zr)[8]) {
+            const int64_t c0 = t0 + (int64_t)c * C;
+            const int L = c < n_chunks ? chunk_len(c) : 0;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int r = 8 * og + u;
+                zr[u] = r < L ? __ldg(reinterpret_cast<const uint2 *>(zg + (c0 + r) * p.z_stride + hv * D + 4 * lane))
+                              : make_uint2(0u, 0u);
+            }
+        };
+        uint2 zr[8];
+        if (zg) load_z(0, zr);
         bool dead = false;
         for (int c = 0; c < n_chunks && !dead; ++c) {
             const int b = c & 1;
             const int64_t c0 = t0 + (int64_t)c * C;
             const int L = chunk_len(c);
-            // z of this warp's 8 tokens (4 values per lane), loaded before the wait.
-            uint2 zr[8];
-            if (zg) {
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int r = 8 * og + u;
-                    zr[u] = r < L ? __ldg(reinterpret_cast<const uint2 *>(zg + (c0 + r) * p.z_stride + hv * D + 4 * lane))
-                                  : make_uint2(0u, 0u);
-                }
-            }
-            bool ok = mbar_wait(bar_oready + b, (uint32_t)(c >> 1) & 1u, kWaitNs);
+            uint2 zn[8];
+            if (zg) load_z(c + 1, zn);
+            bool ok = mbar_wait(bar_oready + b, (uint32_t)(c >> 1) & 1u, kWaitNs) &&
+                      mbar_wait(bar_sc + b, (uint32_t)(c >> 1) & 1u, kWaitNs);  // (long landed)
             if (ok) {
                 // O^T [i][r] = (m e^gamma)_r (S Q^T) + (P Delta)^T, staged as O [r][i].
                 fence_after_sync();
-                const float *sc = rscal(c);
+                const float *sc = scal(c);
                 const int r0 = 32 * half;
 #pragma unroll
                 for (int h16 = 0; h16 < 2; ++h16) {
@@ -697,7 +729,7 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
                     }
                 }
             }
-            // TMEM buffers and the record's scalars go back to the MMA warp and producer.
+            // TMEM buffers and the chunk's scalars go back to the MMA warp and producer.
             fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_ofree + b);
@@ -745,6 +777,8 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
                 }
                 if (r < L) Elem<TOUT>::store4(out + (c0 + r) * p.out_stride + hv * D + 4 * lane, y);
             }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) zr[u] = zn[u];
             // The stage is rewritten by the next chunk.
             group_sync_or(OG_BAR, OG_N, false);
         }

@@ -162,6 +162,22 @@ def test_tc_long_memory_and_reset():
     _check(inp, out, final, torch.bfloat16)
 
 
+@pytest.mark.parametrize("g_scale", [8.0, 40.0])
+@pytest.mark.parametrize("one_kernel", [False, True])
+def test_tc_strong_decay(g_scale, one_kernel):
+    """g = -softplus(N(0,1)) times 8 or 40: the decay across one chunk spans far
+    more than fp32's exponent range, so no intermediate may rescale a chunk's
+    tokens by e^{+-(gamma_r - gamma_s)} beyond what the recurrence itself applies."""
+    lens = [300, 130]
+    inp = synth.make_inputs(lens, 2, 4, 128, seed=35, dtype=torch.bfloat16, s0_std=0.02)
+    inp.g = (inp.g * g_scale).contiguous()
+    ws = None
+    if one_kernel:
+        ws = torch.empty((16 + 4 * len(lens) + 255) // 256 * 256, dtype=torch.uint8, device="cuda")
+    out, final = run_prefill(inp, chunk=64, workspace=ws)
+    _check(inp, out, final, torch.bfloat16)
+
+
 def test_tc_no_l2norm_and_status_word():
     inp = synth.make_inputs([130, 70], 2, 2, 128, seed=33, dtype=torch.bfloat16, s0_std=0.02)
     inp.q = torch.nn.functional.normalize(inp.q.float(), dim=-1).to(torch.bfloat16)

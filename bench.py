@@ -360,6 +360,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=1024)
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="run only the chunked-prefill measurement and print its JSON (profiling)")
+    ap.add_argument("--prefill-reps", type=int, default=5)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -380,6 +383,13 @@ def main():
 
     from linear_attention_recurrence_10_b200 import build
     build.build(quiet=True)
+    if args.prefill_only:
+        pre = prefill_measure(device, reps=args.prefill_reps, world=world)
+        if rank == 0:
+            print(json.dumps(pre), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
 
     bench = DecodeBench(device, seed=1 + rank, B=args.batch, slots=args.slots)
     bench.capture()
@@ -405,7 +415,8 @@ def main():
                          world)
     e2e_gbs = weak_scaling_rate(bench.bytes_per_step * args.e2e_steps, world, ms_e2e) / 1e9
 
-    prefill = None if args.no_prefill else prefill_measure(device, world=world)
+    prefill = None if args.no_prefill else prefill_measure(device, reps=args.prefill_reps,
+                                                           world=world)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_sample()

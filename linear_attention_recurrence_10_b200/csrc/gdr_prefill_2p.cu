@@ -99,18 +99,25 @@ constexpr int PNT = 256;
 constexpr int PSL = 512 / PNT;      // 16-column slices of a 64-column accumulator per thread
 constexpr uint32_t A_KQ = 0;        // bf16 [K;Q] (32 KB)
 constexpr uint32_t A_V = 32768;     // bf16 V (16 KB)
-constexpr uint32_t A_T = 49152;     // fp32 T [64][65]
-constexpr uint32_t A_AX = 65792;    // fp32 A [64][65] and X; once T is built, TB/TW (32 KB) over them
+constexpr int PLD = 68;             // row stride of the fp32 scratch (16-byte aligned rows)
+constexpr uint32_t A_T = 49152;     // fp32 T [64][PLD]
+constexpr uint32_t A_AX = 66560;    // fp32 A [64][PLD] and X; once T is built, TB/TW (32 KB) over them
 constexpr uint32_t A_TBW = A_AX;
-constexpr uint32_t A_GB = 98560;    // g[64], beta[64]
-constexpr uint32_t A_SCAL = 99072;  // scalars, mbarrier
-constexpr uint32_t A_SMEM = A_SCAL + 2048;
+constexpr uint32_t A_GB = 99328;    // g[64], beta[64]
+constexpr uint32_t A_SCAL = 99840;  // scalars, mbarrier
+constexpr uint32_t A_SMEM = A_SCAL + 3072;
 
 struct PrepScalars {
     float gam[C], eg[C], bet[C], nk[C], nq[C], dec[C];
+    // dtab[R][s] = e^{gamma_{16R} - gamma_s} for s < 16R: with the per-row
+    // e^{gamma_r - gamma_{16R}} it gives e^{gamma_r - gamma_s} below the
+    // diagonal 16-block as a product of two factors that are at most one.
+    float dtab[4 * C];
     uint64_t bar;
     uint32_t tmem;
 };
+static_assert(sizeof(PrepScalars) <= A_SMEM - A_SCAL, "prep scalars overflow");
+static_assert(A_T + C * PLD * 4 <= A_AX && A_AX + 32768 <= A_GB, "prep scratch overlap");
 
 __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p, const int *chunk_off,
                                                      unsigned char *records, int *status) {
@@ -137,7 +144,7 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p, con
     const __nv_bfloat16 *vg = static_cast<const __nv_bfloat16 *>(p.v);
     const uint32_t sbase = smem_u32(sm);
     float *Ascr = reinterpret_cast<float *>(sm + A_AX);
-    float *Xscr = Ascr + C * LDA;
+    float *Xscr = Ascr + C * PLD;
     float *Tscr = reinterpret_cast<float *>(sm + A_T);
     float *gbuf = reinterpret_cast<float *>(sm + A_GB);
 
@@ -213,6 +220,10 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p, con
     }
     __syncthreads();
     if (tid < C) sc.dec[tid] = __expf(sc.gam[L - 1] - sc.gam[tid]);
+    {
+        const int R = tid >> 6, s = tid & 63;  // PNT == 4 * C entries
+        sc.dtab[tid] = s < 16 * R ? __expf(sc.gam[16 * R] - sc.gam[s]) : 0.f;
+    }
 
     uint32_t phase = 0;
     auto issue_and_wait = [&](auto issue) -> bool {
@@ -239,30 +250,40 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p, con
         gemm(tm + TM_D1, kq, 128, 2048, 256, kq, 128, 2048, 256, D / 16, ID_KK, false);
     });
     if (alive) {
-        // A (fp32 scratch) and P (hi/lo bf16 straight into the record).
-        const int rr = 32 * (quad & 1) + lane;
+        // A (fp32 scratch) and P (hi/lo bf16 straight into the record).  The
+        // decay e^{gamma_r - gamma_s}: zero above the diagonal 16-block, a
+        // row factor times a table entry below it, exact on it.
+        const int rr = 32 * (quad & 1) + lane, R = rr >> 4;
         const float gr = sc.gam[rr];
+        const float rowf = R > 0 ? __expf(gr - sc.gam[16 * R]) : 1.f;
 #pragma unroll
         for (int sl = 0; sl < PSL; ++sl) {
-        const int s0 = 16 * (part * PSL + sl);
-        float v[16];
+        const int s0 = 16 * (part * PSL + sl), Sb = s0 >> 4;
+        float v[16], e[16];
         tmem_ld16(tm + lane_off + TM_D1 + s0, v);
+        if (Sb < R) {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) e[c] = rowf * sc.dtab[R * C + s0 + c];
+        } else if (Sb == R) {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) e[c] = __expf(gr - sc.gam[s0 + c]);
+        } else {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) e[c] = 0.f;
+        }
         if (quad < 2) {
             const float f = sc.bet[rr] * sc.nk[rr];
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
                 const int s = s0 + c;
-                Ascr[rr * LDA + s] = s < rr ? f * __expf(gr - sc.gam[s]) * sc.nk[s] * v[c] : 0.f;
+                Ascr[rr * PLD + s] = s < rr ? f * e[c] * sc.nk[s] * v[c] : 0.f;
             }
         } else {
-            // P_rs = nq_r e^{gamma_r - gamma_s} n_s QK_rs (s <= r): every factor is
-            // at most one in size whatever the decay, which a rescaled form
-            // (say P diag(1/dn)) would not be.
             const float f = sc.nq[rr];
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
                 const int s = s0 + c;
-                v[c] = s <= rr ? f * __expf(gr - sc.gam[s]) * sc.nk[s] * v[c] : 0.f;
+                v[c] = s <= rr ? f * e[c] * sc.nk[s] * v[c] : 0.f;
             }
 #pragma unroll
             for (int c8 = 0; c8 < 2; ++c8) {
@@ -274,16 +295,17 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p, con
         }
         }
         __syncthreads();
-        invert_unit_lower<PNT>(Ascr, Tscr, Xscr, tid);
+        invert_unit_lower<PNT, PLD>(Ascr, Tscr, Xscr, tid);
         for (int e = tid; e < C * (C / 8); e += PNT) {
             const int r = e & 63, s8 = 8 * (e >> 6);
-            float tb[8], tw[8];
+            float t[8], tb[8], tw[8];
+            *reinterpret_cast<float4 *>(t) = *reinterpret_cast<const float4 *>(Tscr + r * PLD + s8);
+            *reinterpret_cast<float4 *>(t + 4) = *reinterpret_cast<const float4 *>(Tscr + r * PLD + s8 + 4);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int s = s8 + u;
-                const float t = Tscr[r * LDA + s];
-                tb[u] = t * sc.bet[s];
-                tw[u] = t * sc.bet[s] * sc.eg[s] * sc.nk[s];
+                tb[u] = t[u] * sc.bet[s];
+                tw[u] = t[u] * sc.bet[s] * sc.eg[s] * sc.nk[s];
             }
             uint4 h, l;
             split8(tb, h, l);

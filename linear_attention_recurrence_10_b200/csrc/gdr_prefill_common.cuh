@@ -82,20 +82,34 @@ __device__ __forceinline__ void split8(const float *v, uint4 &hi, uint4 &lo) {
 
 // One distance of the blocked triangular inverse: for every pair of 16-blocks
 // (i, j) with i - j = DIST, X = A[i-rows][16j .. 16i) T[16j .. 16i)[j-cols],
-// then T_ij = -T_ii X.  Fully unrolled so the shared-memory loads overlap.
-template <int DIST, int NT>
+// then T_ij = -T_ii X.  Fully unrolled so the shared-memory loads overlap; with
+// a row stride LD that keeps rows 16-byte aligned, the row operand is read four
+// values at a time.
+template <int DIST, int NT, int LD>
 __device__ __forceinline__ void offdiag_stage(const float *Ascr, float *Tscr, float *Xscr, int tid) {
     constexpr int NBLK = 4 - DIST, NOUT = NBLK * 256;
+    constexpr bool VEC = LD % 4 == 0;
 #pragma unroll
     for (int e0 = 0; e0 < NOUT; e0 += NT) {
         const int e = e0 + tid;
         if (NOUT % NT == 0 || e < NOUT) {
             const int j = e >> 8, i = j + DIST, rr = (e >> 4) & 15, cc = e & 15;
-            const float *arow = Ascr + (16 * i + rr) * LDA + 16 * j;
-            const float *tcol = Tscr + 16 * j * LDA + 16 * j + cc;
+            const float *arow = Ascr + (16 * i + rr) * LD + 16 * j;
+            const float *tcol = Tscr + 16 * j * LD + 16 * j + cc;
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            if constexpr (VEC) {
 #pragma unroll
-            for (int k = 0; k < 16 * DIST; ++k) acc[k & 3] = fmaf(arow[k], tcol[k * LDA], acc[k & 3]);
+                for (int k4 = 0; k4 < 4 * DIST; ++k4) {
+                    const float4 a = *reinterpret_cast<const float4 *>(arow + 4 * k4);
+                    acc[0] = fmaf(a.x, tcol[(4 * k4) * LD], acc[0]);
+                    acc[1] = fmaf(a.y, tcol[(4 * k4 + 1) * LD], acc[1]);
+                    acc[2] = fmaf(a.z, tcol[(4 * k4 + 2) * LD], acc[2]);
+                    acc[3] = fmaf(a.w, tcol[(4 * k4 + 3) * LD], acc[3]);
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < 16 * DIST; ++k) acc[k & 3] = fmaf(arow[k], tcol[k * LD], acc[k & 3]);
+            }
             Xscr[e] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
         }
     }
@@ -105,12 +119,23 @@ __device__ __forceinline__ void offdiag_stage(const float *Ascr, float *Tscr, fl
         const int e = e0 + tid;
         if (NOUT % NT == 0 || e < NOUT) {
             const int j = e >> 8, i = j + DIST, rr = (e >> 4) & 15, cc = e & 15;
-            const float *trow = Tscr + (16 * i + rr) * LDA + 16 * i;
+            const float *trow = Tscr + (16 * i + rr) * LD + 16 * i;
             const float *xcol = Xscr + (j << 8) + cc;
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            if constexpr (VEC) {
 #pragma unroll
-            for (int k = 0; k < 16; ++k) acc[k & 3] = fmaf(trow[k], xcol[k * 16], acc[k & 3]);
-            Tscr[(16 * i + rr) * LDA + 16 * j + cc] = -((acc[0] + acc[1]) + (acc[2] + acc[3]));
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    const float4 t = *reinterpret_cast<const float4 *>(trow + 4 * k4);
+                    acc[0] = fmaf(t.x, xcol[(4 * k4) * 16], acc[0]);
+                    acc[1] = fmaf(t.y, xcol[(4 * k4 + 1) * 16], acc[1]);
+                    acc[2] = fmaf(t.z, xcol[(4 * k4 + 2) * 16], acc[2]);
+                    acc[3] = fmaf(t.w, xcol[(4 * k4 + 3) * 16], acc[3]);
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < 16; ++k) acc[k & 3] = fmaf(trow[k], xcol[k * 16], acc[k & 3]);
+            }
+            Tscr[(16 * i + rr) * LD + 16 * j + cc] = -((acc[0] + acc[1]) + (acc[2] + acc[3]));
         }
     }
     __syncthreads();
@@ -118,12 +143,12 @@ __device__ __forceinline__ void offdiag_stage(const float *Ascr, float *Tscr, fl
 
 
 // T = (I + A)^{-1} for the strictly lower-triangular 64 x 64 A in Ascr (fp32,
-// row stride LDA), blocked by 16.  Diagonal blocks first, one column per
+// row stride LD), blocked by 16.  Diagonal blocks first, one column per
 // thread, right-looking (each finished x_s is folded into all later rows at
 // once, so the dependent chain is 16 steps); then the off-diagonal blocks by
 // distance from the diagonal: T_ij = -T_ii sum_{16j <= k < 16i} A[i-rows][k] T[k][j-cols].
 // Every thread of the block calls it; it ends with the block synchronised.
-template <int NT>
+template <int NT, int LD = LDA>
 __device__ __forceinline__ void invert_unit_lower(const float *Ascr, float *Tscr, float *Xscr, int tid) {
     if (tid < C) {
         const int b = tid >> 4, c = tid & 15, base = 16 * b;
@@ -133,20 +158,20 @@ __device__ __forceinline__ void invert_unit_lower(const float *Ascr, float *Tscr
 #pragma unroll
         for (int s = 0; s < 15; ++s) {
 #pragma unroll
-            for (int r = s + 1; r < 16; ++r) x[r] = fmaf(-Ascr[(base + r) * LDA + base + s], x[s], x[r]);
+            for (int r = s + 1; r < 16; ++r) x[r] = fmaf(-Ascr[(base + r) * LD + base + s], x[s], x[r]);
         }
 #pragma unroll
-        for (int r = 0; r < 16; ++r) Tscr[(base + r) * LDA + base + c] = x[r];
+        for (int r = 0; r < 16; ++r) Tscr[(base + r) * LD + base + c] = x[r];
     } else {
         for (int e = tid - C; e < C * C; e += NT - C) {  // zero the blocks above the diagonal
             const int r = e >> 6, s = e & 63;
-            if ((s >> 4) > (r >> 4)) Tscr[r * LDA + s] = 0.f;
+            if ((s >> 4) > (r >> 4)) Tscr[r * LD + s] = 0.f;
         }
     }
     __syncthreads();
-    offdiag_stage<1, NT>(Ascr, Tscr, Xscr, tid);
-    offdiag_stage<2, NT>(Ascr, Tscr, Xscr, tid);
-    offdiag_stage<3, NT>(Ascr, Tscr, Xscr, tid);
+    offdiag_stage<1, NT, LD>(Ascr, Tscr, Xscr, tid);
+    offdiag_stage<2, NT, LD>(Ascr, Tscr, Xscr, tid);
+    offdiag_stage<3, NT, LD>(Ascr, Tscr, Xscr, tid);
 }
 
 }  // namespace tcp

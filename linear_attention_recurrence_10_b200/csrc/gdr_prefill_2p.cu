@@ -119,8 +119,10 @@ struct PrepScalars {
 static_assert(sizeof(PrepScalars) <= A_SMEM - A_SCAL, "prep scalars overflow");
 static_assert(A_T + C * PLD * 4 <= A_AX && A_AX + 32768 <= A_GB, "prep scratch overlap");
 
+// `succ`: block index distance to the unit that most likely takes this block's
+// SM slot next (resident blocks per SM x SMs); its inputs are prefetched to L2.
 __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p, const int *chunk_off,
-                                                     unsigned char *records, int *status) {
+                                                     unsigned char *records, int *status, int succ) {
     extern __shared__ __align__(1024) unsigned char sm[];
     PrepScalars &sc = *reinterpret_cast<PrepScalars *>(sm + A_SCAL);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -176,6 +178,27 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p, con
         cp_async4(gbuf + tid, (tid < C ? p.g : p.beta) + t * p.gb_stride + hv, in ? 4u : 0u);
     }
     cp_async_commit();
+    if (blockIdx.x + succ < gridDim.x) {
+        // Warm L2 for the unit most likely to take this block's SM slot next:
+        // 64 rows x (k, q, v) x two 128-byte lines over the block's threads.
+        const int nb = blockIdx.x + succ, gch = nb / p.H_v, hv2 = nb % p.H_v, hk2 = hv2 / p.hv_per_hk;
+        int a = 0, b = p.n_seq - 1;
+        while (a < b) {
+            const int mid = (a + b + 1) >> 1;
+            if (chunk_off[mid] <= gch) a = mid; else b = mid - 1;
+        }
+        const int64_t n0 = p.cu_seqlens[a] + (int64_t)(gch - chunk_off[a]) * C, n1 = p.cu_seqlens[a + 1];
+        for (int e = tid; e < 3 * 2 * C; e += PNT) {
+            const int r = (e >> 1) & 63, line = e & 1, which = e >> 7;
+            const int64_t t = n0 + r;
+            if (t < n1) {
+                const __nv_bfloat16 *ptr = which == 0 ? kg + t * p.k_stride + hk2 * D
+                                          : which == 1 ? qg + t * p.q_stride + hk2 * D
+                                                       : vg + t * p.v_stride + hv2 * D;
+                prefetch_l2(ptr + 64 * line);
+            }
+        }
+    }
     cp_async_wait<0>();
     fence_before_sync();
     __syncthreads();
@@ -855,8 +878,12 @@ cudaError_t launch_prefill_tc2p(const PrefillParams &p, int64_t n_chunks, void *
         e = cudaFuncSetAttribute(tcp2::prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)tcp2::A_SMEM);
         if (e != cudaSuccess) return e;
-        tcp2::prep_kernel<<<(unsigned)(n_chunks * p.H_v), tcp2::PNT, tcp2::A_SMEM, s>>>(p, chunk_off,
-                                                                                     records, status);
+        int dev = 0, n_sm = 148;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return cudaGetLastError();
+        tcp2::prep_kernel<<<(unsigned)(n_chunks * p.H_v), tcp2::PNT, tcp2::A_SMEM, s>>>(
+            p, chunk_off, records, status, 2 * n_sm);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

@@ -240,6 +240,11 @@ __device__ __forceinline__ void bulk_copy(void *smem_dst, const void *gmem_src, 
         : "memory");
 }
 
+// Ask L2 to fetch the 128-byte line holding `p` (no result, nothing to wait for).
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // Start moving `bytes` (a multiple of 16, 16-byte aligned) of global memory
 // into L2; nothing is written anywhere and nothing needs to be waited for.
 __device__ __forceinline__ void bulk_prefetch_l2(const void *gmem_src, uint32_t bytes) {

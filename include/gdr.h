@@ -127,6 +127,47 @@ typedef struct gdr_decode_args {
 gdr_status gdr_decode_step(const gdr_decode_args *args, gdr_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Several decode tokens per sequence in one call, with optional state slots.
+ *
+ * The same recurrence as gdr_decode_step, applied to n_tokens consecutive
+ * tokens of every sequence; the Swiftlet post checks that advancing token by
+ * token matches processing the tokens together ("Correctness & Validation").
+ * The state is read once and written once per call, whatever n_tokens, which
+ * is the whole point: per token it costs 1/n_tokens of a single step's state
+ * traffic.  State slots let a server keep sequences' states in a pool and
+ * advance any subset of them (the caller owns the state across the generation
+ * loop: Core ML card for Qwen3.5-0.8B, "Usage").
+ *
+ *   base       as for gdr_decode_step, except that every token-indexed tensor
+ *              (q, k, v, z, g, beta, out) holds base.batch * n_tokens rows:
+ *              row b * n_tokens + t is token t of sequence b (same row strides).
+ *              base.batch is the number of sequences.
+ *   n_tokens   1 .. GDR_DECODE_MAX_TOKENS tokens per sequence, applied in order.
+ *   state_slot NULL: sequence b uses state row b, as in gdr_decode_step.
+ *              Otherwise a device array of base.batch int32: sequence b reads
+ *              and writes state row state_slot[b] of state_in / state_out (row
+ *              stride base.state_stride).  Slots must be distinct within a call.
+ *   n_slots    with state_slot: the number of state rows the buffers hold
+ *              (>= 1).  A slot outside [0, n_slots) leaves that sequence's state
+ *              and outputs untouched and, if `status` is given, sets *status to
+ *              GDR_ERR_INVALID_ARG on the device; other sequences proceed.
+ *   status     optional device int32, written only on such an error.
+ * With state_slot the slot table is read after the preceding kernel on the
+ * stream has finished, so it may be produced by that kernel.
+ * ------------------------------------------------------------------------ */
+#define GDR_DECODE_MAX_TOKENS 8
+
+typedef struct gdr_decode_multi_args {
+    gdr_decode_args base;
+    int32_t n_tokens;
+    int32_t n_slots;
+    const int32_t *state_slot;
+    int32_t *status;
+} gdr_decode_multi_args;
+
+gdr_status gdr_decode_multi(const gdr_decode_multi_args *args, gdr_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Chunked prefill over packed variable-length sequences.
  *
  * The pages' Core ML build pairs a prefill model with the decode model

@@ -19,7 +19,7 @@ import torch
 from . import _abi
 from ._abi import GDR_BF16, GDR_F32
 
-__all__ = ["GdrError", "decode_step", "prefill_chunked", "prefill_chunked_noalloc",
+__all__ = ["GdrError", "decode_step", "decode_multi", "prefill_chunked", "prefill_chunked_noalloc",
            "prefill_workspace_size",
            "rmsnorm_gated", "version", "status_string"]
 
@@ -79,20 +79,9 @@ def status_string(status: int) -> str:
     return _abi.lib().gdr_status_string(int(status)).decode()
 
 
-def decode_step(q, k, v, g, beta, state, out, *, z=None, norm_w=None, state_out=None,
-                scale: float = 1.0, eps_l2: float = 1e-6, eps_norm: float = 1e-6,
-                qk_l2norm: bool = True, overlap_state_load: bool = False,
-                stream=None) -> torch.Tensor:
-    """Advance every sequence of the batch by one token (gdr_decode_step).
-
-    q, k [B, H_k, d]; v, z [B, H_v, d] (bf16 or fp32, same dtype); g, beta
-    [B, H_v] fp32; state [B, H_v, d, d] fp32, updated in place unless
-    ``state_out`` is given; out [B, H_v, d] bf16 or fp32.  Batch rows may be
-    strided views (e.g. one step of a [B, T, H, d] tensor).
-    ``overlap_state_load``: GDR_DECODE_OVERLAP_STATE_LOAD -- only when the
-    kernel queued just before this call does not write this state.
-    """
-    B, H_k, d = q.shape
+def _decode_args(q, k, v, g, beta, state, out, z, norm_w, state_out, scale, eps_l2, eps_norm,
+                 qk_l2norm, overlap_state_load, batch):
+    H_k, d = q.shape[1], q.shape[2]
     H_v = v.shape[1]
     for t, name in ((g, "g"), (beta, "beta"), (state, "state"), (norm_w, "norm_w")):
         _f32_tensor(t, name)
@@ -102,7 +91,7 @@ def decode_step(q, k, v, g, beta, state, out, *, z=None, norm_w=None, state_out=
     if state.stride() != so.stride():
         raise ValueError("state and state_out must share one layout")
     a = _abi.DecodeArgs()
-    a.batch, a.H_k, a.H_v, a.d_k, a.d_v = B, H_k, H_v, d, v.shape[2]
+    a.batch, a.H_k, a.H_v, a.d_k, a.d_v = batch, H_k, H_v, d, v.shape[2]
     a.in_dtype = _dtype_code(q, "q")
     for t, name in ((k, "k"), (v, "v"), (z, "z")):
         if t is not None and _dtype_code(t, name) != a.in_dtype:
@@ -121,8 +110,60 @@ def decode_step(q, k, v, g, beta, state, out, *, z=None, norm_w=None, state_out=
     a.g, a.beta = _ptr(g), _ptr(beta)
     a.state_in, a.state_out = _ptr(state), _ptr(so)
     a.norm_w, a.out = _ptr(norm_w), _ptr(out)
+    return a
+
+
+def decode_step(q, k, v, g, beta, state, out, *, z=None, norm_w=None, state_out=None,
+                scale: float = 1.0, eps_l2: float = 1e-6, eps_norm: float = 1e-6,
+                qk_l2norm: bool = True, overlap_state_load: bool = False,
+                stream=None) -> torch.Tensor:
+    """Advance every sequence of the batch by one token (gdr_decode_step).
+
+    q, k [B, H_k, d]; v, z [B, H_v, d] (bf16 or fp32, same dtype); g, beta
+    [B, H_v] fp32; state [B, H_v, d, d] fp32, updated in place unless
+    ``state_out`` is given; out [B, H_v, d] bf16 or fp32.  Batch rows may be
+    strided views (e.g. one step of a [B, T, H, d] tensor).
+    ``overlap_state_load``: GDR_DECODE_OVERLAP_STATE_LOAD -- only when the
+    kernel queued just before this call does not write this state.
+    """
+    a = _decode_args(q, k, v, g, beta, state, out, z, norm_w, state_out, scale, eps_l2, eps_norm,
+                     qk_l2norm, overlap_state_load, q.shape[0])
     _check(_abi.lib().gdr_decode_step(ctypes.byref(a), _stream(stream, q.device)),
            "gdr_decode_step")
+    return out
+
+
+def decode_multi(q, k, v, g, beta, state, out, *, n_tokens: int, z=None, norm_w=None,
+                 state_out=None, slots=None, status=None, scale: float = 1.0,
+                 eps_l2: float = 1e-6, eps_norm: float = 1e-6, qk_l2norm: bool = True,
+                 overlap_state_load: bool = False, stream=None) -> torch.Tensor:
+    """Advance every sequence by ``n_tokens`` tokens in one call (gdr_decode_multi).
+
+    Token-indexed tensors hold B * n_tokens rows, row b * n_tokens + t being
+    token t of sequence b: q, k [B*T, H_k, d]; v, z [B*T, H_v, d]; g, beta
+    [B*T, H_v]; out [B*T, H_v, d].  ``slots`` (int32 [B] on the device, or
+    None) maps sequence b to its row of ``state`` [n_rows, H_v, d, d];
+    ``status`` (int32 [1] on the device) receives GDR_ERR_INVALID_ARG if a
+    slot is out of range.
+    """
+    rows = q.shape[0]
+    if n_tokens < 1 or rows % n_tokens != 0:
+        raise ValueError("q must hold batch * n_tokens rows")
+    batch = rows // n_tokens
+    a = _decode_args(q, k, v, g, beta, state, out, z, norm_w, state_out, scale, eps_l2, eps_norm,
+                     qk_l2norm, overlap_state_load, batch)
+    m = _abi.DecodeMultiArgs()
+    m.base = a
+    m.n_tokens = int(n_tokens)
+    m.n_slots = 0
+    if slots is not None:
+        if slots.dtype != torch.int32 or slots.dim() != 1 or slots.shape[0] != batch:
+            raise ValueError("slots must be an int32 tensor of one entry per sequence")
+        m.n_slots = state.shape[0]
+    m.state_slot = _ptr(slots)
+    m.status = _ptr(status)
+    _check(_abi.lib().gdr_decode_multi(ctypes.byref(m), _stream(stream, q.device)),
+           "gdr_decode_multi")
     return out
 
 

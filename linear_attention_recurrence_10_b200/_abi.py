@@ -41,6 +41,13 @@ class DecodeArgs(ctypes.Structure):
     ]
 
 
+class DecodeMultiArgs(ctypes.Structure):
+    _fields_ = [
+        ("base", DecodeArgs), ("n_tokens", _i32), ("n_slots", _i32),
+        ("state_slot", _vp), ("status", _vp),
+    ]
+
+
 class PrefillArgs(ctypes.Structure):
     _fields_ = [
         ("n_seq", _i32), ("H_k", _i32), ("H_v", _i32), ("d_k", _i32), ("d_v", _i32),

@@ -9,6 +9,8 @@
 
 namespace gdr {
 cudaError_t launch_decode(const DecodeParams &p, int d, int in_bf16, int out_bf16, cudaStream_t s);
+cudaError_t launch_decode_multi(const DecodeParams &p, int d, int in_bf16, int out_bf16,
+                                cudaStream_t s);
 cudaError_t launch_rmsnorm_gated(const NormParams &p, int d, int o_bf16, int z_bf16, int y_bf16,
                                  cudaStream_t s);
 cudaError_t launch_prefill_simt(const PrefillParams &p, int d, int chunk, int in_bf16,
@@ -84,8 +86,9 @@ const char *gdr_status_string(gdr_status s) {
 
 int gdr_version(void) { return 100; }
 
-gdr_status gdr_decode_step(const gdr_decode_args *a, gdr_stream_t stream) {
-    if (!a) return GDR_ERR_INVALID_ARG;
+// Shared validation of the decode arguments.  `slots` is the number of state
+// rows the state buffers hold (batch for the one-token step).
+static gdr_status decode_params(const gdr_decode_args *a, int64_t slots, DecodeParams *out) {
     if (a->batch < 0 || (a->flags & ~GDR_DECODE_OVERLAP_STATE_LOAD) != 0)
         return GDR_ERR_INVALID_ARG;
     if (!dtype_ok(a->in_dtype) || !dtype_ok(a->out_dtype)) return GDR_ERR_INVALID_ARG;
@@ -95,7 +98,7 @@ gdr_status gdr_decode_step(const gdr_decode_args *a, gdr_stream_t stream) {
         return GDR_ERR_INVALID_ARG;
     const int d = a->d_k;
     const size_t ein = dtype_bytes(a->in_dtype), eout = dtype_bytes(a->out_dtype);
-    DecodeParams p;
+    DecodeParams &p = *out;
     memset(&p, 0, sizeof(p));
     GDR_TRY(resolve_stride(a->q_stride, (int64_t)a->H_k * d, ein, &p.q_stride));
     GDR_TRY(resolve_stride(a->k_stride, (int64_t)a->H_k * d, ein, &p.k_stride));
@@ -112,7 +115,7 @@ gdr_status gdr_decode_step(const gdr_decode_args *a, gdr_stream_t stream) {
         return GDR_ERR_MISALIGNED;
     if ((int64_t)a->batch * a->H_v > 0x7fffffffLL) return GDR_ERR_UNSUPPORTED;
     if (a->state_in != a->state_out) {
-        const size_t span = ((size_t)(a->batch - 1) * p.state_stride + (size_t)a->H_v * d * d) * 4;
+        const size_t span = ((size_t)(slots - 1) * p.state_stride + (size_t)a->H_v * d * d) * 4;
         if (ranges_overlap(a->state_in, span, a->state_out, span)) return GDR_ERR_INVALID_ARG;
     }
     p.batch = a->batch;
@@ -128,8 +131,36 @@ gdr_status gdr_decode_step(const gdr_decode_args *a, gdr_stream_t stream) {
     p.g = a->g; p.beta = a->beta;
     p.state_in = a->state_in; p.state_out = a->state_out;
     p.norm_w = a->norm_w; p.out = a->out;
-    return from_cuda(gdr::launch_decode(p, d, a->in_dtype == GDR_BF16, a->out_dtype == GDR_BF16,
-                                        (cudaStream_t)stream));
+    p.n_tokens = 1;
+    return GDR_OK;
+}
+
+gdr_status gdr_decode_step(const gdr_decode_args *a, gdr_stream_t stream) {
+    if (!a) return GDR_ERR_INVALID_ARG;
+    DecodeParams p;
+    GDR_TRY(decode_params(a, a->batch, &p));
+    if (a->batch == 0) return GDR_OK;
+    return from_cuda(gdr::launch_decode(p, a->d_k, a->in_dtype == GDR_BF16,
+                                        a->out_dtype == GDR_BF16, (cudaStream_t)stream));
+}
+
+gdr_status gdr_decode_multi(const gdr_decode_multi_args *m, gdr_stream_t stream) {
+    if (!m) return GDR_ERR_INVALID_ARG;
+    const gdr_decode_args *a = &m->base;
+    if (m->n_tokens < 1 || m->n_tokens > GDR_DECODE_MAX_TOKENS) return GDR_ERR_INVALID_ARG;
+    if (m->state_slot && m->n_slots < 1) return GDR_ERR_INVALID_ARG;
+    if ((m->state_slot && !aligned4(m->state_slot)) || (m->status && !aligned4(m->status)))
+        return GDR_ERR_MISALIGNED;
+    if ((int64_t)a->batch * m->n_tokens > 0x7fffffffLL) return GDR_ERR_UNSUPPORTED;
+    DecodeParams p;
+    GDR_TRY(decode_params(a, m->state_slot ? m->n_slots : a->batch, &p));
+    if (a->batch == 0) return GDR_OK;
+    p.n_tokens = m->n_tokens;
+    p.n_slots = m->state_slot ? m->n_slots : a->batch;
+    p.slot = m->state_slot;
+    p.status = m->status;
+    return from_cuda(gdr::launch_decode_multi(p, a->d_k, a->in_dtype == GDR_BF16,
+                                              a->out_dtype == GDR_BF16, (cudaStream_t)stream));
 }
 
 gdr_status gdr_rmsnorm_gated(const gdr_norm_args *a, gdr_stream_t stream) {

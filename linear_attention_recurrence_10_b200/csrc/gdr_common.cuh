@@ -25,6 +25,11 @@ struct DecodeParams {
     float *state_out;
     const float *norm_w;
     void *out;
+    // Several tokens per sequence (rows b * n_tokens + t of every token-indexed
+    // tensor) and optional state slots; unused by the one-token kernel.
+    int n_tokens, n_slots;
+    const int *slot;
+    int *status;
 };
 
 struct NormParams {

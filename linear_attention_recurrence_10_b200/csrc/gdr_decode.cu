@@ -27,7 +27,10 @@
 
 namespace gdr {
 
-template <int D, typename TIN, typename TOUT>
+// MULTI: p.n_tokens tokens per sequence in order, the state held in registers
+// between them (read once, written once), and optional state slots.  The
+// one-token instantiation (MULTI = false) is the plain decode step.
+template <int D, typename TIN, typename TOUT, bool MULTI>
 __global__ void __launch_bounds__(2 * D) decode_kernel(const DecodeParams p) {
     constexpr int NW = 2 * D / 32;  // warps; each owns 16 state rows
     constexpr int LPR = D / 4;      // lanes per state row (one float4 each)
@@ -42,10 +45,22 @@ __global__ void __launch_bounds__(2 * D) decode_kernel(const DecodeParams p) {
     const int hk = hv / p.hv_per_hk;
     const int col = 4 * gl;
     const int row0 = warp * 16 + rg;  // row of slot s is row0 + s * RPP
+    const int T = MULTI ? p.n_tokens : 1;
 
+    // The state this sequence owns: its own batch row, or its slot.  A slot
+    // table may be written by the preceding kernel, so it is read after it.
+    int sb = b;
+    if (MULTI && p.slot) {
+        wait_for_predecessor();
+        sb = p.slot[b];
+        if (sb < 0 || sb >= p.n_slots) {
+            if (threadIdx.x == 0 && p.status) atomicExch(p.status, 1);  // GDR_ERR_INVALID_ARG
+            return;
+        }
+    }
     const size_t head_off = (size_t)hv * D * D;
-    const float *sin = p.state_in + (size_t)b * p.state_stride + head_off;
-    float *sout = p.state_out + (size_t)b * p.state_stride + head_off;
+    const float *sin = p.state_in + (size_t)sb * p.state_stride + head_off;
+    float *sout = p.state_out + (size_t)sb * p.state_stride + head_off;
 
     // Issue every state load first so the whole tile is in flight at once.  With
     // overlap_state_load the caller guarantees that the kernel before this one
@@ -57,92 +72,98 @@ __global__ void __launch_bounds__(2 * D) decode_kernel(const DecodeParams p) {
     if (p.overlap_state_load) wait_for_predecessor();
     release_dependents();
 
-    const TIN *qp = static_cast<const TIN *>(p.q) + (size_t)b * p.q_stride + hk * D;
-    const TIN *kp = static_cast<const TIN *>(p.k) + (size_t)b * p.k_stride + hk * D;
-    float4 q4 = Elem<TIN>::load4(qp + col);
-    float4 k4 = Elem<TIN>::load4(kp + col);
-    const float g = __ldg(p.g + (size_t)b * p.gb_stride + hv);
-    const float beta = __ldg(p.beta + (size_t)b * p.gb_stride + hv);
-
     // Row this lane finishes: lanes gl < NS need v of it, lanes gl >= NS need z.
     const bool is_a = gl < NS;
     const int my_row = row0 + (gl % NS) * RPP;
-    float vz = 0.f;
-    if (is_a) {
-        vz = Elem<TIN>::load1(static_cast<const TIN *>(p.v) + (size_t)b * p.v_stride + hv * D +
-                              my_row);
-    } else if (p.z) {
-        vz = Elem<TIN>::load1(static_cast<const TIN *>(p.z) + (size_t)b * p.z_stride + hv * D +
-                              my_row);
-    }
+    __shared__ float red[2][NW];
 
-    float qs = p.scale, ks = 1.f;
-    if (p.qk_l2norm) {
-        const float qq = group_sum<LPR>(dot4(q4, q4));
-        const float kk = group_sum<LPR>(dot4(k4, k4));
-        qs *= rsqrtf(qq + p.eps_l2);
-        ks = rsqrtf(kk + p.eps_l2);
-    }
-    q4 = scale4(q4, qs);
-    k4 = scale4(k4, ks);
-    const float kq = group_sum<LPR>(dot4(k4, q4));
-    const float alpha = expf(g);
+    for (int t = 0; t < T; ++t) {
+        const int64_t r = (int64_t)b * T + t;  // token row
+        const TIN *qp = static_cast<const TIN *>(p.q) + r * p.q_stride + hk * D;
+        const TIN *kp = static_cast<const TIN *>(p.k) + r * p.k_stride + hk * D;
+        float4 q4 = Elem<TIN>::load4(qp + col);
+        float4 k4 = Elem<TIN>::load4(kp + col);
+        const float g = __ldg(p.g + r * p.gb_stride + hv);
+        const float beta = __ldg(p.beta + r * p.gb_stride + hv);
+        float vz = 0.f;
+        if (is_a) {
+            vz = Elem<TIN>::load1(static_cast<const TIN *>(p.v) + r * p.v_stride + hv * D + my_row);
+        } else if (p.z) {
+            vz = Elem<TIN>::load1(static_cast<const TIN *>(p.z) + r * p.z_stride + hv * D + my_row);
+        }
 
-    // Partial S k and S q over this lane's 4 columns, for each held row.
-    float x[LPR];
+        float qs = p.scale, ks = 1.f;
+        if (p.qk_l2norm) {
+            const float qq = group_sum<LPR>(dot4(q4, q4));
+            const float kk = group_sum<LPR>(dot4(k4, k4));
+            qs *= rsqrtf(qq + p.eps_l2);
+            ks = rsqrtf(kk + p.eps_l2);
+        }
+        q4 = scale4(q4, qs);
+        k4 = scale4(k4, ks);
+        const float kq = group_sum<LPR>(dot4(k4, q4));
+        const float alpha = expf(g);
+
+        // Partial S k and S q over this lane's 4 columns, for each held row.
+        float x[LPR];
 #pragma unroll
-    for (int s = 0; s < NS; ++s) {
-        x[s] = dot4(S[s], k4);
-        x[NS + s] = dot4(S[s], q4);
-    }
-    // Reduce-scatter: at offset o a lane keeps the half of its 2o values picked
-    // by bit o of gl and adds the partner's copy of that half.
+        for (int s = 0; s < NS; ++s) {
+            x[s] = dot4(S[s], k4);
+            x[NS + s] = dot4(S[s], q4);
+        }
+        // Reduce-scatter: at offset o a lane keeps the half of its 2o values picked
+        // by bit o of gl and adds the partner's copy of that half.
 #pragma unroll
-    for (int o = LPR / 2; o >= 1; o >>= 1) {
-        const bool up = (gl & o) != 0;
+        for (int o = LPR / 2; o >= 1; o >>= 1) {
+            const bool up = (gl & o) != 0;
 #pragma unroll
-        for (int j = 0; j < o; ++j) {
-            const float send = up ? x[j] : x[j + o];
-            const float keep = up ? x[j + o] : x[j];
-            x[j] = keep + __shfl_xor_sync(kFullMask, send, o);
+            for (int j = 0; j < o; ++j) {
+                const float send = up ? x[j] : x[j + o];
+                const float keep = up ? x[j + o] : x[j];
+                x[j] = keep + __shfl_xor_sync(kFullMask, send, o);
+            }
+        }
+        // x[0]: a = (S k)_row on lanes gl < NS, c = (S q)_row on lanes gl >= NS.
+        const float delta = beta * (vz - alpha * x[0]);                      // valid where is_a
+        const float delta_c = __shfl_xor_sync(kFullMask, delta, NS);         // row's delta on c-lanes
+        const float o_val = fmaf(alpha, x[0], delta_c * kq);                 // valid where !is_a
+
+#pragma unroll
+        for (int s = 0; s < NS; ++s) {
+            const float d = __shfl_sync(kFullMask, delta, rg * LPR + s);
+            S[s] = axpby4(S[s], alpha, k4, d);
+            if (!MULTI) st_state4(sout + (size_t)(row0 + s * RPP) * D + col, S[s]);
+        }
+
+        TOUT *op = static_cast<TOUT *>(p.out) + r * p.out_stride + hv * D;
+        if (p.z == nullptr) {
+            if (!is_a) Elem<TOUT>::store1(op + my_row, o_val);
+        } else {
+            // Partials double-buffered by token, so one barrier per token suffices.
+            float ss = is_a ? 0.f : o_val * o_val;
+            ss = group_sum<32>(ss);
+            if (lane == 0) red[t & 1][warp] = ss;
+            __syncthreads();
+            float tot = 0.f;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) tot += red[t & 1][w];
+            if (!is_a) {
+                const float rstd = rsqrtf(tot * (1.0f / D) + p.eps_norm);
+                const float wv = p.norm_w ? __ldg(p.norm_w + my_row) : 1.0f;
+                Elem<TOUT>::store1(op + my_row, o_val * rstd * wv * silu(vz));
+            }
         }
     }
-    // x[0]: a = (S k)_row on lanes gl < NS, c = (S q)_row on lanes gl >= NS.
-    const float delta = beta * (vz - alpha * x[0]);                      // valid where is_a
-    const float delta_c = __shfl_xor_sync(kFullMask, delta, NS);         // row's delta on c-lanes
-    const float o_val = fmaf(alpha, x[0], delta_c * kq);                 // valid where !is_a
-
+    if (MULTI) {
 #pragma unroll
-    for (int s = 0; s < NS; ++s) {
-        const float d = __shfl_sync(kFullMask, delta, rg * LPR + s);
-        S[s] = axpby4(S[s], alpha, k4, d);
-        st_state4(sout + (size_t)(row0 + s * RPP) * D + col, S[s]);
-    }
-
-    TOUT *op = static_cast<TOUT *>(p.out) + (size_t)b * p.out_stride + hv * D;
-    if (p.z == nullptr) {
-        if (!is_a) Elem<TOUT>::store1(op + my_row, o_val);
-        return;
-    }
-    __shared__ float red[NW];
-    float ss = is_a ? 0.f : o_val * o_val;
-    ss = group_sum<32>(ss);
-    if (lane == 0) red[warp] = ss;
-    __syncthreads();
-    float tot = 0.f;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) tot += red[w];
-    if (!is_a) {
-        const float rstd = rsqrtf(tot * (1.0f / D) + p.eps_norm);
-        const float wv = p.norm_w ? __ldg(p.norm_w + my_row) : 1.0f;
-        Elem<TOUT>::store1(op + my_row, o_val * rstd * wv * silu(vz));
+        for (int s = 0; s < NS; ++s) st_state4(sout + (size_t)(row0 + s * RPP) * D + col, S[s]);
     }
 }
 
 // Launched as a programmatic dependent of the previous kernel on the stream:
 // its blocks may be scheduled while that kernel drains, and wait in
 // wait_for_predecessor() before touching anything it may have written.
-template <int D, typename TIN, typename TOUT>
+template <int D, typename TIN, typename TOUT, bool MULTI>
 static cudaError_t launch_decode_t(const DecodeParams &p, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((int64_t)p.batch * p.H_v));
@@ -154,7 +175,7 @@ static cudaError_t launch_decode_t(const DecodeParams &p, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<D, TIN, TOUT>, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<D, TIN, TOUT, MULTI>, p);
     if (e != cudaSuccess) {
         (void)cudaGetLastError();
         return e;
@@ -162,26 +183,37 @@ static cudaError_t launch_decode_t(const DecodeParams &p, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
-template <int D>
+template <int D, bool MULTI>
 static cudaError_t launch_decode_d(const DecodeParams &p, int in_bf16, int out_bf16,
                                    cudaStream_t s) {
     if (in_bf16) {
-        return out_bf16 ? launch_decode_t<D, __nv_bfloat16, __nv_bfloat16>(p, s)
-                        : launch_decode_t<D, __nv_bfloat16, float>(p, s);
+        return out_bf16 ? launch_decode_t<D, __nv_bfloat16, __nv_bfloat16, MULTI>(p, s)
+                        : launch_decode_t<D, __nv_bfloat16, float, MULTI>(p, s);
     }
-    return out_bf16 ? launch_decode_t<D, float, __nv_bfloat16>(p, s)
-                    : launch_decode_t<D, float, float>(p, s);
+    return out_bf16 ? launch_decode_t<D, float, __nv_bfloat16, MULTI>(p, s)
+                    : launch_decode_t<D, float, float, MULTI>(p, s);
+}
+
+template <bool MULTI>
+static cudaError_t launch_decode_m(const DecodeParams &p, int d, int in_bf16, int out_bf16,
+                                   cudaStream_t s) {
+    switch (d) {
+        case 16: return launch_decode_d<16, MULTI>(p, in_bf16, out_bf16, s);
+        case 32: return launch_decode_d<32, MULTI>(p, in_bf16, out_bf16, s);
+        case 64: return launch_decode_d<64, MULTI>(p, in_bf16, out_bf16, s);
+        case 128: return launch_decode_d<128, MULTI>(p, in_bf16, out_bf16, s);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 cudaError_t launch_decode(const DecodeParams &p, int d, int in_bf16, int out_bf16,
                           cudaStream_t s) {
-    switch (d) {
-        case 16: return launch_decode_d<16>(p, in_bf16, out_bf16, s);
-        case 32: return launch_decode_d<32>(p, in_bf16, out_bf16, s);
-        case 64: return launch_decode_d<64>(p, in_bf16, out_bf16, s);
-        case 128: return launch_decode_d<128>(p, in_bf16, out_bf16, s);
-        default: return cudaErrorInvalidValue;
-    }
+    return launch_decode_m<false>(p, d, in_bf16, out_bf16, s);
+}
+
+cudaError_t launch_decode_multi(const DecodeParams &p, int d, int in_bf16, int out_bf16,
+                                cudaStream_t s) {
+    return launch_decode_m<true>(p, d, in_bf16, out_bf16, s);
 }
 
 }  // namespace gdr

@@ -98,6 +98,50 @@ def test_decode_empty_batch_is_noop(lib):
     assert lib.gdr_decode_step(None, None) == INVALID
 
 
+def _decode_multi_args(base=None, **kw):
+    m = _abi.DecodeMultiArgs()
+    m.base = base if base is not None else _decode_args()
+    m.n_tokens, m.n_slots = 4, 0
+    for k, v in kw.items():
+        setattr(m, k, v)
+    return m
+
+
+DECODE_MULTI_CASES = [
+    ("zero_tokens", dict(n_tokens=0), INVALID),
+    ("too_many_tokens", dict(n_tokens=9), INVALID),
+    ("slots_without_count", dict(state_slot=FAKE + (11 << 32), n_slots=0), INVALID),
+    ("misaligned_slots", dict(state_slot=FAKE + (11 << 32) + 2, n_slots=8), MISALIGNED),
+    ("misaligned_status", dict(status=FAKE + (12 << 32) + 1), MISALIGNED),
+]
+
+
+@host_only
+@pytest.mark.parametrize("name,kw,want", DECODE_MULTI_CASES, ids=[c[0] for c in DECODE_MULTI_CASES])
+def test_decode_multi_validation(lib, name, kw, want):
+    assert lib.gdr_decode_multi(ctypes.byref(_decode_multi_args(**kw)), None) == want
+
+
+@host_only
+@pytest.mark.parametrize("name,kw,want", DECODE_CASES, ids=[c[0] for c in DECODE_CASES])
+def test_decode_multi_checks_the_step_arguments(lib, name, kw, want):
+    m = _decode_multi_args(base=_decode_args(**kw))
+    assert lib.gdr_decode_multi(ctypes.byref(m), None) == want
+
+
+@host_only
+def test_decode_multi_slot_pool_overlap(lib):
+    # With slots the state buffers span n_slots rows: a separate state_out that
+    # starts inside that span overlaps even though `batch` rows alone would not.
+    row = 4 * 128 * 128 * 4  # H_v * d * d floats
+    base = _decode_args(state_in=FAKE, state_out=FAKE + 6 * row)
+    assert lib.gdr_decode_multi(ctypes.byref(_decode_multi_args(base=base)), None) != INVALID
+    base = _decode_args(state_in=FAKE, state_out=FAKE + 6 * row)
+    m = _decode_multi_args(base=base, state_slot=FAKE + (11 << 32), n_slots=8)
+    assert lib.gdr_decode_multi(ctypes.byref(m), None) == INVALID
+    assert lib.gdr_decode_multi(None, None) == INVALID
+
+
 def _prefill_args(lens=(5, 0, 9), **kw):
     a = _abi.PrefillArgs()
     cu = [0]

@@ -54,6 +54,14 @@ def decode_bytes_per_layer_step(B, H_k, H_v, d, in_b=IN_BYTES, out_b=OUT_BYTES) 
     return B * H_v * per_value_head + B * H_k * per_key_head
 
 
+def decode_bytes_per_layer_call(B, H_k, H_v, d, T, in_b=IN_BYTES, out_b=OUT_BYTES) -> int:
+    """Algorithmic bytes of one multi-token call over B sequences x T tokens:
+    the state once, the per-token inputs and outputs T times."""
+    state = B * H_v * 2 * d * d * 4
+    per_token = decode_bytes_per_layer_step(B, H_k, H_v, d, in_b, out_b) - state
+    return state + T * per_token
+
+
 def prefill_flops_per_token_head(C, d, gva: bool) -> int:
     # K K^T, Q K^T, U, W, P Delta at 2 C d each; W S^T, Q S^T, state update at 2 d^2 each.
     kk_qk = 0 if gva else 4 * C * d
@@ -232,6 +240,66 @@ def time_region(fn, n, ranks):
     return max_over_ranks(e0.elapsed_time(e1), ranks, device="cuda")
 
 
+def decode_variants(device, B, steps=64, warmup=4, slots=32, T=4, world=1):
+    """Two more views of the headline decode workload (18 layers x B, 16/16
+    heads, d=128), each timed on its own inputs with the states rotating
+    through HBM:
+    - layer-folded: the 18 layers' states as one batch of 18*B rows, one
+      launch per step (the kernel without per-launch ramp and tail);
+    - multi-token: T tokens per sequence per call (gdr_decode_multi), 18
+      launches per call, the state read and written once per call."""
+    import linear_attention_recurrence_10_b200 as gdr
+    from linear_attention_recurrence_10_b200 import synth
+    res = {}
+    # Layer-folded single launch.
+    x = synth.make_decode_inputs(LAYERS, slots, B, H_K, H_V, D, seed=11, s0_std=0.02, device=device)
+    fold = lambda t: t.transpose(0, 1).contiguous().view(slots, LAYERS * B, *t.shape[3:])
+    q, k, v, z, g, beta = (fold(t) for t in (x.q, x.k, x.v, x.z, x.g, x.beta))
+    state = x.s0.view(LAYERS * B, H_V, D, D)
+    out = torch.empty(LAYERS * B, H_V, D, device=device, dtype=torch.bfloat16)
+    del x
+
+    def fold_step(s):
+        t = s % slots
+        gdr.decode_step(q[t], k[t], v[t], g[t], beta[t], state, out, z=z[t], norm_w=None)
+
+    for s in range(warmup):
+        fold_step(s)
+    ms = time_region(lambda: [fold_step(warmup + s) for s in range(steps)], steps, world)
+    nbytes = LAYERS * decode_bytes_per_layer_step(B, H_K, H_V, D)
+    res["layer_folded"] = {
+        "value": nbytes * steps / (ms * 1e-3) / 1e9, "unit": "GB/s", "steps": steps,
+        "us_per_launch": ms * 1e3 / steps, "launch": f"one launch per step over {LAYERS}x{B} rows",
+        "tokens_per_s": B * steps / (ms * 1e-3)}
+    del q, k, v, z, g, beta, state, out
+    # Multi-token calls.
+    x = synth.make_decode_inputs(LAYERS, slots * T, B, H_K, H_V, D, seed=12, s0_std=0.02,
+                                 device=device)
+    # [L, calls, T, B, ...] -> [L, calls, B, T, ...]: each call's rows are b*T + t.
+    per_call = lambda t: t.view(LAYERS, slots, T, B, *t.shape[3:]).transpose(2, 3).contiguous() \
+        .view(LAYERS, slots, B * T, *t.shape[3:])
+    q, k, v, z, g, beta = (per_call(t) for t in (x.q, x.k, x.v, x.z, x.g, x.beta))
+    state = x.s0
+    out = torch.empty(B * T, H_V, D, device=device, dtype=torch.bfloat16)
+    del x
+
+    def multi_call(s):
+        c = s % slots
+        for l in range(LAYERS):
+            gdr.decode_multi(q[l, c], k[l, c], v[l, c], g[l, c], beta[l, c], state[l], out,
+                             n_tokens=T, z=z[l, c], overlap_state_load=True)
+
+    for s in range(warmup):
+        multi_call(s)
+    ms = time_region(lambda: [multi_call(warmup + s) for s in range(steps)], steps, world)
+    nbytes = LAYERS * decode_bytes_per_layer_call(B, H_K, H_V, D, T)
+    res["multi_token"] = {
+        "value": nbytes * steps / (ms * 1e-3) / 1e9, "unit": "GB/s", "tokens_per_call": T,
+        "tokens_per_s": B * T * steps / (ms * 1e-3), "us_per_launch": ms * 1e3 / (steps * LAYERS),
+        "launch": f"{LAYERS} launches per call, {T} tokens per sequence each"}
+    return res
+
+
 # ---------------------------------------------------------------- prefill
 
 def prefill_measure(device, reps=5, world=1):
@@ -360,6 +428,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=1024)
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode-variants", action="store_true")
     ap.add_argument("--prefill-only", action="store_true",
                     help="run only the chunked-prefill measurement and print its JSON (profiling)")
     ap.add_argument("--prefill-reps", type=int, default=5)
@@ -415,6 +484,11 @@ def main():
                          world)
     e2e_gbs = weak_scaling_rate(bench.bytes_per_step * args.e2e_steps, world, ms_e2e) / 1e9
 
+    # Free the headline's inputs before the extra decode views allocate theirs.
+    launches_per_step, h2d_bytes, d2h_bytes = bench.launches_per_step, e2e.h2d_bytes, e2e.d2h_bytes
+    del e2e, bench
+    torch.cuda.empty_cache()
+    variants = None if args.no_decode_variants else decode_variants(device, args.batch, world=world)
     prefill = None if args.no_prefill else prefill_measure(device, reps=args.prefill_reps,
                                                            world=world)
     cpu = None
@@ -442,11 +516,12 @@ def main():
                      "bytes_per_launch": per_launch_bytes, "us_per_launch": per_launch_ms * 1e3,
                      "peak_source": peaks["source"] + " (hbm_gbs, of measured copy bandwidth)"},
         "cpu_baseline": cpu,
-        "e2e": {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": e2e.h2d_bytes,
-                "d2h_bytes_per_step": e2e.d2h_bytes, "steps": args.e2e_steps,
+        "e2e": {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": h2d_bytes,
+                "d2h_bytes_per_step": d2h_bytes, "steps": args.e2e_steps,
                 "ms_per_step": ms_e2e / args.e2e_steps},
-        "gpu_launches": args.steps * bench.launches_per_step,
+        "gpu_launches": args.steps * launches_per_step,
         "clocks": clock_info,
+        "decode_variants": variants,
         "prefill": prefill,
     }
     if rank == 0:

@@ -240,6 +240,37 @@ def time_region(fn, n, ranks):
     return max_over_ranks(e0.elapsed_time(e1), ranks, device="cuda")
 
 
+def decode_batch_sweep(device, batches=(1, 2, 4, 8, 16, 32), steps=64, warmup=4, slots=32,
+                       world=1):
+    """The headline step (18 layers, 16/16 heads, d=128) at each batch size.
+    Where the 18 layer states (18 x B x 1 MiB) total less than twice the L2,
+    L2 is flushed (a 256 MB write) before every step and each step is timed
+    on its own with CUDA events, so no step finds its state in L2; larger
+    batches rotate more state than L2 holds and are timed as one region."""
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    res = {}
+    for B in batches:
+        bench = DecodeBench(device, seed=20 + B, B=B, slots=slots)
+        bench.capture()
+        bench.run(0, warmup)
+        state_bytes = LAYERS * B * H_V * D * D * 4
+        flushed = state_bytes < 2 * l2
+        if flushed:
+            ms = 0.0
+            for s in range(steps):
+                flush.zero_()
+                ms += time_region(lambda: bench.run(warmup + s, 1), 1, world)
+        else:
+            ms = time_region(lambda: bench.run(warmup, steps), steps, world)
+        res[str(B)] = {"value": bench.bytes_per_step * steps / (ms * 1e-3) / 1e9, "unit": "GB/s",
+                       "us_per_launch": ms * 1e3 / (steps * LAYERS),
+                       "l2": "flushed before every step" if flushed else "states exceed L2"}
+        del bench
+        torch.cuda.empty_cache()
+    return res
+
+
 def decode_variants(device, B, steps=64, warmup=4, slots=32, T=4, world=1):
     """Two more views of the headline decode workload (18 layers x B, 16/16
     heads, d=128), each timed on its own inputs with the states rotating
@@ -293,6 +324,7 @@ def decode_variants(device, B, steps=64, warmup=4, slots=32, T=4, world=1):
         multi_call(s)
     ms = time_region(lambda: [multi_call(warmup + s) for s in range(steps)], steps, world)
     nbytes = LAYERS * decode_bytes_per_layer_call(B, H_K, H_V, D, T)
+    res["batch_sweep"] = decode_batch_sweep(device, world=world)
     res["multi_token"] = {
         "value": nbytes * steps / (ms * 1e-3) / 1e9, "unit": "GB/s", "tokens_per_call": T,
         "tokens_per_s": B * T * steps / (ms * 1e-3), "us_per_launch": ms * 1e3 / (steps * LAYERS),

@@ -2,8 +2,8 @@
 
 Only the tests, the smoke check and the benchmark's CPU-baseline leg use it.
 """
-from .oracle import (Result, build, gdr_bruteforce, gdr_chunked, gdr_recurrent, load,
-                     rmsnorm_gated)
+from .oracle import (Result, build, gate_from_raw, gdr_bruteforce, gdr_chunked, gdr_recurrent,
+                     load, rmsnorm_gated)
 
 __all__ = ["Result", "build", "load", "gdr_recurrent", "gdr_chunked", "gdr_bruteforce",
-           "rmsnorm_gated"]
+           "rmsnorm_gated", "gate_from_raw"]

@@ -132,6 +132,26 @@ void orc_rmsnorm_gated(const double *o, const double *z, const double *w, int64_
         rmsnorm_gated_row(o + r * n, z + r * n, w, n, eps, y + r * n);
 }
 
+/* Gate inputs from raw projection outputs (the reading taken where the pages
+ * are silent: the parameterisation of the published Gated DeltaNet and Mamba-2
+ * layers, per value head h):
+ *   g_t    = -exp(A_log[h]) * softplus(a_t + dt_bias[h])
+ *   beta_t = sigmoid(b_t) = 1 / (1 + exp(-b_t))
+ * with softplus(x) = log(1 + exp(x)), evaluated as max(x, 0) + log1p(exp(-|x|)),
+ * the same number without overflow.  a, b, g, beta are [n_tok, H_v]. */
+void orc_gate_from_raw(int64_t n_tok, int H_v, const double *a, const double *b,
+                       const double *A_log, const double *dt_bias, double *g, double *beta) {
+    for (int64_t t = 0; t < n_tok; ++t) {
+        for (int h = 0; h < H_v; ++h) {
+            const size_t i = (size_t)t * H_v + h;
+            const double x = a[i] + dt_bias[h];
+            const double softplus = fmax(x, 0.0) + log1p(exp(-fabs(x)));
+            g[i] = -exp(A_log[h]) * softplus;
+            beta[i] = 1.0 / (1.0 + exp(-b[i]));
+        }
+    }
+}
+
 /* Apply the gate to every (token, value head) row of o produced for a problem. */
 static void gate_outputs(const orc_problem *p, int seq, int hv, const double *o,
                          double *y) {

@@ -87,6 +87,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.orc_rmsnorm_gated.argtypes = [_DP, _DP, _DP, ctypes.c_int64, ctypes.c_int,
                                       ctypes.c_double, _DP]
     lib.orc_rmsnorm_gated.restype = None
+    lib.orc_gate_from_raw.argtypes = [ctypes.c_int64, ctypes.c_int, _DP, _DP, _DP, _DP, _DP, _DP]
+    lib.orc_gate_from_raw.restype = None
     _lib_cache[path] = lib
     return lib
 
@@ -182,6 +184,22 @@ def gdr_bruteforce(q, k, v, g, beta, cu_seqlens, *, z=None, s0=None, w=None, sca
         raise ValueError("brute force takes sequences of at most 8 tokens")
     del keep
     return Result(o, y, s)
+
+
+def gate_from_raw(a, b, A_log, dt_bias, lib: ctypes.CDLL | None = None):
+    """(g, beta) from raw per-token gate projections a, b [n_tok, H_v] and the
+    per-head A_log, dt_bias [H_v]: g = -exp(A_log) softplus(a + dt_bias),
+    beta = sigmoid(b)."""
+    a = _f64(a)
+    b = _f64(b, a.shape)
+    n_tok, H_v = a.shape
+    A_log = _f64(A_log, (H_v,))
+    dt_bias = _f64(dt_bias, (H_v,))
+    g = np.zeros_like(a)
+    beta = np.zeros_like(a)
+    (lib or load()).orc_gate_from_raw(ctypes.c_int64(n_tok), int(H_v), _ptr(a), _ptr(b),
+                                      _ptr(A_log), _ptr(dt_bias), _ptr(g), _ptr(beta))
+    return g, beta
 
 
 def rmsnorm_gated(o, z, w=None, eps=1e-6, lib: ctypes.CDLL | None = None) -> np.ndarray:

@@ -88,8 +88,8 @@ typedef struct CUstream_st *gdr_stream_t;
  *   `scale` still multiplies q.  g = -inf is allowed (state reset).
  *   Supported: d_k == d_v in {16, 32, 64, 128}, H_v a multiple of H_k.
  *   batch == 0 is a no-op.  state_stride must be >= H_v*d_v*d_k (0 = that).
- *   flags: 0 or GDR_DECODE_OVERLAP_STATE_LOAD (below); other bits are
- *   rejected with GDR_ERR_INVALID_ARG.
+ *   flags: GDR_DECODE_OVERLAP_STATE_LOAD, GDR_GATE_FROM_RAW (below) or 0;
+ *   other bits are rejected with GDR_ERR_INVALID_ARG.
  * ------------------------------------------------------------------------ */
 /* gdr_decode_args.flags
  *
@@ -105,6 +105,18 @@ typedef struct CUstream_st *gdr_stream_t;
  * the preceding kernel has finished. */
 #define GDR_DECODE_OVERLAP_STATE_LOAD 1
 
+/* gdr_decode_args.flags and gdr_prefill_args.flags
+ *
+ * GDR_GATE_FROM_RAW: g and beta hold the raw per-token gate projections a and
+ * b instead of the gate values; the kernel forms, per value head h,
+ *     g    = -exp(A_log[h]) * softplus(a + dt_bias[h])
+ *     beta = sigmoid(b)
+ * from the [H_v] fp32 arrays A_log and dt_bias, which must then be given.
+ * The pages do not spell this parameterisation out; it is the one of the
+ * published Gated DeltaNet and Mamba-2 layers, and saves the caller a
+ * separate elementwise pass over g and beta. */
+#define GDR_GATE_FROM_RAW 2
+
 typedef struct gdr_decode_args {
     int32_t batch, H_k, H_v, d_k, d_v;
     int32_t in_dtype;  /* gdr_dtype of q, k, v, z */
@@ -113,7 +125,7 @@ typedef struct gdr_decode_args {
     float scale;       /* multiplies q_hat; 1.0 for the plain o_t = S_t q_t */
     float eps_l2;      /* under the square root of the q/k norms */
     float eps_norm;    /* added to mean(o^2) in RMSNormGated */
-    int32_t flags;     /* 0, or GDR_DECODE_OVERLAP_STATE_LOAD */
+    int32_t flags;     /* 0, or GDR_DECODE_OVERLAP_STATE_LOAD | GDR_GATE_FROM_RAW */
     int64_t q_stride, k_stride, v_stride, z_stride, gb_stride, out_stride;
     int64_t state_stride;
     const void *q, *k, *v, *z;
@@ -122,6 +134,7 @@ typedef struct gdr_decode_args {
     float *state_out;
     const float *norm_w;
     void *out;
+    const float *A_log, *dt_bias; /* [H_v] fp32, with GDR_GATE_FROM_RAW only */
 } gdr_decode_args;
 
 gdr_status gdr_decode_step(const gdr_decode_args *args, gdr_stream_t stream);
@@ -229,6 +242,9 @@ typedef struct gdr_prefill_args {
     float *final_state;
     const float *norm_w;
     void *out;
+    int32_t flags;                /* 0 or GDR_GATE_FROM_RAW; other bits are rejected */
+    int32_t reserved;             /* 0 */
+    const float *A_log, *dt_bias; /* [H_v] fp32, with GDR_GATE_FROM_RAW only */
 } gdr_prefill_args;
 
 /* Bytes of workspace gdr_prefill_chunked needs for these arguments (the same

@@ -79,8 +79,20 @@ def status_string(status: int) -> str:
     return _abi.lib().gdr_status_string(int(status)).decode()
 
 
+def _gate_params(gate_params, H_v):
+    """(A_log, dt_bias) fp32 [H_v] tensors, or None: see GDR_GATE_FROM_RAW."""
+    if gate_params is None:
+        return None, None
+    A_log, dt_bias = gate_params
+    for t, name in ((A_log, "A_log"), (dt_bias, "dt_bias")):
+        _f32_tensor(t, name)
+        if t.dim() != 1 or t.shape[0] != H_v or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous fp32 tensor of H_v entries")
+    return A_log, dt_bias
+
+
 def _decode_args(q, k, v, g, beta, state, out, z, norm_w, state_out, scale, eps_l2, eps_norm,
-                 qk_l2norm, overlap_state_load, batch):
+                 qk_l2norm, overlap_state_load, batch, gate_params=None):
     H_k, d = q.shape[1], q.shape[2]
     H_v = v.shape[1]
     for t, name in ((g, "g"), (beta, "beta"), (state, "state"), (norm_w, "norm_w")):
@@ -110,13 +122,17 @@ def _decode_args(q, k, v, g, beta, state, out, z, norm_w, state_out, scale, eps_
     a.g, a.beta = _ptr(g), _ptr(beta)
     a.state_in, a.state_out = _ptr(state), _ptr(so)
     a.norm_w, a.out = _ptr(norm_w), _ptr(out)
+    A_log, dt_bias = _gate_params(gate_params, H_v)
+    if A_log is not None:
+        a.flags |= _abi.GDR_GATE_FROM_RAW
+        a.A_log, a.dt_bias = _ptr(A_log), _ptr(dt_bias)
     return a
 
 
 def decode_step(q, k, v, g, beta, state, out, *, z=None, norm_w=None, state_out=None,
                 scale: float = 1.0, eps_l2: float = 1e-6, eps_norm: float = 1e-6,
                 qk_l2norm: bool = True, overlap_state_load: bool = False,
-                stream=None) -> torch.Tensor:
+                gate_params=None, stream=None) -> torch.Tensor:
     """Advance every sequence of the batch by one token (gdr_decode_step).
 
     q, k [B, H_k, d]; v, z [B, H_v, d] (bf16 or fp32, same dtype); g, beta
@@ -125,9 +141,11 @@ def decode_step(q, k, v, g, beta, state, out, *, z=None, norm_w=None, state_out=
     strided views (e.g. one step of a [B, T, H, d] tensor).
     ``overlap_state_load``: GDR_DECODE_OVERLAP_STATE_LOAD -- only when the
     kernel queued just before this call does not write this state.
+    ``gate_params`` = (A_log, dt_bias), fp32 [H_v]: g and beta then hold the
+    raw projections a, b (GDR_GATE_FROM_RAW).
     """
     a = _decode_args(q, k, v, g, beta, state, out, z, norm_w, state_out, scale, eps_l2, eps_norm,
-                     qk_l2norm, overlap_state_load, q.shape[0])
+                     qk_l2norm, overlap_state_load, q.shape[0], gate_params)
     _check(_abi.lib().gdr_decode_step(ctypes.byref(a), _stream(stream, q.device)),
            "gdr_decode_step")
     return out
@@ -136,7 +154,8 @@ def decode_step(q, k, v, g, beta, state, out, *, z=None, norm_w=None, state_out=
 def decode_multi(q, k, v, g, beta, state, out, *, n_tokens: int, z=None, norm_w=None,
                  state_out=None, slots=None, status=None, scale: float = 1.0,
                  eps_l2: float = 1e-6, eps_norm: float = 1e-6, qk_l2norm: bool = True,
-                 overlap_state_load: bool = False, stream=None) -> torch.Tensor:
+                 overlap_state_load: bool = False, gate_params=None,
+                 stream=None) -> torch.Tensor:
     """Advance every sequence by ``n_tokens`` tokens in one call (gdr_decode_multi).
 
     Token-indexed tensors hold B * n_tokens rows, row b * n_tokens + t being
@@ -151,7 +170,7 @@ def decode_multi(q, k, v, g, beta, state, out, *, n_tokens: int, z=None, norm_w=
         raise ValueError("q must hold batch * n_tokens rows")
     batch = rows // n_tokens
     a = _decode_args(q, k, v, g, beta, state, out, z, norm_w, state_out, scale, eps_l2, eps_norm,
-                     qk_l2norm, overlap_state_load, batch)
+                     qk_l2norm, overlap_state_load, batch, gate_params)
     m = _abi.DecodeMultiArgs()
     m.base = a
     m.n_tokens = int(n_tokens)
@@ -168,7 +187,8 @@ def decode_multi(q, k, v, g, beta, state, out, *, n_tokens: int, z=None, norm_w=
 
 
 def _prefill_args(q, k, v, g, beta, cu_seqlens, out, cu_seqlens_host, z, norm_w,
-                  initial_state, final_state, chunk, scale, eps_l2, eps_norm, qk_l2norm):
+                  initial_state, final_state, chunk, scale, eps_l2, eps_norm, qk_l2norm,
+                  gate_params=None):
     n_tok, H_k, d = q.shape
     H_v = v.shape[1]
     if cu_seqlens.dtype != torch.int32:
@@ -204,6 +224,10 @@ def _prefill_args(q, k, v, g, beta, cu_seqlens, out, cu_seqlens_host, z, norm_w,
     a.cu_seqlens_host = ctypes.cast(host, ctypes.POINTER(ctypes.c_int32))
     a.initial_state, a.final_state = _ptr(initial_state), _ptr(final_state)
     a.norm_w, a.out = _ptr(norm_w), _ptr(out)
+    A_log, dt_bias = _gate_params(gate_params, H_v)
+    if A_log is not None:
+        a.flags = _abi.GDR_GATE_FROM_RAW
+        a.A_log, a.dt_bias = _ptr(A_log), _ptr(dt_bias)
     return a, host
 
 
@@ -221,7 +245,8 @@ def prefill_workspace_size(q, k, v, g, beta, cu_seqlens, out, *, cu_seqlens_host
 def prefill_chunked(q, k, v, g, beta, cu_seqlens, out, *, cu_seqlens_host=None, z=None,
                     norm_w=None, initial_state=None, final_state=None, chunk: int = 0,
                     workspace=None, scale: float = 1.0, eps_l2: float = 1e-6,
-                    eps_norm: float = 1e-6, qk_l2norm: bool = True, stream=None) -> torch.Tensor:
+                    eps_norm: float = 1e-6, qk_l2norm: bool = True, gate_params=None,
+                    stream=None) -> torch.Tensor:
     """Chunked prefill of packed variable-length sequences (gdr_prefill_chunked).
 
     q, k [n_tok, H_k, d]; v, z, out [n_tok, H_v, d]; g, beta [n_tok, H_v] fp32;
@@ -229,10 +254,12 @@ def prefill_chunked(q, k, v, g, beta, cu_seqlens, out, *, cu_seqlens_host=None, 
     values on the host, read during the call); initial_state / final_state
     [n_seq, H_v, d, d] fp32 or None.  ``workspace``: a uint8 device tensor of
     at least prefill_workspace_size() bytes; allocated here when None.
+    ``gate_params`` = (A_log, dt_bias), fp32 [H_v]: g and beta then hold the
+    raw projections a, b (GDR_GATE_FROM_RAW).
     """
     a, host = _prefill_args(q, k, v, g, beta, cu_seqlens, out, cu_seqlens_host, z, norm_w,
                             initial_state, final_state, chunk, scale, eps_l2, eps_norm,
-                            qk_l2norm)
+                            qk_l2norm, gate_params)
     L = _abi.lib()
     n = ctypes.c_size_t(0)
     _check(L.gdr_prefill_workspace_size(ctypes.byref(a), ctypes.byref(n)),
@@ -250,7 +277,7 @@ def prefill_chunked(q, k, v, g, beta, cu_seqlens, out, *, cu_seqlens_host=None, 
 def prefill_chunked_noalloc(q, k, v, g, beta, cu_seqlens, out, *, cu_seqlens_host=None,
                             z=None, norm_w=None, initial_state=None, final_state=None,
                             chunk: int = 0, scale: float = 1.0, eps_l2: float = 1e-6,
-                            eps_norm: float = 1e-6, qk_l2norm: bool = True,
+                            eps_norm: float = 1e-6, qk_l2norm: bool = True, gate_params=None,
                             stream=None) -> torch.Tensor:
     """gdr_prefill_chunked_noalloc: the same prefill, with no workspace to pass and
     nothing allocated -- for callers that cannot allocate device memory here.
@@ -258,7 +285,7 @@ def prefill_chunked_noalloc(q, k, v, g, beta, cu_seqlens, out, *, cu_seqlens_hos
     share one scratch array per device).  Arguments as prefill_chunked."""
     a, host = _prefill_args(q, k, v, g, beta, cu_seqlens, out, cu_seqlens_host, z, norm_w,
                             initial_state, final_state, chunk, scale, eps_l2, eps_norm,
-                            qk_l2norm)
+                            qk_l2norm, gate_params)
     _check(_abi.lib().gdr_prefill_chunked_noalloc(ctypes.byref(a), _stream(stream, q.device)),
            "gdr_prefill_chunked_noalloc")
     del host

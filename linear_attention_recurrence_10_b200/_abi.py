@@ -16,6 +16,7 @@ HEADER = os.path.join(os.path.dirname(PKG), "include", "gdr.h")
 GDR_F32 = 0
 GDR_BF16 = 1
 GDR_DECODE_OVERLAP_STATE_LOAD = 1
+GDR_GATE_FROM_RAW = 2
 GDR_PREFILL_NOALLOC_MAX_SEQS = 4096
 
 STATUS_NAMES = {
@@ -38,6 +39,7 @@ class DecodeArgs(ctypes.Structure):
         ("gb_stride", _i64), ("out_stride", _i64), ("state_stride", _i64),
         ("q", _vp), ("k", _vp), ("v", _vp), ("z", _vp), ("g", _vp), ("beta", _vp),
         ("state_in", _vp), ("state_out", _vp), ("norm_w", _vp), ("out", _vp),
+        ("A_log", _vp), ("dt_bias", _vp),
     ]
 
 
@@ -59,6 +61,7 @@ class PrefillArgs(ctypes.Structure):
         ("q", _vp), ("k", _vp), ("v", _vp), ("z", _vp), ("g", _vp), ("beta", _vp),
         ("cu_seqlens", _vp), ("cu_seqlens_host", ctypes.POINTER(_i32)),
         ("initial_state", _vp), ("final_state", _vp), ("norm_w", _vp), ("out", _vp),
+        ("flags", _i32), ("reserved", _i32), ("A_log", _vp), ("dt_bias", _vp),
     ]
 
 

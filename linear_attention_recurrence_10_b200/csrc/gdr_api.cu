@@ -86,11 +86,20 @@ const char *gdr_status_string(gdr_status s) {
 
 int gdr_version(void) { return 100; }
 
+// With GDR_GATE_FROM_RAW both per-head gate parameter arrays must be given.
+static gdr_status check_raw_gate(int32_t flags, const float *A_log, const float *dt_bias) {
+    if (!(flags & GDR_GATE_FROM_RAW)) return GDR_OK;
+    if (!A_log || !dt_bias) return GDR_ERR_INVALID_ARG;
+    if (!aligned4(A_log) || !aligned4(dt_bias)) return GDR_ERR_MISALIGNED;
+    return GDR_OK;
+}
+
 // Shared validation of the decode arguments.  `slots` is the number of state
 // rows the state buffers hold (batch for the one-token step).
 static gdr_status decode_params(const gdr_decode_args *a, int64_t slots, DecodeParams *out) {
-    if (a->batch < 0 || (a->flags & ~GDR_DECODE_OVERLAP_STATE_LOAD) != 0)
+    if (a->batch < 0 || (a->flags & ~(GDR_DECODE_OVERLAP_STATE_LOAD | GDR_GATE_FROM_RAW)) != 0)
         return GDR_ERR_INVALID_ARG;
+    GDR_TRY(check_raw_gate(a->flags, a->A_log, a->dt_bias));
     if (!dtype_ok(a->in_dtype) || !dtype_ok(a->out_dtype)) return GDR_ERR_INVALID_ARG;
     GDR_TRY(check_heads(a->H_k, a->H_v, a->d_k, a->d_v));
     if (a->batch == 0) return GDR_OK;
@@ -132,6 +141,10 @@ static gdr_status decode_params(const gdr_decode_args *a, int64_t slots, DecodeP
     p.state_in = a->state_in; p.state_out = a->state_out;
     p.norm_w = a->norm_w; p.out = a->out;
     p.n_tokens = 1;
+    if (a->flags & GDR_GATE_FROM_RAW) {
+        p.A_log = a->A_log;
+        p.dt_bias = a->dt_bias;
+    }
     return GDR_OK;
 }
 
@@ -195,6 +208,8 @@ gdr_status gdr_rmsnorm_gated(const gdr_norm_args *a, gdr_stream_t stream) {
 static gdr_status check_prefill(const gdr_prefill_args *a, int *chunk_out) {
     if (!a) return GDR_ERR_INVALID_ARG;
     if (a->n_seq < 0 || a->n_tok < 0) return GDR_ERR_INVALID_ARG;
+    if ((a->flags & ~GDR_GATE_FROM_RAW) != 0 || a->reserved != 0) return GDR_ERR_INVALID_ARG;
+    GDR_TRY(check_raw_gate(a->flags, a->A_log, a->dt_bias));
     if (!dtype_ok(a->in_dtype) || !dtype_ok(a->out_dtype)) return GDR_ERR_INVALID_ARG;
     GDR_TRY(check_heads(a->H_k, a->H_v, a->d_k, a->d_v));
     int chunk = a->chunk;
@@ -289,6 +304,10 @@ gdr_status gdr_prefill_chunked(const gdr_prefill_args *a, void *workspace, size_
     p.eps_l2 = a->eps_l2;
     p.eps_norm = a->eps_norm;
     p.q = a->q; p.k = a->k; p.v = a->v; p.z = a->z;
+    if (a->flags & GDR_GATE_FROM_RAW) {
+        p.A_log = a->A_log;
+        p.dt_bias = a->dt_bias;
+    }
     p.g = a->g; p.beta = a->beta;
     p.cu_seqlens = a->cu_seqlens;
     p.initial_state = a->initial_state;

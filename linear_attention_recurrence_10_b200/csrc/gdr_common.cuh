@@ -30,7 +30,19 @@ struct DecodeParams {
     int n_tokens, n_slots;
     const int *slot;
     int *status;
+    // Non-null: g and beta hold the raw projections a, b (see gate_g, gate_beta).
+    const float *A_log, *dt_bias;
 };
+
+// Gate values from raw projection outputs (gates passed raw): per value head,
+//   g = -exp(A_log) softplus(a + dt_bias),   beta = sigmoid(b),
+// the parameterisation of the published Gated DeltaNet and Mamba-2 layers;
+// softplus(x) as max(x, 0) + log1p(exp(-|x|)), which cannot overflow.
+__device__ __forceinline__ float gate_g(float a, float A_log, float dt_bias) {
+    const float x = a + dt_bias;
+    return -expf(A_log) * (fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))));
+}
+__device__ __forceinline__ float gate_beta(float b) { return 1.f / (1.f + expf(-b)); }
 
 struct NormParams {
     int64_t rows;
@@ -53,6 +65,8 @@ struct PrefillParams {
     float *final_state;
     const float *norm_w;
     void *out;
+    // Non-null: g and beta hold the raw projections a, b (see gate_g, gate_beta).
+    const float *A_log, *dt_bias;
 };
 
 // ------------------------------------------------------------ typed memory

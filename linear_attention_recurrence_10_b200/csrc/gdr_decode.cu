@@ -83,8 +83,12 @@ __global__ void __launch_bounds__(2 * D) decode_kernel(const DecodeParams p) {
         const TIN *kp = static_cast<const TIN *>(p.k) + r * p.k_stride + hk * D;
         float4 q4 = Elem<TIN>::load4(qp + col);
         float4 k4 = Elem<TIN>::load4(kp + col);
-        const float g = __ldg(p.g + r * p.gb_stride + hv);
-        const float beta = __ldg(p.beta + r * p.gb_stride + hv);
+        float g = __ldg(p.g + r * p.gb_stride + hv);
+        float beta = __ldg(p.beta + r * p.gb_stride + hv);
+        if (p.A_log) {
+            g = gate_g(g, __ldg(p.A_log + hv), __ldg(p.dt_bias + hv));
+            beta = gate_beta(beta);
+        }
         float vz = 0.f;
         if (is_a) {
             vz = Elem<TIN>::load1(static_cast<const TIN *>(p.v) + r * p.v_stride + hv * D + my_row);

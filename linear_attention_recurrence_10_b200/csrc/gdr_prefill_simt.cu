@@ -101,8 +101,17 @@ __global__ void __launch_bounds__(kSimtThreads) prefill_simt_kernel(const Prefil
         }
         if (tid < C) {
             const int64_t t = c0 + tid;
-            gin[tid] = tid < L ? fmaxf(__ldg(p.g + t * p.gb_stride + hv), kGammaFloor) : 0.f;
-            bet[tid] = tid < L ? __ldg(p.beta + t * p.gb_stride + hv) : 0.f;
+            float gv = 0.f, bv = 0.f;
+            if (tid < L) {
+                gv = __ldg(p.g + t * p.gb_stride + hv);
+                bv = __ldg(p.beta + t * p.gb_stride + hv);
+                if (p.A_log) {  // raw projections
+                    gv = gate_g(gv, __ldg(p.A_log + hv), __ldg(p.dt_bias + hv));
+                    bv = gate_beta(bv);
+                }
+            }
+            gin[tid] = tid < L ? fmaxf(gv, kGammaFloor) : 0.f;
+            bet[tid] = bv;
         }
         __syncthreads();
         if (tid == 0) {

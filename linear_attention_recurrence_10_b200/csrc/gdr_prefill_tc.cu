@@ -259,7 +259,15 @@ __global__ void __launch_bounds__(NT, 1) prefill_tc_kernel(const PrefillParams p
             if (tid < 64) sc.nk[r] = r < L ? f : 0.f;
             else sc.nq[r] = r < L ? f * p.scale : 0.f;
         } else if (warp == 4) {
-            float ga = fmaxf(gb[lane], kGammaFloor), gbv = fmaxf(gb[lane + 32], kGammaFloor);
+            float g0 = gb[lane], g1 = gb[lane + 32], b0 = gb[C + lane], b1 = gb[C + lane + 32];
+            if (p.A_log) {  // raw projections; rows past the chunk stay zero
+                const float al = __ldg(p.A_log + hv), db = __ldg(p.dt_bias + hv);
+                g0 = lane < L ? gate_g(g0, al, db) : 0.f;
+                g1 = lane + 32 < L ? gate_g(g1, al, db) : 0.f;
+                b0 = lane < L ? gate_beta(b0) : 0.f;
+                b1 = lane + 32 < L ? gate_beta(b1) : 0.f;
+            }
+            float ga = fmaxf(g0, kGammaFloor), gbv = fmaxf(g1, kGammaFloor);
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const float xa = __shfl_up_sync(kFullMask, ga, o);
@@ -269,8 +277,8 @@ __global__ void __launch_bounds__(NT, 1) prefill_tc_kernel(const PrefillParams p
             gbv += __shfl_sync(kFullMask, ga, 31);
             sc.gam[lane] = ga;
             sc.gam[lane + 32] = gbv;
-            sc.bet[lane] = gb[C + lane];
-            sc.bet[lane + 32] = gb[C + lane + 32];
+            sc.bet[lane] = b0;
+            sc.bet[lane + 32] = b1;
             sc.eg[lane] = __expf(ga);
             sc.eg[lane + 32] = __expf(gbv);
         }

@@ -82,6 +82,11 @@ DECODE_CASES = [
     ("state_stride_small", dict(state_stride=128 * 128), INVALID),
     ("gb_stride_small", dict(gb_stride=2), INVALID),
     ("state_partial_overlap", dict(state_out=FAKE + (6 << 32) + 4096), INVALID),
+    ("raw_gate_without_params", dict(flags=2), INVALID),
+    ("raw_gate_without_dt_bias", dict(flags=2, A_log=FAKE + (13 << 32)), INVALID),
+    ("raw_gate_misaligned", dict(flags=2, A_log=FAKE + (13 << 32) + 2,
+                                 dt_bias=FAKE + (14 << 32)), MISALIGNED),
+    ("unknown_flag_4", dict(flags=4), INVALID),
 ]
 
 
@@ -163,6 +168,11 @@ def _prefill_args(lens=(5, 0, 9), **kw):
 
 
 PREFILL_CASES = [
+    ("unknown_flag", dict(flags=1), INVALID),
+    ("reserved_set", dict(reserved=1), INVALID),
+    ("raw_gate_without_params", dict(flags=2), INVALID),
+    ("raw_gate_misaligned", dict(flags=2, A_log=FAKE + (13 << 32) + 1,
+                                 dt_bias=FAKE + (14 << 32)), MISALIGNED),
     ("chunk48", dict(chunk=48), UNSUPPORTED),
     ("chunk128", dict(chunk=128), UNSUPPORTED),
     ("d100", dict(d_k=100, d_v=100), UNSUPPORTED),

@@ -18,9 +18,10 @@ cudaError_t launch_prefill_simt(const PrefillParams &p, int d, int chunk, int in
 size_t prefill_tc_workspace_bytes(int n_seq);
 cudaError_t launch_prefill_tc(const PrefillParams &p, void *workspace, int out_bf16,
                               cudaStream_t s);
-size_t prefill_tc2p_workspace_bytes(int n_seq, int64_t n_chunks, int H_v);
-cudaError_t launch_prefill_tc2p(const PrefillParams &p, int64_t n_chunks, void *workspace,
-                                int out_bf16, cudaStream_t s);
+size_t prefill_tc2p_workspace_bytes(int n_seq, int64_t n_chunks, int H_v, int n_seg);
+int prefill_tc2p_segments(int n_seq, int H_v, int max_chunks, int n_sm);
+cudaError_t launch_prefill_tc2p(const PrefillParams &p, const int32_t *cu_host, int n_seg,
+                                void *workspace, int out_bf16, cudaStream_t s);
 }  // namespace gdr
 
 namespace {
@@ -238,11 +239,38 @@ static int64_t count_chunks(const gdr_prefill_args *a) {
     return n;
 }
 
-// The tensor-core path runs as two kernels when the workspace holds the
-// per-chunk records, else as one kernel that needs only the sequence order.
+// The longest sequence's chunk count (an upper bound without host offsets).
+static int max_chunks(const gdr_prefill_args *a) {
+    if (!a->cu_seqlens_host) return (int)(a->n_tok / 64 + 1);
+    int m = 0;
+    for (int s = 0; s < a->n_seq; ++s) {
+        const int n = (int)(((int64_t)a->cu_seqlens_host[s + 1] - a->cu_seqlens_host[s] + 63) / 64);
+        m = n > m ? n : m;
+    }
+    return m;
+}
+
+static int device_sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        (void)cudaGetLastError();
+        return 148;
+    }
+    return n;
+}
+
+static int prefill_segments(const gdr_prefill_args *a) {
+    return gdr::prefill_tc2p_segments(a->n_seq, a->H_v, max_chunks(a), device_sm_count());
+}
+
+// The tensor-core path runs as two kernels (prep and recurrence, in segments
+// that overlap when the recurrence leaves SMs idle) when the workspace holds
+// the per-chunk records, else as one kernel that needs only the sequence order.
 static size_t workspace_bytes(const gdr_prefill_args *a, int chunk) {
     if (!tensor_core_path(a, chunk)) return 0;
-    return gdr::prefill_tc2p_workspace_bytes(a->n_seq, count_chunks(a), a->H_v);
+    return gdr::prefill_tc2p_workspace_bytes(a->n_seq, count_chunks(a), a->H_v,
+                                             prefill_segments(a));
 }
 
 gdr_status gdr_prefill_workspace_size(const gdr_prefill_args *a, size_t *bytes) {
@@ -290,7 +318,10 @@ gdr_status gdr_prefill_chunked(const gdr_prefill_args *a, void *workspace, size_
     const bool tc = tensor_core_path(a, chunk);
     const int64_t n_chunks = tc ? count_chunks(a) : 0;
     const size_t need_one = tc ? gdr::prefill_tc_workspace_bytes(a->n_seq) : 0;
-    const size_t need_two = tc ? gdr::prefill_tc2p_workspace_bytes(a->n_seq, n_chunks, a->H_v) : 0;
+    const int n_seg = tc ? prefill_segments(a) : 1;
+    const size_t need_two = tc ? gdr::prefill_tc2p_workspace_bytes(a->n_seq, n_chunks, a->H_v, 1) : 0;
+    const size_t need_seg =
+        tc ? gdr::prefill_tc2p_workspace_bytes(a->n_seq, n_chunks, a->H_v, n_seg) : 0;
     if (tc) {
         if (!workspace || ws_bytes < need_one) return GDR_ERR_WORKSPACE;
         if (!aligned16(workspace)) return GDR_ERR_MISALIGNED;
@@ -315,8 +346,9 @@ gdr_status gdr_prefill_chunked(const gdr_prefill_args *a, void *workspace, size_
     p.norm_w = a->norm_w;
     p.out = a->out;
     if (tc && ws_bytes >= need_two)
-        return from_cuda(gdr::launch_prefill_tc2p(p, n_chunks, workspace, a->out_dtype == GDR_BF16,
-                                                  (cudaStream_t)stream));
+        return from_cuda(gdr::launch_prefill_tc2p(p, a->cu_seqlens_host,
+                                                  ws_bytes >= need_seg ? n_seg : 1, workspace,
+                                                  a->out_dtype == GDR_BF16, (cudaStream_t)stream));
     if (tc)
         return from_cuda(gdr::launch_prefill_tc(p, workspace, a->out_dtype == GDR_BF16,
                                                 (cudaStream_t)stream));

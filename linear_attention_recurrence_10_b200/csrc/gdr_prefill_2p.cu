@@ -40,15 +40,28 @@ __host__ __device__ constexpr uint32_t u_off(int s, int i) {
     return (uint32_t)((s >> 2) * 2048 + i * 16 + (s & 3) * 4);
 }
 
-// Workspace: status word, longest-first order, chunk offsets, then records.
-struct WsLayout {
-    size_t order, chunk_off, rec, total;
+// The prefill may run as up to MAX_SEG segments of chunk indices [lo_k, lo_k+1)
+// of every sequence, so that the prep of segment k+1 overlaps the recurrence
+// of segment k on the SMs the recurrence leaves idle.
+constexpr int MAX_SEG = 3;
+struct SegPlan {
+    int n;                  // segments (1 = one prep and one recurrence pass)
+    int lo[MAX_SEG + 1];    // chunk-index boundaries, lo[n] >= every sequence's chunk count
 };
-__host__ __device__ inline WsLayout ws_layout(int n_seq, int64_t n_chunks, int H_v) {
+
+// Workspace: status word, longest-first order, chunk offsets, per-segment unit
+// offsets, the state carried between segments, then records.
+struct WsLayout {
+    size_t order, chunk_off, seg_off, carry, rec, total;
+};
+__host__ __device__ inline WsLayout ws_layout(int n_seq, int64_t n_chunks, int H_v, int n_seg = 1) {
     WsLayout w;
     w.order = 16;
     w.chunk_off = (w.order + 4 * (size_t)n_seq + 15) & ~(size_t)15;
-    w.rec = (w.chunk_off + 4 * ((size_t)n_seq + 1) + 255) & ~(size_t)255;
+    w.seg_off = (w.chunk_off + 4 * ((size_t)n_seq + 1) + 15) & ~(size_t)15;
+    w.carry = (w.seg_off + 4 * (size_t)n_seg * ((size_t)n_seq + 1) + 255) & ~(size_t)255;
+    const size_t carry_bytes = n_seg > 1 ? (size_t)n_seq * H_v * D * D * 4 : 0;
+    w.rec = (w.carry + carry_bytes + 255) & ~(size_t)255;
     w.total = w.rec + (size_t)n_chunks * H_v * REC_BYTES;
     return w;
 }
@@ -57,7 +70,8 @@ __host__ __device__ inline WsLayout ws_layout(int n_seq, int64_t n_chunks, int H
 // Longest-first order (as the one-kernel path), the status word, and the
 // running count of chunks before each sequence.  One block of 1024 threads.
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *cu, int n_seq, int *status,
-                                                    int *order, int *chunk_off) {
+                                                    int *order, int *chunk_off, SegPlan sp,
+                                                    int *seg_off) {
     __shared__ int part[1024];
     const int tid = threadIdx.x;
     if (tid == 0) *status = 0;
@@ -89,6 +103,32 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *cu, int n_seq
         run += (cu[s + 1] - cu[s] + C - 1) / C;
     }
     if (tid == 1023) chunk_off[n_seq] = part[1023];
+    // Per segment k, the exclusive scan of each sequence's chunk count inside
+    // [lo_k, lo_k+1): the prep grid of segment k is laid out by it.
+    for (int k = 0; k < sp.n; ++k) {
+        auto n_in = [&](int s) {
+            const int n = (cu[s + 1] - cu[s] + C - 1) / C;
+            return max(0, min(n, sp.lo[k + 1]) - sp.lo[k]);
+        };
+        __syncthreads();
+        sum = 0;
+        for (int s = lo; s < hi; ++s) sum += n_in(s);
+        part[tid] = sum;
+        __syncthreads();
+        for (int o = 1; o < 1024; o <<= 1) {
+            const int add = tid >= o ? part[tid - o] : 0;
+            __syncthreads();
+            part[tid] += add;
+            __syncthreads();
+        }
+        int *off = seg_off + (size_t)k * (n_seq + 1);
+        run = tid ? part[tid - 1] : 0;
+        for (int s = lo; s < hi; ++s) {
+            off[s] = run;
+            run += n_in(s);
+        }
+        if (tid == 1023) off[n_seq] = part[1023];
+    }
 }
 
 // ------------------------------------------------------------ prep kernel
@@ -121,23 +161,41 @@ static_assert(A_T + C * PLD * 4 <= A_AX && A_AX + 32768 <= A_GB, "prep scratch o
 
 // `succ`: block index distance to the unit that most likely takes this block's
 // SM slot next (resident blocks per SM x SMs); its inputs are prefetched to L2.
+// The block's unit within a segment: the sequence (the last s with
+// seg_off[s] <= unit) and its chunk index (from the segment's first chunk).
+struct PrepUnit {
+    int seq, chunk;
+};
+__device__ __forceinline__ PrepUnit prep_unit(const int *seg_off, int seg_lo, int n_seq, int unit) {
+    int lo = 0, hi = n_seq - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (seg_off[mid] <= unit) lo = mid; else hi = mid - 1;
+    }
+    return {lo, seg_lo + unit - seg_off[lo]};
+}
+
+// One block per (chunk of the segment, value head).  seg_off: the segment's
+// unit offsets per sequence, seg_lo its first chunk index.
+// wait_prev_at_exit: launched as a programmatic dependent of the previous
+// segment's recurrence; the block of the highest index waits for it before
+// exiting, so that this grid completes only after it (the next recurrence
+// segment, queued after this grid, reads the state it carries).
 __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p, const int *chunk_off,
-                                                     unsigned char *records, int *status, int succ) {
+                                                     const int *seg_off, int seg_lo,
+                                                     unsigned char *records, int *status, int succ,
+                                                     int wait_prev_at_exit) {
     extern __shared__ __align__(1024) unsigned char sm[];
     PrepScalars &sc = *reinterpret_cast<PrepScalars *>(sm + A_SCAL);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int quad = warp & 3, part = warp >> 2;
-    const int gchunk = blockIdx.x / p.H_v, hv = blockIdx.x % p.H_v;
+    const int hv = blockIdx.x % p.H_v;
     const int hk = hv / p.hv_per_hk;
-    // The sequence holding this chunk: the last s with chunk_off[s] <= gchunk.
-    int lo = 0, hi = p.n_seq - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (chunk_off[mid] <= gchunk) lo = mid; else hi = mid - 1;
-    }
-    const int seq = lo;
+    const PrepUnit pu = prep_unit(seg_off, seg_lo, p.n_seq, blockIdx.x / p.H_v);
+    const int seq = pu.seq;
+    const int gchunk = chunk_off[seq] + pu.chunk;
     const int64_t t0 = p.cu_seqlens[seq], t1 = p.cu_seqlens[seq + 1];
-    const int64_t c0 = t0 + (int64_t)(gchunk - chunk_off[seq]) * C;
+    const int64_t c0 = t0 + (int64_t)pu.chunk * C;
     const int L = (int)((t1 - c0) < C ? (t1 - c0) : C);
     unsigned char *rec = records + ((size_t)gchunk * p.H_v + hv) * REC_BYTES;
 
@@ -181,13 +239,9 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p, con
     if (blockIdx.x + succ < gridDim.x) {
         // Warm L2 for the unit most likely to take this block's SM slot next:
         // 64 rows x (k, q, v) x two 128-byte lines over the block's threads.
-        const int nb = blockIdx.x + succ, gch = nb / p.H_v, hv2 = nb % p.H_v, hk2 = hv2 / p.hv_per_hk;
-        int a = 0, b = p.n_seq - 1;
-        while (a < b) {
-            const int mid = (a + b + 1) >> 1;
-            if (chunk_off[mid] <= gch) a = mid; else b = mid - 1;
-        }
-        const int64_t n0 = p.cu_seqlens[a] + (int64_t)(gch - chunk_off[a]) * C, n1 = p.cu_seqlens[a + 1];
+        const int nb = blockIdx.x + succ, hv2 = nb % p.H_v, hk2 = hv2 / p.hv_per_hk;
+        const PrepUnit nu = prep_unit(seg_off, seg_lo, p.n_seq, nb / p.H_v);
+        const int64_t n0 = p.cu_seqlens[nu.seq] + (int64_t)nu.chunk * C, n1 = p.cu_seqlens[nu.seq + 1];
         for (int e = tid; e < 3 * 2 * C; e += PNT) {
             const int r = (e >> 1) & 63, line = e & 1, which = e >> 7;
             const int64_t t = n0 + r;
@@ -386,6 +440,7 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p, con
         fence_after_sync();
         tmem_free(tm, 256);
     }
+    if (wait_prev_at_exit && blockIdx.x == gridDim.x - 1) wait_for_predecessor();
 }
 
 // ----------------------------------------------------------- recur kernel
@@ -427,12 +482,25 @@ constexpr uint32_t B_SMEM = B_BAR + 144;
 constexpr uint32_t SC_BYTES = REC_STAGED - REC_SCAL;
 // TMEM columns: the fp32 state, -S W^T, and two buffers each of S Q^T and P Delta.
 constexpr uint32_t TM_S = 0, TM_D = 128, TM_OI = 192, TM_O2 = 320;
+// A recurrence block holds all 512 TMEM columns, so a prep block (which the
+// next segment may start beside it) must never fit on the same SM: their
+// shared memory together exceeds an SM's (228 KB, 1 KB reserved per block).
+static_assert(B_SMEM + A_SMEM + 2 * 1024 > 228 * 1024,
+              "a prep block could share an SM with a recurrence block");
 
+// Chunks [seg_lo, seg_hi) of every sequence.  The state enters from the
+// caller's initial state in the first segment (seg_lo == 0), else from
+// `carry`; it leaves to the caller's final state in the segment where the
+// sequence ends, else to `carry` (both [n_seq, H_v, d_v, d_k]).
 template <typename TOUT>
 __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, const int *order,
                                                        const int *chunk_off,
-                                                       const unsigned char *records, int *status) {
+                                                       const unsigned char *records, int *status,
+                                                       int seg_lo, int seg_hi, float *carry) {
     extern __shared__ __align__(1024) unsigned char sm[];
+    // The next kernel on the stream (the following segment's prep) may start
+    // on the SMs this grid leaves free; it reads nothing this grid writes.
+    release_dependents();
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + B_BAR);
     uint64_t *bar_q = bars, *bar_k = bars + 1;   // tiles landed (32 producer lanes each)
     uint64_t *bar_w = bars + 2;                  // W landed
@@ -451,9 +519,18 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
     const int seq = order[blockIdx.x / p.H_v];
     const int hv = blockIdx.x % p.H_v;
     const int hk = hv / p.hv_per_hk;
-    const int64_t t0 = p.cu_seqlens[seq], t1 = p.cu_seqlens[seq + 1];
-    const int n_chunks = (int)((t1 - t0 + C - 1) / C);
-    const unsigned char *rec0 = records + ((size_t)chunk_off[seq] * p.H_v + hv) * REC_BYTES;
+    const int64_t t1 = p.cu_seqlens[seq + 1];
+    const int total_chunks = (int)((t1 - p.cu_seqlens[seq] + C - 1) / C);
+    // A sequence that ended in an earlier segment has nothing left to do (an
+    // empty sequence belongs to the first segment, which passes its state on).
+    if (seg_lo > 0 && seg_lo >= total_chunks) return;
+    const int seg_end = total_chunks < seg_hi ? total_chunks : seg_hi;
+    const int n_chunks = seg_end - seg_lo;
+    const int64_t t0 = p.cu_seqlens[seq] + (int64_t)seg_lo * C;  // first token of the segment
+    const float *state_in = seg_lo == 0 ? p.initial_state : carry;
+    float *state_out = seg_end == total_chunks ? p.final_state : carry;
+    const unsigned char *rec0 =
+        records + ((size_t)(chunk_off[seq] + seg_lo) * p.H_v + hv) * REC_BYTES;
     const size_t rec_step = (size_t)p.H_v * REC_BYTES;
     const uint32_t sbase = smem_u32(sm);
     auto chunk_len = [&](int c) {
@@ -644,20 +721,20 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
 
         if (n_chunks == 0) {
             // An empty sequence leaves its state as it came in.
-            if (p.final_state) {
+            if (state_out) {
                 const size_t off = ((size_t)seq * p.H_v + hv) * D * D + (size_t)i * D + 64 * half;
 #pragma unroll 4
                 for (int j4 = 0; j4 < 16; ++j4)
-                    *reinterpret_cast<float4 *>(p.final_state + off + 4 * j4) =
-                        p.initial_state ? __ldg(reinterpret_cast<const float4 *>(p.initial_state + off + 4 * j4))
+                    *reinterpret_cast<float4 *>(state_out + off + 4 * j4) =
+                        state_in ? __ldg(reinterpret_cast<const float4 *>(state_in + off + 4 * j4))
                                         : make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
         bool ok = n_chunks > 0 && wait_all(bar_sc, 0);
         if (ok) {
             const float eL = scal(0)[3 * C];
-            const float *s0 = p.initial_state
-                                  ? p.initial_state + ((size_t)seq * p.H_v + hv) * D * D + (size_t)i * D
+            const float *s0 = state_in
+                                  ? state_in + ((size_t)seq * p.H_v + hv) * D * D + (size_t)i * D
                                   : nullptr;
 #pragma unroll 1
             for (int jj = 0; jj < 2; ++jj) {
@@ -841,11 +918,11 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
-    if (warp < 8 && state_ok && p.final_state) {
+    if (warp < 8 && state_ok && state_out) {
         const int quad = warp & 3, half = warp >> 2;
         const int i = 32 * quad + lane;
         const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
-        float *dst = p.final_state + ((size_t)seq * p.H_v + hv) * D * D + (size_t)i * D;
+        float *dst = state_out + ((size_t)seq * p.H_v + hv) * D * D + (size_t)i * D;
 #pragma unroll 1
         for (int jj = 0; jj < 2; ++jj) {
             const int j0 = 64 * half + 32 * jj;
@@ -867,40 +944,99 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
 
 }  // namespace tcp2
 
-size_t prefill_tc2p_workspace_bytes(int n_seq, int64_t n_chunks, int H_v) {
-    return tcp2::ws_layout(n_seq, n_chunks, H_v).total;
+// How many segments: several only when the recurrence leaves at least half of
+// the SMs idle (so the next segment's prep has room beside it) and the longest
+// sequence is long enough to split.
+int prefill_tc2p_segments(int n_seq, int H_v, int max_chunks, int n_sm) {
+    return (2 * (int64_t)n_seq * H_v <= n_sm && max_chunks >= 12) ? tcp2::MAX_SEG : 1;
 }
 
-cudaError_t launch_prefill_tc2p(const PrefillParams &p, int64_t n_chunks, void *workspace,
-                                int out_bf16, cudaStream_t s) {
-    const tcp2::WsLayout w = tcp2::ws_layout(p.n_seq, n_chunks, p.H_v);
+size_t prefill_tc2p_workspace_bytes(int n_seq, int64_t n_chunks, int H_v, int n_seg) {
+    return tcp2::ws_layout(n_seq, n_chunks, H_v, n_seg).total;
+}
+
+// cu_host: the sequence offsets on the host (segment sizes are planned here).
+// Segment boundaries: 44% and 76% of the longest sequence's chunks, so that
+// each later segment's prep (on the SMs the recurrence leaves free) takes
+// about as long as the recurrence of the segment before it.
+cudaError_t launch_prefill_tc2p(const PrefillParams &p, const int32_t *cu_host, int n_seg,
+                                void *workspace, int out_bf16, cudaStream_t s) {
+    int64_t n_chunks = 0;
+    int max_chunks = 0;
+    for (int q = 0; q < p.n_seq; ++q) {
+        const int n = (cu_host[q + 1] - cu_host[q] + tcp2::C - 1) / tcp2::C;
+        n_chunks += n;
+        max_chunks = n > max_chunks ? n : max_chunks;
+    }
+    tcp2::SegPlan sp = {};
+    sp.n = n_seg < 1 ? 1 : (n_seg > tcp2::MAX_SEG ? tcp2::MAX_SEG : n_seg);
+    if (sp.n == 3) {
+        sp.lo[1] = (int)((max_chunks * 44 + 99) / 100);
+        sp.lo[2] = (int)((max_chunks * 76 + 99) / 100);
+    } else if (sp.n == 2) {
+        sp.lo[1] = (int)((max_chunks * 60 + 99) / 100);
+    }
+    sp.lo[0] = 0;
+    sp.lo[sp.n] = max_chunks;
+    for (int k = 1; k <= sp.n; ++k)
+        if (sp.lo[k] <= sp.lo[k - 1]) sp.n = k - 1 > 0 ? k - 1 : 1, sp.lo[sp.n] = max_chunks;
+    const tcp2::WsLayout w = tcp2::ws_layout(p.n_seq, n_chunks, p.H_v, n_seg);
     unsigned char *ws = static_cast<unsigned char *>(workspace);
     int *status = reinterpret_cast<int *>(ws);
     int *order = reinterpret_cast<int *>(ws + w.order);
     int *chunk_off = reinterpret_cast<int *>(ws + w.chunk_off);
+    int *seg_off = reinterpret_cast<int *>(ws + w.seg_off);
+    float *carry = n_seg > 1 ? reinterpret_cast<float *>(ws + w.carry) : nullptr;
     unsigned char *records = ws + w.rec;
-    tcp2::plan_kernel<<<1, 1024, 0, s>>>(p.cu_seqlens, p.n_seq, status, order, chunk_off);
+    tcp2::plan_kernel<<<1, 1024, 0, s>>>(p.cu_seqlens, p.n_seq, status, order, chunk_off, sp,
+                                          seg_off);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    if (n_chunks > 0) {
-        e = cudaFuncSetAttribute(tcp2::prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)tcp2::A_SMEM);
-        if (e != cudaSuccess) return e;
-        int dev = 0, n_sm = 148;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return cudaGetLastError();
-        tcp2::prep_kernel<<<(unsigned)(n_chunks * p.H_v), tcp2::PNT, tcp2::A_SMEM, s>>>(
-            p, chunk_off, records, status, 2 * n_sm);
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-    }
+    int dev = 0, n_sm = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return cudaGetLastError();
+    e = cudaFuncSetAttribute(tcp2::prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)tcp2::A_SMEM);
+    if (e != cudaSuccess) return e;
     auto kern = out_bf16 ? tcp2::recur_kernel<__nv_bfloat16> : tcp2::recur_kernel<float>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcp2::B_SMEM);
     if (e != cudaSuccess) return e;
-    kern<<<(unsigned)((int64_t)p.n_seq * p.H_v), tcp2::RNT, tcp2::B_SMEM, s>>>(p, order, chunk_off,
-                                                                              records, status);
-    return cudaGetLastError();
+    for (int k = 0; k < sp.n; ++k) {
+        int64_t units = 0;
+        for (int q = 0; q < p.n_seq; ++q) {
+            const int n = (cu_host[q + 1] - cu_host[q] + tcp2::C - 1) / tcp2::C;
+            const int m = (n < sp.lo[k + 1] ? n : sp.lo[k + 1]) - sp.lo[k];
+            units += m > 0 ? m : 0;
+        }
+        const int *seg_off_k = seg_off + (size_t)k * (p.n_seq + 1);
+        if (units > 0) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3((unsigned)(units * p.H_v));
+            cfg.blockDim = dim3(tcp2::PNT);
+            cfg.dynamicSmemBytes = tcp2::A_SMEM;
+            cfg.stream = s;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr[0].val.programmaticStreamSerializationAllowed = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = k > 0 ? 1 : 0;  // later segments overlap the recurrence before them
+            e = cudaLaunchKernelEx(&cfg, tcp2::prep_kernel, p, (const int *)chunk_off, seg_off_k,
+                                   sp.lo[k], records, status, 2 * n_sm, k > 0 ? 1 : 0);
+            if (e != cudaSuccess) {
+                (void)cudaGetLastError();
+                return e;
+            }
+        } else if (k > 0) {
+            continue;  // no sequence reaches this segment
+        }
+        kern<<<(unsigned)((int64_t)p.n_seq * p.H_v), tcp2::RNT, tcp2::B_SMEM, s>>>(
+            p, order, chunk_off, records, status, sp.lo[k], k + 1 == sp.n ? 0x7fffffff : sp.lo[k + 1],
+            carry);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace gdr

@@ -247,3 +247,37 @@ def test_tc_one_kernel_variant(lens):
     ws = torch.empty(small, dtype=torch.uint8, device="cuda")
     out, final = run_prefill(inp, chunk=64, workspace=ws)
     _check(inp, out, final, torch.bfloat16)
+
+
+def _single_pass_workspace(inp, H_v):
+    """A workspace one carry buffer short of the segmented layout, which makes
+    the library run prep and recurrence as a single pass."""
+    cu = torch.tensor(inp.cu_seqlens, dtype=torch.int32, device="cuda")
+    x = inp.to("cuda")
+    out = torch.empty(inp.n_tok, H_v, 128, device="cuda")
+    n = gdr.prefill_workspace_size(x.q, x.k, x.v, x.g, x.beta, cu, out,
+                                   cu_seqlens_host=inp.cu_seqlens, z=x.z, chunk=64)
+    return torch.empty(n - inp.n_seq * H_v * 128 * 128 * 4, dtype=torch.uint8, device="cuda")
+
+
+# Sequences of 20, 9 (= the first segment boundary, 44% of 20 chunks rounded
+# up), 0, 17 and 1 chunks: every segment, an end exactly on a boundary, an empty
+# sequence, and a sequence that ends in the first segment.
+SEG_LENS = [20 * 64 - 5, 9 * 64, 0, 16 * 64 + 3, 40]
+
+
+def test_tc_segmented_varlen():
+    """Few (sequence, head) chains leave SMs free, so the prefill runs in
+    segments whose prep overlaps the previous segment's recurrence; the state
+    crosses segment boundaries through the workspace."""
+    inp = synth.make_inputs(SEG_LENS, 2, 4, 128, seed=36, dtype=torch.bfloat16, s0_std=0.02)
+    out, final = run_prefill(inp, chunk=64)
+    _check(inp, out, final, torch.bfloat16)
+
+
+def test_tc_segmented_equals_single_pass():
+    inp = synth.make_inputs(SEG_LENS, 2, 4, 128, seed=37, dtype=torch.bfloat16, s0_std=0.02)
+    out_seg, fin_seg = run_prefill(inp, chunk=64)
+    out_one, fin_one = run_prefill(inp, chunk=64, workspace=_single_pass_workspace(inp, 4))
+    assert torch.equal(out_seg, out_one)
+    assert torch.equal(fin_seg, fin_one)

@@ -165,15 +165,18 @@ class DecodeBench:
         self.bytes_per_step = layers * decode_bytes_per_layer_step(B, H_K, H_V, D)
         self.launches_per_step = layers
 
-    def launch_step(self, t, x=None, out=None):
+    def launch_layer(self, l, t, x=None, out=None):
         x = x or self.x
         out = self.out if out is None else out
+        # Consecutive launches touch different layers' states, so each may
+        # start loading its state while the previous layer's kernel drains.
+        self.gdr.decode_step(x.q[l, t], x.k[l, t], x.v[l, t], x.g[l, t], x.beta[l, t],
+                             self.state[l], out[l], z=x.z[l, t], norm_w=x.w,
+                             overlap_state_load=self.overlap)
+
+    def launch_step(self, t, x=None, out=None):
         for l in range(self.L):
-            # Consecutive launches touch different layers' states, so each may
-            # start loading its state while the previous layer's kernel drains.
-            self.gdr.decode_step(x.q[l, t], x.k[l, t], x.v[l, t], x.g[l, t], x.beta[l, t],
-                                 self.state[l], out[l], z=x.z[l, t], norm_w=x.w,
-                                 overlap_state_load=self.overlap)
+            self.launch_layer(l, t, x, out)
 
     def capture(self):
         s = torch.cuda.Stream()
@@ -195,33 +198,69 @@ class DecodeBench:
 
 
 class DecodeE2E:
-    """Same steps through the same C ABI, with the step's inputs copied in from
-    pinned host memory and its outputs copied back every step."""
+    """Same steps through the same C ABI, with every step's inputs copied in from
+    pinned host memory and its outputs copied back.
+
+    Each step is one CUDA graph (how a serving loop replays a decode step
+    without paying the Python binding's per-call cost): on a side stream it
+    copies the NEXT step's inputs into the other of two device input buffers,
+    while on the main stream its own 18 library calls read the inputs the
+    previous step copied, then its output is copied back.  So every step moves
+    one step's inputs and outputs, and the copies overlap the kernels."""
 
     def __init__(self, bench: DecodeBench, host_slots=16):
         self.b = bench
         x = bench.x
-        self.host_slots = host_slots
+        self.host_slots = host_slots  # even, so a slot fixes its input buffer
         pin = lambda t: t[:, :host_slots].transpose(0, 1).contiguous().cpu().pin_memory()
         # host tensors [slot, L, ...]
         self.h = {n: pin(getattr(x, n)) for n in ("q", "k", "v", "z", "g", "beta")}
         dev = x.q.device
-        self.d = {n: torch.empty_like(t[0], device=dev) for n, t in self.h.items()}
+        self.d = [{n: torch.empty_like(t[0], device=dev) for n, t in self.h.items()}
+                  for _ in range(2)]
         self.h_out = torch.empty(bench.out.shape, dtype=bench.out.dtype).pin_memory()
         self.h2d_bytes = sum(t[0].numel() * t[0].element_size() for t in self.h.values())
         self.d2h_bytes = self.h_out.numel() * self.h_out.element_size()
         import types
-        self.view = types.SimpleNamespace(
-            q=self.d["q"].unsqueeze(1), k=self.d["k"].unsqueeze(1), v=self.d["v"].unsqueeze(1),
-            z=self.d["z"].unsqueeze(1), g=self.d["g"].unsqueeze(1),
-            beta=self.d["beta"].unsqueeze(1), w=x.w)
+        self.view = [types.SimpleNamespace(
+            q=d["q"].unsqueeze(1), k=d["k"].unsqueeze(1), v=d["v"].unsqueeze(1),
+            z=d["z"].unsqueeze(1), g=d["g"].unsqueeze(1), beta=d["beta"].unsqueeze(1), w=x.w)
+            for d in self.d]
+
+    def _copy_in(self, slot):
+        for n, t in self.h.items():
+            self.d[slot % 2][n].copy_(t[slot], non_blocking=True)
+
+    def _enqueue(self, slot):
+        main = torch.cuda.current_stream()
+        self.side.wait_stream(main)
+        with torch.cuda.stream(self.side):
+            self._copy_in((slot + 1) % self.host_slots)
+        self.b.launch_step(0, x=self.view[slot % 2])
+        self.h_out.copy_(self.b.out, non_blocking=True)
+        main.wait_stream(self.side)
+
+    def capture(self):
+        self.side = torch.cuda.Stream()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self._copy_in(0)
+            self._enqueue(0)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        self.graphs = []
+        for slot in range(self.host_slots):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self._enqueue(slot)
+            self.graphs.append(g)
+        torch.cuda.synchronize()
+        self._copy_in(0)  # the first replayed step's inputs
+        torch.cuda.synchronize()
 
     def step(self, s):
-        slot = s % self.host_slots
-        for n, t in self.h.items():
-            self.d[n].copy_(t[slot], non_blocking=True)
-        self.b.launch_step(0, x=self.view)
-        self.h_out.copy_(self.b.out, non_blocking=True)
+        self.graphs[s % self.host_slots].replay()
 
 
 def time_region(fn, n, ranks):
@@ -314,11 +353,28 @@ def decode_variants(device, B, steps=64, warmup=4, slots=32, T=4, world=1):
     out = torch.empty(B * T, H_V, D, device=device, dtype=torch.bfloat16)
     del x
 
-    def multi_call(s):
-        c = s % slots
+    def enqueue_call(c):
         for l in range(LAYERS):
             gdr.decode_multi(q[l, c], k[l, c], v[l, c], g[l, c], beta[l, c], state[l], out,
                              n_tokens=T, z=z[l, c], overlap_state_load=True)
+
+    # One CUDA graph per call, as for the headline (the binding's per-call host
+    # cost would otherwise exceed the kernels' time).
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        enqueue_call(0)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graphs = []
+    for c in range(slots):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            enqueue_call(c)
+        graphs.append(gr)
+
+    def multi_call(s):
+        graphs[s % slots].replay()
 
     for s in range(warmup):
         multi_call(s)
@@ -328,7 +384,8 @@ def decode_variants(device, B, steps=64, warmup=4, slots=32, T=4, world=1):
     res["multi_token"] = {
         "value": nbytes * steps / (ms * 1e-3) / 1e9, "unit": "GB/s", "tokens_per_call": T,
         "tokens_per_s": B * T * steps / (ms * 1e-3), "us_per_launch": ms * 1e3 / (steps * LAYERS),
-        "launch": f"{LAYERS} launches per call, {T} tokens per sequence each"}
+        "launch": f"{LAYERS} launches per call, {T} tokens per sequence each, one CUDA graph per call"}
+    del graphs
     return res
 
 
@@ -510,10 +567,11 @@ def main():
 
     # End to end through the same ABI with host buffers.
     e2e = DecodeE2E(bench)
+    e2e.capture()
     for s in range(4):
         e2e.step(s)
-    ms_e2e = time_region(lambda: [e2e.step(s) for s in range(args.e2e_steps)], args.e2e_steps,
-                         world)
+    ms_e2e = time_region(lambda: [e2e.step(4 + s) for s in range(args.e2e_steps)],
+                         args.e2e_steps, world)  # consecutive with the warm-up steps
     e2e_gbs = weak_scaling_rate(bench.bytes_per_step * args.e2e_steps, world, ms_e2e) / 1e9
 
     # Free the headline's inputs before the extra decode views allocate theirs.
@@ -550,6 +608,9 @@ def main():
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": h2d_bytes,
                 "d2h_bytes_per_step": d2h_bytes, "steps": args.e2e_steps,
+                "launch": "one CUDA graph per step: the 18 library calls on inputs the previous "
+                          "step copied from pinned host memory, the next step's inputs copied "
+                          "in meanwhile, the outputs copied back",
                 "ms_per_step": ms_e2e / args.e2e_steps},
         "gpu_launches": args.steps * launches_per_step,
         "clocks": clock_info,

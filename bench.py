@@ -211,8 +211,11 @@ class DecodeE2E:
     def __init__(self, bench: DecodeBench, host_slots=16):
         self.b = bench
         x = bench.x
-        self.host_slots = host_slots  # even, so a slot fixes its input buffer
-        pin = lambda t: t[:, :host_slots].transpose(0, 1).contiguous().cpu().pin_memory()
+        # An even number of slots, so that a slot fixes its input buffer.
+        n = max(1, min(host_slots, bench.T))
+        idx = list(range(n)) + ([0] if n % 2 else [])
+        self.host_slots = len(idx)
+        pin = lambda t: t[:, idx].transpose(0, 1).contiguous().cpu().pin_memory()
         # host tensors [slot, L, ...]
         self.h = {n: pin(getattr(x, n)) for n in ("q", "k", "v", "z", "g", "beta")}
         dev = x.q.device
@@ -601,8 +604,8 @@ def main():
         "hbm_frac": gbs / world / peaks["hbm_gbs"],
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                     "traffic": captured_traffic("decode_kernel<128, bf16, bf16>"),
-                     "kernel": "decode_kernel<128, bf16, bf16>",
+                     "traffic": captured_traffic("decode_kernel<128, bf16, bf16, false>"),
+                     "kernel": "decode_kernel<128, bf16, bf16, false>",
                      "bytes_per_launch": per_launch_bytes, "us_per_launch": per_launch_ms * 1e3,
                      "peak_source": peaks["source"] + " (hbm_gbs, of measured copy bandwidth)"},
         "cpu_baseline": cpu,

@@ -472,16 +472,17 @@ constexpr uint32_t B_KQ = 0;                   // bf16 [K;Q] (32 KB)
 constexpr uint32_t B_W = 32768;                // bf16 W of the current chunk (16 KB)
 constexpr uint32_t B_P = 49152;                // bf16 P hi/lo of the current chunk (16 KB)
 constexpr uint32_t B_SC = 65536;               // 2 x scalars (eg, nqe, dn, eL: 1 KB each)
-constexpr uint32_t B_S = 67584;                // bf16 S [i][j] (32 KB)
-constexpr uint32_t B_DL = 100352;              // Delta hi/lo (32 KB)
-constexpr uint32_t B_DT = 133120;              // decayed Delta hi/lo (32 KB)
-constexpr uint32_t B_U = 165888;               // fp32 U of the current chunk (32 KB, record layout)
-constexpr uint32_t B_OS = 198656;              // fp32 O [r][i] of the chunk being output (32 KB)
-constexpr uint32_t B_BAR = 231424;             // 16 mbarriers, then the TMEM address
+constexpr uint32_t B_DL = 67584;               // Delta hi/lo (32 KB)
+constexpr uint32_t B_DT = 100352;              // decayed Delta hi/lo (32 KB)
+constexpr uint32_t B_U = 133120;               // fp32 U of the current chunk (32 KB, record layout)
+constexpr uint32_t B_OS = 165888;              // fp32 O [r][i] of the chunk being output (32 KB)
+constexpr uint32_t B_BAR = 198656;             // 16 mbarriers, then the TMEM address
 constexpr uint32_t B_SMEM = B_BAR + 144;
 constexpr uint32_t SC_BYTES = REC_STAGED - REC_SCAL;
-// TMEM columns: the fp32 state, -S W^T, and two buffers each of S Q^T and P Delta.
-constexpr uint32_t TM_S = 0, TM_D = 128, TM_OI = 192, TM_O2 = 320;
+// TMEM columns: the fp32 state, -S W^T, two buffers of S Q^T, one of P Delta,
+// and the bf16 copy of S (two values per column) that -S W^T and S Q^T read
+// as their A operand.
+constexpr uint32_t TM_S = 0, TM_D = 128, TM_OI = 192, TM_O2 = 320, TM_SB = 384;
 // A recurrence block holds all 512 TMEM columns, so a prep block (which the
 // next segment may start beside it) must never fit on the same SM: their
 // shared memory together exceeds an SM's (228 KB, 1 KB reserved per block).
@@ -582,9 +583,9 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
                 if (!ok) break;
                 fence_after_sync();
                 fence_smem_to_async();
-                gemm(tm + TM_D, sbase + B_S, 2048, 128, 4096, sbase + B_W, 128, 2048, 256, D / 16, ID_D, false);
+                gemm_ta(tm + TM_D, tm + TM_SB, sbase + B_W, 128, 2048, 256, D / 16, ID_D, false);
                 commit(smem_u32(bar_gd));
-                gemm(tm + TM_OI + 64 * b, sbase + B_S, 2048, 128, 4096, kq + 16384, 128, 2048, 256, D / 16, ID_KK, false);
+                gemm_ta(tm + TM_OI + 64 * b, tm + TM_SB, kq + 16384, 128, 2048, 256, D / 16, ID_KK, false);
                 commit(smem_u32(bar_qfree));
                 ok = mbar_wait(bar_dready, ph, kWaitNs) && mbar_wait(bar_k, ph, kWaitNs);
                 if (!ok) break;
@@ -596,11 +597,14 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
                 gemm(tm + TM_S, eh, 2048, 128, 4096, kq, 2048, 128, 4096, C / 16, ID_S, true);
                 gemm(tm + TM_S, el, 2048, 128, 4096, kq, 2048, 128, 4096, C / 16, ID_S, true);
                 commit(smem_u32(bar_gs));
-                ok = mbar_wait(bar_p, ph, kWaitNs);
+                // P Delta has one accumulator: chunk c-1's output must have left it.
+                ok = mbar_wait(bar_p, ph, kWaitNs) &&
+                     (c < 1 || mbar_wait(bar_ofree + ((c - 1) & 1), (uint32_t)((c - 1) >> 1) & 1u, kWaitNs));
                 if (!ok) break;
+                fence_after_sync();
                 fence_smem_to_async();
                 const uint32_t dh = sbase + B_DL, dl = dh + 16384, pb = sbase + B_P, pl = pb + 8192;
-                const uint32_t o2 = tm + TM_O2 + 64 * b;
+                const uint32_t o2 = tm + TM_O2;
                 gemm(o2, dh, 2048, 128, 4096, pb, 1024, 128, 2048, C / 16, ID_KK, false);
                 gemm(o2, dh, 2048, 128, 4096, pl, 1024, 128, 2048, C / 16, ID_KK, true);
                 gemm(o2, dl, 2048, 128, 4096, pb, 1024, 128, 2048, C / 16, ID_KK, true);
@@ -708,12 +712,17 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
             __syncwarp();
             if (lane == 0) mbar_arrive(bar);
         };
-        // Row i of S (32 columns from j0): bf16 copy for the MMAs and, scaled by
-        // e^{gamma_L} of the coming chunk, back into TMEM for its update.
+        // Row i of S (32 columns from j0): bf16 copy (the A operand of the next
+        // chunk's first MMAs) and, scaled by e^{gamma_L} of the coming chunk, the
+        // fp32 state for its update, both into TMEM.
         auto stage_state = [&](float (&v)[32], int j0, float eL) {
+            uint32_t pk[16];
 #pragma unroll
-            for (int j8 = 0; j8 < 4; ++j8)
-                *reinterpret_cast<uint4 *>(sm + B_S + kmaj(i, j0 + 8 * j8, D)) = pack8(v + 8 * j8);
+            for (int u = 0; u < 16; ++u) {
+                const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * u], v[2 * u + 1]);
+                pk[u] = *reinterpret_cast<const uint32_t *>(&b2);
+            }
+            tmem_st16(tm + lane_off + TM_SB + j0 / 2, pk);
 #pragma unroll
             for (int u = 0; u < 32; ++u) v[u] *= eL;
             tmem_st32(tm + lane_off + TM_S + j0, v);
@@ -847,7 +856,7 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
                 for (int h16 = 0; h16 < 2; ++h16) {
                     float a[16], d[16];
                     tmem_ld16(tm + lane_off + TM_OI + 64 * b + r0 + 16 * h16, a);
-                    tmem_ld16(tm + lane_off + TM_O2 + 64 * b + r0 + 16 * h16, d);
+                    tmem_ld16(tm + lane_off + TM_O2 + r0 + 16 * h16, d);
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4) {
                         const int r = r0 + 16 * h16 + 4 * k4;

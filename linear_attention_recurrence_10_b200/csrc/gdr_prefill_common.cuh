@@ -49,6 +49,16 @@ __device__ __forceinline__ void gemm(uint32_t d, uint32_t a, uint32_t a_lbo, uin
                         smem_desc(b + kk * b_step, b_lbo, b_sbo), idesc, (acc || kk > 0) ? 1u : 0u);
 }
 
+// The same with A in tensor memory (see mma_ta): `ksteps` instructions of
+// K = 16, A advancing 8 columns a step.
+__device__ __forceinline__ void gemm_ta(uint32_t d, uint32_t a_tmem, uint32_t b, uint32_t b_lbo,
+                                        uint32_t b_sbo, uint32_t b_step, int ksteps, uint32_t idesc,
+                                        bool acc) {
+    for (int kk = 0; kk < ksteps; ++kk)
+        mma_ta(d, a_tmem + 8 * kk, smem_desc(b + kk * b_step, b_lbo, b_sbo), idesc,
+               (acc || kk > 0) ? 1u : 0u);
+}
+
 // z * sigmoid(z) with the fast exponential (relative error ~1e-7 here).
 __device__ __forceinline__ float fast_silu(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 

@@ -473,7 +473,6 @@ constexpr uint32_t B_W = 32768;                // bf16 W of the current chunk (1
 constexpr uint32_t B_P = 49152;                // bf16 P hi/lo of the current chunk (16 KB)
 constexpr uint32_t B_SC = 65536;               // 2 x scalars (eg, nqe, dn, eL: 1 KB each)
 constexpr uint32_t B_DL = 67584;               // Delta hi/lo (32 KB)
-constexpr uint32_t B_DT = 100352;              // decayed Delta hi/lo (32 KB)
 constexpr uint32_t B_U = 133120;               // fp32 U of the current chunk (32 KB, record layout)
 constexpr uint32_t B_OS = 165888;              // fp32 O [r][i] of the chunk being output (32 KB)
 constexpr uint32_t B_BAR = 198656;             // 16 mbarriers, then the TMEM address
@@ -483,6 +482,9 @@ constexpr uint32_t SC_BYTES = REC_STAGED - REC_SCAL;
 // and the bf16 copy of S (two values per column) that -S W^T and S Q^T read
 // as their A operand.
 constexpr uint32_t TM_S = 0, TM_D = 128, TM_OI = 192, TM_O2 = 320, TM_SB = 384;
+// ... and the decayed Delta^T tiles (hi, lo; two values per column), the A
+// operand of the state update.
+constexpr uint32_t TM_DTH = 448, TM_DTL = 480;
 // A recurrence block holds all 512 TMEM columns, so a prep block (which the
 // next segment may start beside it) must never fit on the same SM: their
 // shared memory together exceeds an SM's (228 KB, 1 KB reserved per block).
@@ -591,11 +593,10 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
                 if (!ok) break;
                 fence_after_sync();
                 fence_smem_to_async();
-                // S <- e^{gamma_L} S + Dt~^T K (hi + lo); then O_intra^T = Delta^T P^T
-                // (hi*hi + hi*lo + lo*hi) into this chunk's output buffer.
-                const uint32_t eh = sbase + B_DT, el = eh + 16384;
-                gemm(tm + TM_S, eh, 2048, 128, 4096, kq, 2048, 128, 4096, C / 16, ID_S, true);
-                gemm(tm + TM_S, el, 2048, 128, 4096, kq, 2048, 128, 4096, C / 16, ID_S, true);
+                // S <- e^{gamma_L} S + Dt~^T K (hi + lo, Dt~^T from TMEM); then
+                // O_intra^T = Delta^T P^T (hi*hi + hi*lo + lo*hi) into its buffer.
+                gemm_ta(tm + TM_S, tm + TM_DTH, kq, 2048, 128, 4096, C / 16, ID_S, true);
+                gemm_ta(tm + TM_S, tm + TM_DTL, kq, 2048, 128, 4096, C / 16, ID_S, true);
                 commit(smem_u32(bar_gs));
                 // P Delta has one accumulator: chunk c-1's output must have left it.
                 ok = mbar_wait(bar_p, ph, kWaitNs) &&
@@ -779,17 +780,21 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
                     w[4 * s4] = v[4 * s4] * dn.x; w[4 * s4 + 1] = v[4 * s4 + 1] * dn.y;
                     w[4 * s4 + 2] = v[4 * s4 + 2] * dn.z; w[4 * s4 + 3] = v[4 * s4 + 3] * dn.w;
                 }
+                uint32_t th[8], tl[8];
 #pragma unroll
                 for (int c8 = 0; c8 < 2; ++c8) {
                     uint4 hi, lo;
-                    const uint32_t o = kmaj(i, s0 + 8 * c8, D);
                     split8(v + 8 * c8, hi, lo);
+                    const uint32_t o = kmaj(i, s0 + 8 * c8, D);
                     *reinterpret_cast<uint4 *>(sm + B_DL + o) = hi;
                     *reinterpret_cast<uint4 *>(sm + B_DL + 16384 + o) = lo;
                     split8(w + 8 * c8, hi, lo);
-                    *reinterpret_cast<uint4 *>(sm + B_DT + o) = hi;
-                    *reinterpret_cast<uint4 *>(sm + B_DT + 16384 + o) = lo;
+                    th[4 * c8] = hi.x; th[4 * c8 + 1] = hi.y; th[4 * c8 + 2] = hi.z; th[4 * c8 + 3] = hi.w;
+                    tl[4 * c8] = lo.x; tl[4 * c8 + 1] = lo.y; tl[4 * c8 + 2] = lo.z; tl[4 * c8 + 3] = lo.w;
                 }
+                // Tokens s0 .. s0+15 of row i: columns s0/2 .. s0/2+7 of each tile.
+                tmem_st8(tm + lane_off + TM_DTH + s0 / 2, th);
+                tmem_st8(tm + lane_off + TM_DTL + s0 / 2, tl);
             }
             publish(bar_dready);
 

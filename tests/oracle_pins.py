@@ -334,10 +334,51 @@ def check_rmsnorm_gated(lib):
     _close(got[0], np.array([0.5 * 0.75 * l3] * 2), 1e-14, "eps of the RMS norm")
 
 
+def check_gate_from_raw_closed_forms(lib):
+    """g = -exp(A_log) softplus(a + dt_bias), beta = sigmoid(b) (the Gated DeltaNet
+    parameterisation; the pages only say the layer is a Gated DeltaNet) at points
+    whose values are known exactly: softplus(0) = ln 2, softplus(x) = x + log1p(e^-x)
+    for large x, no overflow at +-800, sigmoid(0) = 1/2."""
+    a = np.array([[0.0, -3.0], [50.0, -800.0], [800.0, 2.0]])
+    b = np.array([[0.0, 1.0], [-1.0, 40.0], [-800.0, 3.0]])
+    A_log = np.array([0.0, math.log(2.0)])
+    dt_bias = np.array([0.0, 3.0])
+    g, beta = oracle.gate_from_raw(a, b, A_log, dt_bias, lib=lib)
+    # x = a + dt_bias = 0 -> softplus = ln 2; head 1 scales by exp(ln 2) = 2.
+    _close(g[0, 0], -math.log(2.0), 1e-15, "softplus(0)")
+    _close(g[0, 1], -2.0 * math.log(2.0), 1e-15, "dt_bias shift and exp(A_log)")
+    _close(g[1, 0], -(50.0 + math.log1p(math.exp(-50.0))), 1e-15, "softplus(50)")
+    assert g[1, 1] == 0.0, "softplus(-797) underflows to 0"
+    _close(g[2, 0], -800.0, 1e-15, "softplus(800) without overflow")
+    assert beta[0, 0] == 0.5 and beta[2, 0] == 0.0, "sigmoid(0), sigmoid(-800)"
+    assert abs(beta[1, 1] - 1.0) <= 1e-15, "sigmoid(40)"
+    _close(beta[0, 1], 1.0 / (1.0 + math.exp(-1.0)), 1e-15, "sigmoid(1)")
+
+
+def check_gate_from_raw_identities(lib):
+    """softplus(x) - softplus(-x) = x and sigmoid(x) + sigmoid(-x) = 1; A_log = -inf
+    turns the decay off; decays are never positive; dt_bias shifts the argument."""
+    rng = np.random.default_rng(5)
+    a = rng.normal(size=(40, 3)) * 4
+    b = rng.normal(size=(40, 3)) * 4
+    zero = np.zeros(3)
+    g_pos, beta_pos = oracle.gate_from_raw(a, b, zero, zero, lib=lib)
+    g_neg, beta_neg = oracle.gate_from_raw(-a, -b, zero, zero, lib=lib)
+    assert np.max(np.abs(-g_pos + g_neg - a)) <= 1e-13, "softplus(x) - softplus(-x) = x"
+    assert np.max(np.abs(beta_pos + beta_neg - 1.0)) <= 1e-15, "sigmoid(x) + sigmoid(-x) = 1"
+    g_off, _ = oracle.gate_from_raw(a, b, np.full(3, -np.inf), zero, lib=lib)
+    assert np.all(g_off == 0.0) and np.all(g_pos < 0), "no decay at A_log = -inf; g < 0"
+    c = np.array([0.5, -1.0, 2.0])
+    g1, _ = oracle.gate_from_raw(a, b, zero, c, lib=lib)
+    g2, _ = oracle.gate_from_raw(a + c, b, zero, zero, lib=lib)
+    assert np.array_equal(g1, g2), "dt_bias shifts the softplus argument"
+
+
 ALL_CHECKS = [
     check_beta0_g0_identity, check_retrieval_beta1, check_reset_neg_inf, check_pure_decay,
     check_orthonormal_keys, check_handworked, check_bruteforce_equals_recurrent,
     check_chunked_equals_recurrent, check_linearity, check_value_permutation,
     check_gva_equals_expanded, check_varlen_equals_separate, check_split_handoff,
     check_contraction_bound, check_qk_normalisation, check_rmsnorm_gated,
+    check_gate_from_raw_closed_forms, check_gate_from_raw_identities,
 ]

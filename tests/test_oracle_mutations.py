@@ -40,6 +40,11 @@ MUTANTS = [
     ("brute_sign", "a * ((i == j ? 1.0 : 0.0) - b * kh[s * dk + i] * kh[s * dk + j]);",
      "a * ((i == j ? 1.0 : 0.0) + b * kh[s * dk + i] * kh[s * dk + j]);"),
     ("brute_product_order", "for (int r = s + 1; r <= t; ++r) {", "for (int r = s; r <= t; ++r) {"),
+    ("gate_softplus_mirrored", "fmax(x, 0.0) + log1p(exp(-fabs(x)))", "fmax(-x, 0.0) + log1p(exp(-fabs(x)))"),
+    ("gate_alog_not_exponentiated", "g[i] = -exp(A_log[h]) * softplus;", "g[i] = -A_log[h] * softplus;"),
+    ("gate_decay_positive", "g[i] = -exp(A_log[h]) * softplus;", "g[i] = exp(A_log[h]) * softplus;"),
+    ("gate_bias_dropped", "const double x = a[i] + dt_bias[h];", "const double x = a[i];"),
+    ("gate_beta_mirrored", "beta[i] = 1.0 / (1.0 + exp(-b[i]));", "beta[i] = 1.0 / (1.0 + exp(b[i]));"),
 ]
 
 

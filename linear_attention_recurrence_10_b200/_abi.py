@@ -102,6 +102,8 @@ def lib(path: str = LIB_PATH) -> ctypes.CDLL:
     h.gdr_prefill_chunked.restype = ctypes.c_int
     h.gdr_prefill_chunked_noalloc.argtypes = [ctypes.POINTER(PrefillArgs), _vp]
     h.gdr_prefill_chunked_noalloc.restype = ctypes.c_int
+    h.gdr_decode_multi.argtypes = [ctypes.POINTER(DecodeMultiArgs), _vp]
+    h.gdr_decode_multi.restype = ctypes.c_int
     h.gdr_rmsnorm_gated.argtypes = [ctypes.POINTER(NormArgs), _vp]
     h.gdr_rmsnorm_gated.restype = ctypes.c_int
     h.gdr_status_string.argtypes = [ctypes.c_int]

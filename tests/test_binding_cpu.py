@@ -1,6 +1,7 @@
 """The Python binding's marshalling, checked on the host: every field of the argument
 struct a decode call hands to gdr_decode_step, for packed tensors and for strided
-views, and the binding's own refusals.  Nothing is launched."""
+views; the binding's own refusals; and, with no CUDA device present, each entry
+carried through the library's host checks up to the launch.  Nothing runs on a device."""
 import pytest
 import torch
 
@@ -89,3 +90,49 @@ def test_binding_refusals():
         _args(dict(x, beta=torch.randn(B, 2, H_V)[:, 0]), state, out)
     with pytest.raises(ValueError):  # gate parameters of the wrong length
         _args(x, state, out, gate_params=(torch.zeros(H_V + 1), torch.zeros(H_V + 1)))
+
+
+def test_every_entry_reaches_the_launch_without_a_device():
+    """With no CUDA device, each binding call marshals its tensors, passes every host
+    check of the library, and stops at the launch with GDR_ERR_CUDA: so the binding
+    builds arguments the library accepts, through each declared ctypes signature."""
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present: the GPU tests cover these calls")
+    H, D = 2, 128
+    bf = torch.bfloat16
+    w = torch.ones(D)
+
+    def rows(n, dtype=bf):
+        return torch.randn(n, H, D, dtype=dtype)
+
+    def gates(n):
+        return -torch.rand(n, H), torch.rand(n, H)
+
+    state = torch.zeros(4, H, D, D)
+    g, beta = gates(4)
+    g8, beta8 = gates(8)
+    n_tok = 200
+    cu = torch.tensor([0, 80, n_tok], dtype=torch.int32)
+    gp, bp = gates(n_tok)
+    final = torch.zeros(2, H, D, D)
+    pre = dict(cu_seqlens_host=[0, 80, n_tok], z=rows(n_tok), norm_w=w, final_state=final,
+               chunk=64, stream=0)
+    calls = {
+        "gdr_decode_step": lambda: gdr.decode_step(
+            rows(4), rows(4), rows(4), g, beta, state, rows(4), z=rows(4), norm_w=w, stream=0),
+        "gdr_decode_multi": lambda: gdr.decode_multi(
+            rows(8), rows(8), rows(8), g8, beta8, state, rows(8), n_tokens=2, z=rows(8),
+            norm_w=w, slots=torch.arange(4, dtype=torch.int32),
+            status=torch.zeros(1, dtype=torch.int32), stream=0),
+        "gdr_prefill_chunked": lambda: gdr.prefill_chunked(
+            rows(n_tok), rows(n_tok), rows(n_tok), gp, bp, cu, rows(n_tok), **pre),
+        "gdr_prefill_chunked_noalloc": lambda: gdr.prefill_chunked_noalloc(
+            rows(n_tok), rows(n_tok), rows(n_tok), gp, bp, cu, rows(n_tok), **pre),
+        "gdr_rmsnorm_gated": lambda: gdr.rmsnorm_gated(
+            rows(10, torch.float32), rows(10, torch.float32), rows(10, torch.float32), w=w,
+            stream=0),
+    }
+    for name, call in calls.items():
+        with pytest.raises(gdr.GdrError) as e:
+            call()
+        assert e.value.status == 5 and name in str(e.value), (name, str(e.value))  # GDR_ERR_CUDA

@@ -5,8 +5,8 @@
  * The mixer: the pages name it as the "gated delta rule" recurrence with an
  * RMSNormGated output (Qwen3.5 Chat guide, soniqo.audio/de/guides/chat,
  * section "Architektur"), 18 of the 24 layers of Qwen3.5-0.8B; on the Core AI
- * Qwen3.6-35B-A3B card (first section) it runs 32 value heads over 16 key
- * heads, each key/query head shared by two value heads (GVA).  Its state is a
+ * Qwen3.6-35B-A3B card (first section) it has 16 key heads, each serving two
+ * of its 32 value heads (GVA).  Its state is a
  * fixed-size matrix per head, so memory does not grow with context (Swiftlet
  * post, "How It Works").  The equations follow the published gated delta rule
  * (Gated Delta Networks, Yang, Kautz, Hatamizadeh, ICLR 2025).  Per sequence,
@@ -69,9 +69,9 @@ typedef struct CUstream_st *gdr_stream_t;
 /* ------------------------------------------------------------------------
  * One decode step: every sequence in the batch advances by one token.
  *
- * The pages' decoder is a single-step model that owns the recurrent state, so
- * the caller advances one token per call (Core ML card for Qwen3.5-0.8B,
- * section "Model"); the state is held across the generation loop (same card,
+ * The pages' decoder keeps the layer state between calls and moves forward by
+ * a single token each time it is invoked (Core ML card for Qwen3.5-0.8B,
+ * section "Model"); the state lives across the generation loop (same card,
  * "Usage").  Here the caller owns the state buffer and this call updates it.
  *
  *   q, k       [batch, H_k, d_k]   in_dtype    row strides q_stride, k_stride

@@ -8,13 +8,12 @@
  *
  * What it computes (one value head at a time, tokens in order):
  *
- *   The pages name the mixer -- "DeltaNet layers (linear attention with
- *   gated-delta-rule recurrence and RMSNormGated)" in the Qwen3.5 Chat guide
- *   (soniqo.audio/de/guides/chat, section "Architektur"; same text in the
- *   Arabic copy, section "البنية المعمارية"), and "GatedDeltaNet ... 32 value
- *   heads over 16 key heads (GVA: each k/q head is shared across two value
- *   heads)" on the Core AI model-zoo card for Qwen3.6-35B-A3B (first section).
- *   They do not write the equations.  The recurrence used here is the gated
+ *   The pages name the mixer but never write its equations.  The Qwen3.5 Chat
+ *   guide (soniqo.audio/de/guides/chat, section "Architektur"; the Arabic copy
+ *   has the same section) describes these layers as linear attention driven
+ *   by a gated delta rule recurrence and followed by RMSNormGated.  The Core
+ *   AI model-zoo card for Qwen3.6-35B-A3B (first section) gives the head
+ *   layout: 16 key/query heads, each serving two of 32 value heads (GVA).  The recurrence used here is the gated
  *   delta rule as published in "Gated Delta Networks: Improving Mamba2 with
  *   Delta Rule" (Yang, Kautz, Hatamizadeh, ICLR 2025, eq. of the gated delta
  *   rule):
@@ -27,8 +26,8 @@
  *
  *   S is d_v x d_k, row-major, so row i belongs to value dimension i.
  *   Value head h_v reads key head floor(h_v * H_k / H_v) (each key head feeds
- *   H_v/H_k consecutive value heads, the "head-repeat" on the same card,
- *   section "How to reproduce").
+ *   H_v/H_k consecutive value heads: the same card expands key heads by
+ *   repetition, section "How to reproduce").
  *
  * Three independent forms are provided so they can be checked against each
  * other and against closed forms:

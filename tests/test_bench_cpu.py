@@ -35,7 +35,8 @@ def test_decode_bytes_qwen35_batch32():
 
 
 def test_decode_bytes_gva_batch64():
-    # 64 sequences, 32 value heads over 16 key heads: q and k are read once per key head.
+    # 64 sequences, 16 key heads each serving two of 32 value heads: q and k are read once
+    # per key head.
     per_value_head = 131_072 + 256 + 256 + 8 + 256
     want = 64 * 32 * per_value_head + 64 * 16 * 512
     assert want == 270_548_992

@@ -29,7 +29,26 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "gdr_oracle.c")
-_LIB = os.path.join(_HERE, "_build", "liboracle.so")
+# The gated full-attention decode step (the other mixer of the hybrid decoder).
+_SRC_ATTN = os.path.join(_HERE, "gattn_oracle.c")
+
+
+def _host_key() -> str:
+    """A short key of this host's CPU model and flags: the oracle is compiled
+    with -march=native, so a build is only reused on the CPU it was made for."""
+    import hashlib
+    import platform
+    text = platform.machine()
+    try:
+        with open("/proc/cpuinfo") as f:
+            lines = [l for l in f if l.startswith(("model name", "flags", "Features"))]
+        text += "".join(sorted(set(lines)))
+    except OSError:
+        pass
+    return hashlib.sha256(text.encode()).hexdigest()[:12]
+
+
+_LIB = os.path.join(_HERE, "_build", f"liboracle-{_host_key()}.so")
 
 _DP = ctypes.POINTER(ctypes.c_double)
 
@@ -52,15 +71,32 @@ class _Problem(ctypes.Structure):
     ]
 
 
-def build(src: str = _SRC, out: str = _LIB, force: bool = False, werror: bool = True) -> str:
-    """Compile the oracle with the host C compiler (plain -O2, no CPU-specific flags)."""
-    if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(src):
+class _AttnProblem(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("H_q", ctypes.c_int32), ("H_kv", ctypes.c_int32),
+        ("d", ctypes.c_int32), ("rot_dim", ctypes.c_int32), ("max_len", ctypes.c_int32),
+        ("theta", ctypes.c_double), ("scale", ctypes.c_double),
+        ("q", _DP), ("gate", _DP), ("k", _DP), ("v", _DP),
+        ("k_cache", _DP), ("v_cache", _DP),
+        ("cache_len", ctypes.POINTER(ctypes.c_int64)),
+    ]
+
+
+def build(src: str = _SRC, out: str = _LIB, force: bool = False, werror: bool = True,
+          attn_src: str = _SRC_ATTN) -> str:
+    """Compile the oracle with the host C compiler: -O3 -march=native, ISO C11 (so
+    no floating-point contraction or reassociation: the same arithmetic as any
+    other build, only faster).  The file name carries the host's CPU key."""
+    srcs = [src, attn_src]
+    if not force and os.path.exists(out) and all(
+            os.path.getmtime(out) >= os.path.getmtime(f) for f in srcs):
         return out
     os.makedirs(os.path.dirname(out), exist_ok=True)
     tmp = out + f".tmp{os.getpid()}"
     subprocess.run(
-        ["gcc", "-std=c11", "-O2", "-fPIC", "-shared", "-Wall", "-Wextra"]
-        + (["-Werror"] if werror else []) + ["-o", tmp, src, "-lm", "-lpthread"],
+        ["gcc", "-std=c11", "-O3", "-march=native", "-ffp-contract=off", "-fPIC", "-shared",
+         "-Wall", "-Wextra"]
+        + (["-Werror"] if werror else []) + ["-o", tmp, *srcs, "-lm", "-lpthread"],
         check=True,
     )
     os.replace(tmp, out)
@@ -89,6 +125,11 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.orc_rmsnorm_gated.restype = None
     lib.orc_gate_from_raw.argtypes = [ctypes.c_int64, ctypes.c_int, _DP, _DP, _DP, _DP, _DP, _DP]
     lib.orc_gate_from_raw.restype = None
+    lib.orc_rope_partial.argtypes = [_DP, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                                     ctypes.c_double, ctypes.c_double, _DP]
+    lib.orc_rope_partial.restype = None
+    lib.orc_gated_attn_decode.argtypes = [ctypes.POINTER(_AttnProblem), _DP, _DP, _DP]
+    lib.orc_gated_attn_decode.restype = ctypes.c_int
     _lib_cache[path] = lib
     return lib
 
@@ -211,3 +252,46 @@ def rmsnorm_gated(o, z, w=None, eps=1e-6, lib: ctypes.CDLL | None = None) -> np.
     (lib or load()).orc_rmsnorm_gated(_ptr(o), _ptr(z), _ptr(w), o.size // n, n, float(eps),
                                       _ptr(y))
     return y
+
+
+# ----------------------------------------------------- gated full attention
+
+def rope_partial(x, pos, rot_dim, theta=1e7, lib: ctypes.CDLL | None = None) -> np.ndarray:
+    """Rotary embedding of the first rot_dim dims of every row of x [..., d] at
+    one position ("rotate half" pairing: dim i with dim i + rot_dim/2)."""
+    x = _f64(x)
+    d = x.shape[-1]
+    out = np.zeros_like(x)
+    (lib or load()).orc_rope_partial(_ptr(x), x.size // d, d, int(rot_dim), float(pos),
+                                     float(theta), _ptr(out))
+    return out
+
+
+@dataclass
+class AttnResult:
+    y: np.ndarray        # [batch, H_q, d] after the output gate
+    o: np.ndarray        # [batch, H_q, d] attention output before the gate
+    k_rot: np.ndarray    # [batch, H_kv, d] rotated key appended at index cache_len[b]
+
+
+def gated_attn_decode(q, gate, k, v, k_cache, v_cache, cache_len, *, rot_dim, theta=1e7,
+                      scale=None, lib: ctypes.CDLL | None = None) -> AttnResult:
+    """One decode step of the gated full-attention layer for every sequence:
+    q, gate [B, H_q, d]; k, v [B, H_kv, d] (the new token); k_cache, v_cache
+    [B, H_kv, max_len, d] with cache_len[b] valid entries; scale defaults to
+    d^-1/2."""
+    q = _f64(q); gate = _f64(gate, q.shape); k = _f64(k); v = _f64(v, k.shape)
+    B, H_q, d = q.shape
+    H_kv = k.shape[1]
+    k_cache = _f64(k_cache); v_cache = _f64(v_cache, k_cache.shape)
+    if k_cache.shape[:2] != (B, H_kv) or k_cache.shape[3] != d:
+        raise ValueError("k_cache must be [B, H_kv, max_len, d]")
+    cl = np.ascontiguousarray(np.asarray(cache_len, dtype=np.int64))
+    p = _AttnProblem(B, H_q, H_kv, d, int(rot_dim), k_cache.shape[2], float(theta),
+                     float(d ** -0.5 if scale is None else scale), _ptr(q), _ptr(gate), _ptr(k),
+                     _ptr(v), _ptr(k_cache), _ptr(v_cache),
+                     cl.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)))
+    y = np.zeros((B, H_q, d)); o = np.zeros((B, H_q, d)); kr = np.zeros((B, H_kv, d))
+    if (lib or load()).orc_gated_attn_decode(ctypes.byref(p), _ptr(y), _ptr(o), _ptr(kr)):
+        raise ValueError("invalid shape or a full cache")
+    return AttnResult(y, o, kr)

@@ -11,6 +11,12 @@ namespace gdr {
 
 constexpr unsigned kFullMask = 0xffffffffu;
 
+// Workspace of the one-kernel tensor-core prefill: the status word (16 bytes
+// reserved) and the longest-first order of n_seq sequences, rounded up to 256.
+constexpr size_t prefill_tc_ws_bytes(int64_t n_seq) {
+    return (size_t)(16 + 4 * (size_t)n_seq + 255) & ~(size_t)255;
+}
+
 // ----------------------------------------------------------------- params
 
 struct DecodeParams {
@@ -67,6 +73,12 @@ struct PrefillParams {
     void *out;
     // Non-null: g and beta hold the raw projections a, b (see gate_g, gate_beta).
     const float *A_log, *dt_bias;
+    // Diagnostics only, zero in every ordinary call: a limit for the device
+    // waits of the tensor-core recurrence (0 = the default), and a flag that
+    // withholds every (sequence, head)'s first key tile so that those waits
+    // run out and the kernel's unwinding path runs.
+    uint64_t wait_ns;
+    int withhold_first_k;
 };
 
 // ------------------------------------------------------------ typed memory

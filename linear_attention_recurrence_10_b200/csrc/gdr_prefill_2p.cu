@@ -450,10 +450,12 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p, con
 // and the next state needs Delta.  The output of a chunk (O = (m e^gamma) Q S^T
 // + P Delta, then RMSNormGated) feeds nothing later, so the CTA is split into
 // four roles that run concurrently and hand work over on mbarriers:
-//   warps 0-7   state group: the Delta epilogue (hi/lo tiles of Delta and of
-//               its decayed, k-normalised copy) and, once the state update is
-//               done, the bf16 copy of S for the next chunk's products, with
-//               the next chunk's e^{gamma_L} folded into the same pass;
+//   warps 0-7   state group: the Delta epilogue -- first the decayed,
+//               k-normalised copy of Delta^T as hi/lo tiles in TMEM, all the
+//               state update waits for, then Delta's hi/lo tiles for P Delta --
+//               and, once the update is done, the bf16 copy of S that the next
+//               chunk's first products wait for, then the state pre-scaled by
+//               the next chunk's e^{gamma_L}, which only its update waits for;
 //   warps 8-15  output group, one chunk behind: S Q^T and P Delta out of
 //               double-buffered TMEM, staged through shared memory so that
 //               one warp normalises, gates and stores whole tokens;
@@ -475,8 +477,8 @@ constexpr uint32_t B_SC = 65536;               // 2 x scalars (eg, nqe, dn, eL: 
 constexpr uint32_t B_DL = 67584;               // Delta hi/lo (32 KB)
 constexpr uint32_t B_U = 133120;               // fp32 U of the current chunk (32 KB, record layout)
 constexpr uint32_t B_OS = 165888;              // fp32 O [r][i] of the chunk being output (32 KB)
-constexpr uint32_t B_BAR = 198656;             // 16 mbarriers, then the TMEM address
-constexpr uint32_t B_SMEM = B_BAR + 144;
+constexpr uint32_t B_BAR = 198656;             // 18 mbarriers, then the TMEM address
+constexpr uint32_t B_SMEM = B_BAR + 160;
 constexpr uint32_t SC_BYTES = REC_STAGED - REC_SCAL;
 // TMEM columns: the fp32 state, -S W^T, two buffers of S Q^T, one of P Delta,
 // and the bf16 copy of S (two values per column) that -S W^T and S Q^T read
@@ -516,8 +518,10 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
     uint64_t *bar_oready = bars + 10;            // [2] P Delta (and S Q^T) of a chunk done
     uint64_t *bar_ofree = bars + 12;             // [2] output group done with a chunk's buffers
     uint64_t *bar_sready = bars + 14;            // state group: bf16 S staged (8 warps)
-    uint64_t *bar_dready = bars + 15;            // state group: Delta tiles staged (8 warps)
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + B_BAR + 128);
+    uint64_t *bar_dready = bars + 15;            // state group: Delta tiles for P Delta staged (8 warps)
+    uint64_t *bar_dtready = bars + 16;           // state group: decayed Delta^T in TMEM (8 warps)
+    uint64_t *bar_scaled = bars + 17;            // state group: fp32 S pre-scaled for the update (8 warps)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + B_BAR + 144);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int seq = order[blockIdx.x / p.H_v];
     const int hv = blockIdx.x % p.H_v;
@@ -541,6 +545,9 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
         return (int)(left < C ? left : C);
     };
     auto fail = [&]() { atomicExch(status, kTimeoutStatus); };
+    // Every wait below gives up after wait_ns (2 s unless a diagnostic call
+    // shortens it) and the CTA then unwinds: status word, copies, TMEM.
+    const uint64_t wait_ns = p.wait_ns ? p.wait_ns : kWaitNs;
     auto scal = [&](int c) { return reinterpret_cast<const float *>(sm + B_SC + (c & 1) * SC_BYTES); };
 
     if (warp == 0) tmem_alloc(tmem_slot, 512);
@@ -560,6 +567,8 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
         mbar_init(bar_gs, 1);
         mbar_init(bar_sready, 8);
         mbar_init(bar_dready, 8);
+        mbar_init(bar_dtready, 8);
+        mbar_init(bar_scaled, 8);
         mbar_fence_init();
     }
     fence_before_sync();
@@ -579,9 +588,9 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
             for (int c = 0; c < n_chunks && ok; ++c) {
                 const int b = c & 1;
                 const uint32_t ph = (uint32_t)c & 1u;
-                ok = mbar_wait(bar_sready, ph, kWaitNs) && mbar_wait(bar_w, ph, kWaitNs) &&
-                     mbar_wait(bar_q, ph, kWaitNs) &&
-                     (c < 2 || mbar_wait(bar_ofree + b, (uint32_t)((c >> 1) - 1) & 1u, kWaitNs));
+                ok = mbar_wait(bar_sready, ph, wait_ns) && mbar_wait(bar_w, ph, wait_ns) &&
+                     mbar_wait(bar_q, ph, wait_ns) &&
+                     (c < 2 || mbar_wait(bar_ofree + b, (uint32_t)((c >> 1) - 1) & 1u, wait_ns));
                 if (!ok) break;
                 fence_after_sync();
                 fence_smem_to_async();
@@ -589,7 +598,10 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
                 commit(smem_u32(bar_gd));
                 gemm_ta(tm + TM_OI + 64 * b, tm + TM_SB, kq + 16384, 128, 2048, 256, D / 16, ID_KK, false);
                 commit(smem_u32(bar_qfree));
-                ok = mbar_wait(bar_dready, ph, kWaitNs) && mbar_wait(bar_k, ph, kWaitNs);
+                // The update needs only the decayed Delta^T tiles (TMEM) and the
+                // pre-scaled state; the Delta tiles of P Delta may still be coming.
+                ok = mbar_wait(bar_dtready, ph, wait_ns) && mbar_wait(bar_k, ph, wait_ns) &&
+                     mbar_wait(bar_scaled, ph, wait_ns);
                 if (!ok) break;
                 fence_after_sync();
                 fence_smem_to_async();
@@ -599,8 +611,8 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
                 gemm_ta(tm + TM_S, tm + TM_DTL, kq, 2048, 128, 4096, C / 16, ID_S, true);
                 commit(smem_u32(bar_gs));
                 // P Delta has one accumulator: chunk c-1's output must have left it.
-                ok = mbar_wait(bar_p, ph, kWaitNs) &&
-                     (c < 1 || mbar_wait(bar_ofree + ((c - 1) & 1), (uint32_t)((c - 1) >> 1) & 1u, kWaitNs));
+                ok = mbar_wait(bar_p, ph, wait_ns) && mbar_wait(bar_dready, ph, wait_ns) &&
+                     (c < 1 || mbar_wait(bar_ofree + ((c - 1) & 1), (uint32_t)((c - 1) >> 1) & 1u, wait_ns));
                 if (!ok) break;
                 fence_after_sync();
                 fence_smem_to_async();
@@ -657,29 +669,30 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
             const int L = chunk_len(c);
             const uint32_t pp = (uint32_t)(c - 1) & 1u;  // phase of chunk c-1's events
             // Q and W of chunk c once chunk c-1's S Q^T (issued after -S W^T) is done.
-            if (c > 0) ok = mbar_wait(bar_qfree, pp, kWaitNs);
+            if (c > 0) ok = mbar_wait(bar_qfree, pp, wait_ns);
             if (!ok) break;
             fetch(c0, L, true);
             bulk(B_W, REC_W, REC_P - REC_W, bar_w, c);
             ++n_w;
             // U once chunk c-1's Delta epilogue is done with the stage.
-            if (c > 0) ok = mbar_wait(bar_dready, pp, kWaitNs);
+            if (c > 0) ok = mbar_wait(bar_dready, pp, wait_ns);
             if (!ok) break;
             bulk(B_U, REC_U, REC_BYTES - REC_U, bar_u, c);
             ++n_u;
-            // K once chunk c-1's state update is done.
-            if (c > 0) ok = mbar_wait(bar_gs, pp, kWaitNs);
+            // K once chunk c-1's state update is done.  A diagnostic call may
+            // withhold chunk 0's K tile, so that the waits on it run out.
+            if (c > 0) ok = mbar_wait(bar_gs, pp, wait_ns);
             if (!ok) break;
-            fetch(c0, L, false);
+            if (!(p.withhold_first_k && c == 0)) fetch(c0, L, false);
             // P once chunk c-1's P Delta is done.
-            if (c > 0) ok = mbar_wait(bar_oready + ((c - 1) & 1), (uint32_t)((c - 1) >> 1) & 1u, kWaitNs);
+            if (c > 0) ok = mbar_wait(bar_oready + ((c - 1) & 1), (uint32_t)((c - 1) >> 1) & 1u, wait_ns);
             if (!ok) break;
             bulk(B_P, REC_P, REC_SCAL - REC_P, bar_p, c);
             ++n_p;
             // Scalars of chunk c+1 replace chunk c-1's once the output group is
             // done with them; the record after that goes to L2.
             if (c >= 1 && c + 1 < n_chunks) {
-                ok = mbar_wait(bar_ofree + ((c + 1) & 1), (uint32_t)((c - 1) >> 1) & 1u, kWaitNs);
+                ok = mbar_wait(bar_ofree + ((c + 1) & 1), (uint32_t)((c - 1) >> 1) & 1u, wait_ns);
                 if (!ok) break;
                 bulk(B_SC + ((c + 1) & 1) * SC_BYTES, REC_SCAL, SC_BYTES, bar_sc + ((c + 1) & 1), c + 1);
                 ++n_sc[(c + 1) & 1];
@@ -690,11 +703,11 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
         if (!ok) {
             if (lane == 0) fail();
             // No bulk copy may land after the CTA ends.
-            if (n_w) mbar_wait(bar_w, (uint32_t)(n_w - 1) & 1u, kWaitNs);
-            if (n_p) mbar_wait(bar_p, (uint32_t)(n_p - 1) & 1u, kWaitNs);
-            if (n_u) mbar_wait(bar_u, (uint32_t)(n_u - 1) & 1u, kWaitNs);
+            if (n_w) mbar_wait(bar_w, (uint32_t)(n_w - 1) & 1u, wait_ns);
+            if (n_p) mbar_wait(bar_p, (uint32_t)(n_p - 1) & 1u, wait_ns);
+            if (n_u) mbar_wait(bar_u, (uint32_t)(n_u - 1) & 1u, wait_ns);
             for (int b = 0; b < 2; ++b)
-                if (n_sc[b]) mbar_wait(bar_sc + b, (uint32_t)(n_sc[b] - 1) & 1u, kWaitNs);
+                if (n_sc[b]) mbar_wait(bar_sc + b, (uint32_t)(n_sc[b] - 1) & 1u, wait_ns);
         }
         __syncwarp();
     } else if (warp < 8) {
@@ -704,7 +717,7 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
         const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
         // Every wait's outcome is made warp-uniform, so a warp stops as a whole.
         auto wait_all = [&](uint64_t *bar, uint32_t parity) {
-            return __all_sync(0xffffffffu, mbar_wait(bar, parity, kWaitNs)) != 0;
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, wait_ns)) != 0;
         };
         // Hand the staged tiles and TMEM to the MMA warp: one arrival per warp.
         auto publish = [&](uint64_t *bar) {
@@ -713,10 +726,9 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
             __syncwarp();
             if (lane == 0) mbar_arrive(bar);
         };
-        // Row i of S (32 columns from j0): bf16 copy (the A operand of the next
-        // chunk's first MMAs) and, scaled by e^{gamma_L} of the coming chunk, the
-        // fp32 state for its update, both into TMEM.
-        auto stage_state = [&](float (&v)[32], int j0, float eL) {
+        // Row i of S (32 columns from j0): the bf16 copy, the A operand of the
+        // next chunk's first MMAs ...
+        auto stage_bf16 = [&](const float (&v)[32], int j0) {
             uint32_t pk[16];
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
@@ -724,6 +736,10 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
                 pk[u] = *reinterpret_cast<const uint32_t *>(&b2);
             }
             tmem_st16(tm + lane_off + TM_SB + j0 / 2, pk);
+        };
+        // ... and, scaled by e^{gamma_L} of the coming chunk, the fp32 state for
+        // its update.
+        auto stage_scaled = [&](float (&v)[32], int j0, float eL) {
 #pragma unroll
             for (int u = 0; u < 32; ++u) v[u] *= eL;
             tmem_st32(tm + lane_off + TM_S + j0, v);
@@ -756,9 +772,11 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
                                         : make_float4(0.f, 0.f, 0.f, 0.f);
                     v[4 * j4] = x.x; v[4 * j4 + 1] = x.y; v[4 * j4 + 2] = x.z; v[4 * j4 + 3] = x.w;
                 }
-                stage_state(v, j0, eL);
+                stage_bf16(v, j0);
+                stage_scaled(v, j0, eL);
             }
             publish(bar_sready);
+            publish(bar_scaled);
         }
         int c = 0;
         for (; c < n_chunks && ok; ++c) {
@@ -767,11 +785,14 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
             ok = wait_all(bar_gd, (uint32_t)c & 1u) && wait_all(bar_u, (uint32_t)c & 1u);
             if (!ok) break;
             fence_after_sync();
+            // Decayed Delta^T first: it is all the state update waits for.
+            float dv[2][16];
 #pragma unroll
             for (int h16 = 0; h16 < 2; ++h16) {
                 const int s0 = 32 * half + 16 * h16;
-                float v[16], w[16];
-                tmem_ld16(tm + lane_off + TM_D + s0, v);
+                float *v = dv[h16];
+                float w[16];
+                tmem_ld16(tm + lane_off + TM_D + s0, dv[h16]);
 #pragma unroll
                 for (int s4 = 0; s4 < 4; ++s4) {
                     const float4 u = *reinterpret_cast<const float4 *>(sm + B_U + u_off(s0 + 4 * s4, i));
@@ -784,10 +805,6 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
 #pragma unroll
                 for (int c8 = 0; c8 < 2; ++c8) {
                     uint4 hi, lo;
-                    split8(v + 8 * c8, hi, lo);
-                    const uint32_t o = kmaj(i, s0 + 8 * c8, D);
-                    *reinterpret_cast<uint4 *>(sm + B_DL + o) = hi;
-                    *reinterpret_cast<uint4 *>(sm + B_DL + 16384 + o) = lo;
                     split8(w + 8 * c8, hi, lo);
                     th[4 * c8] = hi.x; th[4 * c8 + 1] = hi.y; th[4 * c8 + 2] = hi.z; th[4 * c8 + 3] = hi.w;
                     tl[4 * c8] = lo.x; tl[4 * c8 + 1] = lo.y; tl[4 * c8 + 2] = lo.z; tl[4 * c8 + 3] = lo.w;
@@ -796,9 +813,24 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
                 tmem_st8(tm + lane_off + TM_DTH + s0 / 2, th);
                 tmem_st8(tm + lane_off + TM_DTL + s0 / 2, tl);
             }
+            publish(bar_dtready);
+            // Then Delta itself as hi/lo tiles in shared memory, the B operand of P Delta.
+#pragma unroll
+            for (int h16 = 0; h16 < 2; ++h16) {
+                const int s0 = 32 * half + 16 * h16;
+#pragma unroll
+                for (int c8 = 0; c8 < 2; ++c8) {
+                    uint4 hi, lo;
+                    split8(dv[h16] + 8 * c8, hi, lo);
+                    const uint32_t o = kmaj(i, s0 + 8 * c8, D);
+                    *reinterpret_cast<uint4 *>(sm + B_DL + o) = hi;
+                    *reinterpret_cast<uint4 *>(sm + B_DL + 16384 + o) = lo;
+                }
+            }
             publish(bar_dready);
 
-            // Once the state update is done: the next chunk's bf16 S and scaled S.
+            // Once the state update is done: the next chunk's bf16 S (what its
+            // first products wait for), then the state scaled for its update.
             ok = wait_all(bar_gs, (uint32_t)c & 1u);
             if (!ok || c + 1 == n_chunks) continue;
             ok = wait_all(bar_sc + ((c + 1) & 1), (uint32_t)((c + 1) >> 1) & 1u);
@@ -810,9 +842,17 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
                 const int j0 = 64 * half + 32 * jj;
                 float v[32];
                 tmem_ld32(tm + lane_off + TM_S + j0, v);
-                stage_state(v, j0, eL);
+                stage_bf16(v, j0);
             }
             publish(bar_sready);
+#pragma unroll 1
+            for (int jj = 0; jj < 2; ++jj) {
+                const int j0 = 64 * half + 32 * jj;
+                float v[32];
+                tmem_ld32(tm + lane_off + TM_S + j0, v);
+                stage_scaled(v, j0, eL);
+            }
+            publish(bar_scaled);
         }
         state_ok = ok && n_chunks > 0 && c == n_chunks;
         if (n_chunks > 0 && !state_ok && lane == 0) fail();
@@ -850,8 +890,8 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
             const int L = chunk_len(c);
             uint2 zn[8];
             if (zg) load_z(c + 1, zn);
-            bool ok = mbar_wait(bar_oready + b, (uint32_t)(c >> 1) & 1u, kWaitNs) &&
-                      mbar_wait(bar_sc + b, (uint32_t)(c >> 1) & 1u, kWaitNs);  // (long landed)
+            bool ok = mbar_wait(bar_oready + b, (uint32_t)(c >> 1) & 1u, wait_ns) &&
+                      mbar_wait(bar_sc + b, (uint32_t)(c >> 1) & 1u, wait_ns);  // (long landed)
             if (ok) {
                 // O^T [i][r] = (m e^gamma)_r (S Q^T) + (P Delta)^T, staged as O [r][i].
                 fence_after_sync();

@@ -39,26 +39,6 @@ __device__ __forceinline__ uint32_t w_off(int j, int r) {
     return (uint32_t)((r >> 3) * 2048 + (j >> 3) * 128 + (j & 7) * 16 + (r & 7) * 2);
 }
 
-// D (+)= A B, `ksteps` bf16 instructions of K = 16, advancing A and B by the
-// given byte steps.
-__device__ __forceinline__ void gemm(uint32_t d, uint32_t a, uint32_t a_lbo, uint32_t a_sbo,
-                                     uint32_t a_step, uint32_t b, uint32_t b_lbo, uint32_t b_sbo,
-                                     uint32_t b_step, int ksteps, uint32_t idesc, bool acc) {
-    for (int kk = 0; kk < ksteps; ++kk)
-        mma<Kind::BF16>(d, smem_desc(a + kk * a_step, a_lbo, a_sbo),
-                        smem_desc(b + kk * b_step, b_lbo, b_sbo), idesc, (acc || kk > 0) ? 1u : 0u);
-}
-
-// The same with A in tensor memory (see mma_ta): `ksteps` instructions of
-// K = 16, A advancing 8 columns a step.
-__device__ __forceinline__ void gemm_ta(uint32_t d, uint32_t a_tmem, uint32_t b, uint32_t b_lbo,
-                                        uint32_t b_sbo, uint32_t b_step, int ksteps, uint32_t idesc,
-                                        bool acc) {
-    for (int kk = 0; kk < ksteps; ++kk)
-        mma_ta(d, a_tmem + 8 * kk, smem_desc(b + kk * b_step, b_lbo, b_sbo), idesc,
-               (acc || kk > 0) ? 1u : 0u);
-}
-
 // z * sigmoid(z) with the fast exponential (relative error ~1e-7 here).
 __device__ __forceinline__ float fast_silu(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
@@ -92,13 +72,11 @@ __device__ __forceinline__ void split8(const float *v, uint4 &hi, uint4 &lo) {
 
 // One distance of the blocked triangular inverse: for every pair of 16-blocks
 // (i, j) with i - j = DIST, X = A[i-rows][16j .. 16i) T[16j .. 16i)[j-cols],
-// then T_ij = -T_ii X.  Fully unrolled so the shared-memory loads overlap; with
-// a row stride LD that keeps rows 16-byte aligned, the row operand is read four
-// values at a time.
+// then T_ij = -T_ii X.  One output per thread, fully unrolled so the
+// shared-memory loads overlap; for row strides that are not 16-byte aligned.
 template <int DIST, int NT, int LD>
 __device__ __forceinline__ void offdiag_stage(const float *Ascr, float *Tscr, float *Xscr, int tid) {
     constexpr int NBLK = 4 - DIST, NOUT = NBLK * 256;
-    constexpr bool VEC = LD % 4 == 0;
 #pragma unroll
     for (int e0 = 0; e0 < NOUT; e0 += NT) {
         const int e = e0 + tid;
@@ -107,19 +85,8 @@ __device__ __forceinline__ void offdiag_stage(const float *Ascr, float *Tscr, fl
             const float *arow = Ascr + (16 * i + rr) * LD + 16 * j;
             const float *tcol = Tscr + 16 * j * LD + 16 * j + cc;
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
-            if constexpr (VEC) {
 #pragma unroll
-                for (int k4 = 0; k4 < 4 * DIST; ++k4) {
-                    const float4 a = *reinterpret_cast<const float4 *>(arow + 4 * k4);
-                    acc[0] = fmaf(a.x, tcol[(4 * k4) * LD], acc[0]);
-                    acc[1] = fmaf(a.y, tcol[(4 * k4 + 1) * LD], acc[1]);
-                    acc[2] = fmaf(a.z, tcol[(4 * k4 + 2) * LD], acc[2]);
-                    acc[3] = fmaf(a.w, tcol[(4 * k4 + 3) * LD], acc[3]);
-                }
-            } else {
-#pragma unroll
-                for (int k = 0; k < 16 * DIST; ++k) acc[k & 3] = fmaf(arow[k], tcol[k * LD], acc[k & 3]);
-            }
+            for (int k = 0; k < 16 * DIST; ++k) acc[k & 3] = fmaf(arow[k], tcol[k * LD], acc[k & 3]);
             Xscr[e] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
         }
     }
@@ -132,25 +99,67 @@ __device__ __forceinline__ void offdiag_stage(const float *Ascr, float *Tscr, fl
             const float *trow = Tscr + (16 * i + rr) * LD + 16 * i;
             const float *xcol = Xscr + (j << 8) + cc;
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
-            if constexpr (VEC) {
 #pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) {
-                    const float4 t = *reinterpret_cast<const float4 *>(trow + 4 * k4);
-                    acc[0] = fmaf(t.x, xcol[(4 * k4) * 16], acc[0]);
-                    acc[1] = fmaf(t.y, xcol[(4 * k4 + 1) * 16], acc[1]);
-                    acc[2] = fmaf(t.z, xcol[(4 * k4 + 2) * 16], acc[2]);
-                    acc[3] = fmaf(t.w, xcol[(4 * k4 + 3) * 16], acc[3]);
-                }
-            } else {
-#pragma unroll
-                for (int k = 0; k < 16; ++k) acc[k & 3] = fmaf(trow[k], xcol[k * 16], acc[k & 3]);
-            }
+            for (int k = 0; k < 16; ++k) acc[k & 3] = fmaf(trow[k], xcol[k * 16], acc[k & 3]);
             Tscr[(16 * i + rr) * LD + 16 * j + cc] = -((acc[0] + acc[1]) + (acc[2] + acc[3]));
         }
     }
     __syncthreads();
 }
 
+// The same distance stage with 16-byte aligned rows (LD % 4 == 0): each thread
+// computes a strip of four adjacent outputs, so every operand load is a
+// 16-byte vector that feeds four (row operand) or sixteen (column operand)
+// FMAs instead of one.  X is kept as dense 16 x 16 blocks.
+template <int DIST, int NT, int LD>
+__device__ __forceinline__ void offdiag_stage_strips(const float *Ascr, float *Tscr, float *Xscr,
+                                                     int tid) {
+    static_assert(LD % 4 == 0, "rows must be 16-byte aligned");
+    constexpr int NSTRIP = (4 - DIST) * 64;  // 16 rows x 4 strips per block pair
+    for (int e = tid; e < NSTRIP; e += NT) {
+        const int j = e >> 6, i = j + DIST, rr = (e >> 2) & 15, c4 = 4 * (e & 3);
+        const float *arow = Ascr + (16 * i + rr) * LD + 16 * j;
+        const float *tcol = Tscr + 16 * j * LD + 16 * j + c4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k4 = 0; k4 < 4 * DIST; ++k4) {
+            const float4 a = *reinterpret_cast<const float4 *>(arow + 4 * k4);
+            const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float4 t = *reinterpret_cast<const float4 *>(tcol + (4 * k4 + u) * LD);
+                acc.x = fmaf(av[u], t.x, acc.x);
+                acc.y = fmaf(av[u], t.y, acc.y);
+                acc.z = fmaf(av[u], t.z, acc.z);
+                acc.w = fmaf(av[u], t.w, acc.w);
+            }
+        }
+        *reinterpret_cast<float4 *>(Xscr + (j << 8) + rr * 16 + c4) = acc;
+    }
+    __syncthreads();
+    for (int e = tid; e < NSTRIP; e += NT) {
+        const int j = e >> 6, i = j + DIST, rr = (e >> 2) & 15, c4 = 4 * (e & 3);
+        const float *trow = Tscr + (16 * i + rr) * LD + 16 * i;
+        const float *xblk = Xscr + (j << 8) + c4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+            const float4 t = *reinterpret_cast<const float4 *>(trow + 4 * k4);
+            const float tv[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float4 x = *reinterpret_cast<const float4 *>(xblk + (4 * k4 + u) * 16);
+                acc.x = fmaf(tv[u], x.x, acc.x);
+                acc.y = fmaf(tv[u], x.y, acc.y);
+                acc.z = fmaf(tv[u], x.z, acc.z);
+                acc.w = fmaf(tv[u], x.w, acc.w);
+            }
+        }
+        *reinterpret_cast<float4 *>(Tscr + (16 * i + rr) * LD + 16 * j + c4) =
+            make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+    }
+    __syncthreads();
+}
 
 // T = (I + A)^{-1} for the strictly lower-triangular 64 x 64 A in Ascr (fp32,
 // row stride LD), blocked by 16.  Diagonal blocks first, one column per
@@ -179,9 +188,15 @@ __device__ __forceinline__ void invert_unit_lower(const float *Ascr, float *Tscr
         }
     }
     __syncthreads();
-    offdiag_stage<1, NT, LD>(Ascr, Tscr, Xscr, tid);
-    offdiag_stage<2, NT, LD>(Ascr, Tscr, Xscr, tid);
-    offdiag_stage<3, NT, LD>(Ascr, Tscr, Xscr, tid);
+    if constexpr (LD % 4 == 0) {
+        offdiag_stage_strips<1, NT, LD>(Ascr, Tscr, Xscr, tid);
+        offdiag_stage_strips<2, NT, LD>(Ascr, Tscr, Xscr, tid);
+        offdiag_stage_strips<3, NT, LD>(Ascr, Tscr, Xscr, tid);
+    } else {
+        offdiag_stage<1, NT, LD>(Ascr, Tscr, Xscr, tid);
+        offdiag_stage<2, NT, LD>(Ascr, Tscr, Xscr, tid);
+        offdiag_stage<3, NT, LD>(Ascr, Tscr, Xscr, tid);
+    }
 }
 
 }  // namespace tcp

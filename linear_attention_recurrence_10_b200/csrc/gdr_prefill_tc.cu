@@ -514,9 +514,7 @@ __global__ void lpt_order_kernel(const int32_t *cu, int n_seq, int *order, int *
 
 }  // namespace tcp
 
-size_t prefill_tc_workspace_bytes(int n_seq) {
-    return (size_t)(16 + 4 * (size_t)n_seq + 255) & ~(size_t)255;
-}
+size_t prefill_tc_workspace_bytes(int n_seq) { return prefill_tc_ws_bytes(n_seq); }
 
 cudaError_t launch_prefill_tc(const PrefillParams &p, void *workspace, int out_bf16,
                               cudaStream_t s) {

@@ -36,15 +36,15 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
     return d;
 }
 
-enum class Kind { BF16, TF32 };
+enum class Kind { BF16 };
 
-// Instruction descriptor for kind::f16 (bf16 inputs) and kind::tf32, fp32 accumulate.
+// Instruction descriptor for kind::f16 with bf16 inputs, fp32 accumulate.
 template <Kind K>
 __host__ __device__ constexpr uint32_t instr_desc(int M, int N, bool a_mn_major, bool b_mn_major,
                                                   bool negate_a = false) {
     return (1u << 4)                                      // D: fp32
-           | ((K == Kind::BF16 ? 1u : 2u) << 7)           // A format: bf16 = 1, tf32 = 2
-           | ((K == Kind::BF16 ? 1u : 2u) << 10)          // B format
+           | (1u << 7)                                    // A format: bf16
+           | (1u << 10)                                   // B format: bf16
            | ((negate_a ? 1u : 0u) << 13)
            | ((a_mn_major ? 1u : 0u) << 15)
            | ((b_mn_major ? 1u : 0u) << 16)
@@ -58,17 +58,11 @@ __host__ __device__ constexpr uint32_t instr_desc(int M, int N, bool a_mn_major,
 template <Kind K>
 __device__ __forceinline__ void mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                     uint32_t idesc, uint32_t accumulate) {
-    if constexpr (K == Kind::BF16) {
-        asm volatile(
-            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-            "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
-    } else {
-        asm volatile(
-            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-            "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-            "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
-    }
+    static_assert(K == Kind::BF16, "bf16 operands only");
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 
 // D[tmem] (+)= A[tmem] * B[smem] (kind::f16): A is M rows in M TMEM lanes, its
@@ -80,6 +74,26 @@ __device__ __forceinline__ void mma_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+
+// D (+)= A B, `ksteps` bf16 instructions of K = 16, advancing A and B by the
+// given byte steps.
+__device__ __forceinline__ void gemm(uint32_t d, uint32_t a, uint32_t a_lbo, uint32_t a_sbo,
+                                     uint32_t a_step, uint32_t b, uint32_t b_lbo, uint32_t b_sbo,
+                                     uint32_t b_step, int ksteps, uint32_t idesc, bool acc) {
+    for (int kk = 0; kk < ksteps; ++kk)
+        mma<Kind::BF16>(d, smem_desc(a + kk * a_step, a_lbo, a_sbo),
+                        smem_desc(b + kk * b_step, b_lbo, b_sbo), idesc, (acc || kk > 0) ? 1u : 0u);
+}
+
+// The same with A in tensor memory (see mma_ta): `ksteps` instructions of
+// K = 16, A advancing 8 columns a step.
+__device__ __forceinline__ void gemm_ta(uint32_t d, uint32_t a_tmem, uint32_t b, uint32_t b_lbo,
+                                        uint32_t b_sbo, uint32_t b_step, int ksteps, uint32_t idesc,
+                                        bool acc) {
+    for (int kk = 0; kk < ksteps; ++kk)
+        mma_ta(d, a_tmem + 8 * kk, smem_desc(b + kk * b_step, b_lbo, b_sbo), idesc,
+               (acc || kk > 0) ? 1u : 0u);
 }
 
 // Arrive on an mbarrier once all tcgen05 work issued so far by this thread is done.
@@ -312,13 +326,6 @@ __device__ __forceinline__ bool group_sync_or(int id, int n, bool pred) {
         : "r"((uint32_t)pred), "r"(id), "r"(n)
         : "memory");
     return r != 0;
-}
-
-// fp32 -> tf32 (round to nearest, ties away), kept in a 32-bit container.
-__device__ __forceinline__ float to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return __uint_as_float(r);
 }
 
 }  // namespace tc

@@ -11,7 +11,7 @@ import pytest
 import torch
 
 import linear_attention_recurrence_10_b200 as gdr
-from gdr_testutil import TOL, f64, oracle_full, rel_l2, run_decode
+from gdr_testutil import TOL, f64, oracle_full, assert_close, rel_l2, run_decode
 from linear_attention_recurrence_10_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -41,8 +41,8 @@ def test_matches_oracle(T, dtype, heads, d):
     ref = oracle_full(inp)
     out, state = run_multi(inp, T)
     tol = TOL[dtype]
-    assert rel_l2(f64(out), ref.y) <= tol["out"]
-    assert rel_l2(f64(state), ref.state) <= tol["state"]
+    assert_close(f64(out), ref.y, tol["out"])
+    assert_close(f64(state), ref.state, tol["state"])
 
 
 @pytest.mark.parametrize("T", [2, 5, 8])
@@ -70,8 +70,8 @@ def test_state_slots_gather_and_scatter():
     slots = torch.tensor(slot_of, dtype=torch.int32, device="cuda")
     out, pool_after = run_multi(inp, T, state=pool_state, slots=slots)
     ref = oracle_full(inp)
-    assert rel_l2(f64(out), ref.y) <= 2e-3
-    assert rel_l2(f64(pool_after[slots.long()]), ref.state) <= 1e-3
+    assert_close(f64(out), ref.y, 2e-3)
+    assert_close(f64(pool_after[slots.long()]), ref.state, 1e-3)
     untouched = [s for s in range(pool) if s not in slot_of]
     assert torch.equal(pool_after[untouched], before[untouched])
 
@@ -92,8 +92,8 @@ def test_bad_slot_reports_and_leaves_its_sequence_alone():
     ref = oracle_full(inp)
     good = [0, 1, 3]
     rows = np.concatenate([np.arange(b * T, (b + 1) * T) for b in good])
-    assert rel_l2(f64(out[rows]), ref.y[rows]) <= 1e-5
-    assert rel_l2(f64(pool_after[good]), ref.state[good]) <= 1e-5
+    assert_close(f64(out[rows]), ref.y[rows], 1e-5)
+    assert_close(f64(pool_after[good]), ref.state[good], 1e-5)
 
 
 def test_many_sequences_full_size():
@@ -102,5 +102,5 @@ def test_many_sequences_full_size():
     inp = synth.make_inputs([T] * 32, 16, 16, 128, seed=440, dtype=torch.bfloat16, s0_std=0.02)
     ref = oracle_full(inp, threads=16)
     out, state = run_multi(inp, T)
-    assert rel_l2(f64(out), ref.y) <= 2e-3
-    assert rel_l2(f64(state), ref.state) <= 1e-3
+    assert_close(f64(out), ref.y, 2e-3)
+    assert_close(f64(state), ref.state, 1e-3)

@@ -13,7 +13,7 @@ import torch
 
 import linear_attention_recurrence_10_b200 as gdr
 import oracle
-from gdr_testutil import TOL, f64, rel_l2, run_decode, run_prefill
+from gdr_testutil import TOL, f64, assert_close, rel_l2, run_decode, run_prefill
 from linear_attention_recurrence_10_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -53,8 +53,8 @@ def test_decode(dtype):
     raw, _, params, g, beta = raw_gate_problem([T] * 5, 2, 4, 128, 600, dtype)
     ref = oracle_ref(raw, g, beta)
     out, final = run_decode(raw, T, gate_params=params)
-    assert rel_l2(f64(out), ref.y) <= TOL[dtype]["out"]
-    assert rel_l2(f64(final), ref.state) <= TOL[dtype]["state"]
+    assert_close(f64(out), ref.y, TOL[dtype]["out"])
+    assert_close(f64(final), ref.state, TOL[dtype]["state"])
 
 
 def test_decode_multi():
@@ -67,8 +67,8 @@ def test_decode_multi():
     gdr.decode_multi(x.q, x.k, x.v, x.g, x.beta, state, out, n_tokens=T, z=x.z, norm_w=x.w,
                      gate_params=params)
     torch.cuda.synchronize()
-    assert rel_l2(f64(out), ref.y) <= 2e-3
-    assert rel_l2(f64(state), ref.state) <= 1e-3
+    assert_close(f64(out), ref.y, 2e-3)
+    assert_close(f64(state), ref.state, 1e-3)
 
 
 @pytest.mark.parametrize("path", ["two_kernel", "one_kernel", "cuda_cores"])
@@ -83,8 +83,8 @@ def test_prefill(path):
         ws = torch.empty((16 + 4 * len(lens) + 255) // 256 * 256, dtype=torch.uint8, device="cuda")
     out, final = run_prefill(raw, chunk=64 if path != "cuda_cores" else 32, workspace=ws,
                              gate_params=params)
-    assert rel_l2(f64(out), ref.y) <= TOL[dtype]["out"]
-    assert rel_l2(f64(final), ref.state) <= TOL[dtype]["state"]
+    assert_close(f64(out), ref.y, TOL[dtype]["out"])
+    assert_close(f64(final), ref.state, TOL[dtype]["state"])
 
 
 def test_raw_matches_precomputed_gates_on_device():
@@ -93,5 +93,5 @@ def test_raw_matches_precomputed_gates_on_device():
     raw, gated, params, _, _ = raw_gate_problem([64, 33], 2, 2, 128, 620, torch.bfloat16)
     out_r, fin_r = run_prefill(raw, gate_params=params)
     out_g, fin_g = run_prefill(gated)
-    assert rel_l2(f64(out_r), f64(out_g)) <= 1e-5
-    assert rel_l2(f64(fin_r), f64(fin_g)) <= 1e-5
+    assert_close(f64(out_r), f64(out_g), 1e-5)
+    assert_close(f64(fin_r), f64(fin_g), 1e-5)

@@ -6,7 +6,7 @@ import torch
 
 import linear_attention_recurrence_10_b200 as gdr
 import oracle
-from gdr_testutil import f64, rel_l2
+from gdr_testutil import f64, assert_close, rel_l2
 from linear_attention_recurrence_10_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -24,12 +24,12 @@ def test_norm(d, o_dtype, z_dtype):
     out = torch.empty(rows, d, device="cuda")
     gdr.rmsnorm_gated(o.cuda(), z.cuda(), out, w=w.cuda(), eps=1e-6)
     torch.cuda.synchronize()
-    assert rel_l2(f64(out), want) <= 1e-6
+    assert_close(f64(out), want, 1e-6)
     out16 = torch.empty(rows, d, device="cuda", dtype=torch.bfloat16)
     gdr.rmsnorm_gated(o.cuda(), z.cuda(), out16, w=w.cuda(), eps=1e-6)
     torch.cuda.synchronize()
     want16 = torch.from_numpy(want).to(torch.bfloat16).double().numpy()
-    assert rel_l2(f64(out16), want16) <= 2e-3
+    assert_close(f64(out16), want16, 2e-3, bf16_ulp=True)
 
 
 def test_norm_in_place_and_no_weight():
@@ -38,7 +38,7 @@ def test_norm_in_place_and_no_weight():
     want = oracle.rmsnorm_gated(f64(o).reshape(-1, 128), f64(z).reshape(-1, 128), None, eps=1e-5)
     gdr.rmsnorm_gated(o, z, o, eps=1e-5)
     torch.cuda.synchronize()
-    assert rel_l2(f64(o).reshape(-1, 128), want) <= 1e-6
+    assert_close(f64(o).reshape(-1, 128), want, 1e-6)
 
 
 def test_norm_empty():

@@ -11,15 +11,18 @@
 // In host code `g_prefill_scratch` names a host-side stand-in, not a device
 // address.  Its device address is looked up once per device, with that device
 // current, through cudaGetSymbolAddress; the prefill kernels only ever see
-// that address.
+// that address.  The lookup is cached per device index for the life of the
+// process: it belongs to the device's primary context, so callers that reset
+// the device (cudaDeviceReset) or run in a context of their own are not
+// served by this entry point.
 #include <mutex>
 
 #include "gdr.h"
+#include "gdr_common.cuh"
 
 namespace {
 
-constexpr size_t kScratchBytes =
-    ((16 + 4 * (size_t)GDR_PREFILL_NOALLOC_MAX_SEQS) + 255) & ~(size_t)255;
+constexpr size_t kScratchBytes = gdr::prefill_tc_ws_bytes(GDR_PREFILL_NOALLOC_MAX_SEQS);
 
 static __device__ __align__(256) unsigned char g_prefill_scratch[kScratchBytes];
 
@@ -44,6 +47,13 @@ void *scratch_on_current_device() {
     return g_scratch_addr[dev];
 }
 
+// The calls that run on the tensor cores write the scratch status word; the
+// others (CUDA-core shapes, no sequences) leave it alone.
+bool writes_status_word(const gdr_prefill_args *a) {
+    return a->n_seq > 0 && a->in_dtype == GDR_BF16 && a->d_k == 128 &&
+           (a->chunk == 0 || a->chunk == 64);
+}
+
 }  // namespace
 
 extern "C" gdr_status gdr_prefill_chunked_noalloc(const gdr_prefill_args *args,
@@ -55,5 +65,24 @@ extern "C" gdr_status gdr_prefill_chunked_noalloc(const gdr_prefill_args *args,
     // Everything the kernels read from the scratch is written first by the same
     // call (the status word is cleared and the sequence order rebuilt), so the
     // previous call's contents never leak into this one.
-    return gdr_prefill_chunked(args, scratch, kScratchBytes, stream);
+    const gdr_status st = gdr_prefill_chunked(args, scratch, kScratchBytes, stream);
+    if (st != GDR_OK || writes_status_word(args)) return st;
+    // A call that does not write the status word still leaves it reading 0.
+    if (cudaMemsetAsync(scratch, 0, sizeof(int32_t), (cudaStream_t)stream) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return GDR_ERR_CUDA;
+    }
+    return GDR_OK;
+}
+
+extern "C" gdr_status gdr_prefill_noalloc_status(int32_t *status, gdr_stream_t stream) {
+    if (!status) return GDR_ERR_INVALID_ARG;
+    void *scratch = scratch_on_current_device();
+    if (!scratch) return GDR_ERR_CUDA;
+    if (cudaMemcpyAsync(status, scratch, sizeof(int32_t), cudaMemcpyDefault,
+                        (cudaStream_t)stream) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return GDR_ERR_CUDA;
+    }
+    return GDR_OK;
 }

@@ -31,6 +31,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "gdr_oracle.c")
 # The gated full-attention decode step (the other mixer of the hybrid decoder).
 _SRC_ATTN = os.path.join(_HERE, "gattn_oracle.c")
+# The routed-expert MoE feed-forward block.
+_SRC_MOE = os.path.join(_HERE, "moe_oracle.c")
 
 
 def _host_key() -> str:
@@ -82,12 +84,21 @@ class _AttnProblem(ctypes.Structure):
     ]
 
 
+class _MoeProblem(ctypes.Structure):
+    _fields_ = [
+        ("n_tok", ctypes.c_int32), ("hidden", ctypes.c_int32), ("n_exp", ctypes.c_int32),
+        ("top_k", ctypes.c_int32), ("inter", ctypes.c_int32), ("s_inter", ctypes.c_int32),
+        ("x", _DP), ("w_router", _DP), ("w_gate", _DP), ("w_up", _DP), ("w_down", _DP),
+        ("ws_gate", _DP), ("ws_up", _DP), ("ws_down", _DP), ("w_sgate", _DP),
+    ]
+
+
 def build(src: str = _SRC, out: str = _LIB, force: bool = False, werror: bool = True,
-          attn_src: str = _SRC_ATTN) -> str:
+          attn_src: str = _SRC_ATTN, moe_src: str = _SRC_MOE) -> str:
     """Compile the oracle with the host C compiler: -O3 -march=native, ISO C11 (so
     no floating-point contraction or reassociation: the same arithmetic as any
     other build, only faster).  The file name carries the host's CPU key."""
-    srcs = [src, attn_src]
+    srcs = [src, attn_src, moe_src]
     if not force and os.path.exists(out) and all(
             os.path.getmtime(out) >= os.path.getmtime(f) for f in srcs):
         return out
@@ -130,6 +141,11 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.orc_rope_partial.restype = None
     lib.orc_gated_attn_decode.argtypes = [ctypes.POINTER(_AttnProblem), _DP, _DP, _DP]
     lib.orc_gated_attn_decode.restype = ctypes.c_int
+    ip = ctypes.POINTER(ctypes.c_int32)
+    lib.orc_moe_route.argtypes = [ctypes.POINTER(_MoeProblem), _DP, ip, _DP]
+    lib.orc_moe_route.restype = None
+    lib.orc_moe_forward.argtypes = [ctypes.POINTER(_MoeProblem), ip, _DP, _DP]
+    lib.orc_moe_forward.restype = ctypes.c_int
     _lib_cache[path] = lib
     return lib
 
@@ -295,3 +311,64 @@ def gated_attn_decode(q, gate, k, v, k_cache, v_cache, cache_len, *, rot_dim, th
     if (lib or load()).orc_gated_attn_decode(ctypes.byref(p), _ptr(y), _ptr(o), _ptr(kr)):
         raise ValueError("invalid shape or a full cache")
     return AttnResult(y, o, kr)
+
+
+# ------------------------------------------------------- routed-expert MoE
+
+@dataclass
+class MoeRoute:
+    probs: np.ndarray    # [n_tok, n_exp] softmax of the router logits
+    idx: np.ndarray      # [n_tok, top_k] int32, experts in decreasing probability
+    w: np.ndarray        # [n_tok, top_k] renormalised weights
+
+
+def _moe_problem(x, w_router, w_gate, w_up, w_down, top_k, shared):
+    x = _f64(x)
+    n_tok, H = x.shape
+    w_router = _f64(w_router)
+    E = w_router.shape[0]
+    w_gate = _f64(w_gate); w_up = _f64(w_up, w_gate.shape)
+    I = w_gate.shape[1]
+    w_down = _f64(w_down, (E, H, I))
+    if shared is not None:
+        ws_gate, ws_up, ws_down, w_sgate = (_f64(a) for a in shared)
+        SI = ws_gate.shape[0]
+    else:
+        ws_gate = ws_up = ws_down = w_sgate = None
+        SI = 0
+    keep = (x, w_router, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, w_sgate)
+    p = _MoeProblem(n_tok, H, E, int(top_k), I, SI, _ptr(x), _ptr(w_router), _ptr(w_gate),
+                    _ptr(w_up), _ptr(w_down), _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down),
+                    _ptr(w_sgate))
+    return p, keep, (n_tok, H, E)
+
+
+def moe_route(x, w_router, top_k, lib: ctypes.CDLL | None = None) -> MoeRoute:
+    """Router probabilities, top-k experts and renormalised weights per token."""
+    E, H = np.shape(w_router)
+    dummy = np.zeros((E, 1, H))
+    p, keep, (n_tok, H, E) = _moe_problem(x, w_router, dummy, dummy, np.zeros((E, H, 1)),
+                                          top_k, None)
+    probs = np.zeros((n_tok, E)); w = np.zeros((n_tok, top_k))
+    idx = np.zeros((n_tok, top_k), dtype=np.int32)
+    (lib or load()).orc_moe_route(ctypes.byref(p), _ptr(probs),
+                                  idx.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), _ptr(w))
+    del keep
+    return MoeRoute(probs, idx, w)
+
+
+def moe_forward(x, w_router, w_gate, w_up, w_down, idx, w, *, shared=None,
+                lib: ctypes.CDLL | None = None) -> np.ndarray:
+    """The MoE block's output [n_tok, hidden] for the routing (idx, w):
+    sum_k w_k SwitchGLU_{idx_k}(x) + sigmoid(w_sgate . x) SwitchGLU_shared(x);
+    shared = (ws_gate, ws_up, ws_down, w_sgate) or None."""
+    idx = np.ascontiguousarray(np.asarray(idx, dtype=np.int32))
+    w = _f64(w, idx.shape)
+    p, keep, (n_tok, H, E) = _moe_problem(x, w_router, w_gate, w_up, w_down, idx.shape[1], shared)
+    y = np.zeros((n_tok, H))
+    if (lib or load()).orc_moe_forward(ctypes.byref(p),
+                                       idx.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                                       _ptr(w), _ptr(y)):
+        raise ValueError("expert index out of range")
+    del keep
+    return y

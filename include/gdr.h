@@ -278,10 +278,55 @@ gdr_status gdr_prefill_chunked(const gdr_prefill_args *args, void *workspace,
  *   ordering between them) race on it and must not be made.  Each call
  *   rewrites everything it reads from the array before reading it, so
  *   results never depend on an earlier call.
+ *   The looked-up address belongs to the device's primary context and is kept
+ *   for the life of the process: after cudaDeviceReset, or from a context the
+ *   caller created itself, this entry point must not be used.
+ *   The array's first 4 bytes are the status word gdr_prefill_chunked writes
+ *   to its workspace; gdr_prefill_noalloc_status reads it back.
  * ------------------------------------------------------------------------ */
 #define GDR_PREFILL_NOALLOC_MAX_SEQS 4096
 
 gdr_status gdr_prefill_chunked_noalloc(const gdr_prefill_args *args, gdr_stream_t stream);
+
+/* Queue on `stream` a copy of the current device's status word of
+ * gdr_prefill_chunked_noalloc (an int32: 0, or GDR_ERR_TIMEOUT if a bounded
+ * device-side wait of the last call on this device gave up, its outputs then
+ * being incomplete) into `status`, which may be device memory or host memory
+ * (with pageable host memory the copy completes before the call returns).
+ * Read it once the prefill's work on the stream has finished.  Like the
+ * prefill, it has no counterpart in the pages and allocates nothing.
+ * Returns GDR_ERR_INVALID_ARG for a NULL `status`, GDR_ERR_CUDA if the copy
+ * cannot be queued. */
+gdr_status gdr_prefill_noalloc_status(int32_t *status, gdr_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Diagnostics: the expiry path of the prefill's bounded device waits.
+ *
+ * The pages have no counterpart; this exists so that a test can watch the
+ * failure handling of the tensor-core prefill without faulting or hanging a
+ * GPU.  Every device-side wait of that prefill gives up after a deadline,
+ * records GDR_ERR_TIMEOUT in the workspace status word, waits (again bounded)
+ * for its own copies in flight, frees its tensor memory and returns.  This
+ * call runs gdr_prefill_chunked's two-kernel tensor-core path with the
+ * recurrence's waits limited to `wait_ns` nanoseconds and each (sequence,
+ * value head)'s first key tile never delivered, so those waits run out:
+ * once the work has finished, the status word reads GDR_ERR_TIMEOUT, the
+ * outputs and final states are incomplete (unspecified), and the device is
+ * left usable for the calls that follow.
+ *
+ *   args, workspace, workspace_bytes: as for gdr_prefill_chunked; the shape
+ *   must take the tensor-core path (else GDR_ERR_UNSUPPORTED) with a
+ *   workspace of at least gdr_prefill_workspace_size() bytes (else
+ *   GDR_ERR_WORKSPACE), and n_seq >= 1.
+ *   wait_ns in [GDR_SELFTEST_MIN_WAIT_NS, GDR_SELFTEST_MAX_WAIT_NS], else
+ *   GDR_ERR_INVALID_ARG.
+ * ------------------------------------------------------------------------ */
+#define GDR_SELFTEST_MIN_WAIT_NS 100000ull      /* 0.1 ms */
+#define GDR_SELFTEST_MAX_WAIT_NS 2000000000ull  /* 2 s, the ordinary limit */
+
+gdr_status gdr_prefill_selftest_wait_expiry(const gdr_prefill_args *args, void *workspace,
+                                            size_t workspace_bytes, uint64_t wait_ns,
+                                            gdr_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * RMSNormGated on its own (the output gate of the mixer; Qwen3.5 Chat guide,
@@ -308,6 +353,113 @@ typedef struct gdr_norm_args {
 } gdr_norm_args;
 
 gdr_status gdr_rmsnorm_gated(const gdr_norm_args *args, gdr_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * One decode step of the gated full-attention layer: the other mixer of the
+ * hybrid decoder, one layer in four (Qwen3.5 Chat guide, "Architektur":
+ * GatedAttention layers, standard scaled-dot-product attention over a KV
+ * cache; Core AI card for Qwen3.6-35B-A3B, first section: head_dim 256,
+ * 16 query heads over 2 key/value heads, partial rotary embedding with
+ * theta = 1e7).  For every sequence b, with L = cache_len[b] tokens cached
+ * before this step and kv head g = floor(h * H_kv / H_q) of query head h:
+ *
+ *     q_rot, k_rot = RoPE(q, L), RoPE(k, L): the first rot_dim dims turned in
+ *                    pairs (i, i + rot_dim/2) by L * theta^(-2i/rot_dim)
+ *     cache[b, g, L] = (k_rot, v)                              (appended)
+ *     o_h = sum_{t <= L} softmax_t(scale * q_rot_h . k_cache[t]) v_cache[t]
+ *     y_h = o_h * sigmoid(gate_h)                              (elementwise)
+ *
+ * For text tokens the three position components of mRoPE coincide, which
+ * makes it this one-dimensional rotation.  The new key is stored and
+ * attended as bf16, like every cached key.
+ *
+ *   q, gate    [batch, H_q, d]  bf16   row strides q_stride, gate_stride
+ *   k, v       [batch, H_kv, d] bf16   row strides k_stride, v_stride
+ *   k_cache, v_cache  [batch, H_kv, max_len, d] bf16, packed; row L of each
+ *              (b, g) is written by this call, rows < L are read.
+ *   cache_len  device int32 [batch]; read, not updated (the caller advances it)
+ *   kv_bound   host: an upper bound of cache_len over the batch, < max_len;
+ *              it sizes the split of the work.  A cache_len outside
+ *              [0, kv_bound] is not attended past kv_bound, is not appended
+ *              and sets the status word to GDR_ERR_INVALID_ARG.
+ *   out        [batch, H_q, d] out_dtype, row stride out_stride
+ *   rot_dim    even, 0 .. d (64 in the Qwen3.5 / 3.6 layers); rope_theta;
+ *   scale      multiplies q.k (d^-1/2 for standard attention)
+ *   Supported: d = 256, H_q a multiple of H_kv with H_q / H_kv <= 16.
+ *   batch == 0 is a no-op.
+ *   workspace: device memory, 16-byte aligned, of gdr_attn_decode_workspace_size
+ *   bytes (per-split partial results); its first 4 bytes (int32) hold, once
+ *   the work has finished, 0, GDR_ERR_INVALID_ARG (a cache_len out of range)
+ *   or GDR_ERR_TIMEOUT (a bounded device-side wait gave up; outputs incomplete).
+ * ------------------------------------------------------------------------ */
+typedef struct gdr_attn_decode_args {
+    int32_t batch, H_q, H_kv, d;
+    int32_t rot_dim, max_len, kv_bound;
+    int32_t out_dtype;                /* gdr_dtype of out */
+    float rope_theta, scale;
+    int64_t q_stride, gate_stride, k_stride, v_stride, out_stride;
+    const void *q, *gate, *k, *v;
+    void *k_cache, *v_cache;
+    const int32_t *cache_len;
+    void *out;
+} gdr_attn_decode_args;
+
+/* Workspace bytes gdr_attn_decode_step needs for these arguments (only sizes
+ * are read).  Returns the status gdr_attn_decode_step's checks would. */
+gdr_status gdr_attn_decode_workspace_size(const gdr_attn_decode_args *args, size_t *bytes);
+
+gdr_status gdr_attn_decode_step(const gdr_attn_decode_args *args, void *workspace,
+                                size_t workspace_bytes, gdr_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * The routed-expert MoE feed-forward block at decode time (the FFN of the
+ * hybrid decoder's MoE models: Core AI card for Qwen3.6-35B-A3B, first
+ * section -- a router over the experts, an fp32 softmax, the top k
+ * renormalised by their sum, SwitchGLU experts gathered by index, and an
+ * always-on shared SwitchGLU scaled by sigmoid(shared_expert_gate(x)); its
+ * "Speed" section puts a decode step's cost in reading only the routed
+ * experts' weights).  Per token x:
+ *
+ *     p = softmax(W_router x);  top_k experts by p (ties to the lower index)
+ *     w_e = p_e / sum_{top_k} p
+ *     y = sum_e w_e W_down,e (silu(W_gate,e x) * (W_up,e x))
+ *       + sigmoid(w_sgate . x) W_down,s (silu(W_gate,s x) * (W_up,s x))
+ *
+ * Only the experts some token chose are read, each once for all the tokens
+ * that chose it.  bf16 weights and activations, fp32 arithmetic.
+ *
+ *   x          [n_tok, hidden] bf16, row stride x_stride
+ *   w_router   [n_exp, hidden] bf16
+ *   w_gate_up  [n_exp, 2 * inter, hidden] bf16: rows 0 .. inter-1 of an
+ *              expert are its gate matrix, rows inter .. 2 inter - 1 its up
+ *   w_down     [n_exp, hidden, inter] bf16
+ *   ws_gate_up [2 * s_inter, hidden], ws_down [hidden, s_inter], w_sgate
+ *              [hidden] bf16: the shared expert and its gate row; ws_gate_up
+ *              NULL (and s_inter 0) for a block without a shared expert
+ *   out        [n_tok, hidden] out_dtype, row stride out_stride
+ *   topk_idx, topk_w   optional device outputs [n_tok, top_k]: the chosen
+ *              experts (int32, in decreasing probability) and their weights
+ *   Supported: hidden and inter (s_inter) multiples of 8, inter and s_inter
+ *   <= 1024; 1 <= top_k <= 32, top_k <= n_exp <= 1024; n_tok <= 4096.
+ *   n_tok == 0 is a no-op.
+ *   workspace: gdr_moe_workspace_size bytes, 16-byte aligned.
+ * ------------------------------------------------------------------------ */
+typedef struct gdr_moe_args {
+    int32_t n_tok, hidden, n_exp, top_k, inter, s_inter;
+    int32_t out_dtype;                /* gdr_dtype of out */
+    int32_t reserved;                 /* 0 */
+    int64_t x_stride, out_stride;
+    const void *x, *w_router, *w_gate_up, *w_down;
+    const void *ws_gate_up, *ws_down, *w_sgate;
+    void *out;
+    int32_t *topk_idx;
+    float *topk_w;
+} gdr_moe_args;
+
+gdr_status gdr_moe_workspace_size(const gdr_moe_args *args, size_t *bytes);
+
+gdr_status gdr_moe_decode(const gdr_moe_args *args, void *workspace, size_t workspace_bytes,
+                          gdr_stream_t stream);
 
 /* Static, human-readable name of a status (never NULL). */
 const char *gdr_status_string(gdr_status status);

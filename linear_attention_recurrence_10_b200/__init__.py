@@ -9,6 +9,9 @@ kernels.  PyTorch is used for device memory and streams only.
     decode_step(q, k, v, g, beta, state, out, ...)        one token per sequence
     prefill_chunked(q, k, v, g, beta, cu_seqlens, out, ...)  packed varlen prompts
     rmsnorm_gated(o, z, out, ...)                          the output gate alone
+    attn_decode_step(q, gate, k, v, k_cache, v_cache, cache_len, out, ...)
+                                                           gated full-attention decode
+    moe_decode(x, w_router, w_gate_up, w_down, out, ...)    routed-expert MoE block
 """
 from __future__ import annotations
 
@@ -20,7 +23,8 @@ from . import _abi
 from ._abi import GDR_BF16, GDR_F32
 
 __all__ = ["GdrError", "decode_step", "decode_multi", "prefill_chunked", "prefill_chunked_noalloc",
-           "prefill_workspace_size",
+           "prefill_noalloc_status", "prefill_workspace_size", "attn_decode_step",
+           "attn_decode_workspace_size", "moe_decode", "moe_workspace_size",
            "rmsnorm_gated", "version", "status_string"]
 
 
@@ -290,6 +294,19 @@ def prefill_chunked_noalloc(q, k, v, g, beta, cu_seqlens, out, *, cu_seqlens_hos
     return out
 
 
+def prefill_noalloc_status(stream=None) -> int:
+    """The status word of the last prefill_chunked_noalloc call on the current
+    device (gdr_prefill_noalloc_status): 0, or GDR_ERR_TIMEOUT if a bounded
+    device wait gave up.  ``stream``: a torch CUDA stream (default: the current
+    one), which is synchronised, since the value is read back to the host."""
+    s = stream if stream is not None else torch.cuda.current_stream()
+    host = torch.zeros(1, dtype=torch.int32).pin_memory()
+    _check(_abi.lib().gdr_prefill_noalloc_status(host.data_ptr(), ctypes.c_void_p(s.cuda_stream)),
+           "gdr_prefill_noalloc_status")
+    s.synchronize()
+    return int(host.item())
+
+
 def rmsnorm_gated(o, z, out, *, w=None, eps: float = 1e-6, stream=None) -> torch.Tensor:
     """y = o / sqrt(mean(o^2) + eps) * w * z * sigmoid(z) over the last dim (gdr_rmsnorm_gated).
 
@@ -309,4 +326,125 @@ def rmsnorm_gated(o, z, out, *, w=None, eps: float = 1e-6, stream=None) -> torch
     a.o, a.z, a.w, a.out = _ptr(o2), _ptr(z2), _ptr(w), _ptr(out2)
     _check(_abi.lib().gdr_rmsnorm_gated(ctypes.byref(a), _stream(stream, o.device)),
            "gdr_rmsnorm_gated")
+    return out
+
+
+def _attn_args(q, gate, k, v, k_cache, v_cache, cache_len, out, kv_bound, rot_dim, rope_theta,
+               scale):
+    B, H_q, d = q.shape
+    H_kv = k.shape[1]
+    for t, name in ((q, "q"), (gate, "gate"), (k, "k"), (v, "v"), (k_cache, "k_cache"),
+                    (v_cache, "v_cache")):
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be bf16")
+    for t, name in ((k_cache, "k_cache"), (v_cache, "v_cache")):
+        if t.dim() != 4 or t.shape[:2] != (B, H_kv) or t.shape[3] != d or not t.is_contiguous():
+            raise ValueError(f"{name} must be a packed [batch, H_kv, max_len, d] tensor")
+    if cache_len.dtype != torch.int32:
+        raise TypeError("cache_len must be int32")
+    return _abi.AttnDecodeArgs(
+        batch=B, H_q=H_q, H_kv=H_kv, d=d, rot_dim=int(rot_dim), max_len=k_cache.shape[2],
+        kv_bound=int(kv_bound), out_dtype=_dtype_code(out, "out"), rope_theta=float(rope_theta),
+        scale=float(d ** -0.5 if scale is None else scale),
+        q_stride=_row_stride(q, "q"), gate_stride=_row_stride(gate, "gate"),
+        k_stride=_row_stride(k, "k"), v_stride=_row_stride(v, "v"),
+        out_stride=_row_stride(out, "out"), q=_ptr(q), gate=_ptr(gate), k=_ptr(k), v=_ptr(v),
+        k_cache=_ptr(k_cache), v_cache=_ptr(v_cache), cache_len=_ptr(cache_len), out=_ptr(out))
+
+
+def attn_decode_workspace_size(q, gate, k, v, k_cache, v_cache, cache_len, out, *, kv_bound,
+                               rot_dim=64, rope_theta=1e7, scale=None) -> int:
+    a = _attn_args(q, gate, k, v, k_cache, v_cache, cache_len, out, kv_bound, rot_dim,
+                   rope_theta, scale)
+    n = ctypes.c_size_t(0)
+    _check(_abi.lib().gdr_attn_decode_workspace_size(ctypes.byref(a), ctypes.byref(n)),
+           "gdr_attn_decode_workspace_size")
+    return int(n.value)
+
+
+def attn_decode_step(q, gate, k, v, k_cache, v_cache, cache_len, out, *, kv_bound, rot_dim=64,
+                     rope_theta=1e7, scale=None, workspace=None, stream=None) -> torch.Tensor:
+    """One decode step of the gated full-attention layer (gdr_attn_decode_step).
+
+    q, gate [B, H_q, 256]; k, v [B, H_kv, 256] (the new token, bf16);
+    k_cache, v_cache [B, H_kv, max_len, 256] bf16 (row cache_len[b] receives the
+    rotated key and the value); cache_len int32 [B] on the device; ``kv_bound``
+    an upper bound of cache_len on the host; out [B, H_q, 256] bf16 or fp32.
+    ``workspace``: a uint8 device tensor of attn_decode_workspace_size() bytes,
+    allocated here when None.
+    """
+    a = _attn_args(q, gate, k, v, k_cache, v_cache, cache_len, out, kv_bound, rot_dim,
+                   rope_theta, scale)
+    L = _abi.lib()
+    n = ctypes.c_size_t(0)
+    _check(L.gdr_attn_decode_workspace_size(ctypes.byref(a), ctypes.byref(n)),
+           "gdr_attn_decode_workspace_size")
+    if workspace is None and n.value:
+        workspace = torch.empty(int(n.value), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(L.gdr_attn_decode_step(ctypes.byref(a), _ptr(workspace), ws_bytes,
+                                  _stream(stream, q.device)), "gdr_attn_decode_step")
+    return out
+
+
+def _moe_args(x, w_router, w_gate_up, w_down, out, top_k, shared, topk_idx, topk_w):
+    n_tok, H = x.shape
+    E = w_router.shape[0]
+    I = w_gate_up.shape[1] // 2
+    for t, name in ((x, "x"), (w_router, "w_router"), (w_gate_up, "w_gate_up"),
+                    (w_down, "w_down")):
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be bf16")
+    for t, name, shape in ((w_router, "w_router", (E, H)), (w_gate_up, "w_gate_up", (E, 2 * I, H)),
+                           (w_down, "w_down", (E, H, I))):
+        if tuple(t.shape) != shape or not t.is_contiguous():
+            raise ValueError(f"{name} must be a packed {list(shape)} tensor")
+    ws_gate_up = ws_down = w_sgate = None
+    SI = 0
+    if shared is not None:
+        ws_gate_up, ws_down, w_sgate = shared
+        SI = ws_gate_up.shape[0] // 2
+        for t, name, shape in ((ws_gate_up, "ws_gate_up", (2 * SI, H)), (ws_down, "ws_down", (H, SI)),
+                               (w_sgate, "w_sgate", (H,))):
+            if t.dtype != torch.bfloat16 or tuple(t.shape) != shape or not t.is_contiguous():
+                raise ValueError(f"{name} must be a packed bf16 {list(shape)} tensor")
+    if topk_idx is not None and topk_idx.dtype != torch.int32:
+        raise TypeError("topk_idx must be int32")
+    _f32_tensor(topk_w, "topk_w")
+    return _abi.MoeArgs(
+        n_tok=n_tok, hidden=H, n_exp=E, top_k=int(top_k), inter=I, s_inter=SI,
+        out_dtype=_dtype_code(out, "out"), reserved=0,
+        x_stride=_row_stride(x, "x"), out_stride=_row_stride(out, "out"),
+        x=_ptr(x), w_router=_ptr(w_router), w_gate_up=_ptr(w_gate_up), w_down=_ptr(w_down),
+        ws_gate_up=_ptr(ws_gate_up), ws_down=_ptr(ws_down), w_sgate=_ptr(w_sgate), out=_ptr(out),
+        topk_idx=_ptr(topk_idx), topk_w=_ptr(topk_w))
+
+
+def moe_workspace_size(x, w_router, w_gate_up, w_down, out, *, top_k=8, shared=None) -> int:
+    a = _moe_args(x, w_router, w_gate_up, w_down, out, top_k, shared, None, None)
+    n = ctypes.c_size_t(0)
+    _check(_abi.lib().gdr_moe_workspace_size(ctypes.byref(a), ctypes.byref(n)),
+           "gdr_moe_workspace_size")
+    return int(n.value)
+
+
+def moe_decode(x, w_router, w_gate_up, w_down, out, *, top_k=8, shared=None, topk_idx=None,
+               topk_w=None, workspace=None, stream=None) -> torch.Tensor:
+    """The routed-expert MoE block for a decode batch (gdr_moe_decode).
+
+    x [n_tok, hidden] bf16; w_router [n_exp, hidden]; w_gate_up [n_exp, 2*inter,
+    hidden] (gate rows, then up rows); w_down [n_exp, hidden, inter], all bf16;
+    ``shared`` = (ws_gate_up [2*s_inter, hidden], ws_down [hidden, s_inter],
+    w_sgate [hidden]) bf16 or None; out [n_tok, hidden] bf16 or fp32;
+    ``topk_idx`` (int32) / ``topk_w`` (fp32) [n_tok, top_k] receive the routing.
+    """
+    a = _moe_args(x, w_router, w_gate_up, w_down, out, top_k, shared, topk_idx, topk_w)
+    L = _abi.lib()
+    n = ctypes.c_size_t(0)
+    _check(L.gdr_moe_workspace_size(ctypes.byref(a), ctypes.byref(n)), "gdr_moe_workspace_size")
+    if workspace is None and n.value:
+        workspace = torch.empty(int(n.value), dtype=torch.uint8, device=x.device)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(L.gdr_moe_decode(ctypes.byref(a), _ptr(workspace), ws_bytes, _stream(stream, x.device)),
+           "gdr_moe_decode")
     return out

@@ -74,6 +74,29 @@ class NormArgs(ctypes.Structure):
     ]
 
 
+class AttnDecodeArgs(ctypes.Structure):
+    _fields_ = [
+        ("batch", _i32), ("H_q", _i32), ("H_kv", _i32), ("d", _i32),
+        ("rot_dim", _i32), ("max_len", _i32), ("kv_bound", _i32), ("out_dtype", _i32),
+        ("rope_theta", _f32), ("scale", _f32),
+        ("q_stride", _i64), ("gate_stride", _i64), ("k_stride", _i64), ("v_stride", _i64),
+        ("out_stride", _i64),
+        ("q", _vp), ("gate", _vp), ("k", _vp), ("v", _vp),
+        ("k_cache", _vp), ("v_cache", _vp), ("cache_len", _vp), ("out", _vp),
+    ]
+
+
+class MoeArgs(ctypes.Structure):
+    _fields_ = [
+        ("n_tok", _i32), ("hidden", _i32), ("n_exp", _i32), ("top_k", _i32), ("inter", _i32),
+        ("s_inter", _i32), ("out_dtype", _i32), ("reserved", _i32),
+        ("x_stride", _i64), ("out_stride", _i64),
+        ("x", _vp), ("w_router", _vp), ("w_gate_up", _vp), ("w_down", _vp),
+        ("ws_gate_up", _vp), ("ws_down", _vp), ("w_sgate", _vp), ("out", _vp),
+        ("topk_idx", _vp), ("topk_w", _vp),
+    ]
+
+
 _lib = None
 
 
@@ -102,10 +125,24 @@ def lib(path: str = LIB_PATH) -> ctypes.CDLL:
     h.gdr_prefill_chunked.restype = ctypes.c_int
     h.gdr_prefill_chunked_noalloc.argtypes = [ctypes.POINTER(PrefillArgs), _vp]
     h.gdr_prefill_chunked_noalloc.restype = ctypes.c_int
+    h.gdr_prefill_selftest_wait_expiry.argtypes = [ctypes.POINTER(PrefillArgs), _vp,
+                                                   ctypes.c_size_t, ctypes.c_uint64, _vp]
+    h.gdr_prefill_selftest_wait_expiry.restype = ctypes.c_int
+    h.gdr_prefill_noalloc_status.argtypes = [_vp, _vp]
+    h.gdr_prefill_noalloc_status.restype = ctypes.c_int
     h.gdr_decode_multi.argtypes = [ctypes.POINTER(DecodeMultiArgs), _vp]
     h.gdr_decode_multi.restype = ctypes.c_int
     h.gdr_rmsnorm_gated.argtypes = [ctypes.POINTER(NormArgs), _vp]
     h.gdr_rmsnorm_gated.restype = ctypes.c_int
+    h.gdr_attn_decode_workspace_size.argtypes = [ctypes.POINTER(AttnDecodeArgs),
+                                                 ctypes.POINTER(ctypes.c_size_t)]
+    h.gdr_attn_decode_workspace_size.restype = ctypes.c_int
+    h.gdr_attn_decode_step.argtypes = [ctypes.POINTER(AttnDecodeArgs), _vp, ctypes.c_size_t, _vp]
+    h.gdr_attn_decode_step.restype = ctypes.c_int
+    h.gdr_moe_workspace_size.argtypes = [ctypes.POINTER(MoeArgs), ctypes.POINTER(ctypes.c_size_t)]
+    h.gdr_moe_workspace_size.restype = ctypes.c_int
+    h.gdr_moe_decode.argtypes = [ctypes.POINTER(MoeArgs), _vp, ctypes.c_size_t, _vp]
+    h.gdr_moe_decode.restype = ctypes.c_int
     h.gdr_status_string.argtypes = [ctypes.c_int]
     h.gdr_status_string.restype = ctypes.c_char_p
     h.gdr_version.argtypes = []

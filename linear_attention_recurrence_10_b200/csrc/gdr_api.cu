@@ -22,6 +22,14 @@ size_t prefill_tc2p_workspace_bytes(int n_seq, int64_t n_chunks, int H_v, int n_
 int prefill_tc2p_segments(int n_seq, int H_v, int max_chunks, int n_sm);
 cudaError_t launch_prefill_tc2p(const PrefillParams &p, const int32_t *cu_host, int n_seg,
                                 void *workspace, int out_bf16, cudaStream_t s);
+struct AttnParams;
+size_t attn_workspace_bytes(int batch, int H_kv, int n_items);
+void attn_plan(int batch, int H_kv, int kv_bound, int n_sm, int *n_split, int *split_tok);
+cudaError_t launch_attn_decode_args(const gdr_attn_decode_args *a, int n_split, int split_tok,
+                                    void *workspace, cudaStream_t s);
+size_t moe_workspace_bytes(int n_tok, int n_exp, int top_k, int inter, int s_inter, int hidden);
+size_t moe_route_smem_bytes(int n_tok, int n_exp, int top_k);
+cudaError_t launch_moe_args(const gdr_moe_args *a, void *workspace, cudaStream_t s);
 }  // namespace gdr
 
 namespace {
@@ -281,8 +289,13 @@ gdr_status gdr_prefill_workspace_size(const gdr_prefill_args *a, size_t *bytes) 
     return GDR_OK;
 }
 
-gdr_status gdr_prefill_chunked(const gdr_prefill_args *a, void *workspace, size_t ws_bytes,
-                               gdr_stream_t stream) {
+}  // extern "C"
+
+// The prefill behind gdr_prefill_chunked.  diag_wait_ns / diag_withhold: zero
+// for every ordinary call; the wait-expiry self-test sets them (and then needs
+// the two-kernel tensor-core path).
+static gdr_status prefill_impl(const gdr_prefill_args *a, void *workspace, size_t ws_bytes,
+                               gdr_stream_t stream, uint64_t diag_wait_ns, int diag_withhold) {
     int chunk = 0;
     GDR_TRY(check_prefill(a, &chunk));
     if (a->n_seq == 0) return GDR_OK;
@@ -345,6 +358,12 @@ gdr_status gdr_prefill_chunked(const gdr_prefill_args *a, void *workspace, size_
     p.final_state = a->final_state;
     p.norm_w = a->norm_w;
     p.out = a->out;
+    if (diag_withhold) {
+        if (!tc) return GDR_ERR_UNSUPPORTED;
+        if (ws_bytes < need_two) return GDR_ERR_WORKSPACE;
+        p.wait_ns = diag_wait_ns;
+        p.withhold_first_k = 1;
+    }
     if (tc && ws_bytes >= need_two)
         return from_cuda(gdr::launch_prefill_tc2p(p, a->cu_seqlens_host,
                                                   ws_bytes >= need_seg ? n_seg : 1, workspace,
@@ -354,6 +373,141 @@ gdr_status gdr_prefill_chunked(const gdr_prefill_args *a, void *workspace, size_
                                                 (cudaStream_t)stream));
     return from_cuda(gdr::launch_prefill_simt(p, d, chunk, a->in_dtype == GDR_BF16,
                                               a->out_dtype == GDR_BF16, (cudaStream_t)stream));
+}
+
+extern "C" {
+
+gdr_status gdr_prefill_chunked(const gdr_prefill_args *a, void *workspace, size_t ws_bytes,
+                               gdr_stream_t stream) {
+    return prefill_impl(a, workspace, ws_bytes, stream, 0, 0);
+}
+
+gdr_status gdr_prefill_selftest_wait_expiry(const gdr_prefill_args *a, void *workspace,
+                                            size_t ws_bytes, uint64_t wait_ns,
+                                            gdr_stream_t stream) {
+    if (wait_ns < GDR_SELFTEST_MIN_WAIT_NS || wait_ns > GDR_SELFTEST_MAX_WAIT_NS)
+        return GDR_ERR_INVALID_ARG;
+    if (!a || a->n_seq == 0) return GDR_ERR_INVALID_ARG;
+    return prefill_impl(a, workspace, ws_bytes, stream, wait_ns, 1);
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------ gated attention
+
+// Shape and pointer checks of the attention step; fills the work split.
+static gdr_status attn_check(const gdr_attn_decode_args *a, int *n_split, int *split_tok,
+                             size_t *ws_bytes) {
+    if (!a) return GDR_ERR_INVALID_ARG;
+    if (a->batch < 0 || a->H_q <= 0 || a->H_kv <= 0 || a->d <= 0) return GDR_ERR_INVALID_ARG;
+    if (a->H_q % a->H_kv != 0) return GDR_ERR_INVALID_ARG;
+    if (a->H_q / a->H_kv > 16 || a->d != 256) return GDR_ERR_UNSUPPORTED;
+    if (a->rot_dim < 0 || a->rot_dim > a->d || (a->rot_dim & 1)) return GDR_ERR_INVALID_ARG;
+    if (a->max_len < 1 || a->kv_bound < 0 || a->kv_bound >= a->max_len) return GDR_ERR_INVALID_ARG;
+    if (!dtype_ok(a->out_dtype)) return GDR_ERR_INVALID_ARG;
+    if (!(a->rope_theta > 0.f)) return GDR_ERR_INVALID_ARG;
+    if ((int64_t)a->batch * a->H_kv * a->max_len * a->d > ((int64_t)1 << 40)) return GDR_ERR_UNSUPPORTED;
+    gdr::attn_plan(a->batch, a->H_kv, a->kv_bound, device_sm_count(), n_split, split_tok);
+    if ((int64_t)a->batch * a->H_kv * *n_split > 0x7fffffffLL) return GDR_ERR_UNSUPPORTED;
+    *ws_bytes = gdr::attn_workspace_bytes(a->batch, a->H_kv, a->batch * a->H_kv * *n_split);
+    return GDR_OK;
+}
+
+extern "C" {
+
+gdr_status gdr_attn_decode_workspace_size(const gdr_attn_decode_args *a, size_t *bytes) {
+    if (!bytes) return GDR_ERR_INVALID_ARG;
+    int n_split = 0, split_tok = 0;
+    size_t need = 0;
+    GDR_TRY(attn_check(a, &n_split, &split_tok, &need));
+    *bytes = a->batch == 0 ? 0 : need;
+    return GDR_OK;
+}
+
+gdr_status gdr_attn_decode_step(const gdr_attn_decode_args *a, void *workspace,
+                                size_t ws_bytes, gdr_stream_t stream) {
+    int n_split = 0, split_tok = 0;
+    size_t need = 0;
+    GDR_TRY(attn_check(a, &n_split, &split_tok, &need));
+    if (a->batch == 0) return GDR_OK;
+    if (!a->q || !a->gate || !a->k || !a->v || !a->k_cache || !a->v_cache || !a->cache_len ||
+        !a->out)
+        return GDR_ERR_INVALID_ARG;
+    const int64_t d = a->d;
+    int64_t qs, gs, ks, vs, os;
+    GDR_TRY(resolve_stride(a->q_stride, a->H_q * d, 2, &qs));
+    GDR_TRY(resolve_stride(a->gate_stride, a->H_q * d, 2, &gs));
+    GDR_TRY(resolve_stride(a->k_stride, a->H_kv * d, 2, &ks));
+    GDR_TRY(resolve_stride(a->v_stride, a->H_kv * d, 2, &vs));
+    GDR_TRY(resolve_stride(a->out_stride, a->H_q * d, dtype_bytes(a->out_dtype), &os));
+    const void *p16[] = {a->q, a->gate, a->k, a->v, a->k_cache, a->v_cache, a->out};
+    for (const void *ptr : p16)
+        if (!aligned16(ptr)) return GDR_ERR_MISALIGNED;
+    if (!aligned4(a->cache_len)) return GDR_ERR_MISALIGNED;
+    if (!workspace || ws_bytes < need) return GDR_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return GDR_ERR_MISALIGNED;
+    gdr_attn_decode_args r = *a;
+    r.q_stride = qs;
+    r.gate_stride = gs;
+    r.k_stride = ks;
+    r.v_stride = vs;
+    r.out_stride = os;
+    return from_cuda(gdr::launch_attn_decode_args(&r, n_split, split_tok, workspace,
+                                                  (cudaStream_t)stream));
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ MoE
+
+static gdr_status moe_check(const gdr_moe_args *a) {
+    if (!a) return GDR_ERR_INVALID_ARG;
+    if (a->n_tok < 0 || a->hidden <= 0 || a->n_exp <= 0 || a->inter <= 0 || a->reserved != 0)
+        return GDR_ERR_INVALID_ARG;
+    if (a->top_k < 1 || a->top_k > a->n_exp) return GDR_ERR_INVALID_ARG;
+    if (a->top_k > 32 || a->n_tok > 4096 || a->n_exp > 1024) return GDR_ERR_UNSUPPORTED;
+    if (a->ws_gate_up && a->s_inter <= 0) return GDR_ERR_INVALID_ARG;
+    if (a->hidden % 8 || a->inter % 8 || (a->ws_gate_up && a->s_inter % 8)) return GDR_ERR_UNSUPPORTED;
+    if (a->inter > 1024 || (a->ws_gate_up && a->s_inter > 1024)) return GDR_ERR_UNSUPPORTED;
+    if (!dtype_ok(a->out_dtype)) return GDR_ERR_INVALID_ARG;
+    if (gdr::moe_route_smem_bytes(a->n_tok, a->n_exp, a->top_k) > 200 * 1024) return GDR_ERR_UNSUPPORTED;
+    return GDR_OK;
+}
+
+extern "C" {
+
+gdr_status gdr_moe_workspace_size(const gdr_moe_args *a, size_t *bytes) {
+    if (!bytes) return GDR_ERR_INVALID_ARG;
+    GDR_TRY(moe_check(a));
+    *bytes = a->n_tok == 0 ? 0
+                           : gdr::moe_workspace_bytes(a->n_tok, a->n_exp, a->top_k, a->inter,
+                                                      a->ws_gate_up ? a->s_inter : 0, a->hidden);
+    return GDR_OK;
+}
+
+gdr_status gdr_moe_decode(const gdr_moe_args *a, void *workspace, size_t ws_bytes,
+                          gdr_stream_t stream) {
+    GDR_TRY(moe_check(a));
+    if (a->n_tok == 0) return GDR_OK;
+    if (!a->x || !a->w_router || !a->w_gate_up || !a->w_down || !a->out) return GDR_ERR_INVALID_ARG;
+    if (a->ws_gate_up && (!a->ws_down || !a->w_sgate)) return GDR_ERR_INVALID_ARG;
+    int64_t xs, os;
+    GDR_TRY(resolve_stride(a->x_stride, a->hidden, 2, &xs));
+    GDR_TRY(resolve_stride(a->out_stride, a->hidden, dtype_bytes(a->out_dtype), &os));
+    const void *p16[] = {a->x, a->w_router, a->w_gate_up, a->w_down, a->ws_gate_up, a->ws_down,
+                         a->w_sgate, a->out};
+    for (const void *ptr : p16)
+        if (ptr && !aligned16(ptr)) return GDR_ERR_MISALIGNED;
+    if ((a->topk_idx && !aligned4(a->topk_idx)) || (a->topk_w && !aligned4(a->topk_w)))
+        return GDR_ERR_MISALIGNED;
+    const size_t need = gdr::moe_workspace_bytes(a->n_tok, a->n_exp, a->top_k, a->inter,
+                                                 a->ws_gate_up ? a->s_inter : 0, a->hidden);
+    if (!workspace || ws_bytes < need) return GDR_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return GDR_ERR_MISALIGNED;
+    gdr_moe_args r = *a;
+    r.x_stride = xs;
+    r.out_stride = os;
+    return from_cuda(gdr::launch_moe_args(&r, workspace, (cudaStream_t)stream));
 }
 
 }  // extern "C"

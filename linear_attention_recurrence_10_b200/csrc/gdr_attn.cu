@@ -1,0 +1,666 @@
+// gdr_attn.cu -- one decode step of the gated full-attention layer, the other
+// mixer of the hybrid decoder (GatedAttention in the Qwen3.5 Chat guide,
+// section "Architektur": standard scaled-dot-product attention over a KV
+// cache; on the Core AI Qwen3.6-35B-A3B card, first section: head_dim 256,
+// 16 query heads over 2 key/value heads, partial rotary embedding with
+// theta = 1e7).  Per sequence b with L = cache_len[b] tokens already cached:
+//
+//   q_rot, k_rot = RoPE(q), RoPE(k) at position L on the first rot_dim dims
+//                  (dim i paired with i + rot_dim/2, angle L theta^(-2i/rot_dim))
+//   cache[L]     = (k_rot, v)                               (appended)
+//   o_h          = sum_{t <= L} softmax_t(scale q_rot_h . k_t) v_t
+//   y_h          = o_h * sigmoid(gate_h)
+//
+// Three kernels on the caller's stream, each a programmatic dependent of the
+// one before:
+//   rope_append: per (b, kv head): rotates q (the group's query heads) and k in
+//     fp32 with angles taken in double, appends the key and value at row L,
+//     and stages the rotated queries as the bf16 MMA operand tile of the group.
+//   attend: persistent; each work item is one (b, kv head, split of the
+//     tokens).  A producer warp streams the K and V rows through a six-slot
+//     ring of 32 KB shared-memory slots (one d-half of a 128-token tile each,
+//     cp.async with zero fill past the split's end); an MMA warp issues
+//     S^T = K Q^T (M = 128 tokens, N = 16 query-head columns, K = 256) and
+//     O^T += V^T P^T (M = 128 dims per half, N = 16, K = 128 tokens) on
+//     tcgen05 with the accumulators in TMEM; four softmax warps (thread = TMEM
+//     lane) keep the running maxima and sums, write P as bf16 and rescale O^T
+//     when a maximum moves.  The item's (m, l, O) go to the workspace.
+//   combine: per (b, kv head): merges the splits' partials and applies the
+//     output gate.
+//
+// The contraction per token and key/value head is 2 x 256 MACs per query head:
+// at decode the layer is bound by HBM, reading the cache once.  Every wait is
+// bounded (2 s); on expiry the kernel records GDR_ERR_TIMEOUT in the workspace
+// status word, waits (bounded) for its copies in flight, frees its tensor
+// memory and returns.
+#include <math.h>
+
+#include "gdr.h"
+#include "gdr_common.cuh"
+#include "gdr_tc.cuh"
+
+namespace gdr {
+
+struct AttnParams {
+    int batch, H_q, H_kv, n_rep, rot_dim, max_len, kv_bound;
+    int n_split, split_tok, n_items;
+    float scale;
+    double log2_theta;
+    int64_t q_stride, gate_stride, k_stride, v_stride, out_stride;
+    const __nv_bfloat16 *q, *gate, *k, *v;
+    __nv_bfloat16 *k_cache, *v_cache;
+    const int32_t *cache_len;
+    void *out;
+    // workspace
+    int *status;             // [0]: the call's status (combine block 0); [1]: wait expired
+    __nv_bfloat16 *q_tiles;  // [batch * H_kv][16 x 256] bf16, operand layout
+    float *part_o;           // [n_items][16][256]
+    float *part_ml;          // [n_items][16][2]
+};
+
+namespace attn {
+
+using namespace gdr::tc;
+
+constexpr int D = 256;
+constexpr int TILE = 128;                 // tokens per tile
+constexpr int NH = 16;                    // query-head columns per key/value head
+constexpr int NSLOT = 6;
+constexpr uint32_t SLOT = 32768;          // one d-half of a K or V tile, bf16
+constexpr uint32_t QTILE = NH * D * 2;    // 8 KB
+constexpr uint32_t PTILE = NH * TILE * 2; // 4 KB
+constexpr uint32_t S_RING = 0;
+constexpr uint32_t S_Q = S_RING + NSLOT * SLOT;   // 2 x Q tile
+constexpr uint32_t S_P = S_Q + 2 * QTILE;         // 2 x P tile
+constexpr uint32_t S_RED = S_P + 2 * PTILE;       // 4 warps x 16 floats
+constexpr uint32_t S_BAR = S_RED + 256;
+constexpr uint32_t S_BYTES = S_BAR + 256;
+constexpr int NTHR = 224;  // warps 0-3 softmax, 4 producer, 5 S^T issue, 6 O^T issue
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr int kTimeout = 6;  // GDR_ERR_TIMEOUT
+constexpr int kBadLen = 1;   // GDR_ERR_INVALID_ARG
+// TMEM columns: S^T double buffer, O^T two d-halves.
+constexpr uint32_t TM_S = 0, TM_O = 32, TM_COLS = 64;
+
+// Tile operand layouts (no swizzle, 16-byte chunks of 8 bf16).
+// K / V slot: row r (token) of 128, chunk c (8 dims) of 16:
+//   byte = (r / 8) * 2048 + c * 128 + (r % 8) * 16
+// read as K-major A for S^T (rows = tokens: SBO 2048, LBO 128) and as
+// MN-major A for O^T (M = dims: SBO 128 between chunks, LBO 2048 between
+// 8-token groups).
+__host__ __device__ constexpr uint32_t slot_off(int r, int c) {
+    return (uint32_t)((r >> 3) * 2048 + c * 128 + (r & 7) * 16);
+}
+// Q tile: query-head column h of 16, dim chunk c of 32 (K-major B for S^T):
+//   byte = c * 256 + h * 16   (LBO 256 between chunks, SBO 128 between 8-head groups)
+__host__ __device__ constexpr uint32_t q_off(int h, int c) { return (uint32_t)(c * 256 + h * 16); }
+// P tile: column h, token t (K-major B for O^T): byte = (t/8) * 256 + h * 16 + (t%8) * 2
+__host__ __device__ constexpr uint32_t p_off(int h, int t) {
+    return (uint32_t)((t >> 3) * 256 + h * 16 + (t & 7) * 2);
+}
+
+struct Item {
+    int b, g, t0, t1;  // tokens [t0, t1) of the cache rows of (b, g)
+};
+__device__ __forceinline__ Item item_of(const AttnParams &p, int it) {
+    Item w;
+    const int bg = it / p.n_split, s = it - bg * p.n_split;
+    w.b = bg / p.H_kv;
+    w.g = bg - w.b * p.H_kv;
+    int L = p.cache_len[w.b];
+    // Attended rows: 0 .. L (the new token was appended at row L).  A length
+    // outside the checked range reads nothing past the bound.
+    int end = min(L, min(p.kv_bound, p.max_len - 1)) + 1;
+    if (L < 0) end = 0;
+    w.t0 = s * p.split_tok;
+    w.t1 = min(end, w.t0 + p.split_tok);
+    if (w.t1 < w.t0) w.t1 = w.t0;
+    return w;
+}
+
+// ------------------------------------------------------------ rope_append
+// One block of 256 threads (thread = dim) per (b, kv head).
+__global__ void __launch_bounds__(256) rope_append_kernel(const AttnParams p) {
+    wait_for_predecessor();
+    release_dependents();
+    const int bg = blockIdx.x, b = bg / p.H_kv, g = bg - b * p.H_kv, d = threadIdx.x;
+    const int L = p.cache_len[b];
+    const bool ok = L >= 0 && L < p.max_len && L <= p.kv_bound;
+    if (bg == 0 && d == 0) p.status[1] = 0;  // the attend kernel's expiry flag
+    const int half = p.rot_dim >> 1;
+    float c = 1.f, s = 0.f;
+    int partner = d;
+    float sign = 0.f;
+    if (d < p.rot_dim && ok) {
+        const int i = d < half ? d : d - half;
+        // angle = L * theta^(-2i/rot_dim), in double so that large positions keep
+        // their precision.
+        const double ang = (double)L * exp2(-(2.0 * i / p.rot_dim) * p.log2_theta);
+        double sd, cd;
+        sincos(ang, &sd, &cd);
+        c = (float)cd;
+        s = (float)sd;
+        partner = d < half ? d + half : d - half;
+        sign = d < half ? -1.f : 1.f;  // x_i c - x_{i+h} s ;  x_{i+h} c + x_i s
+    }
+    auto rot = [&](const __nv_bfloat16 *row) {
+        const float x = __bfloat162float(row[d]);
+        if (d >= p.rot_dim) return x;
+        return x * c + sign * __bfloat162float(row[partner]) * s;
+    };
+    if (ok) {
+        const __nv_bfloat16 *kr = p.k + (int64_t)b * p.k_stride + g * D;
+        const __nv_bfloat16 *vr = p.v + (int64_t)b * p.v_stride + g * D;
+        const size_t crow = (((size_t)b * p.H_kv + g) * p.max_len + L) * D;
+        p.k_cache[crow + d] = __float2bfloat16_rn(rot(kr));
+        p.v_cache[crow + d] = vr[d];
+    }
+    unsigned char *qt = reinterpret_cast<unsigned char *>(p.q_tiles) + (size_t)bg * QTILE;
+    for (int h = 0; h < NH; ++h) {
+        float x = 0.f;
+        if (h < p.n_rep && ok) x = rot(p.q + (int64_t)b * p.q_stride + (g * p.n_rep + h) * D);
+        *reinterpret_cast<__nv_bfloat16 *>(qt + q_off(h, d >> 3) + (d & 7) * 2) =
+            __float2bfloat16_rn(x);
+    }
+}
+
+// ---------------------------------------------------------------- attend
+__global__ void __launch_bounds__(NTHR, 1) attend_kernel(const AttnParams p) {
+    extern __shared__ __align__(1024) unsigned char sm[];
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + S_BAR);
+    uint64_t *full = bars;           // [6] slot landed (32 producer lanes)
+    uint64_t *empty = bars + 6;      // [6] slot consumed (MMA commit)
+    uint64_t *bar_s = bars + 12;     // [2] S^T of a tile in TMEM
+    uint64_t *bar_p = bars + 14;     // [2] P of a tile staged, O^T rescaled (4 warps)
+    uint64_t *bar_o = bars + 16;     // [2] O^T += V^T P^T of a tile done (by P buffer)
+    uint64_t *bar_q = bars + 18;     // [2] Q tile of an item landed
+    uint64_t *bar_qfree = bars + 20; // [2] an item's S^T products done with its Q tile
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + S_BAR + 176);
+    float *red = reinterpret_cast<float *>(sm + S_RED);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const uint32_t sbase = smem_u32(sm);
+
+    if (warp == 0) tmem_alloc(tmem_slot, TM_COLS);
+    if (tid == 0) {
+        for (int i = 0; i < NSLOT; ++i) {
+            mbar_init(full + i, 32);
+            mbar_init(empty + i, 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar_s + i, 1);
+            mbar_init(bar_p + i, 4);
+            mbar_init(bar_q + i, 1);
+            mbar_init(bar_qfree + i, 1);
+            mbar_init(bar_o + i, 1);
+        }
+        mbar_fence_init();
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tm = *tmem_slot;
+    // The set-up above overlaps the kernel before; everything below reads what
+    // it wrote.  Dependents start only when this grid completes.
+    wait_for_predecessor();
+    auto fail = [&]() { atomicExch(p.status + 1, kTimeout); };
+    auto n_tiles_of = [&](const Item &w) { return (w.t1 - w.t0 + TILE - 1) / TILE; };
+
+    if (warp == 4) {
+        // ------------------------------------------------------ producer
+        // Slot uses are counted in one sequence (c) over this CTA's non-empty
+        // items (nq), tiles and the tile's K0, K1, V0, V1 quarters; the MMA
+        // warp walks the same sequence.
+        int c = 0, nq = 0, n_qcopy[2] = {0, 0};
+        bool ok = true;
+        for (int it = blockIdx.x; it < p.n_items && ok; it += gridDim.x) {
+            const Item w = item_of(p, it);
+            const int nt = n_tiles_of(w);
+            if (nt == 0) continue;
+            const int qb = nq & 1;
+            // The item's Q tile, once the item two back is done with the buffer.
+            if (nq >= 2 && lane == 0) ok = mbar_wait(bar_qfree + qb, (uint32_t)((nq - 2) >> 1) & 1u, kWaitNs);
+            ok = __shfl_sync(kFullMask, ok, 0);
+            if (!ok) break;
+            if (lane == 0) {
+                bulk_expect(bar_q + qb, QTILE);
+                bulk_copy(sm + S_Q + qb * QTILE,
+                          reinterpret_cast<const unsigned char *>(p.q_tiles) +
+                              (size_t)(w.b * p.H_kv + w.g) * QTILE,
+                          QTILE, bar_q + qb);
+            }
+            ++n_qcopy[qb];
+            ++nq;
+            const size_t head_row = ((size_t)w.b * p.H_kv + w.g) * p.max_len;
+            for (int j = 0; j < nt && ok; ++j) {
+                const int r0 = w.t0 + j * TILE;
+                const int nvalid = min(TILE, w.t1 - r0);
+#pragma unroll 1
+                for (int q4 = 0; q4 < 4; ++q4, ++c) {
+                    const int slot = c % NSLOT, round = c / NSLOT;
+                    if (round > 0) ok = mbar_wait(empty + slot, (uint32_t)(round - 1) & 1u, kWaitNs);
+                    ok = __all_sync(kFullMask, ok) != 0;
+                    if (!ok) break;
+                    // Lane l copies, at step k, row (k / 4) * 8 + l % 8 and chunk
+                    // (k % 4) * 4 + l / 8: 8 rows x 4 chunks per step, 512
+                    // contiguous bytes of the slot.  Everything but k folds into
+                    // two per-lane base addresses, so a full tile is one
+                    // instruction per 16-byte copy.
+                    const __nv_bfloat16 *src = (q4 < 2 ? p.k_cache : p.v_cache) +
+                                               (head_row + r0 + (lane & 7)) * D + (q4 & 1) * 128 +
+                                               (lane >> 3) * 8;
+                    const uint32_t dst = sbase + S_RING + slot * SLOT + (lane >> 3) * 128 + (lane & 7) * 16;
+                    if (nvalid == TILE) {
+#pragma unroll
+                        for (int k = 0; k < 64; ++k)
+                            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                                             dst + (k >> 2) * 2048 + (k & 3) * 512),
+                                         "l"(src + (size_t)((k >> 2) * 8) * D + (k & 3) * 32)
+                                         : "memory");
+                    } else {
+                        // The split's last, partial tile: rows past it are zero-filled
+                        // (their source address is the tile's first row, never read).
+#pragma unroll 4
+                        for (int k = 0; k < 64; ++k) {
+                            const int r = (k >> 2) * 8 + (lane & 7);
+                            const bool in = r < nvalid;
+                            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
+                                             dst + (k >> 2) * 2048 + (k & 3) * 512),
+                                         "l"(in ? src + (size_t)((k >> 2) * 8) * D + (k & 3) * 32
+                                                : src - (size_t)(lane & 7) * D),
+                                         "r"(in ? 16u : 0u)
+                                         : "memory");
+                        }
+                    }
+                    cp_async_arrive(full + slot);
+                }
+            }
+        }
+        cp_async_wait_all();
+        if (!ok && lane == 0) {
+            fail();
+            // No bulk copy may land after the CTA ends.
+            for (int b = 0; b < 2; ++b)
+                if (n_qcopy[b]) mbar_wait(bar_q + b, (uint32_t)(n_qcopy[b] - 1) & 1u, kWaitNs);
+        }
+        __syncwarp();
+    } else if (warp == 5 || warp == 6) {
+        // ------------------------------------------- MMA issue, two threads
+        // Warp 5 issues S^T = K Q^T of each tile as soon as its K has landed
+        // (and the softmax is done with the S^T buffer it reuses); warp 6
+        // issues O^T += V^T P^T of each tile as soon as its P and V are ready.
+        // Neither waits behind the other's operands.
+        if (lane == 0) {
+            const bool s_role = warp == 5;
+            const uint32_t ID_S = instr_desc<Kind::BF16>(128, NH, false, false);
+            const uint32_t ID_O = instr_desc<Kind::BF16>(128, NH, true, false);
+            bool ok = true;
+            int c = 0, jt = 0, nq = 0;
+            for (int it = blockIdx.x; it < p.n_items && ok; it += gridDim.x) {
+                const Item w = item_of(p, it);
+                const int nt = n_tiles_of(w);
+                if (nt == 0) continue;
+                const int qb = nq & 1;
+                if (s_role) ok = mbar_wait(bar_q + qb, (uint32_t)(nq >> 1) & 1u, kWaitNs);
+                ++nq;
+                for (int j = 0; j < nt && ok; ++j, ++jt, c += 4) {
+                    if (s_role) {
+                        // K halves in uses c, c + 1 of the ring; S^T buffer jt & 1
+                        // was read by the softmax of tile jt - 2.
+                        const int s0 = c % NSLOT, s1 = (c + 1) % NSLOT;
+                        ok = mbar_wait(full + s0, (uint32_t)(c / NSLOT) & 1u, kWaitNs) &&
+                             mbar_wait(full + s1, (uint32_t)((c + 1) / NSLOT) & 1u, kWaitNs) &&
+                             (jt < 2 || mbar_wait(bar_p + (jt & 1), (uint32_t)((jt - 2) >> 1) & 1u, kWaitNs));
+                        if (!ok) break;
+                        fence_after_sync();
+                        const uint32_t d = tm + TM_S + 16 * (jt & 1);
+                        const uint32_t qa = sbase + S_Q + qb * QTILE;
+                        gemm(d, sbase + S_RING + s0 * SLOT, 128, 2048, 256, qa, 256, 128, 512, 8, ID_S,
+                             false);
+                        gemm(d, sbase + S_RING + s1 * SLOT, 128, 2048, 256, qa + 4096, 256, 128, 512, 8,
+                             ID_S, true);
+                        commit(smem_u32(bar_s + (jt & 1)));
+                        commit(smem_u32(empty + s0));
+                        commit(smem_u32(empty + s1));
+                        if (j == nt - 1) commit(smem_u32(bar_qfree + qb));
+                    } else {
+                        const int v0 = (c + 2) % NSLOT, v1 = (c + 3) % NSLOT;
+                        ok = mbar_wait(bar_p + (jt & 1), (uint32_t)(jt >> 1) & 1u, kWaitNs) &&
+                             mbar_wait(full + v0, (uint32_t)((c + 2) / NSLOT) & 1u, kWaitNs) &&
+                             mbar_wait(full + v1, (uint32_t)((c + 3) / NSLOT) & 1u, kWaitNs);
+                        if (!ok) break;
+                        fence_after_sync();
+                        const uint32_t pb = sbase + S_P + (jt & 1) * PTILE;
+                        gemm(tm + TM_O, sbase + S_RING + v0 * SLOT, 2048, 128, 4096, pb, 256, 128, 512,
+                             8, ID_O, j > 0);
+                        gemm(tm + TM_O + 16, sbase + S_RING + v1 * SLOT, 2048, 128, 4096, pb, 256, 128,
+                             512, 8, ID_O, j > 0);
+                        commit(smem_u32(bar_o + (jt & 1)));
+                        commit(smem_u32(empty + v0));
+                        commit(smem_u32(empty + v1));
+                    }
+                }
+            }
+            if (!ok) fail();
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------ softmax warps
+        // Every decision that leads to a named barrier is made by all four
+        // warps together (an OR over the barrier), so none waits for a warp
+        // that has stopped.
+        //
+        // The weights are taken against a reference maximum m_ref that only
+        // moves when a tile's maximum passes it by more than kLazy (so P stays
+        // below e^kLazy): then O^T and l are rescaled, which needs the previous
+        // tile's O^T product finished.  Otherwise a tile waits only for the
+        // product two tiles back, whose P buffer it reuses.
+        constexpr float kLazy = 8.0f;
+        const int t = tid;  // TMEM lane: token of the tile for S^T, dim for O^T
+        const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+        bool dead = false;
+        int jt = 0;
+        auto wait_o = [&](int tile) {  // O^T product of `tile` done
+            return mbar_wait(bar_o + (tile & 1), (uint32_t)(tile >> 1) & 1u, kWaitNs);
+        };
+        for (int it = blockIdx.x; it < p.n_items && !dead; it += gridDim.x) {
+            const Item w = item_of(p, it);
+            const int nt = n_tiles_of(w);
+            float *po = p.part_o + (size_t)it * NH * D;
+            float *pml = p.part_ml + (size_t)it * NH * 2;
+            if (nt == 0) {
+                if (t < NH) {
+                    pml[2 * t] = -INFINITY;
+                    pml[2 * t + 1] = 0.f;
+                }
+                continue;
+            }
+            float m_ref[NH], l_run[NH];
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+                m_ref[h] = -INFINITY;
+                l_run[h] = 0.f;
+            }
+            const int jt0 = jt;
+            for (int j = 0; j < nt; ++j, ++jt) {
+                const int nvalid = min(TILE, w.t1 - (w.t0 + j * TILE));
+                bool ok = mbar_wait(bar_s + (jt & 1), (uint32_t)(jt >> 1) & 1u, kWaitNs);
+                // P's buffer was last read by the product two tiles back.
+                if (ok && jt >= 2) ok = wait_o(jt - 2);
+                dead = group_sync_or(1, 128, !ok);
+                if (dead) break;
+                fence_after_sync();
+                float s[NH];
+                tmem_ld16(tm + lane_off + TM_S + 16 * (jt & 1), s);
+                const bool valid = t < nvalid;
+                float tmax[NH];
+                // Columns past the group's query heads are padding: their
+                // weights stay zero and they cost no reductions.
+#pragma unroll
+                for (int h = 0; h < NH; ++h) {
+                    s[h] = valid && h < p.n_rep ? s[h] * p.scale : -INFINITY;
+                    float x = s[h];
+                    if (h < p.n_rep) {
+#pragma unroll
+                        for (int o = 16; o >= 1; o >>= 1) x = fmaxf(x, __shfl_xor_sync(kFullMask, x, o));
+                    }
+                    tmax[h] = x;
+                }
+                if (lane < NH) {
+                    float mine = tmax[0];
+#pragma unroll
+                    for (int h = 1; h < NH; ++h) mine = lane == h ? tmax[h] : mine;
+                    red[warp * NH + lane] = mine;
+                }
+                group_sync_or(1, 128, false);
+                float alpha[NH];
+                bool moved = false;
+#pragma unroll
+                for (int h = 0; h < NH; ++h) {
+                    const float m4 = fmaxf(fmaxf(red[h], red[NH + h]), fmaxf(red[2 * NH + h], red[3 * NH + h]));
+                    alpha[h] = 1.f;
+                    if (m_ref[h] == -INFINITY) {
+                        m_ref[h] = m4;  // first tile of the item: O^T starts from zero
+                    } else if (m4 > m_ref[h] + kLazy) {
+                        alpha[h] = __expf(m_ref[h] - m4);
+                        m_ref[h] = m4;
+                        moved = true;
+                    }
+                    const float pv = (valid && h < p.n_rep && m_ref[h] > -INFINITY) ? __expf(s[h] - m_ref[h]) : 0.f;
+                    l_run[h] = l_run[h] * alpha[h] + pv;
+                    s[h] = pv;
+                }
+                // P as bf16: column h = query head, row t = token.
+                unsigned char *pt = sm + S_P + (jt & 1) * PTILE;
+#pragma unroll
+                for (int h = 0; h < NH; ++h)
+                    *reinterpret_cast<__nv_bfloat16 *>(pt + p_off(h, t)) = __float2bfloat16_rn(s[h]);
+                // Rescale O^T (lane = dim) when a reference maximum moved: the
+                // previous tile's product must have finished adding into it.
+                // (`moved` is the same in every thread: it comes from red[].)
+                if (moved) {
+                    const bool ok2 = jt == jt0 || wait_o(jt - 1);
+                    dead = group_sync_or(1, 128, !ok2);
+                    if (dead) break;
+                    fence_after_sync();
+#pragma unroll
+                    for (int hd = 0; hd < 2; ++hd) {
+                        float o[16];
+                        tmem_ld16(tm + lane_off + TM_O + 16 * hd, o);
+                        uint32_t ou[16];
+#pragma unroll
+                        for (int h = 0; h < NH; ++h) ou[h] = __float_as_uint(o[h] * alpha[h]);
+                        tmem_st16(tm + lane_off + TM_O + 16 * hd, ou);
+                    }
+                }
+                fence_smem_to_async();
+                fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_p + (jt & 1));
+                group_sync_or(1, 128, false);  // red[] is rewritten next
+            }
+            if (dead) break;
+            // Item done: the partial (m, l, O) of every query head of the group.
+            const bool ok = wait_o(jt - 1);
+            dead = group_sync_or(1, 128, !ok);
+            if (dead) break;
+            fence_after_sync();
+#pragma unroll
+            for (int hd = 0; hd < 2; ++hd) {
+                float o[16];
+                tmem_ld16(tm + lane_off + TM_O + 16 * hd, o);
+#pragma unroll
+                for (int h = 0; h < NH; ++h)
+                    if (h < p.n_rep) po[(size_t)h * D + 128 * hd + t] = o[h];
+            }
+            // l: sum over the 128 token lanes.
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+                float x = l_run[h];
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(kFullMask, x, o);
+                l_run[h] = x;
+            }
+            if (lane < NH) {
+                float mine = l_run[0];
+#pragma unroll
+                for (int h = 1; h < NH; ++h) mine = lane == h ? l_run[h] : mine;
+                red[warp * NH + lane] = mine;
+            }
+            group_sync_or(1, 128, false);
+            if (t < NH) {
+                float m = m_ref[0];
+#pragma unroll
+                for (int h = 1; h < NH; ++h) m = t == h ? m_ref[h] : m;
+                pml[2 * t] = m;
+                pml[2 * t + 1] = (red[t] + red[NH + t]) + (red[2 * NH + t] + red[3 * NH + t]);
+            }
+            group_sync_or(1, 128, false);
+        }
+        if (dead && tid == 0) fail();
+    }
+
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        fence_after_sync();
+        tmem_free(tm, TM_COLS);
+    }
+}
+
+// --------------------------------------------------------------- combine
+// One block of 256 threads (thread = dim) per (b, kv head): every query head of
+// the group merges its splits, y = (sum_s e^{m_s - m} O_s) / (sum_s e^{m_s - m} l_s)
+// * sigmoid(gate).
+template <typename TOUT>
+__global__ void __launch_bounds__(256) combine_kernel(const AttnParams p) {
+    wait_for_predecessor();
+    release_dependents();
+    const int bg = blockIdx.x, b = bg / p.H_kv, g = bg - b * p.H_kv, d = threadIdx.x;
+    const size_t it0 = (size_t)bg * p.n_split;
+    if (bg == 0) {
+        // The call's status: an expired wait, else a cache length out of range.
+        __shared__ int bad;
+        if (d == 0) bad = 0;
+        __syncthreads();
+        for (int i = d; i < p.batch; i += blockDim.x) {
+            const int L = p.cache_len[i];
+            if (L < 0 || L >= p.max_len || L > p.kv_bound) bad = 1;
+        }
+        __syncthreads();
+        if (d == 0) p.status[0] = p.status[1] ? kTimeout : (bad ? kBadLen : 0);
+    }
+    for (int h = 0; h < p.n_rep; ++h) {
+        float m = -INFINITY;
+        for (int s = 0; s < p.n_split; ++s) m = fmaxf(m, p.part_ml[((it0 + s) * NH + h) * 2]);
+        float o = 0.f, l = 0.f;
+        if (m > -INFINITY) {
+            for (int s = 0; s < p.n_split; ++s) {
+                const float ms = p.part_ml[((it0 + s) * NH + h) * 2];
+                if (ms == -INFINITY) continue;
+                const float f = __expf(ms - m);
+                l += f * p.part_ml[((it0 + s) * NH + h) * 2 + 1];
+                o += f * p.part_o[((it0 + s) * NH + h) * D + d];
+            }
+        }
+        const int hq = g * p.n_rep + h;
+        const float gt = __bfloat162float(p.gate[(int64_t)b * p.gate_stride + hq * D + d]);
+        const float y = (l > 0.f ? o / l : 0.f) / (1.f + __expf(-gt));
+        Elem<TOUT>::store1(static_cast<TOUT *>(p.out) + (int64_t)b * p.out_stride + hq * D + d, y);
+    }
+}
+
+}  // namespace attn
+
+size_t attn_workspace_bytes(int batch, int H_kv, int n_items) {
+    size_t off = 256;  // status word
+    off += (size_t)batch * H_kv * attn::QTILE;
+    off = (off + 255) & ~(size_t)255;
+    off += (size_t)n_items * attn::NH * attn::D * 4;
+    off += (size_t)n_items * attn::NH * 2 * 4;
+    return (off + 255) & ~(size_t)255;
+}
+
+// Cost of starting and finishing one work item (waiting for its last
+// product, writing its partials), in tiles of 128 tokens.
+#ifndef GDR_ATTN_ITEM_COST
+#define GDR_ATTN_ITEM_COST 1.0
+#endif
+
+// Splits of the attended tokens per (b, kv head): the count that minimises the
+// busiest CTA's work (tiles plus per-item cost) over the persistent grid.
+void attn_plan(int batch, int H_kv, int kv_bound, int n_sm, int *n_split, int *split_tok) {
+    const int tiles = (kv_bound + 1 + attn::TILE - 1) / attn::TILE;
+    const int bg = batch * H_kv;
+    int best = 1;
+    double best_cost = 1e30;
+    for (int s = 1; s <= tiles && s <= 64; ++s) {
+        const int per = (tiles + s - 1) / s;  // tiles per split
+        const long items = (long)bg * s;
+        const long rounds = (items + n_sm - 1) / n_sm;
+        const double cost = (double)rounds * (per + GDR_ATTN_ITEM_COST);
+        if (cost < best_cost - 1e-9) {
+            best_cost = cost;
+            best = s;
+        }
+    }
+    *n_split = best;
+    *split_tok = ((tiles + best - 1) / best) * attn::TILE;
+}
+
+cudaError_t launch_attn_decode(AttnParams p, void *workspace, int out_bf16, cudaStream_t s) {
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    p.status = reinterpret_cast<int *>(ws);
+    size_t off = 256;
+    p.q_tiles = reinterpret_cast<__nv_bfloat16 *>(ws + off);
+    off += (size_t)p.batch * p.H_kv * attn::QTILE;
+    off = (off + 255) & ~(size_t)255;
+    p.part_o = reinterpret_cast<float *>(ws + off);
+    off += (size_t)p.n_items * attn::NH * attn::D * 4;
+    p.part_ml = reinterpret_cast<float *>(ws + off);
+    cudaError_t e;
+    int dev = 0, n_sm = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return cudaGetLastError();
+    e = cudaFuncSetAttribute(attn::attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)attn::S_BYTES);
+    if (e != cudaSuccess) return e;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    auto launch = [&](auto kern, unsigned grid, unsigned block, size_t smem) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(block);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cudaError_t r = cudaLaunchKernelEx(&cfg, kern, p);
+        if (r != cudaSuccess) (void)cudaGetLastError();
+        return r;
+    };
+    const unsigned bg = (unsigned)(p.batch * p.H_kv);
+    if ((e = launch(attn::rope_append_kernel, bg, 256, 0)) != cudaSuccess) return e;
+    const unsigned grid = (unsigned)(p.n_items < n_sm ? p.n_items : n_sm);
+    if ((e = launch(attn::attend_kernel, grid, attn::NTHR, attn::S_BYTES)) != cudaSuccess) return e;
+    if (out_bf16)
+        e = launch(attn::combine_kernel<__nv_bfloat16>, bg, 256, 0);
+    else
+        e = launch(attn::combine_kernel<float>, bg, 256, 0);
+    return e;
+}
+
+// Fills the kernels' parameters from checked ABI arguments (strides resolved).
+cudaError_t launch_attn_decode_args(const gdr_attn_decode_args *a, int n_split, int split_tok,
+                                    void *workspace, cudaStream_t s) {
+    AttnParams p = {};
+    p.batch = a->batch;
+    p.H_q = a->H_q;
+    p.H_kv = a->H_kv;
+    p.n_rep = a->H_q / a->H_kv;
+    p.rot_dim = a->rot_dim;
+    p.max_len = a->max_len;
+    p.kv_bound = a->kv_bound;
+    p.n_split = n_split;
+    p.split_tok = split_tok;
+    p.n_items = a->batch * a->H_kv * n_split;
+    p.scale = a->scale;
+    p.log2_theta = log2((double)a->rope_theta);
+    p.q_stride = a->q_stride;
+    p.gate_stride = a->gate_stride;
+    p.k_stride = a->k_stride;
+    p.v_stride = a->v_stride;
+    p.out_stride = a->out_stride;
+    p.q = static_cast<const __nv_bfloat16 *>(a->q);
+    p.gate = static_cast<const __nv_bfloat16 *>(a->gate);
+    p.k = static_cast<const __nv_bfloat16 *>(a->k);
+    p.v = static_cast<const __nv_bfloat16 *>(a->v);
+    p.k_cache = static_cast<__nv_bfloat16 *>(a->k_cache);
+    p.v_cache = static_cast<__nv_bfloat16 *>(a->v_cache);
+    p.cache_len = a->cache_len;
+    p.out = a->out;
+    return launch_attn_decode(p, workspace, a->out_dtype == GDR_BF16, s);
+}
+
+}  // namespace gdr

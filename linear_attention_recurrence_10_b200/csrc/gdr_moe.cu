@@ -1,0 +1,463 @@
+// gdr_moe.cu -- the routed-expert MoE feed-forward block at decode time, reading
+// only the experts the router picks.
+//
+// The Core AI card for the Qwen3.6-35B-A3B text decoder (first section) makes
+// every FFN a 256-expert top-8 mixture with a shared expert: a router
+// Linear(hidden, 256), a softmax over all experts in fp32, the top 8
+// renormalised by their sum, SwitchGLU experts gathered by index, and an
+// always-on shared SwitchGLU scaled by sigmoid(shared_expert_gate(x)); its
+// "Speed" section puts the cost of a decode step in reading only the routed
+// experts' weights instead of all of them.  Per token x:
+//
+//   p     = softmax(W_router x)                 (fp32)
+//   top-k by p (ties to the lower index), w_e = p_e / sum_{top-k} p
+//   y     = sum_e w_e W_down,e (silu(W_gate,e x) * (W_up,e x))
+//         + sigmoid(w_sgate . x) W_down,s (silu(W_gate,s x) * (W_up,s x))
+//
+// Five kernels on the caller's stream, each a programmatic dependent of the
+// one before: it waits for it before reading what it wrote, and each block
+// lets the next kernel launch only once its own stores are issued, so blocks
+// of the next kernel never sit on an SM the current one still needs:
+//   router:  one warp per router row (and one for the shared gate row): the
+//            row's dot products with every token, fp32.
+//   route:   one block: per token the softmax, the top-k and the weights; then
+//            the (token, slot) pairs grouped by expert, the shared expert last
+//            with every token, so that each expert's weights are read once
+//            for all the tokens that chose it.
+//   gate_up: per (active expert, 16 intermediate rows): the gate and up rows
+//            against each of the expert's tokens, h = silu(g) * u (fp32).
+//   down:    per (active expert, 32 output rows): w * (W_down h) per pair.
+//   combine: per token, the sum of its pairs' partial outputs.
+// Weights are bf16; all arithmetic is fp32.  Bound by HBM on the weights read.
+#include "gdr.h"
+#include "gdr_common.cuh"
+
+namespace gdr {
+
+struct MoeParams {
+    int n_tok, hidden, n_exp, top_k, inter, s_inter;
+    int64_t x_stride, out_stride;
+    const __nv_bfloat16 *x, *w_router, *w_gate_up, *w_down, *ws_gate_up, *ws_down, *w_sgate;
+    void *out;
+    int32_t *topk_idx;
+    float *topk_w;
+    // workspace
+    float *logits;      // [n_tok][n_exp + 1]  (the last column: the shared gate's dot product)
+    int *n_active;      // active experts (shared expert included)
+    int *act_expert;    // [n_exp + 1] expert of active slot a (n_exp = the shared expert)
+    int *act_off;       // [n_exp + 2] first pair of slot a
+    int *pair_tok;      // [n_pairs] token of pair i (pairs grouped by expert)
+    float *pair_w;      // [n_pairs] the pair's weight
+    int *tok_pair;      // [n_tok][top_k + 1] pair index of (token, slot); the shared one last
+    float *h;           // [n_pairs][max(inter, s_inter)]
+    float *part;        // [n_pairs][hidden]
+};
+
+namespace moe {
+
+constexpr int GU_ROWS = 16;   // intermediate rows per gate_up block (x 2: gate and up)
+constexpr int DN_ROWS = 32;   // output rows per down block
+constexpr int ROUTE_THREADS = 1024;
+constexpr int MAXE_LANE = 32;  // experts per lane in the router's softmax: n_exp <= 1024
+
+// Dot products of ROWS bf16 rows with one bf16 vector x of n values (n a
+// multiple of 8), by one warp: lane l takes 16-byte chunks l, l + 32, ...; the
+// rows' chunks for a batch of 8 chunk steps are all loaded before any is used,
+// so each lane keeps 8 * ROWS 16-byte loads in flight.  Returns the warp sums.
+template <int ROWS>
+__device__ __forceinline__ void warp_dots_bf16(const __nv_bfloat16 *const (&w)[ROWS],
+                                               const __nv_bfloat16 *x, int n, int lane,
+                                               float (&out)[ROWS]) {
+    float acc[ROWS];
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r) acc[r] = 0.f;
+    const int nc = n / 8;
+    for (int c0 = 0; c0 < nc; c0 += 32 * 8) {
+        uint4 a[ROWS][8], b[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int c = c0 + lane + 32 * u;
+            b[u] = c < nc ? __ldg(reinterpret_cast<const uint4 *>(x) + c) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int r = 0; r < ROWS; ++r)
+                a[r][u] = c < nc ? __ldg(reinterpret_cast<const uint4 *>(w[r]) + c) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&b[u]);
+#pragma unroll
+            for (int r = 0; r < ROWS; ++r) {
+                const __nv_bfloat162 *a2 = reinterpret_cast<const __nv_bfloat162 *>(&a[r][u]);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const float2 fa = __bfloat1622float2(a2[v]), fb = __bfloat1622float2(b2[v]);
+                    acc[r] = fmaf(fa.x, fb.x, fmaf(fa.y, fb.y, acc[r]));
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r) out[r] = group_sum<32>(acc[r]);
+}
+
+// ------------------------------------------------------------------ router
+// One warp per router row e (e == n_exp: the shared-expert gate), every token.
+__global__ void __launch_bounds__(256) router_kernel(const MoeParams p) {
+    wait_for_predecessor();
+    const int lane = threadIdx.x & 31;
+    const int e = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const bool shared_row = e == p.n_exp;
+    if (e > p.n_exp || (shared_row && p.s_inter == 0)) return;
+    const __nv_bfloat16 *w[1] = {shared_row ? p.w_sgate : p.w_router + (size_t)e * p.hidden};
+    for (int t = 0; t < p.n_tok; ++t) {
+        float d[1];
+        warp_dots_bf16<1>(w, p.x + (int64_t)t * p.x_stride, p.hidden, lane, d);
+        if (lane == 0) p.logits[(size_t)t * (p.n_exp + 1) + e] = d[0];
+    }
+    release_dependents();
+}
+
+// ------------------------------------------------------------------- route
+// One block: softmax, top-k and weights per token (one warp per token), then
+// the pairs grouped by expert.
+__global__ void __launch_bounds__(ROUTE_THREADS) route_kernel(const MoeParams p) {
+    wait_for_predecessor();
+    extern __shared__ int rsm[];
+    int *cnt = rsm;                      // [n_exp + 1] tokens per expert
+    int *fill = cnt + (p.n_exp + 1);     // [n_exp + 1] running fill per expert
+    int *slot_of = fill + (p.n_exp + 1); // [n_exp + 1] active slot of expert e (or -1)
+    int *sel = slot_of + (p.n_exp + 1);  // [n_tok][top_k] selected experts
+    float *selw = reinterpret_cast<float *>(sel + p.n_tok * p.top_k);  // [n_tok][top_k]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int E = p.n_exp, K = p.top_k;
+    const bool has_shared = p.s_inter > 0;
+    for (int e = tid; e <= E; e += blockDim.x) cnt[e] = 0;
+    __syncthreads();
+    for (int t = warp; t < p.n_tok; t += blockDim.x / 32) {
+        // Lane l holds the probabilities of experts l, l + 32, ... in registers.
+        const float *lg = p.logits + (size_t)t * (E + 1);
+        float pr[MAXE_LANE];
+        float m = -INFINITY;
+#pragma unroll
+        for (int u = 0; u < MAXE_LANE; ++u) {
+            const int e = lane + 32 * u;
+            pr[u] = e < E ? lg[e] : -INFINITY;
+            m = fmaxf(m, pr[u]);
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
+        float z = 0.f;
+#pragma unroll
+        for (int u = 0; u < MAXE_LANE; ++u) {
+            pr[u] = lane + 32 * u < E ? expf(pr[u] - m) : 0.f;
+            z += pr[u];
+        }
+        z = group_sum<32>(z);
+        const float rz = 1.f / z;
+#pragma unroll
+        for (int u = 0; u < MAXE_LANE; ++u) pr[u] = lane + 32 * u < E ? pr[u] * rz : -1.f;
+        // Top-k, ties to the lower index: k rounds of a warp arg-max over each
+        // lane's best untaken expert; the winner's lane marks it taken.
+        uint32_t taken = 0;
+        float wsum = 0.f;
+        for (int k = 0; k < K; ++k) {
+            float bv = -1.f;
+            int bi = 0x7fffffff;
+#pragma unroll
+            for (int u = 0; u < MAXE_LANE; ++u) {
+                if (!((taken >> u) & 1u) && pr[u] > bv) {  // u ascending: ties keep the lower index
+                    bv = pr[u];
+                    bi = lane + 32 * u;
+                }
+            }
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) {
+                const float ov = __shfl_xor_sync(kFullMask, bv, o);
+                const int oi = __shfl_xor_sync(kFullMask, bi, o);
+                if (ov > bv || (ov == bv && oi < bi)) {
+                    bv = ov;
+                    bi = oi;
+                }
+            }
+            if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+            if (lane == 0) {
+                sel[t * K + k] = bi;
+                selw[t * K + k] = bv;
+                atomicAdd(&cnt[bi], 1);
+            }
+            wsum += bv;
+        }
+        __syncwarp();
+        if (lane < K) {
+            const float wk = selw[t * K + lane] / wsum;
+            selw[t * K + lane] = wk;
+            if (p.topk_idx) p.topk_idx[(size_t)t * K + lane] = sel[t * K + lane];
+            if (p.topk_w) p.topk_w[(size_t)t * K + lane] = wk;
+        }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        // Active slots in expert order, the shared expert last; pair offsets.
+        int a = 0, off = 0;
+        for (int e = 0; e < E; ++e) {
+            slot_of[e] = -1;
+            if (cnt[e] > 0) {
+                slot_of[e] = a;
+                p.act_expert[a] = e;
+                p.act_off[a] = off;
+                fill[e] = off;
+                off += cnt[e];
+                ++a;
+            }
+        }
+        if (has_shared) {
+            slot_of[E] = a;
+            p.act_expert[a] = E;
+            p.act_off[a] = off;
+            fill[E] = off;
+            off += p.n_tok;
+            ++a;
+        }
+        p.act_off[a] = off;
+        *p.n_active = a;
+    }
+    __syncthreads();
+    // Pairs: (token, slot k) under its expert, in token order (one thread per token).
+    for (int t = tid; t < p.n_tok; t += blockDim.x) {
+        for (int k = 0; k < K; ++k) {
+            const int e = sel[t * K + k];
+            const int i = atomicAdd(&fill[e], 1);
+            p.pair_tok[i] = t;
+            p.pair_w[i] = selw[t * K + k];
+            p.tok_pair[(size_t)t * (K + 1) + k] = i;
+        }
+        if (has_shared) {
+            const int i = p.act_off[slot_of[E]] + t;
+            const float s = p.logits[(size_t)t * (E + 1) + E];
+            p.pair_tok[i] = t;
+            p.pair_w[i] = 1.f / (1.f + expf(-s));
+            p.tok_pair[(size_t)t * (K + 1) + K] = i;
+        }
+    }
+    release_dependents();
+}
+
+// ---------------------------------------------------------------- gate_up
+// Block (a, j0): rows j0 .. j0+15 of the gate and up matrices of active
+// expert a; warp w takes rows j0 + 2w, j0 + 2w + 1.  h = silu(g) * u per pair.
+__global__ void __launch_bounds__(256) gate_up_kernel(const MoeParams p) {
+    wait_for_predecessor();
+    const int a = blockIdx.y;
+    if (a >= *p.n_active) return;
+    const int e = p.act_expert[a];
+    const bool sh = e == p.n_exp;
+    const int I = sh ? p.s_inter : p.inter;
+    const int j0 = blockIdx.x * GU_ROWS;
+    if (j0 >= I) return;
+    const __nv_bfloat16 *W = sh ? p.ws_gate_up : p.w_gate_up + (size_t)e * 2 * p.inter * p.hidden;
+    const int p0 = p.act_off[a], p1 = p.act_off[a + 1];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int hmax = p.inter > p.s_inter ? p.inter : p.s_inter;
+    // The warp's two rows of the gate matrix and the same two of the up matrix,
+    // all four streamed together for each of the expert's tokens.
+    const int j = j0 + 2 * warp;
+    if (j >= I) return;
+    const int j1 = j + 1 < I ? j + 1 : j;
+    const __nv_bfloat16 *w[4] = {W + (size_t)j * p.hidden, W + (size_t)j1 * p.hidden,
+                                 W + (size_t)(I + j) * p.hidden, W + (size_t)(I + j1) * p.hidden};
+    for (int i = p0; i < p1; ++i) {
+        float d[4];
+        warp_dots_bf16<4>(w, p.x + (int64_t)p.pair_tok[i] * p.x_stride, p.hidden, lane, d);
+        if (lane == 0) {
+            p.h[(size_t)i * hmax + j] = d[0] / (1.f + expf(-d[0])) * d[2];
+            if (j1 != j) p.h[(size_t)i * hmax + j1] = d[1] / (1.f + expf(-d[1])) * d[3];
+        }
+    }
+    release_dependents();
+}
+
+// ------------------------------------------------------------------- down
+// Block (a, i0): output rows i0 .. i0+31 of active expert a's down matrix;
+// warp w takes rows i0 + 4w .. i0 + 4w + 3.  part[pair] = w_pair * W_down h.
+__global__ void __launch_bounds__(256) down_kernel(const MoeParams p) {
+    wait_for_predecessor();
+    const int a = blockIdx.y;
+    if (a >= *p.n_active) return;
+    const int e = p.act_expert[a];
+    const bool sh = e == p.n_exp;
+    const int I = sh ? p.s_inter : p.inter;
+    const __nv_bfloat16 *W = sh ? p.ws_down : p.w_down + (size_t)e * p.hidden * p.inter;
+    const int p0 = p.act_off[a], p1 = p.act_off[a + 1];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int hmax = p.inter > p.s_inter ? p.inter : p.s_inter;
+    // The warp's four rows, their weights loaded once into registers (the rows
+    // are I values: I / 256 16-byte chunks per lane), then every pair's h.
+    constexpr int MAXC = 4;  // chunks per lane: I <= 1024
+    const int row0 = blockIdx.x * DN_ROWS + 4 * warp;
+    if (row0 >= p.hidden) return;
+    const int nc = I / 8;
+    uint4 wv[4][MAXC];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int row = min(row0 + r, p.hidden - 1);
+#pragma unroll
+        for (int u = 0; u < MAXC; ++u) {
+            const int c = lane + 32 * u;
+            wv[r][u] = c < nc ? __ldg(reinterpret_cast<const uint4 *>(W + (size_t)row * I) + c)
+                              : make_uint4(0, 0, 0, 0);
+        }
+    }
+    for (int i = p0; i < p1; ++i) {
+        const float *hp = p.h + (size_t)i * hmax;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int u = 0; u < MAXC; ++u) {
+            const int c = lane + 32 * u;
+            if (c >= nc) break;
+            const float4 h0 = *reinterpret_cast<const float4 *>(hp + 8 * c);
+            const float4 h1 = *reinterpret_cast<const float4 *>(hp + 8 * c + 4);
+            const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const __nv_bfloat162 *w2 = reinterpret_cast<const __nv_bfloat162 *>(&wv[r][u]);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const float2 f = __bfloat1622float2(w2[v]);
+                    acc[r] = fmaf(f.x, hv[2 * v], fmaf(f.y, hv[2 * v + 1], acc[r]));
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const float a = group_sum<32>(acc[r]);
+            if (lane == 0 && row0 + r < p.hidden)
+                p.part[(size_t)i * p.hidden + row0 + r] = p.pair_w[i] * a;
+        }
+    }
+    release_dependents();
+}
+
+// ---------------------------------------------------------------- combine
+template <typename TOUT>
+__global__ void __launch_bounds__(256) combine_kernel(const MoeParams p) {
+    wait_for_predecessor();
+    const int t = blockIdx.x;
+    const int np = p.top_k + (p.s_inter > 0 ? 1 : 0);
+    const int *tp = p.tok_pair + (size_t)t * (p.top_k + 1);
+    TOUT *out = static_cast<TOUT *>(p.out) + (int64_t)t * p.out_stride;
+    for (int i = threadIdx.x; i < p.hidden; i += blockDim.x) {
+        float y = 0.f;
+        for (int k = 0; k < np; ++k) y += p.part[(size_t)tp[k] * p.hidden + i];
+        Elem<TOUT>::store1(out + i, y);
+    }
+    release_dependents();
+}
+
+}  // namespace moe
+
+// Workspace layout (256-byte aligned pieces).
+struct MoeWs {
+    size_t logits, n_active, act_expert, act_off, pair_tok, pair_w, tok_pair, h, part, total;
+};
+static MoeWs moe_ws(int n_tok, int n_exp, int top_k, int inter, int s_inter, int hidden) {
+    auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t pairs = (size_t)n_tok * (top_k + (s_inter > 0 ? 1 : 0));
+    const int hmax = inter > s_inter ? inter : s_inter;
+    MoeWs w;
+    size_t o = 0;
+    w.logits = o; o = al(o + (size_t)n_tok * (n_exp + 1) * 4);
+    w.n_active = o; o = al(o + 4);
+    w.act_expert = o; o = al(o + (size_t)(n_exp + 1) * 4);
+    w.act_off = o; o = al(o + (size_t)(n_exp + 2) * 4);
+    w.pair_tok = o; o = al(o + pairs * 4);
+    w.pair_w = o; o = al(o + pairs * 4);
+    w.tok_pair = o; o = al(o + (size_t)n_tok * (top_k + 1) * 4);
+    w.h = o; o = al(o + pairs * hmax * 4);
+    w.part = o; o = al(o + pairs * hidden * 4);
+    w.total = o;
+    return w;
+}
+
+size_t moe_workspace_bytes(int n_tok, int n_exp, int top_k, int inter, int s_inter, int hidden) {
+    return moe_ws(n_tok, n_exp, top_k, inter, s_inter, hidden).total;
+}
+
+size_t moe_route_smem_bytes(int n_tok, int n_exp, int top_k) {
+    return (size_t)3 * (n_exp + 1) * 4 + (size_t)n_tok * top_k * 8;
+}
+
+cudaError_t launch_moe_args(const gdr_moe_args *a, void *workspace, cudaStream_t s) {
+    MoeParams p = {};
+    p.n_tok = a->n_tok;
+    p.hidden = a->hidden;
+    p.n_exp = a->n_exp;
+    p.top_k = a->top_k;
+    p.inter = a->inter;
+    p.s_inter = a->ws_gate_up ? a->s_inter : 0;
+    p.x_stride = a->x_stride;
+    p.out_stride = a->out_stride;
+    p.x = static_cast<const __nv_bfloat16 *>(a->x);
+    p.w_router = static_cast<const __nv_bfloat16 *>(a->w_router);
+    p.w_gate_up = static_cast<const __nv_bfloat16 *>(a->w_gate_up);
+    p.w_down = static_cast<const __nv_bfloat16 *>(a->w_down);
+    p.ws_gate_up = static_cast<const __nv_bfloat16 *>(a->ws_gate_up);
+    p.ws_down = static_cast<const __nv_bfloat16 *>(a->ws_down);
+    p.w_sgate = static_cast<const __nv_bfloat16 *>(a->w_sgate);
+    p.out = a->out;
+    p.topk_idx = a->topk_idx;
+    p.topk_w = a->topk_w;
+    const MoeWs w = moe_ws(p.n_tok, p.n_exp, p.top_k, p.inter, p.s_inter, p.hidden);
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    p.logits = reinterpret_cast<float *>(ws + w.logits);
+    p.n_active = reinterpret_cast<int *>(ws + w.n_active);
+    p.act_expert = reinterpret_cast<int *>(ws + w.act_expert);
+    p.act_off = reinterpret_cast<int *>(ws + w.act_off);
+    p.pair_tok = reinterpret_cast<int *>(ws + w.pair_tok);
+    p.pair_w = reinterpret_cast<float *>(ws + w.pair_w);
+    p.tok_pair = reinterpret_cast<int *>(ws + w.tok_pair);
+    p.h = reinterpret_cast<float *>(ws + w.h);
+    p.part = reinterpret_cast<float *>(ws + w.part);
+
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    auto launch = [&](auto kern, dim3 grid, unsigned block, size_t smem) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = grid;
+        cfg.blockDim = dim3(block);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cudaError_t r = cudaLaunchKernelEx(&cfg, kern, p);
+        if (r != cudaSuccess) (void)cudaGetLastError();
+        return r;
+    };
+    cudaError_t e;
+    const int rows = p.n_exp + 1;
+    if ((e = launch(moe::router_kernel, dim3((rows + 7) / 8), 256, 0)) != cudaSuccess) return e;
+    const size_t rsm = moe_route_smem_bytes(p.n_tok, p.n_exp, p.top_k);
+    if (rsm > 48 * 1024) {
+        e = cudaFuncSetAttribute(moe::route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)rsm);
+        if (e != cudaSuccess) return e;
+    }
+    if ((e = launch(moe::route_kernel, dim3(1), moe::ROUTE_THREADS, rsm)) != cudaSuccess) return e;
+    // Active slots: at most min(n_tok * top_k, n_exp) routed experts and the shared one.
+    const long routed = (long)p.n_tok * p.top_k < p.n_exp ? (long)p.n_tok * p.top_k : p.n_exp;
+    const unsigned max_active = (unsigned)(routed + (p.s_inter > 0 ? 1 : 0));
+    const int imax = p.inter > p.s_inter ? p.inter : p.s_inter;
+    if ((e = launch(moe::gate_up_kernel, dim3((imax + moe::GU_ROWS - 1) / moe::GU_ROWS, max_active),
+                    256, 0)) != cudaSuccess)
+        return e;
+    if ((e = launch(moe::down_kernel, dim3((p.hidden + moe::DN_ROWS - 1) / moe::DN_ROWS, max_active),
+                    256, 0)) != cudaSuccess)
+        return e;
+    if (a->out_dtype == GDR_BF16)
+        e = launch(moe::combine_kernel<__nv_bfloat16>, dim3(p.n_tok), 256, 0);
+    else
+        e = launch(moe::combine_kernel<float>, dim3(p.n_tok), 256, 0);
+    return e;
+}
+
+}  // namespace gdr

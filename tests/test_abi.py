@@ -275,3 +275,139 @@ def test_norm_zero_rows_is_noop(lib):
 def test_binding_fails_loudly_without_library(tmp_path):
     with pytest.raises(RuntimeError, match="missing"):
         _abi.lib(str(tmp_path / "libgdr.so"))
+
+
+@host_only
+def test_selftest_wait_expiry_host_checks(lib):
+    """The wait-expiry self-test refuses, before anything is queued, a wait limit
+    outside its range, a shape that does not take the tensor cores, a workspace
+    too small for the two-kernel path and an empty batch."""
+    f = lib.gdr_prefill_selftest_wait_expiry
+    a, host = _prefill_args()
+    n = ctypes.c_size_t(0)
+    assert lib.gdr_prefill_workspace_size(ctypes.byref(a), ctypes.byref(n)) == OK
+    ws = FAKE + (40 << 32)
+    assert f(ctypes.byref(a), ws, n.value, 10, None) == INVALID                # < 0.1 ms
+    assert f(ctypes.byref(a), ws, n.value, 3_000_000_000, None) == INVALID     # > 2 s
+    assert f(ctypes.byref(a), ws, 256, 20_000_000, None) == WORKSPACE
+    b, host_b = _prefill_args(in_dtype=0)                                      # fp32 inputs
+    assert f(ctypes.byref(b), ws, n.value, 20_000_000, None) == UNSUPPORTED
+    c, host_c = _prefill_args(lens=())
+    assert f(ctypes.byref(c), ws, n.value, 20_000_000, None) == INVALID
+
+
+@host_only
+def test_noalloc_status_rejects_null(lib):
+    assert lib.gdr_prefill_noalloc_status(None, None) == INVALID
+
+
+def _attn_args(**kw):
+    a = _abi.AttnDecodeArgs()
+    a.batch, a.H_q, a.H_kv, a.d = 4, 16, 2, 256
+    a.rot_dim, a.max_len, a.kv_bound, a.out_dtype = 64, 512, 511, 0
+    a.rope_theta, a.scale = 1e7, 1.0 / 16
+    for i, name in enumerate(["q", "gate", "k", "v", "k_cache", "v_cache", "cache_len", "out"]):
+        setattr(a, name, FAKE + (i << 32))
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+ATTN_CASES = [
+    ("null_q", dict(q=None), INVALID),
+    ("null_cache_len", dict(cache_len=None), INVALID),
+    ("heads_not_multiple", dict(H_q=15), INVALID),
+    ("too_many_query_heads_per_kv", dict(H_q=64, H_kv=2), UNSUPPORTED),
+    ("d128", dict(d=128), UNSUPPORTED),
+    ("odd_rot_dim", dict(rot_dim=63), INVALID),
+    ("rot_dim_past_d", dict(rot_dim=258), INVALID),
+    ("bound_past_capacity", dict(kv_bound=512), INVALID),
+    ("negative_bound", dict(kv_bound=-1), INVALID),
+    ("bad_theta", dict(rope_theta=0.0), INVALID),
+    ("bad_out_dtype", dict(out_dtype=4), INVALID),
+    ("misaligned_k_cache", dict(k_cache=FAKE + 8), MISALIGNED),
+    ("misaligned_cache_len", dict(cache_len=FAKE + 2), MISALIGNED),
+    ("stride_too_small", dict(q_stride=256), INVALID),
+]
+
+
+@host_only
+@pytest.mark.parametrize("name,kw,want", ATTN_CASES, ids=[c[0] for c in ATTN_CASES])
+def test_attn_validation(lib, name, kw, want):
+    a = _attn_args(**kw)
+    n = ctypes.c_size_t(1 << 30)
+    assert lib.gdr_attn_decode_step(ctypes.byref(a), FAKE + (50 << 32), n, None) == want
+
+
+@host_only
+def test_attn_workspace(lib):
+    a = _attn_args()
+    n = ctypes.c_size_t(0)
+    assert lib.gdr_attn_decode_workspace_size(ctypes.byref(a), ctypes.byref(n)) == OK
+    assert n.value > 4 * 2 * 256 * 16 * 4  # at least one split's partials per (b, kv head)
+    assert lib.gdr_attn_decode_step(ctypes.byref(a), FAKE + (50 << 32), n.value - 16, None) == WORKSPACE
+    assert lib.gdr_attn_decode_step(ctypes.byref(a), None, n.value, None) == WORKSPACE
+    empty = _attn_args(batch=0)
+    assert lib.gdr_attn_decode_workspace_size(ctypes.byref(empty), ctypes.byref(n)) == OK
+    assert n.value == 0
+    assert lib.gdr_attn_decode_step(ctypes.byref(empty), None, 0, None) == OK
+
+
+def _moe_args(**kw):
+    a = _abi.MoeArgs()
+    a.n_tok, a.hidden, a.n_exp, a.top_k, a.inter, a.s_inter = 4, 2048, 256, 8, 512, 512
+    a.out_dtype = 0
+    for i, name in enumerate(["x", "w_router", "w_gate_up", "w_down", "ws_gate_up", "ws_down",
+                              "w_sgate", "out", "topk_idx", "topk_w"]):
+        setattr(a, name, FAKE + (i << 32))
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+MOE_CASES = [
+    ("null_x", dict(x=None), INVALID),
+    ("null_down", dict(w_down=None), INVALID),
+    ("shared_without_down", dict(ws_down=None), INVALID),
+    ("shared_without_width", dict(s_inter=0), INVALID),
+    ("top_k_zero", dict(top_k=0), INVALID),
+    ("top_k_past_experts", dict(n_exp=4, top_k=8), INVALID),
+    ("top_k_too_large", dict(n_exp=64, top_k=33), UNSUPPORTED),
+    ("hidden_not_multiple_of_8", dict(hidden=2044), UNSUPPORTED),
+    ("negative_tokens", dict(n_tok=-1), INVALID),
+    ("reserved_set", dict(reserved=1), INVALID),
+    ("misaligned_weights", dict(w_gate_up=FAKE + 8), MISALIGNED),
+    ("misaligned_topk", dict(topk_idx=FAKE + 2), MISALIGNED),
+    ("stride_too_small", dict(x_stride=1024), INVALID),
+]
+
+
+@host_only
+@pytest.mark.parametrize("name,kw,want", MOE_CASES, ids=[c[0] for c in MOE_CASES])
+def test_moe_validation(lib, name, kw, want):
+    a = _moe_args(**kw)
+    assert lib.gdr_moe_decode(ctypes.byref(a), FAKE + (60 << 32), 1 << 30, None) == want
+
+
+@host_only
+def test_moe_workspace(lib):
+    a = _moe_args()
+    n = ctypes.c_size_t(0)
+    assert lib.gdr_moe_workspace_size(ctypes.byref(a), ctypes.byref(n)) == OK
+    # at least the per-pair partial outputs: 4 tokens x (8 + 1) pairs x 2048 fp32
+    assert n.value >= 4 * 9 * 2048 * 4
+    assert lib.gdr_moe_decode(ctypes.byref(a), FAKE + (60 << 32), n.value - 256, None) == WORKSPACE
+    no_shared = _moe_args(ws_gate_up=None, ws_down=None, w_sgate=None, s_inter=0)
+    m = ctypes.c_size_t(0)
+    assert lib.gdr_moe_workspace_size(ctypes.byref(no_shared), ctypes.byref(m)) == OK
+    assert m.value < n.value
+    empty = _moe_args(n_tok=0)
+    assert lib.gdr_moe_workspace_size(ctypes.byref(empty), ctypes.byref(m)) == OK and m.value == 0
+    assert lib.gdr_moe_decode(ctypes.byref(empty), None, 0, None) == OK
+
+
+@host_only
+@pytest.mark.parametrize("kw", [dict(inter=1032), dict(s_inter=2048), dict(n_exp=1025, top_k=8)])
+def test_moe_size_limits(lib, kw):
+    a = _moe_args(**kw)
+    assert lib.gdr_moe_decode(ctypes.byref(a), FAKE + (60 << 32), 1 << 30, None) == UNSUPPORTED

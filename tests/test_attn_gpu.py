@@ -1,0 +1,141 @@
+"""Gated full-attention decode step (gdr_attn_decode_step) against the fp64 oracle.
+
+The layer is the other mixer of the hybrid decoder (GatedAttention in the Qwen3.5
+Chat guide, section "Architektur"; head_dim 256, GQA 16/2, partial rotary
+embedding with theta 1e7 on the Core AI Qwen3.6-35B-A3B card, first section).
+The oracle receives the exact bf16 inputs widened to fp64.
+
+Tolerance.  Three roundings to bf16 sit inside the kernel: the rotated query
+(the MMA operand), the rotated new key (stored in the cache, like every cached
+key) and the softmax weights P (the operand of P V).  Each is a relative error
+of at most 2^-9 per element, about 1.1e-3 RMS; they enter the output roughly
+independently, ~2e-3 together, so the bar is a relative L2 of 5e-3 (2.5x that)
+with the element-wise bound of gdr_testutil.  bf16 outputs are compared with
+the oracle rounded to bf16 at the same bar plus one bf16 ulp per element.
+"""
+import numpy as np
+import pytest
+import torch
+
+import linear_attention_recurrence_10_b200 as gdr
+import oracle
+from gdr_testutil import assert_close, f64
+
+pytestmark = pytest.mark.gpu
+
+TOL = 5e-3
+D = 256
+
+
+def _inputs(B, H_q, H_kv, max_len, lens, seed, fill=float("nan")):
+    g = torch.Generator().manual_seed(seed)
+    bf = lambda *s: torch.randn(*s, generator=g).to(torch.bfloat16)
+    x = dict(q=bf(B, H_q, D), gate=bf(B, H_q, D), k=bf(B, H_kv, D), v=bf(B, H_kv, D),
+             k_cache=bf(B, H_kv, max_len, D), v_cache=bf(B, H_kv, max_len, D))
+    for b, L in enumerate(lens):  # rows past the cached ones hold garbage
+        x["k_cache"][b, :, L:] = fill
+        x["v_cache"][b, :, L:] = fill
+    x["cache_len"] = torch.tensor(lens, dtype=torch.int32)
+    return x
+
+
+def _run(x, kv_bound, rot_dim=64, out_dtype=torch.float32, theta=1e7):
+    d = {k: v.cuda() for k, v in x.items()}
+    B, H_q = x["q"].shape[:2]
+    out = torch.full((B, H_q, D), float("nan"), device="cuda", dtype=out_dtype)
+    n = gdr.attn_decode_workspace_size(d["q"], d["gate"], d["k"], d["v"], d["k_cache"],
+                                       d["v_cache"], d["cache_len"], out, kv_bound=kv_bound,
+                                       rot_dim=rot_dim, rope_theta=theta)
+    ws = torch.full((n,), 0xAB, dtype=torch.uint8, device="cuda")
+    gdr.attn_decode_step(d["q"], d["gate"], d["k"], d["v"], d["k_cache"], d["v_cache"],
+                         d["cache_len"], out, kv_bound=kv_bound, rot_dim=rot_dim,
+                         rope_theta=theta, workspace=ws)
+    torch.cuda.synchronize()
+    return out, d, int(ws[:4].view(torch.int32).item())
+
+
+def _oracle(x, rot_dim=64, theta=1e7):
+    return oracle.gated_attn_decode(f64(x["q"]), f64(x["gate"]), f64(x["k"]), f64(x["v"]),
+                                    np.nan_to_num(f64(x["k_cache"])),
+                                    np.nan_to_num(f64(x["v_cache"])),
+                                    x["cache_len"].numpy(), rot_dim=rot_dim, theta=theta)
+
+
+def _check_cache(x, d, ref):
+    """Row cache_len[b] holds the rotated key (bf16 of the oracle's, one ulp)
+    and the value; every other row is bit-for-bit what it was."""
+    kc, vc = d["k_cache"].cpu(), d["v_cache"].cpu()
+    for b, L in enumerate(x["cache_len"].tolist()):
+        want = torch.from_numpy(ref.k_rot[b]).to(torch.bfloat16).double().numpy()
+        got = f64(kc[b, :, L])
+        assert np.all(np.abs(got - want) <= np.abs(want) * 2.0 ** -7 + 1e-6), b
+        assert torch.equal(vc[b, :, L].view(torch.int16), x["v"][b].view(torch.int16))
+        keep = [t for t in range(kc.shape[2]) if t != L]
+        assert torch.equal(kc[b, :, keep].view(torch.int16), x["k_cache"][b, :, keep].view(torch.int16))
+        assert torch.equal(vc[b, :, keep].view(torch.int16), x["v_cache"][b, :, keep].view(torch.int16))
+
+
+@pytest.mark.parametrize("heads", [(16, 2), (2, 2), (32, 2), (8, 8)])
+def test_ragged_lengths_match_oracle(heads):
+    H_q, H_kv = heads
+    lens = [0, 37, 255, 128, 1]
+    x = _inputs(len(lens), H_q, H_kv, 300, lens, seed=700 + H_q)
+    out, d, status = _run(x, kv_bound=299)
+    assert status == 0
+    ref = _oracle(x)
+    assert_close(f64(out), ref.y, TOL, "outputs")
+    _check_cache(x, d, ref)
+
+
+@pytest.mark.parametrize("rot_dim", [0, 64, 256])
+def test_rotary_dims_and_bf16_output(rot_dim):
+    lens = [300, 5, 129]
+    x = _inputs(3, 16, 2, 320, lens, seed=710 + rot_dim)
+    ref = _oracle(x, rot_dim=rot_dim)
+    out, d, status = _run(x, kv_bound=319, rot_dim=rot_dim)
+    assert status == 0
+    assert_close(f64(out), ref.y, TOL, "fp32 outputs")
+    out16, _, _ = _run(x, kv_bound=319, rot_dim=rot_dim, out_dtype=torch.bfloat16)
+    ref16 = torch.from_numpy(ref.y).to(torch.bfloat16).double().numpy()
+    assert_close(f64(out16), ref16, TOL, "bf16 outputs", bf16_ulp=True)
+
+
+def test_two_steps_attend_the_appended_token():
+    """Step 1 appends at row L; step 2 (cache_len + 1) attends over it."""
+    lens = [40, 200]
+    x = _inputs(2, 16, 2, 256, lens, seed=720)
+    out1, d, status = _run(x, kv_bound=255)
+    assert status == 0
+    x2 = _inputs(2, 16, 2, 256, lens, seed=721)
+    x2["k_cache"], x2["v_cache"] = d["k_cache"].cpu(), d["v_cache"].cpu()
+    x2["cache_len"] = x["cache_len"] + 1
+    out2, _, status = _run(x2, kv_bound=255)
+    assert status == 0
+    assert_close(f64(out2), _oracle(x2).y, TOL, "second step")
+
+
+def test_length_past_the_bound_is_reported():
+    lens = [10, 90]
+    x = _inputs(2, 16, 2, 128, lens, seed=730)
+    out, d, status = _run(x, kv_bound=50)
+    assert status == 1  # GDR_ERR_INVALID_ARG
+    # The sequence within the bound is still right and appended; the other is not appended.
+    ref = _oracle(x)
+    assert_close(f64(out[0]), ref.y[0], TOL, "sequence within the bound")
+    assert torch.equal(d["k_cache"][1, :, 90].cpu().view(torch.int16),
+                       x["k_cache"][1, :, 90].view(torch.int16))
+
+
+@pytest.mark.slow
+def test_qwen36_attention_decode_full():
+    """Qwen3.6-35B-A3B-shaped gated attention decode: B=64, 16/2 heads, d=256,
+    4096 cached tokens per sequence; every output and appended row."""
+    B, L = 64, 4096
+    x = _inputs(B, 16, 2, L + 1, [L] * B, seed=740, fill=0.0)
+    out, d, status = _run(x, kv_bound=L)
+    assert status == 0
+    ref = _oracle(x)
+    assert_close(f64(out), ref.y, TOL, "outputs")
+    kc = d["k_cache"][:, :, L].cpu()
+    want = torch.from_numpy(ref.k_rot).to(torch.bfloat16).double().numpy()
+    assert np.all(np.abs(f64(kc) - want) <= np.abs(want) * 2.0 ** -7 + 1e-6)

@@ -128,6 +128,18 @@ def test_every_entry_reaches_the_launch_without_a_device():
             rows(n_tok), rows(n_tok), rows(n_tok), gp, bp, cu, rows(n_tok), **pre),
         "gdr_prefill_chunked_noalloc": lambda: gdr.prefill_chunked_noalloc(
             rows(n_tok), rows(n_tok), rows(n_tok), gp, bp, cu, rows(n_tok), **pre),
+        "gdr_attn_decode_step": lambda: gdr.attn_decode_step(
+            torch.randn(3, 16, 256, dtype=bf), torch.randn(3, 16, 256, dtype=bf),
+            torch.randn(3, 2, 256, dtype=bf), torch.randn(3, 2, 256, dtype=bf),
+            torch.zeros(3, 2, 64, 256, dtype=bf), torch.zeros(3, 2, 64, 256, dtype=bf),
+            torch.tensor([1, 5, 0], dtype=torch.int32), torch.empty(3, 16, 256),
+            kv_bound=63, stream=0),
+        "gdr_moe_decode": lambda: gdr.moe_decode(
+            torch.randn(2, 256, dtype=bf), torch.randn(8, 256, dtype=bf),
+            torch.randn(8, 64, 256, dtype=bf), torch.randn(8, 256, 32, dtype=bf),
+            torch.empty(2, 256), top_k=2,
+            shared=(torch.randn(32, 256, dtype=bf), torch.randn(256, 16, dtype=bf),
+                    torch.randn(256, dtype=bf)), stream=0),
         "gdr_rmsnorm_gated": lambda: gdr.rmsnorm_gated(
             rows(10, torch.float32), rows(10, torch.float32), rows(10, torch.float32), w=w,
             stream=0),

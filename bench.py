@@ -44,6 +44,20 @@ SLOTS = 512  # distinct per-step inputs (the workload's 512 decode steps), cycle
 IN_BYTES, OUT_BYTES = 2, 2
 # Chunked prefill (reported beside the headline): Qwen3.5-0.8B-shaped prompt batch.
 P_SEQS, P_LEN, P_H, P_CHUNK = 4, 4096, 16, 64
+# Qwen3.6-35B-A3B-shaped GVA decode: 30 GDN layers' states, batch 64, 16 key /
+# 32 value heads, 256 distinct decode steps.
+GVA_LAYERS, GVA_B, GVA_HK, GVA_HV, GVA_STEPS = 30, 64, 16, 32, 256
+# Qwen3.6-35B-A3B-shaped gated full-attention decode: its 10 attention layers
+# (one mixer in four of 40), batch 64, 16 query / 2 key-value heads, head_dim
+# 256, 4096 cached tokens per sequence, rotary embedding on 64 dims, theta 1e7.
+ATT_LAYERS, ATT_B, ATT_HQ, ATT_HKV, ATT_D, ATT_CTX, ATT_ROT = 10, 64, 16, 2, 256, 4096, 64
+# Qwen3.6-35B-A3B-shaped routed-expert MoE block at decode: hidden 2048, 256
+# experts, top 8, expert and shared intermediate 512; 8 layers' weights (12.7 GB
+# in bf16) rotate, one token per step (the pages' single-sequence decode).
+MOE_LAYERS, MOE_H, MOE_E, MOE_K, MOE_I, MOE_SI = 8, 2048, 256, 8, 512, 512
+# Long-context GVA prefill: 8 sequences of U{1024..32768} tokens (seed 4),
+# 16 key / 32 value heads, exp(g) in [0.9, 1).
+LC_SEQS, LC_LO, LC_HI, LC_HK, LC_HV, LC_SEED = 8, 1024, 32768, 16, 32, 4
 
 HEADLINE = "GDN decode state-update GB/s"
 
@@ -62,10 +76,11 @@ def decode_bytes_per_layer_call(B, H_k, H_v, d, T, in_b=IN_BYTES, out_b=OUT_BYTE
     return state + T * per_token
 
 
-def prefill_flops_per_token_head(C, d, gva: bool) -> int:
-    # K K^T, Q K^T, U, W, P Delta at 2 C d each; W S^T, Q S^T, state update at 2 d^2 each.
-    kk_qk = 0 if gva else 4 * C * d
-    return kk_qk + 6 * C * d + 6 * d * d
+def prefill_flops_per_token_head(C, d, hv_per_hk: int = 1) -> int:
+    """Algorithmic FLOPs per (token, value head): K K^T, Q K^T, U, W, P Delta at
+    2 C d each, W S^T, Q S^T and the state update at 2 d^2 each; K K^T and
+    Q K^T belong to the key head, so value heads sharing it share them."""
+    return 4 * C * d // hv_per_hk + 6 * C * d + 6 * d * d
 
 
 def load_peaks():
@@ -150,19 +165,23 @@ class ClockSampler:
 # ----------------------------------------------------------------- decode
 
 class DecodeBench:
-    def __init__(self, device, seed=1, B=BATCH, layers=LAYERS, slots=SLOTS):
+    """One decode token through `layers` independent layer states per step, one
+    library call per layer, replayed from one CUDA graph per step."""
+
+    def __init__(self, device, seed=1, B=BATCH, layers=LAYERS, slots=SLOTS, H_k=H_K, H_v=H_V):
         import linear_attention_recurrence_10_b200 as gdr
         from linear_attention_recurrence_10_b200 import synth
         self.gdr = gdr
         self.B, self.L, self.T = B, layers, slots
-        x = synth.make_decode_inputs(layers, slots, B, H_K, H_V, D, seed=seed, s0_std=0.02,
+        x = synth.make_decode_inputs(layers, slots, B, H_k, H_v, D, seed=seed, s0_std=0.02,
                                      device=device)
         self.x = x
         self.state = x.s0.clone()
-        self.out = torch.empty(layers, B, H_V, D, device=device, dtype=torch.bfloat16)
+        self.out = torch.empty(layers, B, H_v, D, device=device, dtype=torch.bfloat16)
         self.graphs = []
         self.overlap = layers > 1
-        self.bytes_per_step = layers * decode_bytes_per_layer_step(B, H_K, H_V, D)
+        self.bytes_per_launch = decode_bytes_per_layer_step(B, H_k, H_v, D)
+        self.bytes_per_step = layers * self.bytes_per_launch
         self.launches_per_step = layers
 
     def launch_layer(self, l, t, x=None, out=None):
@@ -195,6 +214,56 @@ class DecodeBench:
     def run(self, first, n):
         for s in range(first, first + n):
             self.graphs[s % self.T].replay()
+
+
+class DecodeMultiBench:
+    """The headline layers with T tokens per sequence per call (gdr_decode_multi):
+    each call-step runs the 18 layers once, every launch with
+    GDR_DECODE_OVERLAP_STATE_LOAD, replayed from one CUDA graph per call-step.
+    The state is read and written once per call whatever T."""
+
+    def __init__(self, device, seed=12, B=BATCH, layers=LAYERS, slots=32, T=4):
+        import linear_attention_recurrence_10_b200 as gdr
+        from linear_attention_recurrence_10_b200 import synth
+        self.gdr = gdr
+        self.B, self.L, self.T, self.slots = B, layers, T, slots
+        x = synth.make_decode_inputs(layers, slots * T, B, H_K, H_V, D, seed=seed, s0_std=0.02,
+                                     device=device)
+        # [L, calls, T, B, ...] -> [L, calls, B, T, ...]: each call's rows are b*T + t.
+        per_call = lambda t: t.view(layers, slots, T, B, *t.shape[3:]).transpose(2, 3) \
+            .contiguous().view(layers, slots, B * T, *t.shape[3:])
+        self.q, self.k, self.v, self.z, self.g, self.beta = (
+            per_call(t) for t in (x.q, x.k, x.v, x.z, x.g, x.beta))
+        self.w = x.w
+        self.state = x.s0
+        self.out = torch.empty(layers, B * T, H_V, D, device=device, dtype=torch.bfloat16)
+        self.graphs = []
+        self.bytes_per_call = layers * decode_bytes_per_layer_call(B, H_K, H_V, D, T)
+
+    def enqueue_call(self, c):
+        for l in range(self.L):
+            self.gdr.decode_multi(self.q[l, c], self.k[l, c], self.v[l, c], self.g[l, c],
+                                  self.beta[l, c], self.state[l], self.out[l], n_tokens=self.T,
+                                  z=self.z[l, c], overlap_state_load=True)
+
+    def capture(self):
+        # The binding's per-call host cost would otherwise exceed the kernels' time.
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self.enqueue_call(0)  # load the library and kernels before capture
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        for c in range(self.slots):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr):
+                self.enqueue_call(c)
+            self.graphs.append(gr)
+        torch.cuda.synchronize()
+
+    def run(self, first, n):
+        for s in range(first, first + n):
+            self.graphs[s % self.slots].replay()
 
 
 class DecodeE2E:
@@ -346,61 +415,35 @@ def decode_variants(device, B, steps=64, warmup=4, slots=32, T=4, world=1):
         "tokens_per_s": B * steps / (ms * 1e-3)}
     del q, k, v, z, g, beta, state, out
     # Multi-token calls.
-    x = synth.make_decode_inputs(LAYERS, slots * T, B, H_K, H_V, D, seed=12, s0_std=0.02,
-                                 device=device)
-    # [L, calls, T, B, ...] -> [L, calls, B, T, ...]: each call's rows are b*T + t.
-    per_call = lambda t: t.view(LAYERS, slots, T, B, *t.shape[3:]).transpose(2, 3).contiguous() \
-        .view(LAYERS, slots, B * T, *t.shape[3:])
-    q, k, v, z, g, beta = (per_call(t) for t in (x.q, x.k, x.v, x.z, x.g, x.beta))
-    state = x.s0
-    out = torch.empty(B * T, H_V, D, device=device, dtype=torch.bfloat16)
-    del x
-
-    def enqueue_call(c):
-        for l in range(LAYERS):
-            gdr.decode_multi(q[l, c], k[l, c], v[l, c], g[l, c], beta[l, c], state[l], out,
-                             n_tokens=T, z=z[l, c], overlap_state_load=True)
-
-    # One CUDA graph per call, as for the headline (the binding's per-call host
-    # cost would otherwise exceed the kernels' time).
-    side = torch.cuda.Stream()
-    side.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(side):
-        enqueue_call(0)
-    torch.cuda.current_stream().wait_stream(side)
-    torch.cuda.synchronize()
-    graphs = []
-    for c in range(slots):
-        gr = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gr):
-            enqueue_call(c)
-        graphs.append(gr)
-
-    def multi_call(s):
-        graphs[s % slots].replay()
-
-    for s in range(warmup):
-        multi_call(s)
-    ms = time_region(lambda: [multi_call(warmup + s) for s in range(steps)], steps, world)
-    nbytes = LAYERS * decode_bytes_per_layer_call(B, H_K, H_V, D, T)
+    mb = DecodeMultiBench(device, seed=12, B=B, slots=slots, T=T)
+    mb.capture()
+    mb.run(0, warmup)
+    ms = time_region(lambda: mb.run(warmup, steps), steps, world)
+    nbytes = mb.bytes_per_call
+    del mb
+    torch.cuda.empty_cache()
     res["batch_sweep"] = decode_batch_sweep(device, world=world)
     res["multi_token"] = {
         "value": nbytes * steps / (ms * 1e-3) / 1e9, "unit": "GB/s", "tokens_per_call": T,
         "tokens_per_s": B * T * steps / (ms * 1e-3), "us_per_launch": ms * 1e3 / (steps * LAYERS),
         "launch": f"{LAYERS} launches per call, {T} tokens per sequence each, one CUDA graph per call"}
-    del graphs
     return res
 
 
 # ---------------------------------------------------------------- prefill
 
-def prefill_measure(device, reps=5, world=1):
+def prefill_measure(device, lens=None, H_k=P_H, H_v=P_H, seed=2, g_mode="softplus",
+                    workload=None, reps=5, world=1):
+    """Median time of one chunked prefill over the packed sequences `lens` (default:
+    the Qwen3.5-0.8B-shaped 4 x 4096 prompt batch), L2 flushed before every
+    repetition; tokens/s and algorithmic TFLOP/s against the bf16 peak."""
     import linear_attention_recurrence_10_b200 as gdr
     from linear_attention_recurrence_10_b200 import synth
-    inp = synth.make_inputs([P_LEN] * P_SEQS, P_H, P_H, D, seed=2, device=device)
+    lens = lens or [P_LEN] * P_SEQS
+    inp = synth.make_inputs(lens, H_k, H_v, D, seed=seed, g_mode=g_mode, device=device)
     cu = torch.tensor(inp.cu_seqlens, dtype=torch.int32, device=device)
-    out = torch.empty(inp.n_tok, P_H, D, device=device, dtype=torch.bfloat16)
-    final = torch.empty(P_SEQS, P_H, D, D, device=device)
+    out = torch.empty(inp.n_tok, H_v, D, device=device, dtype=torch.bfloat16)
+    final = torch.empty(len(lens), H_v, D, D, device=device)
     ws_bytes = gdr.prefill_workspace_size(inp.q, inp.k, inp.v, inp.g, inp.beta, cu, out,
                                           cu_seqlens_host=inp.cu_seqlens, z=inp.z, chunk=P_CHUNK)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device)
@@ -420,18 +463,218 @@ def prefill_measure(device, reps=5, world=1):
         times.append(time_region(call, 1, world))  # max over ranks
     ms = statistics.median(times)
     n_tok = inp.n_tok * world
-    flops = n_tok * P_H * prefill_flops_per_token_head(P_CHUNK, D, gva=False)
+    fpt = prefill_flops_per_token_head(P_CHUNK, D, H_v // H_k)
+    flops = n_tok * H_v * fpt
     per_gpu_tflops = flops / world / (ms * 1e-3) / 1e12
     peaks = load_peaks()
     tflops = flops / (ms * 1e-3) / 1e12
+    workload = workload or (f"Qwen3.5-0.8B-shaped prefill: {P_SEQS} x {P_LEN} tokens, "
+                            f"{H_k}/{H_v} heads, d={D}, bf16, chunk {P_CHUNK}, S_0=0")
     return {"metric": "chunked-prefill tokens/s", "value": n_tok / (ms * 1e-3), "unit": "tokens/s",
-            "ms": ms, "workload": f"Qwen3.5-0.8B-shaped prefill: {P_SEQS} x {P_LEN} tokens, "
-                                  f"{P_H}/{P_H} heads, d={D}, bf16, chunk {P_CHUNK}, S_0=0",
-            "n_gpus": world, "scaling": "weak",
-            "tflops": tflops, "tc_frac": per_gpu_tflops / peaks["bf16_tflops"],
-            "tc_peak_tflops": peaks["bf16_tflops"], "flops_per_token_head":
-                prefill_flops_per_token_head(P_CHUNK, D, gva=False),
+            "ms": ms, "workload": workload, "tokens": inp.n_tok, "n_gpus": world,
+            "scaling": "weak", "tflops": tflops, "tc_frac": per_gpu_tflops / peaks["bf16_tflops"],
+            "tc_peak_tflops": peaks["bf16_tflops"], "flops_per_token_head": fpt,
+            "roofline": {"bound": "tensor", "achieved": per_gpu_tflops,
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": per_gpu_tflops / peaks["bf16_tflops"], "traffic": None,
+                         "peak_source": peaks["source"] + " (bf16_tflops, burst)"},
             "l2": "flushed (256 MB write) before each repetition", "reps": reps}
+
+
+def long_context_prefill_measure(device, reps=3, world=1):
+    """Long-context GVA prefill: 8 sequences of U{1024..32768} tokens (seed 4),
+    16 key / 32 value heads, d=128, bf16, chunk 64, exp(g) in [0.9, 1), S_0 = 0."""
+    from linear_attention_recurrence_10_b200 import synth
+    lens = synth.lengths(LC_SEQS, LC_SEED, LC_LO, LC_HI)
+    return prefill_measure(
+        device, lens, LC_HK, LC_HV, seed=LC_SEED, g_mode="long", reps=reps, world=world,
+        workload=f"long-context GVA prefill: {LC_SEQS} sequences of U{{{LC_LO}..{LC_HI}}} tokens "
+                 f"({sum(lens)} in all), {LC_HK}/{LC_HV} heads, d={D}, bf16, chunk {P_CHUNK}, "
+                 f"exp(g) in [0.9, 1), S_0=0")
+
+
+def attn_decode_bytes_per_layer(B, H_q, H_kv, d, ctx, out_b=OUT_BYTES) -> int:
+    """Algorithmic bytes of one gated-attention decode step of one layer: the
+    cache rows read (ctx cached + the appended one, keys and values), the new
+    key and value read and appended, q and gate read, the output written."""
+    cache = B * H_kv * (ctx + 1) * 2 * d * 2
+    new_kv = B * H_kv * 2 * d * 2 * 2
+    q_gate = B * H_q * 2 * d * 2
+    return cache + new_kv + q_gate + B * H_q * d * out_b
+
+
+def attn_decode_measure(device, steps=16, warmup=4, world=1, layers=ATT_LAYERS):
+    """Qwen3.6-35B-A3B-shaped gated full-attention decode: 10 layers' KV caches
+    (64 x 2 heads x 4097 rows x 256, bf16: 5.4 GB in all) rotate through HBM;
+    one step runs the 10 layers' decode calls from one CUDA graph."""
+    import linear_attention_recurrence_10_b200 as gdr
+    from linear_attention_recurrence_10_b200 import synth
+    L, B, Hq, Hkv, d, ctx = layers, ATT_B, ATT_HQ, ATT_HKV, ATT_D, ATT_CTX
+    nrm = lambda shape, name: synth.normal(shape, 9, name, device=device).to(torch.bfloat16)
+    q, gate = nrm((L, B, Hq, d), "att_q"), nrm((L, B, Hq, d), "att_gate")
+    k, v = nrm((L, B, Hkv, d), "att_k"), nrm((L, B, Hkv, d), "att_v")
+    kc = torch.empty(L, B, Hkv, ctx + 1, d, device=device, dtype=torch.bfloat16)
+    vc = torch.empty_like(kc)
+    for l in range(L):  # the cached rows, drawn layer by layer
+        kc[l] = nrm((B, Hkv, ctx + 1, d), f"att_kc{l}")
+        vc[l] = nrm((B, Hkv, ctx + 1, d), f"att_vc{l}")
+    cache_len = torch.full((B,), ctx, dtype=torch.int32, device=device)
+    out = torch.empty(L, B, Hq, d, device=device, dtype=torch.bfloat16)
+    n = gdr.attn_decode_workspace_size(q[0], gate[0], k[0], v[0], kc[0], vc[0], cache_len, out[0],
+                                       kv_bound=ctx, rot_dim=ATT_ROT)
+    ws = torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+    def step():
+        for l in range(L):
+            gdr.attn_decode_step(q[l], gate[l], k[l], v[l], kc[l], vc[l], cache_len, out[l],
+                                 kv_bound=ctx, rot_dim=ATT_ROT, workspace=ws)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for _ in range(warmup):
+        graph.replay()
+    ms = time_region(lambda: [graph.replay() for _ in range(steps)], steps, world)
+    status = int(ws[:4].view(torch.int32).item())
+    from linear_attention_recurrence_10_b200.ranks import weak_scaling_rate
+    per_layer = attn_decode_bytes_per_layer(B, Hq, Hkv, d, ctx)
+    peaks = load_peaks()
+    achieved = per_layer * L * steps / (ms * 1e-3) / 1e9
+    res = {"metric": "gated-attention decode GB/s", "unit": "GB/s",
+           "value": weak_scaling_rate(per_layer * L * steps, world, ms) / 1e9,
+           "steps": steps, "ms_per_step": ms / steps, "status_word": status,
+           "tokens_per_s": weak_scaling_rate(B * steps, world, ms),
+           "workload": f"Qwen3.6-35B-A3B-shaped gated attention decode: {L} layers x B={B}, "
+                       f"{Hq}/{Hkv} heads, head_dim {d}, {ctx} cached tokens, RoPE on {ATT_ROT} "
+                       f"dims, bf16 cache and outputs",
+           "l2": f"inputs larger than L2: {L} layers' caches "
+                 f"({2 * kc.numel() * 2 / 1e9:.1f} GB) rotate every step",
+           "launch": "one CUDA graph per step: 3 kernels per layer (rope/append, attend, combine)",
+           "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                        "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                        "bytes_per_layer": per_layer,
+                        "us_per_layer": ms * 1e3 / (steps * L),
+                        "peak_source": peaks["source"] + " (hbm_gbs, of measured copy bandwidth)"}}
+    del graph, q, gate, k, v, kc, vc, out, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def moe_bytes_per_layer(n_tok, n_active, E=MOE_E, H=MOE_H, I=MOE_I, SI=MOE_SI, out_b=OUT_BYTES) -> int:
+    """Algorithmic bytes of one MoE decode step of one layer: the router and
+    shared-gate rows, the gate/up and down weights of the n_active experts the
+    tokens chose and of the shared expert (bf16), the tokens in, the outputs out."""
+    return (E * H + H) * 2 + n_active * 3 * I * H * 2 + 3 * SI * H * 2 + n_tok * H * (2 + out_b)
+
+
+def moe_decode_measure(device, B=1, steps=32, warmup=4, world=1, slots=16):
+    """Qwen3.6-35B-A3B-shaped MoE decode: 8 layers' expert weights rotate through
+    HBM; each step runs B tokens through the 8 layers (one CUDA graph per step,
+    five kernels per layer).  The bytes are counted from each step's routing:
+    only the experts some token chose are read."""
+    import linear_attention_recurrence_10_b200 as gdr
+    from linear_attention_recurrence_10_b200 import synth
+    L, H, E, K, I, SI = MOE_LAYERS, MOE_H, MOE_E, MOE_K, MOE_I, MOE_SI
+    nrm = lambda shape, name, std: (synth.normal(shape, 10, name, device=device) * std).to(torch.bfloat16)
+    layers = []
+    for l in range(L):
+        layers.append(dict(
+            w_router=nrm((E, H), f"moe_r{l}", H ** -0.5),
+            w_gate_up=nrm((E, 2 * I, H), f"moe_gu{l}", H ** -0.5),
+            w_down=nrm((E, H, I), f"moe_d{l}", I ** -0.5),
+            shared=(nrm((2 * SI, H), f"moe_sgu{l}", H ** -0.5), nrm((H, SI), f"moe_sd{l}", SI ** -0.5),
+                    nrm((H,), f"moe_sg{l}", H ** -0.5))))
+    x = nrm((slots, L, B, H), "moe_x", 1.0)
+    out = torch.empty(L, B, H, device=device, dtype=torch.bfloat16)
+    idx = torch.empty(slots, L, B, K, dtype=torch.int32, device=device)
+    w0 = layers[0]
+    n = gdr.moe_workspace_size(x[0, 0], w0["w_router"], w0["w_gate_up"], w0["w_down"], out[0],
+                               top_k=K, shared=w0["shared"])
+    ws = torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+    def step(sl):
+        for l, w in enumerate(layers):
+            gdr.moe_decode(x[sl, l], w["w_router"], w["w_gate_up"], w["w_down"], out[l], top_k=K,
+                           shared=w["shared"], topk_idx=idx[sl, l], workspace=ws)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for sl in range(slots):
+            step(sl)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    routing = idx.cpu()
+    per_step = [sum(moe_bytes_per_layer(B, len(set(routing[sl, l].flatten().tolist())))
+                    for l in range(L)) for sl in range(slots)]
+    graphs = []
+    for sl in range(slots):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            step(sl)
+        graphs.append(gr)
+    for s_ in range(warmup):
+        graphs[s_ % slots].replay()
+    ms = time_region(lambda: [graphs[(warmup + s_) % slots].replay() for s_ in range(steps)], steps,
+                     world)
+    nbytes = sum(per_step[(warmup + s_) % slots] for s_ in range(steps))
+    from linear_attention_recurrence_10_b200.ranks import weak_scaling_rate
+    peaks = load_peaks()
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    res = {"metric": "MoE decode GB/s (routed experts read)", "unit": "GB/s",
+           "value": weak_scaling_rate(nbytes, world, ms) / 1e9, "steps": steps,
+           "ms_per_step": ms / steps, "us_per_layer": ms * 1e3 / (steps * L),
+           "tokens_per_s": weak_scaling_rate(B * steps, world, ms),
+           "bytes_per_step": nbytes / steps,
+           "workload": f"Qwen3.6-35B-A3B-shaped MoE decode: {L} layers x B={B} tokens, hidden {H}, "
+                       f"{E} experts top-{K}, intermediate {I}, shared expert {SI}, bf16 weights",
+           "l2": f"inputs larger than L2: {L} layers' weights "
+                 f"({L * (E * 3 * I * H + 3 * SI * H + E * H) * 2 / 1e9:.1f} GB) rotate; each step "
+                 f"reads ~{nbytes / steps / 1e6:.0f} MB",
+           "launch": "one CUDA graph per step: 5 kernels per layer (router, route, gate_up, down, "
+                     "combine)",
+           "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                        "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                        "peak_source": peaks["source"] + " (hbm_gbs, of measured copy bandwidth)"}}
+    del graphs, layers, x, out, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def gva_decode_measure(device, steps=32, warmup=4, world=1):
+    """Qwen3.6-35B-A3B-shaped GVA decode: B=64, 16 key / 32 value heads, 30 layer
+    states (4.0 GB, rotating through HBM), 256 distinct steps cycled; one CUDA
+    graph of 30 decode launches per step."""
+    b = DecodeBench(device, seed=3, B=GVA_B, layers=GVA_LAYERS, slots=GVA_STEPS, H_k=GVA_HK,
+                    H_v=GVA_HV)
+    b.capture()
+    b.run(0, warmup)
+    ms = time_region(lambda: b.run(warmup, steps), steps, world)
+    from linear_attention_recurrence_10_b200.ranks import weak_scaling_rate
+    per_launch_ms = ms / (steps * b.L)
+    achieved = b.bytes_per_launch / (per_launch_ms * 1e-3) / 1e9
+    peaks = load_peaks()
+    res = {"metric": HEADLINE, "value": weak_scaling_rate(b.bytes_per_step * steps, world, ms) / 1e9,
+           "unit": "GB/s", "steps": steps, "ms_per_step": ms / steps,
+           "tokens_per_s": weak_scaling_rate(GVA_B * steps, world, ms),
+           "workload": f"Qwen3.6-35B-A3B-shaped GVA decode: {GVA_LAYERS} layers x B={GVA_B}, "
+                       f"{GVA_HK}/{GVA_HV} heads, d={D}, bf16 q/k/v/z/out, fp32 state",
+           "l2": f"inputs larger than L2: {GVA_LAYERS} layer states "
+                 f"({GVA_LAYERS * GVA_B * GVA_HV * D * D * 4 / 1e9:.1f} GB) rotate every step",
+           "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                        "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                        "bytes_per_launch": b.bytes_per_launch,
+                        "us_per_launch": per_launch_ms * 1e3,
+                        "peak_source": peaks["source"] + " (hbm_gbs, of measured copy bandwidth)"}}
+    del b
+    torch.cuda.empty_cache()
+    return res
 
 
 # ------------------------------------------------------------- CPU oracle
@@ -521,6 +764,15 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode-variants", action="store_true")
+    ap.add_argument("--no-gva-decode", action="store_true")
+    ap.add_argument("--no-attn-decode", action="store_true")
+    ap.add_argument("--no-moe", action="store_true")
+    ap.add_argument("--moe-only", action="store_true",
+                    help="run only the MoE decode measurements and print their JSON")
+    ap.add_argument("--attn-only", action="store_true",
+                    help="run only the gated-attention decode measurement and print its JSON")
+    ap.add_argument("--attn-layers", type=int, default=ATT_LAYERS,
+                    help="layers' caches rotated in the attention measurement (fewer for profiling)")
     ap.add_argument("--prefill-only", action="store_true",
                     help="run only the chunked-prefill measurement and print its JSON (profiling)")
     ap.add_argument("--prefill-reps", type=int, default=5)
@@ -544,8 +796,24 @@ def main():
 
     from linear_attention_recurrence_10_b200 import build
     build.build(quiet=True)
+    if args.moe_only:
+        res = {"B1": moe_decode_measure(device, B=1, world=world),
+               "B8": moe_decode_measure(device, B=8, world=world)}
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+    if args.attn_only:
+        res = attn_decode_measure(device, world=world, layers=args.attn_layers)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
     if args.prefill_only:
         pre = prefill_measure(device, reps=args.prefill_reps, world=world)
+        pre["long_context_prefill"] = long_context_prefill_measure(device, world=world)
         if rank == 0:
             print(json.dumps(pre), flush=True)
         if world > 1:
@@ -582,11 +850,19 @@ def main():
     del e2e, bench
     torch.cuda.empty_cache()
     variants = None if args.no_decode_variants else decode_variants(device, args.batch, world=world)
+    gva = None if args.no_gva_decode else gva_decode_measure(device, world=world)
+    attn = None if args.no_attn_decode else attn_decode_measure(device, world=world)
+    moe = None if args.no_moe else {"B1": moe_decode_measure(device, B=1, world=world),
+                                    "B8": moe_decode_measure(device, B=8, world=world)}
     prefill = None if args.no_prefill else prefill_measure(device, reps=args.prefill_reps,
                                                            world=world)
+    long_prefill = None if args.no_prefill else long_context_prefill_measure(device, world=world)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_sample()
+        one = oracle_sample(n_tokens=32, threads=1)
+        cpu["single_thread"] = {"value": one["value"], "unit": one["unit"], "cores": 1,
+                                "seconds": one["seconds"], "sample": one["sample"]}
 
     line = {
         "metric": HEADLINE, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -604,8 +880,8 @@ def main():
         "hbm_frac": gbs / world / peaks["hbm_gbs"],
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                     "traffic": captured_traffic("decode_kernel<128, bf16, bf16, false>"),
-                     "kernel": "decode_kernel<128, bf16, bf16, false>",
+                     "traffic": captured_traffic("decode_rb_kernel<bf16, bf16>"),
+                     "kernel": "decode_rb_kernel<bf16, bf16>",
                      "bytes_per_launch": per_launch_bytes, "us_per_launch": per_launch_ms * 1e3,
                      "peak_source": peaks["source"] + " (hbm_gbs, of measured copy bandwidth)"},
         "cpu_baseline": cpu,
@@ -618,7 +894,11 @@ def main():
         "gpu_launches": args.steps * launches_per_step,
         "clocks": clock_info,
         "decode_variants": variants,
+        "gva_decode": gva,
+        "attn_decode": attn,
+        "moe_decode": moe,
         "prefill": prefill,
+        "long_context_prefill": long_prefill,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

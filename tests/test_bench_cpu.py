@@ -34,6 +34,24 @@ def test_decode_bytes_qwen35_batch32():
     assert bench.decode_bytes_per_layer_step(32, 16, 16, 128) == want
 
 
+def test_prefill_flops_per_token_head():
+    # Chunk 64, d 128: KK^T, QK^T, U, W, P Delta at 2 C d (16,384) each, W S^T, Q S^T and
+    # the state update at 2 d^2 (32,768) each; under GVA (two value heads per key head)
+    # KK^T and QK^T are counted once per key head.
+    assert bench.prefill_flops_per_token_head(64, 128) == 5 * 16_384 + 3 * 32_768 == 180_224
+    assert bench.prefill_flops_per_token_head(64, 128, 2) == 4 * 16_384 + 3 * 32_768 == 163_840
+
+
+def test_attn_decode_bytes_qwen36():
+    # 64 sequences x 2 key/value heads x (4096 + 1) cache rows x (key + value) x 256 x bf16,
+    # the new key and value read and appended, q and gate of 16 heads read, output written.
+    cache = 64 * 2 * 4097 * 2 * 256 * 2
+    new_kv = 64 * 2 * 2 * 256 * 2 * 2
+    q_gate = 64 * 16 * 2 * 256 * 2
+    out = 64 * 16 * 256 * 2
+    assert bench.attn_decode_bytes_per_layer(64, 16, 2, 256, 4096) == cache + new_kv + q_gate + out
+
+
 def test_decode_bytes_gva_batch64():
     # 64 sequences, 16 key heads each serving two of 32 value heads: q and k are read once
     # per key head.

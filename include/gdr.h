@@ -385,8 +385,10 @@ gdr_status gdr_rmsnorm_gated(const gdr_norm_args *args, gdr_stream_t stream);
  *   out        [batch, H_q, d] out_dtype, row stride out_stride
  *   rot_dim    even, 0 .. d (64 in the Qwen3.5 / 3.6 layers); rope_theta;
  *   scale      multiplies q.k (d^-1/2 for standard attention)
- *   Supported: d = 256, H_q a multiple of H_kv with H_q / H_kv <= 16.
- *   batch == 0 is a no-op.
+ *   Supported: d = 256, H_q a multiple of H_kv with H_q / H_kv <= 16,
+ *   batch * H_kv * max_len < 2^31 (GDR_ERR_UNSUPPORTED otherwise).
+ *   batch == 0 is a no-op.  k_cache and v_cache are read with TMA tensor
+ *   copies: they need 16-byte alignment, like every pointer here.
  *   workspace: device memory, 16-byte aligned, of gdr_attn_decode_workspace_size
  *   bytes (per-split partial results); its first 4 bytes (int32) hold, once
  *   the work has finished, 0, GDR_ERR_INVALID_ARG (a cache_len out of range)

@@ -406,7 +406,8 @@ static gdr_status attn_check(const gdr_attn_decode_args *a, int *n_split, int *s
     if (a->max_len < 1 || a->kv_bound < 0 || a->kv_bound >= a->max_len) return GDR_ERR_INVALID_ARG;
     if (!dtype_ok(a->out_dtype)) return GDR_ERR_INVALID_ARG;
     if (!(a->rope_theta > 0.f)) return GDR_ERR_INVALID_ARG;
-    if ((int64_t)a->batch * a->H_kv * a->max_len * a->d > ((int64_t)1 << 40)) return GDR_ERR_UNSUPPORTED;
+    // Cache rows are addressed with 32-bit signed coordinates.
+    if ((int64_t)a->batch * a->H_kv * a->max_len > 0x7fffffffLL) return GDR_ERR_UNSUPPORTED;
     gdr::attn_plan(a->batch, a->H_kv, a->kv_bound, device_sm_count(), n_split, split_tok);
     if ((int64_t)a->batch * a->H_kv * *n_split > 0x7fffffffLL) return GDR_ERR_UNSUPPORTED;
     *ws_bytes = gdr::attn_workspace_bytes(a->batch, a->H_kv, a->batch * a->H_kv * *n_split);

@@ -17,9 +17,10 @@
 //     fp32 with angles taken in double, appends the key and value at row L,
 //     and stages the rotated queries as the bf16 MMA operand tile of the group.
 //   attend: persistent; each work item is one (b, kv head, split of the
-//     tokens).  A producer warp streams the K and V rows through a six-slot
-//     ring of 32 KB shared-memory slots (one d-half of a 128-token tile each,
-//     cp.async with zero fill past the split's end); an MMA warp issues
+//     tokens).  One thread streams the K and V rows through a six-slot ring
+//     of 32 KB shared-memory slots (one d-half of a 128-token tile each) with
+//     TMA tensor copies into 128-byte-swizzled tiles, so that the memory
+//     instruction pipe stays free for the softmax warps; MMA warps issue
 //     S^T = K Q^T (M = 128 tokens, N = 16 query-head columns, K = 256) and
 //     O^T += V^T P^T (M = 128 dims per half, N = 16, K = 128 tokens) on
 //     tcgen05 with the accumulators in TMEM; four softmax warps (thread = TMEM
@@ -33,6 +34,7 @@
 // bounded (2 s); on expiry the kernel records GDR_ERR_TIMEOUT in the workspace
 // status word, waits (bounded) for its copies in flight, frees its tensor
 // memory and returns.
+#include <cuda.h>  // CUtensorMap and its encoder's types (fetched from the driver at run time)
 #include <math.h>
 
 #include "gdr.h"
@@ -42,6 +44,9 @@
 namespace gdr {
 
 struct AttnParams {
+    // 2-D TMA maps of the caches: [batch * H_kv * max_len rows][256] bf16,
+    // boxes of 64 dims x 128 rows, 128-byte swizzle.
+    CUtensorMap tm_k, tm_v;
     int batch, H_q, H_kv, n_rep, rot_dim, max_len, kv_bound;
     int n_split, split_tok, n_items;
     float scale;
@@ -67,6 +72,7 @@ constexpr int TILE = 128;                 // tokens per tile
 constexpr int NH = 16;                    // query-head columns per key/value head
 constexpr int NSLOT = 6;
 constexpr uint32_t SLOT = 32768;          // one d-half of a K or V tile, bf16
+constexpr uint32_t BOX = 16384;           // one TMA box: 128 tokens x 64 dims
 constexpr uint32_t QTILE = NH * D * 2;    // 8 KB
 constexpr uint32_t PTILE = NH * TILE * 2; // 4 KB
 constexpr uint32_t S_RING = 0;
@@ -75,6 +81,7 @@ constexpr uint32_t S_P = S_Q + 2 * QTILE;         // 2 x P tile
 constexpr uint32_t S_RED = S_P + 2 * PTILE;       // 4 warps x 16 floats
 constexpr uint32_t S_BAR = S_RED + 256;
 constexpr uint32_t S_BYTES = S_BAR + 256;
+constexpr uint32_t S_ALLOC = S_BYTES + 1024;  // room to align the ring to 1024 bytes
 constexpr int NTHR = 224;  // warps 0-3 softmax, 4 producer, 5 S^T issue, 6 O^T issue
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr int kTimeout = 6;  // GDR_ERR_TIMEOUT
@@ -82,15 +89,13 @@ constexpr int kBadLen = 1;   // GDR_ERR_INVALID_ARG
 // TMEM columns: S^T double buffer, O^T two d-halves.
 constexpr uint32_t TM_S = 0, TM_O = 32, TM_COLS = 64;
 
-// Tile operand layouts (no swizzle, 16-byte chunks of 8 bf16).
-// K / V slot: row r (token) of 128, chunk c (8 dims) of 16:
-//   byte = (r / 8) * 2048 + c * 128 + (r % 8) * 16
-// read as K-major A for S^T (rows = tokens: SBO 2048, LBO 128) and as
-// MN-major A for O^T (M = dims: SBO 128 between chunks, LBO 2048 between
-// 8-token groups).
-__host__ __device__ constexpr uint32_t slot_off(int r, int c) {
-    return (uint32_t)((r >> 3) * 2048 + c * 128 + (r & 7) * 16);
-}
+// K / V slot: two TMA boxes (dims 0-63 and 64-127 of the half), each 128
+// token rows of 128 bytes with 128-byte swizzle: the 16-byte chunk j (8 dims)
+// of row r sits at box + r * 128 + (j ^ (r % 8)) * 16.  Read as K-major A for
+// S^T (M = tokens: SBO 1024 between 8-row groups; a K step of 16 dims moves
+// the start 32 bytes inside the row, a box every 4 steps) and as MN-major A
+// for O^T (M = dims: LBO = BOX between the two 64-dim boxes, SBO 1024 between
+// 8-token groups; a K step of 16 tokens moves the start 2048 bytes).
 // Q tile: query-head column h of 16, dim chunk c of 32 (K-major B for S^T):
 //   byte = c * 256 + h * 16   (LBO 256 between chunks, SBO 128 between 8-head groups)
 __host__ __device__ constexpr uint32_t q_off(int h, int c) { return (uint32_t)(c * 256 + h * 16); }
@@ -165,27 +170,32 @@ __global__ void __launch_bounds__(256) rope_append_kernel(const AttnParams p) {
 }
 
 // ---------------------------------------------------------------- attend
-__global__ void __launch_bounds__(NTHR, 1) attend_kernel(const AttnParams p) {
-    extern __shared__ __align__(1024) unsigned char sm[];
+__global__ void __launch_bounds__(NTHR, 1) attend_kernel(const __grid_constant__ AttnParams p) {
+    extern __shared__ __align__(1024) unsigned char sm_raw[];
+    // The swizzled ring must start on a 1024-byte boundary.
+    unsigned char *sm = sm_raw + ((1024u - (smem_u32(sm_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + S_BAR);
-    uint64_t *full = bars;           // [6] slot landed (32 producer lanes)
+    uint64_t *full = bars;           // [6] slot landed (TMA bytes, or the producer's arrival)
     uint64_t *empty = bars + 6;      // [6] slot consumed (MMA commit)
     uint64_t *bar_s = bars + 12;     // [2] S^T of a tile in TMEM
     uint64_t *bar_p = bars + 14;     // [2] P of a tile staged, O^T rescaled (4 warps)
     uint64_t *bar_o = bars + 16;     // [2] O^T += V^T P^T of a tile done (by P buffer)
     uint64_t *bar_q = bars + 18;     // [2] Q tile of an item landed
     uint64_t *bar_qfree = bars + 20; // [2] an item's S^T products done with its Q tile
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + S_BAR + 176);
+    uint64_t *bar_aux = bars + 22;   // a partial V quarter landed (before its zero fill)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + S_BAR + 192);
     float *red = reinterpret_cast<float *>(sm + S_RED);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t sbase = smem_u32(sm);
+    const uint32_t ring = sbase + S_RING;
 
     if (warp == 0) tmem_alloc(tmem_slot, TM_COLS);
     if (tid == 0) {
         for (int i = 0; i < NSLOT; ++i) {
-            mbar_init(full + i, 32);
+            mbar_init(full + i, 1);
             mbar_init(empty + i, 1);
         }
+        mbar_init(bar_aux, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar_s + i, 1);
             mbar_init(bar_p + i, 4);
@@ -207,11 +217,21 @@ __global__ void __launch_bounds__(NTHR, 1) attend_kernel(const AttnParams p) {
 
     if (warp == 4) {
         // ------------------------------------------------------ producer
-        // Slot uses are counted in one sequence (c) over this CTA's non-empty
-        // items (nq), tiles and the tile's K0, K1, V0, V1 quarters; the MMA
-        // warp walks the same sequence.
-        int c = 0, nq = 0, n_qcopy[2] = {0, 0};
-        bool ok = true;
+        // Lane 0 streams each quarter of a tile (K0, K1, V0, V1: one d-half)
+        // as two TMA box copies.  Slot uses are counted in one sequence (c)
+        // over this CTA's non-empty items (nq), tiles and quarters; the MMA
+        // warps walk the same sequence.  Past the end of a split's last,
+        // partial tile the rows hold other tokens (or zeros past the tensor):
+        // the softmax gives them zero weight, and in V the warp overwrites
+        // them with zeros before it releases the slot, so that no value stored
+        // there (a NaN in an unwritten cache row) can reach O.
+        int c = 0, ci = 0, nq = 0, n_qcopy[2] = {0, 0}, n_aux = 0;
+        bool ok = true, aux_pending = false;
+        if (lane == 0) {
+            tma_prefetch_map(&p.tm_k);
+            tma_prefetch_map(&p.tm_v);
+            fence_proxy_async_global();  // the rows appended by the kernel before
+        }
         for (int it = blockIdx.x; it < p.n_items && ok; it += gridDim.x) {
             const Item w = item_of(p, it);
             const int nt = n_tiles_of(w);
@@ -230,57 +250,61 @@ __global__ void __launch_bounds__(NTHR, 1) attend_kernel(const AttnParams p) {
             }
             ++n_qcopy[qb];
             ++nq;
-            const size_t head_row = ((size_t)w.b * p.H_kv + w.g) * p.max_len;
+            // Cache row of (b, g, token 0); below 2^31 (checked on the host).
+            const int head_row = (w.b * p.H_kv + w.g) * p.max_len;
             for (int j = 0; j < nt && ok; ++j) {
                 const int r0 = w.t0 + j * TILE;
                 const int nvalid = min(TILE, w.t1 - r0);
 #pragma unroll 1
                 for (int q4 = 0; q4 < 4; ++q4, ++c) {
                     const int slot = c % NSLOT, round = c / NSLOT;
-                    if (round > 0) ok = mbar_wait(empty + slot, (uint32_t)(round - 1) & 1u, kWaitNs);
-                    ok = __all_sync(kFullMask, ok) != 0;
+                    if (round > 0 && lane == 0) ok = mbar_wait(empty + slot, (uint32_t)(round - 1) & 1u, kWaitNs);
+                    ok = __shfl_sync(kFullMask, ok, 0);
                     if (!ok) break;
-                    // Lane l copies, at step k, row (k / 4) * 8 + l % 8 and chunk
-                    // (k % 4) * 4 + l / 8: 8 rows x 4 chunks per step, 512
-                    // contiguous bytes of the slot.  Everything but k folds into
-                    // two per-lane base addresses, so a full tile is one
-                    // instruction per 16-byte copy.
-                    const __nv_bfloat16 *src = (q4 < 2 ? p.k_cache : p.v_cache) +
-                                               (head_row + r0 + (lane & 7)) * D + (q4 & 1) * 128 +
-                                               (lane >> 3) * 8;
-                    const uint32_t dst = sbase + S_RING + slot * SLOT + (lane >> 3) * 128 + (lane & 7) * 16;
-                    if (nvalid == TILE) {
-#pragma unroll
-                        for (int k = 0; k < 64; ++k)
-                            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                                             dst + (k >> 2) * 2048 + (k & 3) * 512),
-                                         "l"(src + (size_t)((k >> 2) * 8) * D + (k & 3) * 32)
-                                         : "memory");
-                    } else {
-                        // The split's last, partial tile: rows past it are zero-filled
-                        // (their source address is the tile's first row, never read).
-#pragma unroll 4
-                        for (int k = 0; k < 64; ++k) {
-                            const int r = (k >> 2) * 8 + (lane & 7);
-                            const bool in = r < nvalid;
-                            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
-                                             dst + (k >> 2) * 2048 + (k & 3) * 512),
-                                         "l"(in ? src + (size_t)((k >> 2) * 8) * D + (k & 3) * 32
-                                                : src - (size_t)(lane & 7) * D),
-                                         "r"(in ? 16u : 0u)
-                                         : "memory");
-                        }
+                    const uint32_t dst = ring + slot * SLOT;
+                    const void *map = q4 < 2 ? static_cast<const void *>(&p.tm_k)
+                                             : static_cast<const void *>(&p.tm_v);
+                    const bool zero_tail = q4 >= 2 && nvalid < TILE;
+                    uint64_t *bar = zero_tail ? bar_aux : full + slot;
+                    if (lane == 0) {
+                        bulk_expect(bar, SLOT);
+                        tma_load_2d(dst, map, (q4 & 1) * 128, head_row + r0, bar);
+                        tma_load_2d(dst + BOX, map, (q4 & 1) * 128 + 64, head_row + r0, bar);
                     }
-                    cp_async_arrive(full + slot);
+                    if (!zero_tail) {
+                        ci = c + 1;
+                        continue;
+                    }
+                    aux_pending = true;
+                    ok = __all_sync(kFullMask, mbar_wait(bar_aux, (uint32_t)n_aux & 1u, kWaitNs)) != 0;
+                    if (!ok) break;
+                    aux_pending = false;
+                    ++n_aux;
+                    // Rows nvalid .. 127 of both boxes: a row keeps its 128 bytes
+                    // under the swizzle, which only permutes chunks inside it.
+                    for (int i = nvalid * 8 + lane; i < TILE * 8; i += 32) {
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst + i * 16), "r"(0u)
+                                     : "memory");
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst + BOX + i * 16),
+                                     "r"(0u)
+                                     : "memory");
+                    }
+                    fence_smem_to_async();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(full + slot);
+                    ci = c + 1;
                 }
             }
         }
-        cp_async_wait_all();
         if (!ok && lane == 0) {
             fail();
-            // No bulk copy may land after the CTA ends.
+            // No copy may land after the CTA ends: the Q tiles, the last use
+            // of every slot, a partial V quarter.
             for (int b = 0; b < 2; ++b)
                 if (n_qcopy[b]) mbar_wait(bar_q + b, (uint32_t)(n_qcopy[b] - 1) & 1u, kWaitNs);
+            for (int u = ci > NSLOT ? ci - NSLOT : 0; u < ci; ++u)
+                mbar_wait(full + u % NSLOT, (uint32_t)(u / NSLOT) & 1u, kWaitNs);
+            if (aux_pending) mbar_wait(bar_aux, (uint32_t)n_aux & 1u, kWaitNs);
         }
         __syncwarp();
     } else if (warp == 5 || warp == 6) {
@@ -314,10 +338,15 @@ __global__ void __launch_bounds__(NTHR, 1) attend_kernel(const AttnParams p) {
                         fence_after_sync();
                         const uint32_t d = tm + TM_S + 16 * (jt & 1);
                         const uint32_t qa = sbase + S_Q + qb * QTILE;
-                        gemm(d, sbase + S_RING + s0 * SLOT, 128, 2048, 256, qa, 256, 128, 512, 8, ID_S,
-                             false);
-                        gemm(d, sbase + S_RING + s1 * SLOT, 128, 2048, 256, qa + 4096, 256, 128, 512, 8,
-                             ID_S, true);
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const uint32_t a0 = ring + (hh ? s1 : s0) * SLOT;
+#pragma unroll
+                            for (int kk = 0; kk < 8; ++kk)
+                                mma<Kind::BF16>(
+                                    d, smem_desc_sw128(a0 + (kk >> 2) * BOX + (kk & 3) * 32, 16, 1024),
+                                    smem_desc(qa + hh * 4096 + kk * 512, 256, 128), ID_S, (hh | kk) ? 1u : 0u);
+                        }
                         commit(smem_u32(bar_s + (jt & 1)));
                         commit(smem_u32(empty + s0));
                         commit(smem_u32(empty + s1));
@@ -330,10 +359,15 @@ __global__ void __launch_bounds__(NTHR, 1) attend_kernel(const AttnParams p) {
                         if (!ok) break;
                         fence_after_sync();
                         const uint32_t pb = sbase + S_P + (jt & 1) * PTILE;
-                        gemm(tm + TM_O, sbase + S_RING + v0 * SLOT, 2048, 128, 4096, pb, 256, 128, 512,
-                             8, ID_O, j > 0);
-                        gemm(tm + TM_O + 16, sbase + S_RING + v1 * SLOT, 2048, 128, 4096, pb, 256, 128,
-                             512, 8, ID_O, j > 0);
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const uint32_t a0 = ring + (hh ? v1 : v0) * SLOT;
+#pragma unroll
+                            for (int kk = 0; kk < 8; ++kk)
+                                mma<Kind::BF16>(tm + TM_O + 16 * hh, smem_desc_sw128(a0 + kk * 2048, BOX, 1024),
+                                                smem_desc(pb + kk * 512, 256, 128), ID_O,
+                                                (j > 0 || kk > 0) ? 1u : 0u);
+                        }
                         commit(smem_u32(bar_o + (jt & 1)));
                         commit(smem_u32(empty + v0));
                         commit(smem_u32(empty + v1));
@@ -587,7 +621,47 @@ void attn_plan(int batch, int H_kv, int kv_bound, int n_sm, int *n_split, int *s
     *split_tok = ((tiles + best - 1) / best) * attn::TILE;
 }
 
+namespace {
+
+using EncodeTiledFn = decltype(&cuTensorMapEncodeTiled);
+
+// The driver's tensor-map encoder, looked up once through the runtime (no
+// link-time dependency on the driver library).
+EncodeTiledFn encode_tiled() {
+    static const EncodeTiledFn fn = []() -> EncodeTiledFn {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault,
+                                             &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess) {
+            (void)cudaGetLastError();
+            return nullptr;
+        }
+        return reinterpret_cast<EncodeTiledFn>(f);
+    }();
+    return fn;
+}
+
+// A cache as `rows` rows of 256 bf16 (512-byte stride); boxes of 64 dims x
+// 128 rows, 128-byte swizzle, rows past the end read as zero.
+bool encode_cache_map(CUtensorMap *m, void *base, uint64_t rows) {
+    const EncodeTiledFn fn = encode_tiled();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)attn::D, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)attn::D * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)attn::TILE};
+    const cuuint32_t elem_strides[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, elem_strides,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
 cudaError_t launch_attn_decode(AttnParams p, void *workspace, int out_bf16, cudaStream_t s) {
+    const uint64_t rows = (uint64_t)p.batch * p.H_kv * p.max_len;
+    if (!encode_cache_map(&p.tm_k, p.k_cache, rows) || !encode_cache_map(&p.tm_v, p.v_cache, rows))
+        return cudaErrorInvalidValue;
     unsigned char *ws = static_cast<unsigned char *>(workspace);
     p.status = reinterpret_cast<int *>(ws);
     size_t off = 256;
@@ -603,7 +677,7 @@ cudaError_t launch_attn_decode(AttnParams p, void *workspace, int out_bf16, cuda
         cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return cudaGetLastError();
     e = cudaFuncSetAttribute(attn::attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)attn::S_BYTES);
+                             (int)attn::S_ALLOC);
     if (e != cudaSuccess) return e;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -623,7 +697,7 @@ cudaError_t launch_attn_decode(AttnParams p, void *workspace, int out_bf16, cuda
     const unsigned bg = (unsigned)(p.batch * p.H_kv);
     if ((e = launch(attn::rope_append_kernel, bg, 256, 0)) != cudaSuccess) return e;
     const unsigned grid = (unsigned)(p.n_items < n_sm ? p.n_items : n_sm);
-    if ((e = launch(attn::attend_kernel, grid, attn::NTHR, attn::S_BYTES)) != cudaSuccess) return e;
+    if ((e = launch(attn::attend_kernel, grid, attn::NTHR, attn::S_ALLOC)) != cudaSuccess) return e;
     if (out_bf16)
         e = launch(attn::combine_kernel<__nv_bfloat16>, bg, 256, 0);
     else

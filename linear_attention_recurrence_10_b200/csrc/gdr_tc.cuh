@@ -36,6 +36,17 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
     return d;
 }
 
+// The same for a 128-byte-swizzled operand (the layout a TMA tensor copy with
+// 128-byte swizzle writes: 8 rows of 128 bytes per 1024-byte atom, 16-byte
+// chunk j of row r stored at chunk j ^ (r % 8)).  The atoms must start on
+// 1024-byte boundaries.  K-major: SBO = stride of 8-row groups (LBO unused);
+// a K step inside the 128-byte row advances the start address.  MN-major:
+// LBO = stride of 64-element (128-byte) groups along M or N, SBO = stride of
+// 8-row groups along K.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return smem_desc(saddr, lbo, sbo) | ((uint64_t)2 << 61);  // layout type: 128-byte swizzle
+}
+
 enum class Kind { BF16 };
 
 // Instruction descriptor for kind::f16 with bf16 inputs, fp32 accumulate.
@@ -282,6 +293,29 @@ __device__ __forceinline__ void bulk_copy(void *smem_dst, const void *gmem_src, 
             smem_u32(smem_dst)),
         "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
+}
+
+// 2-D tensor copy global -> shared through the tensor map at `tmap` (a
+// kernel parameter): the box at element coordinates (x, y), x innermost;
+// elements outside the tensor read as zero.  Completion is counted on `bar`
+// in bytes of the whole box (see bulk_expect).  x * element size must be a
+// multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_2d(uint32_t smem_dst, const void *tmap, int x, int y,
+                                            uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+// Bring a tensor map into the descriptor cache ahead of its first use.
+__device__ __forceinline__ void tma_prefetch_map(const void *tmap) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
+}
+// Order this thread's earlier generic-proxy global accesses (and those it has
+// observed) before its later async-proxy ones (TMA reads of global memory).
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // Ask L2 to fetch the 128-byte line holding `p` (no result, nothing to wait for).

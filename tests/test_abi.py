@@ -328,6 +328,8 @@ ATTN_CASES = [
     ("misaligned_k_cache", dict(k_cache=FAKE + 8), MISALIGNED),
     ("misaligned_cache_len", dict(cache_len=FAKE + 2), MISALIGNED),
     ("stride_too_small", dict(q_stride=256), INVALID),
+    ("cache_rows_past_int32", dict(batch=1 << 16, H_kv=2, H_q=16, max_len=1 << 15, kv_bound=100),
+     UNSUPPORTED),
 ]
 
 

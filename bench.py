@@ -573,14 +573,14 @@ def moe_bytes_per_layer(n_tok, n_active, E=MOE_E, H=MOE_H, I=MOE_I, SI=MOE_SI, o
     return (E * H + H) * 2 + n_active * 3 * I * H * 2 + 3 * SI * H * 2 + n_tok * H * (2 + out_b)
 
 
-def moe_decode_measure(device, B=1, steps=32, warmup=4, world=1, slots=16):
+def moe_decode_measure(device, B=1, steps=32, warmup=4, world=1, slots=16, layers=MOE_LAYERS):
     """Qwen3.6-35B-A3B-shaped MoE decode: 8 layers' expert weights rotate through
     HBM; each step runs B tokens through the 8 layers (one CUDA graph per step,
     five kernels per layer).  The bytes are counted from each step's routing:
     only the experts some token chose are read."""
     import linear_attention_recurrence_10_b200 as gdr
     from linear_attention_recurrence_10_b200 import synth
-    L, H, E, K, I, SI = MOE_LAYERS, MOE_H, MOE_E, MOE_K, MOE_I, MOE_SI
+    L, H, E, K, I, SI = layers, MOE_H, MOE_E, MOE_K, MOE_I, MOE_SI
     nrm = lambda shape, name, std: (synth.normal(shape, 10, name, device=device) * std).to(torch.bfloat16)
     layers = []
     for l in range(L):
@@ -769,6 +769,8 @@ def main():
     ap.add_argument("--no-moe", action="store_true")
     ap.add_argument("--moe-only", action="store_true",
                     help="run only the MoE decode measurements and print their JSON")
+    ap.add_argument("--moe-layers", type=int, default=MOE_LAYERS,
+                    help="layers' expert weights rotated in the MoE measurement (fewer for profiling)")
     ap.add_argument("--attn-only", action="store_true",
                     help="run only the gated-attention decode measurement and print its JSON")
     ap.add_argument("--attn-layers", type=int, default=ATT_LAYERS,
@@ -797,8 +799,8 @@ def main():
     from linear_attention_recurrence_10_b200 import build
     build.build(quiet=True)
     if args.moe_only:
-        res = {"B1": moe_decode_measure(device, B=1, world=world),
-               "B8": moe_decode_measure(device, B=8, world=world)}
+        res = {"B1": moe_decode_measure(device, B=1, world=world, layers=args.moe_layers),
+               "B8": moe_decode_measure(device, B=8, world=world, layers=args.moe_layers)}
         if rank == 0:
             print(json.dumps(res), flush=True)
         if world > 1:

@@ -15,9 +15,7 @@
 //         + sigmoid(w_sgate . x) W_down,s (silu(W_gate,s x) * (W_up,s x))
 //
 // Five kernels on the caller's stream, each a programmatic dependent of the
-// one before: it waits for it before reading what it wrote, and each block
-// lets the next kernel launch only once its own stores are issued, so blocks
-// of the next kernel never sit on an SM the current one still needs:
+// one before (each waits for it before reading what it wrote):
 //   router:  one warp per router row (and one for the shared gate row): the
 //            row's dot products with every token, fp32.
 //   route:   one block: per token the softmax, the top-k and the weights; then
@@ -27,7 +25,7 @@
 //   gate_up: per (active expert, 16 intermediate rows): the gate and up rows
 //            against each of the expert's tokens, h = silu(g) * u (fp32).
 //   down:    per (active expert, 32 output rows): w * (W_down h) per pair.
-//   combine: per token, the sum of its pairs' partial outputs.
+//   combine: per (token, 256 outputs), the sum of its pairs' partial outputs.
 // Weights are bf16; all arithmetic is fp32.  Bound by HBM on the weights read.
 #include "gdr.h"
 #include "gdr_common.cuh"
@@ -57,8 +55,7 @@ namespace moe {
 
 constexpr int GU_ROWS = 16;   // intermediate rows per gate_up block (x 2: gate and up)
 constexpr int DN_ROWS = 32;   // output rows per down block
-constexpr int ROUTE_THREADS = 1024;
-constexpr int MAXE_LANE = 32;  // experts per lane in the router's softmax: n_exp <= 1024
+constexpr int ROUTE_THREADS = 1024;  // also the most experts (one thread each in the scans)
 
 // Dot products of ROWS bf16 rows with one bf16 vector x of n values (n a
 // multiple of 8), by one warp: lane l takes 16-byte chunks l, l + 32, ...; the
@@ -104,6 +101,7 @@ __device__ __forceinline__ void warp_dots_bf16(const __nv_bfloat16 *const (&w)[R
 // One warp per router row e (e == n_exp: the shared-expert gate), every token.
 __global__ void __launch_bounds__(256) router_kernel(const MoeParams p) {
     wait_for_predecessor();
+    release_dependents();
     const int lane = threadIdx.x & 31;
     const int e = blockIdx.x * 8 + (threadIdx.x >> 5);
     const bool shared_row = e == p.n_exp;
@@ -114,19 +112,65 @@ __global__ void __launch_bounds__(256) router_kernel(const MoeParams p) {
         warp_dots_bf16<1>(w, p.x + (int64_t)t * p.x_stride, p.hidden, lane, d);
         if (lane == 0) p.logits[(size_t)t * (p.n_exp + 1) + e] = d[0];
     }
-    release_dependents();
+}
+
+// Exclusive prefix sums of a and c over the block's threads (in thread order)
+// and their totals; every thread of the block calls it.
+__device__ __forceinline__ void block_scan2(int a, int c, int &ea, int &ec, int &ta, int &tc,
+                                            int *scratch /* 2 * 32 ints */) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int ia = a, ic = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int xa = __shfl_up_sync(kFullMask, ia, o), xc = __shfl_up_sync(kFullMask, ic, o);
+        if (lane >= o) {
+            ia += xa;
+            ic += xc;
+        }
+    }
+    if (lane == 31) {
+        scratch[warp] = ia;
+        scratch[32 + warp] = ic;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int wa = lane < nw ? scratch[lane] : 0, wc = lane < nw ? scratch[32 + lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int xa = __shfl_up_sync(kFullMask, wa, o), xc = __shfl_up_sync(kFullMask, wc, o);
+            if (lane >= o) {
+                wa += xa;
+                wc += xc;
+            }
+        }
+        if (lane < nw) {
+            scratch[lane] = wa;  // inclusive over warps 0..lane
+            scratch[32 + lane] = wc;
+        }
+    }
+    __syncthreads();
+    const int pa = warp > 0 ? scratch[warp - 1] : 0, pc = warp > 0 ? scratch[32 + warp - 1] : 0;
+    ea = pa + ia - a;
+    ec = pc + ic - c;
+    ta = scratch[nw - 1];
+    tc = scratch[32 + nw - 1];
+    __syncthreads();
 }
 
 // ------------------------------------------------------------------- route
 // One block: softmax, top-k and weights per token (one warp per token), then
-// the pairs grouped by expert.
+// the pairs grouped by expert.  MAXE: experts per lane in the softmax
+// (n_exp <= 32 * MAXE), held in registers.
+template <int MAXE>
 __global__ void __launch_bounds__(ROUTE_THREADS) route_kernel(const MoeParams p) {
     wait_for_predecessor();
+    release_dependents();
     extern __shared__ int rsm[];
     int *cnt = rsm;                      // [n_exp + 1] tokens per expert
     int *fill = cnt + (p.n_exp + 1);     // [n_exp + 1] running fill per expert
     int *slot_of = fill + (p.n_exp + 1); // [n_exp + 1] active slot of expert e (or -1)
-    int *sel = slot_of + (p.n_exp + 1);  // [n_tok][top_k] selected experts
+    int *scan = slot_of + (p.n_exp + 1); // [64] block-scan scratch
+    int *sel = scan + 64;                // [n_tok][top_k] selected experts
     float *selw = reinterpret_cast<float *>(sel + p.n_tok * p.top_k);  // [n_tok][top_k]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int E = p.n_exp, K = p.top_k;
@@ -136,10 +180,10 @@ __global__ void __launch_bounds__(ROUTE_THREADS) route_kernel(const MoeParams p)
     for (int t = warp; t < p.n_tok; t += blockDim.x / 32) {
         // Lane l holds the probabilities of experts l, l + 32, ... in registers.
         const float *lg = p.logits + (size_t)t * (E + 1);
-        float pr[MAXE_LANE];
+        float pr[MAXE];
         float m = -INFINITY;
 #pragma unroll
-        for (int u = 0; u < MAXE_LANE; ++u) {
+        for (int u = 0; u < MAXE; ++u) {
             const int e = lane + 32 * u;
             pr[u] = e < E ? lg[e] : -INFINITY;
             m = fmaxf(m, pr[u]);
@@ -148,14 +192,14 @@ __global__ void __launch_bounds__(ROUTE_THREADS) route_kernel(const MoeParams p)
         for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
         float z = 0.f;
 #pragma unroll
-        for (int u = 0; u < MAXE_LANE; ++u) {
+        for (int u = 0; u < MAXE; ++u) {
             pr[u] = lane + 32 * u < E ? expf(pr[u] - m) : 0.f;
             z += pr[u];
         }
         z = group_sum<32>(z);
         const float rz = 1.f / z;
 #pragma unroll
-        for (int u = 0; u < MAXE_LANE; ++u) pr[u] = lane + 32 * u < E ? pr[u] * rz : -1.f;
+        for (int u = 0; u < MAXE; ++u) pr[u] = lane + 32 * u < E ? pr[u] * rz : -1.f;
         // Top-k, ties to the lower index: k rounds of a warp arg-max over each
         // lane's best untaken expert; the winner's lane marks it taken.
         uint32_t taken = 0;
@@ -164,7 +208,7 @@ __global__ void __launch_bounds__(ROUTE_THREADS) route_kernel(const MoeParams p)
             float bv = -1.f;
             int bi = 0x7fffffff;
 #pragma unroll
-            for (int u = 0; u < MAXE_LANE; ++u) {
+            for (int u = 0; u < MAXE; ++u) {
                 if (!((taken >> u) & 1u) && pr[u] > bv) {  // u ascending: ties keep the lower index
                     bv = pr[u];
                     bi = lane + 32 * u;
@@ -196,30 +240,34 @@ __global__ void __launch_bounds__(ROUTE_THREADS) route_kernel(const MoeParams p)
         }
     }
     __syncthreads();
-    if (tid == 0) {
-        // Active slots in expert order, the shared expert last; pair offsets.
-        int a = 0, off = 0;
-        for (int e = 0; e < E; ++e) {
-            slot_of[e] = -1;
-            if (cnt[e] > 0) {
-                slot_of[e] = a;
-                p.act_expert[a] = e;
-                p.act_off[a] = off;
+    // Active slots in expert order (thread e = expert e), the shared expert
+    // last; pair offsets.  Exclusive scans of "chosen at all" and of the counts.
+    {
+        const int e = tid;
+        const int ce = e < E ? cnt[e] : 0;
+        int slot, off, n_routed, n_pairs;
+        block_scan2(ce > 0 ? 1 : 0, ce, slot, off, n_routed, n_pairs, scan);
+        if (e < E) {
+            slot_of[e] = ce > 0 ? slot : -1;
+            if (ce > 0) {
+                p.act_expert[slot] = e;
+                p.act_off[slot] = off;
                 fill[e] = off;
-                off += cnt[e];
-                ++a;
             }
         }
-        if (has_shared) {
-            slot_of[E] = a;
-            p.act_expert[a] = E;
-            p.act_off[a] = off;
-            fill[E] = off;
-            off += p.n_tok;
-            ++a;
+        if (tid == 0) {
+            int a = n_routed, end_off = n_pairs;
+            if (has_shared) {
+                slot_of[E] = a;
+                p.act_expert[a] = E;
+                p.act_off[a] = end_off;
+                fill[E] = end_off;
+                end_off += p.n_tok;
+                ++a;
+            }
+            p.act_off[a] = end_off;
+            *p.n_active = a;
         }
-        p.act_off[a] = off;
-        *p.n_active = a;
     }
     __syncthreads();
     // Pairs: (token, slot k) under its expert, in token order (one thread per token).
@@ -239,7 +287,6 @@ __global__ void __launch_bounds__(ROUTE_THREADS) route_kernel(const MoeParams p)
             p.tok_pair[(size_t)t * (K + 1) + K] = i;
         }
     }
-    release_dependents();
 }
 
 // ---------------------------------------------------------------- gate_up
@@ -247,6 +294,7 @@ __global__ void __launch_bounds__(ROUTE_THREADS) route_kernel(const MoeParams p)
 // expert a; warp w takes rows j0 + 2w, j0 + 2w + 1.  h = silu(g) * u per pair.
 __global__ void __launch_bounds__(256) gate_up_kernel(const MoeParams p) {
     wait_for_predecessor();
+    release_dependents();
     const int a = blockIdx.y;
     if (a >= *p.n_active) return;
     const int e = p.act_expert[a];
@@ -273,7 +321,6 @@ __global__ void __launch_bounds__(256) gate_up_kernel(const MoeParams p) {
             if (j1 != j) p.h[(size_t)i * hmax + j1] = d[1] / (1.f + expf(-d[1])) * d[3];
         }
     }
-    release_dependents();
 }
 
 // ------------------------------------------------------------------- down
@@ -281,6 +328,7 @@ __global__ void __launch_bounds__(256) gate_up_kernel(const MoeParams p) {
 // warp w takes rows i0 + 4w .. i0 + 4w + 3.  part[pair] = w_pair * W_down h.
 __global__ void __launch_bounds__(256) down_kernel(const MoeParams p) {
     wait_for_predecessor();
+    release_dependents();
     const int a = blockIdx.y;
     if (a >= *p.n_active) return;
     const int e = p.act_expert[a];
@@ -334,23 +382,24 @@ __global__ void __launch_bounds__(256) down_kernel(const MoeParams p) {
                 p.part[(size_t)i * p.hidden + row0 + r] = p.pair_w[i] * a;
         }
     }
-    release_dependents();
 }
 
 // ---------------------------------------------------------------- combine
+// Block (t, c): outputs 256c .. 256c+255 of token t, one per thread, each the
+// sum of the token's pairs' partials (their loads all in flight together).
 template <typename TOUT>
 __global__ void __launch_bounds__(256) combine_kernel(const MoeParams p) {
     wait_for_predecessor();
-    const int t = blockIdx.x;
-    const int np = p.top_k + (p.s_inter > 0 ? 1 : 0);
-    const int *tp = p.tok_pair + (size_t)t * (p.top_k + 1);
-    TOUT *out = static_cast<TOUT *>(p.out) + (int64_t)t * p.out_stride;
-    for (int i = threadIdx.x; i < p.hidden; i += blockDim.x) {
-        float y = 0.f;
-        for (int k = 0; k < np; ++k) y += p.part[(size_t)tp[k] * p.hidden + i];
-        Elem<TOUT>::store1(out + i, y);
-    }
     release_dependents();
+    __shared__ int tp[33];  // top_k <= 32, and the shared pair
+    const int t = blockIdx.x, i = blockIdx.y * 256 + threadIdx.x;
+    const int np = p.top_k + (p.s_inter > 0 ? 1 : 0);
+    if (threadIdx.x < np) tp[threadIdx.x] = p.tok_pair[(size_t)t * (p.top_k + 1) + threadIdx.x];
+    __syncthreads();
+    if (i >= p.hidden) return;
+    float y = 0.f;
+    for (int k = 0; k < np; ++k) y += p.part[(size_t)tp[k] * p.hidden + i];
+    Elem<TOUT>::store1(static_cast<TOUT *>(p.out) + (int64_t)t * p.out_stride + i, y);
 }
 
 }  // namespace moe
@@ -383,7 +432,7 @@ size_t moe_workspace_bytes(int n_tok, int n_exp, int top_k, int inter, int s_int
 }
 
 size_t moe_route_smem_bytes(int n_tok, int n_exp, int top_k) {
-    return (size_t)3 * (n_exp + 1) * 4 + (size_t)n_tok * top_k * 8;
+    return (size_t)3 * (n_exp + 1) * 4 + 64 * 4 + (size_t)n_tok * top_k * 8;
 }
 
 cudaError_t launch_moe_args(const gdr_moe_args *a, void *workspace, cudaStream_t s) {
@@ -437,12 +486,13 @@ cudaError_t launch_moe_args(const gdr_moe_args *a, void *workspace, cudaStream_t
     const int rows = p.n_exp + 1;
     if ((e = launch(moe::router_kernel, dim3((rows + 7) / 8), 256, 0)) != cudaSuccess) return e;
     const size_t rsm = moe_route_smem_bytes(p.n_tok, p.n_exp, p.top_k);
+    // Fewer experts per lane in registers when they fit.
+    auto route = p.n_exp <= 256 ? moe::route_kernel<8> : moe::route_kernel<32>;
     if (rsm > 48 * 1024) {
-        e = cudaFuncSetAttribute(moe::route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)rsm);
+        e = cudaFuncSetAttribute(route, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsm);
         if (e != cudaSuccess) return e;
     }
-    if ((e = launch(moe::route_kernel, dim3(1), moe::ROUTE_THREADS, rsm)) != cudaSuccess) return e;
+    if ((e = launch(route, dim3(1), moe::ROUTE_THREADS, rsm)) != cudaSuccess) return e;
     // Active slots: at most min(n_tok * top_k, n_exp) routed experts and the shared one.
     const long routed = (long)p.n_tok * p.top_k < p.n_exp ? (long)p.n_tok * p.top_k : p.n_exp;
     const unsigned max_active = (unsigned)(routed + (p.s_inter > 0 ? 1 : 0));
@@ -453,10 +503,11 @@ cudaError_t launch_moe_args(const gdr_moe_args *a, void *workspace, cudaStream_t
     if ((e = launch(moe::down_kernel, dim3((p.hidden + moe::DN_ROWS - 1) / moe::DN_ROWS, max_active),
                     256, 0)) != cudaSuccess)
         return e;
+    const dim3 cgrid(p.n_tok, (p.hidden + 255) / 256);
     if (a->out_dtype == GDR_BF16)
-        e = launch(moe::combine_kernel<__nv_bfloat16>, dim3(p.n_tok), 256, 0);
+        e = launch(moe::combine_kernel<__nv_bfloat16>, cgrid, 256, 0);
     else
-        e = launch(moe::combine_kernel<float>, dim3(p.n_tok), 256, 0);
+        e = launch(moe::combine_kernel<float>, cgrid, 256, 0);
     return e;
 }
 

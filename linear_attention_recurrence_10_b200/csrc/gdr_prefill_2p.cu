@@ -700,6 +700,11 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
             prefetch(c + 2);
         }
         cp_async_wait_all();
+        // The last chunk's S Q^T commit is the one tcgen05 arrival nobody else
+        // waits for; it must land before the CTA ends (after an expired wait,
+        // only if its product was issued: it comes within microseconds then).
+        if (lane == 0 && n_chunks > 0)
+            mbar_wait(bar_qfree, (uint32_t)(n_chunks - 1) & 1u, ok ? wait_ns : 1000000ull);
         if (!ok) {
             if (lane == 0) fail();
             // No bulk copy may land after the CTA ends.

@@ -555,9 +555,12 @@ def attn_decode_measure(device, steps=16, warmup=4, world=1, layers=ATT_LAYERS):
                        f"dims, bf16 cache and outputs",
            "l2": f"inputs larger than L2: {L} layers' caches "
                  f"({2 * kc.numel() * 2 / 1e9:.1f} GB) rotate every step",
-           "launch": "one CUDA graph per step: 3 kernels per layer (rope/append, attend, combine)",
+           "launch": "one CUDA graph per step: rope/append and attend per layer (one work item "
+                     "per (sequence, kv head): the attend kernel stores the gated output, no "
+                     "combine)",
            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
-                        "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                        "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                        "traffic": captured_traffic("attend_kernel"), "kernel": "attend_kernel",
                         "bytes_per_layer": per_layer,
                         "us_per_layer": ms * 1e3 / (steps * L),
                         "peak_source": peaks["source"] + " (hbm_gbs, of measured copy bandwidth)"}}
@@ -679,9 +682,10 @@ def gva_decode_measure(device, steps=32, warmup=4, world=1):
 
 # ------------------------------------------------------------- CPU oracle
 
-def oracle_sample(n_tokens=512, seed=1, threads=None):
+def oracle_sample(n_tokens=512, seed=1, threads=None, reps=30):
     """Time the fp64 oracle on one layer of the decode workload: B sequences x
-    16 heads x n_tokens steps, on every host core."""
+    16 heads x n_tokens steps, on every host core, `reps` times over (about ten
+    seconds of CPU work with the defaults)."""
     import numpy as np
     import oracle
     from linear_attention_recurrence_10_b200 import synth
@@ -690,14 +694,16 @@ def oracle_sample(n_tokens=512, seed=1, threads=None):
     f = lambda t: t.to(torch.float64).numpy()
     args = dict(q=f(inp.q), k=f(inp.k), v=f(inp.v), g=f(inp.g), beta=f(inp.beta),
                 cu_seqlens=np.array(inp.cu_seqlens), z=f(inp.z), s0=f(inp.s0), w=f(inp.w))
+    lib = oracle.load()
     t0 = time.perf_counter()
-    oracle.gdr_recurrent(**args, threads=threads)
+    for _ in range(reps):
+        oracle.gdr_recurrent(**args, threads=threads, lib=lib)
     dt = time.perf_counter() - t0
-    nbytes = n_tokens * decode_bytes_per_layer_step(BATCH, H_K, H_V, D)
+    nbytes = reps * n_tokens * decode_bytes_per_layer_step(BATCH, H_K, H_V, D)
     return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
             "seconds": dt,
             "sample": f"one layer of the decode workload: {BATCH} sequences x {H_V} heads x "
-                      f"{n_tokens} tokens, fp64 recurrence, {threads} threads"}
+                      f"{n_tokens} tokens, fp64 recurrence, {threads} threads, {reps} times"}
 
 
 def run_reference(args, rank, world):
@@ -862,7 +868,7 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_sample()
-        one = oracle_sample(n_tokens=32, threads=1)
+        one = oracle_sample(n_tokens=32, threads=1, reps=30)
         cpu["single_thread"] = {"value": one["value"], "unit": one["unit"], "cores": 1,
                                 "seconds": one["seconds"], "sample": one["sample"]}
 

@@ -47,6 +47,7 @@ struct MoeParams {
     int *pair_tok;      // [n_pairs] token of pair i (pairs grouped by expert)
     float *pair_w;      // [n_pairs] the pair's weight
     int *tok_pair;      // [n_tok][top_k + 1] pair index of (token, slot); the shared one last
+    int router_tg;      // tokens the router stages in shared memory per pass (1..8)
     float *h;           // [n_pairs][max(inter, s_inter)]
     float *part;        // [n_pairs][hidden]
 };
@@ -97,20 +98,62 @@ __device__ __forceinline__ void warp_dots_bf16(const __nv_bfloat16 *const (&w)[R
     for (int r = 0; r < ROWS; ++r) out[r] = group_sum<32>(acc[r]);
 }
 
+// The dot product of 8 bf16 weights with 8 bf16 inputs, added to acc (fp32),
+// in the order warp_dots_bf16 uses.
+__device__ __forceinline__ float dot8_bf16(const uint4 &a, const uint4 &b, float acc) {
+    const __nv_bfloat162 *a2 = reinterpret_cast<const __nv_bfloat162 *>(&a);
+    const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&b);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+        const float2 fa = __bfloat1622float2(a2[v]), fb = __bfloat1622float2(b2[v]);
+        acc = fmaf(fa.x, fb.x, fmaf(fa.y, fb.y, acc));
+    }
+    return acc;
+}
+
+constexpr int TG = 8;  // tokens that share one pass over a weight row
+
 // ------------------------------------------------------------------ router
 // One warp per router row e (e == n_exp: the shared-expert gate), every token.
+// The block stages up to router_tg token rows in shared memory at a time, and
+// each warp streams its row past them once per group: one load per 16-byte
+// chunk of the row, the token values read from shared memory.
 __global__ void __launch_bounds__(256) router_kernel(const MoeParams p) {
     wait_for_predecessor();
     release_dependents();
+    extern __shared__ uint4 xs[];  // [router_tg][hidden / 8]
     const int lane = threadIdx.x & 31;
     const int e = blockIdx.x * 8 + (threadIdx.x >> 5);
     const bool shared_row = e == p.n_exp;
-    if (e > p.n_exp || (shared_row && p.s_inter == 0)) return;
-    const __nv_bfloat16 *w[1] = {shared_row ? p.w_sgate : p.w_router + (size_t)e * p.hidden};
-    for (int t = 0; t < p.n_tok; ++t) {
-        float d[1];
-        warp_dots_bf16<1>(w, p.x + (int64_t)t * p.x_stride, p.hidden, lane, d);
-        if (lane == 0) p.logits[(size_t)t * (p.n_exp + 1) + e] = d[0];
+    const bool active = e < p.n_exp || (shared_row && p.s_inter > 0);
+    const uint4 *w = reinterpret_cast<const uint4 *>(
+        shared_row ? p.w_sgate : p.w_router + (size_t)min(e, p.n_exp - 1) * p.hidden);
+    const int nc = p.hidden / 8;
+    for (int t0 = 0; t0 < p.n_tok; t0 += p.router_tg) {
+        const int ng = min(p.router_tg, p.n_tok - t0);
+        __syncthreads();  // the previous group is done with xs
+        for (int i = threadIdx.x; i < ng * nc; i += blockDim.x) {
+            const int t = i / nc, c = i - t * nc;
+            xs[i] = __ldg(reinterpret_cast<const uint4 *>(p.x + (int64_t)(t0 + t) * p.x_stride) + c);
+        }
+        __syncthreads();
+        if (!active) continue;
+        float acc[TG];
+#pragma unroll
+        for (int t = 0; t < TG; ++t) acc[t] = 0.f;
+#pragma unroll 8
+        for (int c = lane; c < nc; c += 32) {
+            const uint4 wv = __ldg(w + c);
+#pragma unroll
+            for (int t = 0; t < TG; ++t)
+                if (t < ng) acc[t] = dot8_bf16(wv, xs[t * nc + c], acc[t]);
+        }
+#pragma unroll
+        for (int t = 0; t < TG; ++t) {
+            if (t >= ng) break;
+            const float d = group_sum<32>(acc[t]);
+            if (lane == 0) p.logits[(size_t)(t0 + t) * (p.n_exp + 1) + e] = d;
+        }
     }
 }
 
@@ -292,7 +335,7 @@ __global__ void __launch_bounds__(ROUTE_THREADS) route_kernel(const MoeParams p)
 // ---------------------------------------------------------------- gate_up
 // Block (a, j0): rows j0 .. j0+15 of the gate and up matrices of active
 // expert a; warp w takes rows j0 + 2w, j0 + 2w + 1.  h = silu(g) * u per pair.
-__global__ void __launch_bounds__(256) gate_up_kernel(const MoeParams p) {
+__global__ void __launch_bounds__(256, 2) gate_up_kernel(const MoeParams p) {
     wait_for_predecessor();
     release_dependents();
     const int a = blockIdx.y;
@@ -313,12 +356,55 @@ __global__ void __launch_bounds__(256) gate_up_kernel(const MoeParams p) {
     const int j1 = j + 1 < I ? j + 1 : j;
     const __nv_bfloat16 *w[4] = {W + (size_t)j * p.hidden, W + (size_t)j1 * p.hidden,
                                  W + (size_t)(I + j) * p.hidden, W + (size_t)(I + j1) * p.hidden};
-    for (int i = p0; i < p1; ++i) {
+    if (p1 - p0 == 1) {
+        // One token (every routed expert at small batch): all of the four rows'
+        // loads in flight at once.
         float d[4];
-        warp_dots_bf16<4>(w, p.x + (int64_t)p.pair_tok[i] * p.x_stride, p.hidden, lane, d);
+        warp_dots_bf16<4>(w, p.x + (int64_t)p.pair_tok[p0] * p.x_stride, p.hidden, lane, d);
         if (lane == 0) {
-            p.h[(size_t)i * hmax + j] = d[0] / (1.f + expf(-d[0])) * d[2];
-            if (j1 != j) p.h[(size_t)i * hmax + j1] = d[1] / (1.f + expf(-d[1])) * d[3];
+            p.h[(size_t)p0 * hmax + j] = d[0] / (1.f + expf(-d[0])) * d[2];
+            if (j1 != j) p.h[(size_t)p0 * hmax + j1] = d[1] / (1.f + expf(-d[1])) * d[3];
+        }
+        return;
+    }
+    // Several tokens (the shared expert, or a popular one): each chunk of the
+    // four rows is loaded once per group of up to GU_TG tokens.
+    constexpr int GU_TG = 4;
+    const int nc = p.hidden / 8;
+    for (int g0 = p0; g0 < p1; g0 += GU_TG) {
+        const int ng = min(GU_TG, p1 - g0);
+        const uint4 *xr[GU_TG];
+#pragma unroll
+        for (int t = 0; t < GU_TG; ++t)
+            xr[t] = reinterpret_cast<const uint4 *>(p.x + (int64_t)p.pair_tok[g0 + min(t, ng - 1)] * p.x_stride);
+        float acc[GU_TG][4];
+#pragma unroll
+        for (int t = 0; t < GU_TG; ++t)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) acc[t][r] = 0.f;
+#pragma unroll 2
+        for (int c = lane; c < nc; c += 32) {
+            uint4 wv[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) wv[r] = __ldg(reinterpret_cast<const uint4 *>(w[r]) + c);
+#pragma unroll
+            for (int t = 0; t < GU_TG; ++t) {  // rows past ng repeat the last token (unused)
+                const uint4 xv = __ldg(xr[t] + c);
+#pragma unroll
+                for (int r = 0; r < 4; ++r) acc[t][r] = dot8_bf16(wv[r], xv, acc[t][r]);
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < GU_TG; ++t) {
+            if (t >= ng) break;
+            float d[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) d[r] = group_sum<32>(acc[t][r]);
+            if (lane == 0) {
+                const size_t i = (size_t)(g0 + t);
+                p.h[i * hmax + j] = d[0] / (1.f + expf(-d[0])) * d[2];
+                if (j1 != j) p.h[i * hmax + j1] = d[1] / (1.f + expf(-d[1])) * d[3];
+            }
         }
     }
 }
@@ -326,7 +412,7 @@ __global__ void __launch_bounds__(256) gate_up_kernel(const MoeParams p) {
 // ------------------------------------------------------------------- down
 // Block (a, i0): output rows i0 .. i0+31 of active expert a's down matrix;
 // warp w takes rows i0 + 4w .. i0 + 4w + 3.  part[pair] = w_pair * W_down h.
-__global__ void __launch_bounds__(256) down_kernel(const MoeParams p) {
+__global__ void __launch_bounds__(256, 2) down_kernel(const MoeParams p) {
     wait_for_predecessor();
     release_dependents();
     const int a = blockIdx.y;
@@ -338,49 +424,93 @@ __global__ void __launch_bounds__(256) down_kernel(const MoeParams p) {
     const int p0 = p.act_off[a], p1 = p.act_off[a + 1];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int hmax = p.inter > p.s_inter ? p.inter : p.s_inter;
-    // The warp's four rows, their weights loaded once into registers (the rows
-    // are I values: I / 256 16-byte chunks per lane), then every pair's h.
-    constexpr int MAXC = 4;  // chunks per lane: I <= 1024
     const int row0 = blockIdx.x * DN_ROWS + 4 * warp;
-    if (row0 >= p.hidden) return;
+    const bool wactive = row0 < p.hidden;
     const int nc = I / 8;
-    uint4 wv[4][MAXC];
+    const uint4 *wr[4];
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const int row = min(row0 + r, p.hidden - 1);
+    for (int r = 0; r < 4; ++r)
+        wr[r] = reinterpret_cast<const uint4 *>(W + (size_t)min(row0 + r, p.hidden - 1) * I);
+    // 8 weights (one 16-byte chunk) against 8 fp32 values of h.
+    auto dot8_h = [](const uint4 &w, const float4 &h0, const float4 &h1, float acc) {
+        const __nv_bfloat162 *w2 = reinterpret_cast<const __nv_bfloat162 *>(&w);
+        const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
 #pragma unroll
-        for (int u = 0; u < MAXC; ++u) {
-            const int c = lane + 32 * u;
-            wv[r][u] = c < nc ? __ldg(reinterpret_cast<const uint4 *>(W + (size_t)row * I) + c)
-                              : make_uint4(0, 0, 0, 0);
+        for (int v = 0; v < 4; ++v) {
+            const float2 f = __bfloat1622float2(w2[v]);
+            acc = fmaf(f.x, hv[2 * v], fmaf(f.y, hv[2 * v + 1], acc));
         }
-    }
-    for (int i = p0; i < p1; ++i) {
-        const float *hp = p.h + (size_t)i * hmax;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int u = 0; u < MAXC; ++u) {
-            const int c = lane + 32 * u;
-            if (c >= nc) break;
-            const float4 h0 = *reinterpret_cast<const float4 *>(hp + 8 * c);
-            const float4 h1 = *reinterpret_cast<const float4 *>(hp + 8 * c + 4);
-            const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const __nv_bfloat162 *w2 = reinterpret_cast<const __nv_bfloat162 *>(&wv[r][u]);
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    const float2 f = __bfloat1622float2(w2[v]);
-                    acc[r] = fmaf(f.x, hv[2 * v], fmaf(f.y, hv[2 * v + 1], acc[r]));
-                }
-            }
-        }
+        return acc;
+    };
+    auto store = [&](int i, const float (&acc)[4]) {
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
             const float a = group_sum<32>(acc[r]);
             if (lane == 0 && row0 + r < p.hidden)
                 p.part[(size_t)i * p.hidden + row0 + r] = p.pair_w[i] * a;
         }
+    };
+    if (p1 - p0 == 1) {
+        // One pair (every routed expert at small batch): the four rows stream
+        // past once, all of a lane's chunks in flight together.
+        if (!wactive) return;
+        constexpr int MAXC = 4;  // chunks per lane: I <= 1024
+        const float *hp = p.h + (size_t)p0 * hmax;
+        uint4 wv[4][MAXC];
+        float4 h0[MAXC], h1[MAXC];
+#pragma unroll
+        for (int u = 0; u < MAXC; ++u) {
+            const int c = lane + 32 * u;
+            const bool in = c < nc;
+#pragma unroll
+            for (int r = 0; r < 4; ++r) wv[r][u] = in ? __ldg(wr[r] + c) : make_uint4(0, 0, 0, 0);
+            h0[u] = in ? *reinterpret_cast<const float4 *>(hp + 8 * c) : make_float4(0.f, 0.f, 0.f, 0.f);
+            h1[u] = in ? *reinterpret_cast<const float4 *>(hp + 8 * c + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int u = 0; u < MAXC; ++u)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) acc[r] = dot8_h(wv[r][u], h0[u], h1[u], acc[r]);
+        store(p0, acc);
+        return;
+    }
+    // Several pairs (the shared expert, or a popular one): up to DN_G pairs' h
+    // staged in shared memory, and each chunk of the four rows applied to all
+    // of them once it is loaded.
+    constexpr int DN_G = 8;
+    __shared__ __align__(16) float hs[DN_G][1024];
+    for (int g0 = p0; g0 < p1; g0 += DN_G) {
+        const int ng = min(DN_G, p1 - g0);
+        __syncthreads();  // the previous group is done with hs
+        for (int e = threadIdx.x; e < ng * (I / 4); e += blockDim.x) {
+            const int t = e / (I / 4), c4 = e - t * (I / 4);
+            *reinterpret_cast<float4 *>(&hs[t][4 * c4]) =
+                *reinterpret_cast<const float4 *>(p.h + (size_t)(g0 + t) * hmax + 4 * c4);
+        }
+        __syncthreads();
+        if (!wactive) continue;
+        float acc[DN_G][4];
+#pragma unroll
+        for (int t = 0; t < DN_G; ++t)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) acc[t][r] = 0.f;
+        for (int c = lane; c < nc; c += 32) {
+            uint4 wv[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) wv[r] = __ldg(wr[r] + c);
+#pragma unroll
+            for (int t = 0; t < DN_G; ++t) {  // rows past ng repeat the last pair (unused)
+                const float *hp = hs[min(t, ng - 1)];
+                const float4 a = *reinterpret_cast<const float4 *>(hp + 8 * c);
+                const float4 b = *reinterpret_cast<const float4 *>(hp + 8 * c + 4);
+#pragma unroll
+                for (int r = 0; r < 4; ++r) acc[t][r] = dot8_h(wv[r], a, b, acc[t][r]);
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < DN_G; ++t)
+            if (t < ng) store(g0 + t, acc[t]);
     }
 }
 
@@ -484,7 +614,18 @@ cudaError_t launch_moe_args(const gdr_moe_args *a, void *workspace, cudaStream_t
     };
     cudaError_t e;
     const int rows = p.n_exp + 1;
-    if ((e = launch(moe::router_kernel, dim3((rows + 7) / 8), 256, 0)) != cudaSuccess) return e;
+    // Token rows staged per router pass: up to TG, within 96 KB of shared memory.
+    const size_t row_bytes = (size_t)p.hidden * 2;
+    size_t tg = (96 * 1024) / row_bytes;
+    tg = tg < 1 ? 1 : (tg > (size_t)moe::TG ? (size_t)moe::TG : tg);
+    p.router_tg = (int)tg;
+    const size_t xsm = tg * row_bytes;
+    if (xsm > 48 * 1024) {
+        e = cudaFuncSetAttribute(moe::router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)xsm);
+        if (e != cudaSuccess) return e;
+    }
+    if ((e = launch(moe::router_kernel, dim3((rows + 7) / 8), 256, xsm)) != cudaSuccess) return e;
     const size_t rsm = moe_route_smem_bytes(p.n_tok, p.n_exp, p.top_k);
     // Fewer experts per lane in registers when they fit.
     auto route = p.n_exp <= 256 ? moe::route_kernel<8> : moe::route_kernel<32>;

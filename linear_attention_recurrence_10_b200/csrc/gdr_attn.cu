@@ -36,7 +36,7 @@
 // bounded (2 s); on expiry the kernel records GDR_ERR_TIMEOUT in the workspace
 // status word, waits (bounded) for its copies in flight, frees its tensor
 // memory and returns.
-#include <cuda.h>  // CUtensorMap and its encoder's types (fetched from the driver at run time)
+#include "gdr_tmap.cuh"
 #include <math.h>
 
 #include "gdr.h"
@@ -750,37 +750,10 @@ void attn_plan(int batch, int H_kv, int kv_bound, int n_sm, int *n_split, int *s
 
 namespace {
 
-using EncodeTiledFn = decltype(&cuTensorMapEncodeTiled);
-
-// The driver's tensor-map encoder, looked up once through the runtime (no
-// link-time dependency on the driver library).
-EncodeTiledFn encode_tiled() {
-    static const EncodeTiledFn fn = []() -> EncodeTiledFn {
-        void *f = nullptr;
-        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault,
-                                             &q) != cudaSuccess ||
-            q != cudaDriverEntryPointSuccess) {
-            (void)cudaGetLastError();
-            return nullptr;
-        }
-        return reinterpret_cast<EncodeTiledFn>(f);
-    }();
-    return fn;
-}
-
 // A cache as `rows` rows of 256 bf16 (512-byte stride); boxes of 64 dims x
 // 128 rows, 128-byte swizzle, rows past the end read as zero.
 bool encode_cache_map(CUtensorMap *m, void *base, uint64_t rows) {
-    const EncodeTiledFn fn = encode_tiled();
-    if (!fn) return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)attn::D, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)attn::D * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)attn::TILE};
-    const cuuint32_t elem_strides[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, elem_strides,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return encode_bf16_2d(m, base, attn::D, rows, (uint64_t)attn::D * 2, 64, attn::TILE);
 }
 
 }  // namespace

@@ -20,6 +20,7 @@
 // Arithmetic, operand precisions (bf16 MMAs, hi + lo pairs for T, P, Delta)
 // and layouts are those of the one-kernel version in gdr_prefill_tc.cu.
 #include "gdr_prefill_common.cuh"
+#include "gdr_tmap.cuh"
 
 namespace gdr {
 namespace tcp2 {
@@ -146,6 +147,8 @@ constexpr uint32_t A_TBW = A_AX;
 constexpr uint32_t A_GB = 99328;    // g[64], beta[64]
 constexpr uint32_t A_SCAL = 99840;  // scalars, mbarrier
 constexpr uint32_t A_SMEM = A_SCAL + 3072;
+constexpr uint32_t A_SMEM_LAUNCH = A_SMEM + 1024;  // with the alignment slack
+static_assert(2 * (A_SMEM_LAUNCH + 1024) <= 228 * 1024, "two prep blocks must share an SM");
 
 struct PrepScalars {
     float gam[C], eg[C], bet[C], nk[C], nq[C], dec[C];
@@ -154,10 +157,23 @@ struct PrepScalars {
     // diagonal 16-block as a product of two factors that are at most one.
     float dtab[4 * C];
     uint64_t bar;
+    uint64_t tbar;  // the K, Q, V tiles landed (tensor-copy path)
     uint32_t tmem;
 };
 static_assert(sizeof(PrepScalars) <= A_SMEM - A_SCAL, "prep scalars overflow");
 static_assert(A_T + C * PLD * 4 <= A_AX && A_AX + 32768 <= A_GB, "prep scratch overlap");
+
+// Tensor maps of the packed q, k and v (rows = tokens; boxes of 64 elements x
+// 64 tokens, 128-byte swizzle) for the prep kernel's tensor copies.
+struct PrepMaps {
+    CUtensorMap k, q, v;
+};
+// The [K;Q] tile as the tensor copies leave it: per half of d (64 values),
+// 64 rows of K then 64 of Q, 128 bytes a row, 16-byte chunks swizzled by the
+// row's index mod 8.
+__device__ __forceinline__ uint32_t kq_sw(int row, int jc) {
+    return (uint32_t)((jc >> 3) * 16384 + row * 128 + (((jc & 7) ^ (row & 7)) << 4));
+}
 
 // `succ`: block index distance to the unit that most likely takes this block's
 // SM slot next (resident blocks per SM x SMs); its inputs are prefetched to L2.
@@ -181,11 +197,17 @@ __device__ __forceinline__ PrepUnit prep_unit(const int *seg_off, int seg_lo, in
 // segment's recurrence; the block of the highest index waits for it before
 // exiting, so that this grid completes only after it (the next recurrence
 // segment, queued after this grid, reads the state it carries).
-__global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p, const int *chunk_off,
+// K, Q and V come by tensor copies (maps) into 128-byte-swizzled tiles.
+__global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p,
+                                                     const __grid_constant__ PrepMaps maps,
+                                                     const int *chunk_off,
                                                      const int *seg_off, int seg_lo,
                                                      unsigned char *records, int *status, int succ,
                                                      int wait_prev_at_exit) {
-    extern __shared__ __align__(1024) unsigned char sm[];
+    extern __shared__ __align__(1024) unsigned char sm_raw[];
+    // The swizzled tiles must start on a 1024-byte boundary (A_SMEM_LAUNCH
+    // leaves room to round up).
+    unsigned char *sm = sm_raw + ((1024u - (smem_u32(sm_raw) & 1023u)) & 1023u);
     PrepScalars &sc = *reinterpret_cast<PrepScalars *>(sm + A_SCAL);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int quad = warp & 3, part = warp >> 2;
@@ -199,9 +221,6 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p, con
     const int L = (int)((t1 - c0) < C ? (t1 - c0) : C);
     unsigned char *rec = records + ((size_t)gchunk * p.H_v + hv) * REC_BYTES;
 
-    const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(p.q);
-    const __nv_bfloat16 *kg = static_cast<const __nv_bfloat16 *>(p.k);
-    const __nv_bfloat16 *vg = static_cast<const __nv_bfloat16 *>(p.v);
     const uint32_t sbase = smem_u32(sm);
     float *Ascr = reinterpret_cast<float *>(sm + A_AX);
     float *Xscr = Ascr + C * PLD;
@@ -211,23 +230,18 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p, con
     if (warp == 0) tmem_alloc(&sc.tmem, 256);
     if (tid == 0) {
         mbar_init(&sc.bar, 1);
+        mbar_init(&sc.tbar, 1);
         mbar_fence_init();
-    }
-    for (int e = tid; e < 128 * 16; e += PNT) {
-        const int row = (e & 7) + 8 * ((e >> 5) & 15);
-        const int jc = ((e >> 3) & 3) + 4 * (e >> 9);
-        const int r = row & 63;
-        const bool in = r < L;
-        const int64_t t = in ? c0 + r : c0;
-        const __nv_bfloat16 *src = row < 64 ? kg + t * p.k_stride + hk * D : qg + t * p.q_stride + hk * D;
-        cp_async16(sm + A_KQ + kq_off(row, 8 * jc), src + 8 * jc, in ? 16u : 0u);
-    }
-    for (int e = tid; e < C * 16; e += PNT) {
-        const int s = (e & 7) + 8 * ((e >> 5) & 7);
-        const int ic = ((e >> 3) & 3) + 4 * (e >> 8);
-        const bool in = s < L;
-        const int64_t t = in ? c0 + s : c0;
-        cp_async16(sm + A_V + v_off(s, 8 * ic), vg + t * p.v_stride + hv * D + 8 * ic, in ? 16u : 0u);
+        // Six boxes of 64 tokens x 64 values: K and Q (each d half), V.
+        // Tokens past the sequence belong to the next one (zeroed below) or
+        // lie past the tensor (read as zero).
+        bulk_expect(&sc.tbar, 6 * 8192);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            tma_load_2d(sbase + A_KQ + h * 16384, &maps.k, hk * D + 64 * h, (int)c0, &sc.tbar);
+            tma_load_2d(sbase + A_KQ + h * 16384 + 8192, &maps.q, hk * D + 64 * h, (int)c0, &sc.tbar);
+            tma_load_2d(sbase + A_V + h * 8192, &maps.v, hv * D + 64 * h, (int)c0, &sc.tbar);
+        }
     }
     if (tid < 2 * C) {
         const int r = tid & 63;
@@ -236,27 +250,38 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p, con
         cp_async4(gbuf + tid, (tid < C ? p.g : p.beta) + t * p.gb_stride + hv, in ? 4u : 0u);
     }
     cp_async_commit();
-    if (blockIdx.x + succ < gridDim.x) {
-        // Warm L2 for the unit most likely to take this block's SM slot next:
-        // 64 rows x (k, q, v) x two 128-byte lines over the block's threads.
+    if (tid == 0 && blockIdx.x + succ < gridDim.x) {
+        // Warm L2 for the unit most likely to take this block's SM slot next.
         const int nb = blockIdx.x + succ, hv2 = nb % p.H_v, hk2 = hv2 / p.hv_per_hk;
         const PrepUnit nu = prep_unit(seg_off, seg_lo, p.n_seq, nb / p.H_v);
-        const int64_t n0 = p.cu_seqlens[nu.seq] + (int64_t)nu.chunk * C, n1 = p.cu_seqlens[nu.seq + 1];
-        for (int e = tid; e < 3 * 2 * C; e += PNT) {
-            const int r = (e >> 1) & 63, line = e & 1, which = e >> 7;
-            const int64_t t = n0 + r;
-            if (t < n1) {
-                const __nv_bfloat16 *ptr = which == 0 ? kg + t * p.k_stride + hk2 * D
-                                          : which == 1 ? qg + t * p.q_stride + hk2 * D
-                                                       : vg + t * p.v_stride + hv2 * D;
-                prefetch_l2(ptr + 64 * line);
-            }
+        const int n0 = (int)(p.cu_seqlens[nu.seq] + (int64_t)nu.chunk * C);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            tma_prefetch_2d(&maps.k, hk2 * D + 64 * h, n0);
+            tma_prefetch_2d(&maps.q, hk2 * D + 64 * h, n0);
+            tma_prefetch_2d(&maps.v, hv2 * D + 64 * h, n0);
         }
     }
     cp_async_wait<0>();
+    // g and beta landed, the barriers' initialisation seen by every thread.
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
+    const bool loads_ok = mbar_wait(&sc.tbar, 0u, kWaitNs);
+    // Rows past a ragged chunk's end are zero (the products scale them by zero
+    // factors too, but the next sequence's values must not reach them).
+    if (loads_ok && L < C) {
+        const int nz = (C - L) * 8;
+        for (int e = tid; e < 6 * nz; e += PNT) {
+            const int box = e / nz, r = L + ((e - box * nz) >> 3), ch = e & 7;
+            const uint32_t at = box < 4 ? A_KQ + box * 8192 : A_V + (box - 4) * 8192;
+            *reinterpret_cast<uint4 *>(sm + at + r * 128 + ch * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+    fence_before_sync();
+    const bool loads_bad = __syncthreads_or(!loads_ok) != 0;
+    fence_after_sync();
+    if (loads_bad && tid == 0) atomicExch(status, kTimeoutStatus);
     const uint32_t tm = sc.tmem;
     const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
     constexpr uint32_t TM_D1 = 0, TM_U = 64, TM_W = 128;
@@ -266,7 +291,8 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p, con
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int jc = 0; jc < 16; ++jc) {
-            const uint4 raw = *reinterpret_cast<const uint4 *>(sm + A_KQ + kq_off(tid, 8 * jc));
+            const uint4 raw =
+                *reinterpret_cast<const uint4 *>(sm + A_KQ + kq_sw(tid, jc));
             const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
@@ -331,8 +357,13 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p, con
     const uint32_t ID_U = instr_desc<Kind::BF16>(128, 64, true, false);
     const uint32_t kq = sbase + A_KQ;
 
-    bool alive = issue_and_wait([&] {
-        gemm(tm + TM_D1, kq, 128, 2048, 256, kq, 128, 2048, 256, D / 16, ID_KK, false);
+    bool alive = !loads_bad && issue_and_wait([&] {
+        // K-major, 128-byte swizzle: a K step is 32 bytes inside a row, the
+        // second half of d 16 KB on.
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t dk = smem_desc_sw128(kq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+            mma<Kind::BF16>(tm + TM_D1, dk, dk, ID_KK, kk > 0 ? 1u : 0u);
+        }
     });
     if (alive) {
         // A (fp32 scratch) and P (hi/lo bf16 straight into the record).  The
@@ -402,10 +433,18 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p, con
         }
         alive = issue_and_wait([&] {
             const uint32_t tbw = sbase + A_TBW;
-            gemm(tm + TM_U, sbase + A_V, 128, 1024, 256, tbw, 1024, 128, 2048, C / 16, ID_U, false);
-            gemm(tm + TM_U, sbase + A_V, 128, 1024, 256, tbw + 8192, 1024, 128, 2048, C / 16, ID_U, true);
-            gemm(tm + TM_W, kq, 2048, 128, 4096, tbw + 16384, 1024, 128, 2048, C / 16, ID_U, false);
-            gemm(tm + TM_W, kq, 2048, 128, 4096, tbw + 24576, 1024, 128, 2048, C / 16, ID_U, true);
+            // V and K as MN-major A (d across 64-value atoms, the tokens as K,
+            // 16 of them = 2 KB a step); B = T diag(beta) (hi, lo) and the
+            // same scaled for W (hi, lo).
+            for (int kk = 0; kk < C / 16; ++kk) {
+                const uint64_t av = smem_desc_sw128(sbase + A_V + kk * 2048, 8192, 1024);
+                const uint64_t ak = smem_desc_sw128(kq + kk * 2048, 16384, 1024);
+                const uint32_t acc = kk > 0 ? 1u : 0u;
+                mma<Kind::BF16>(tm + TM_U, av, smem_desc(tbw + kk * 2048, 1024, 128), ID_U, acc);
+                mma<Kind::BF16>(tm + TM_U, av, smem_desc(tbw + 8192 + kk * 2048, 1024, 128), ID_U, 1u);
+                mma<Kind::BF16>(tm + TM_W, ak, smem_desc(tbw + 16384 + kk * 2048, 1024, 128), ID_U, acc);
+                mma<Kind::BF16>(tm + TM_W, ak, smem_desc(tbw + 24576 + kk * 2048, 1024, 128), ID_U, 1u);
+            }
         });
     }
     if (alive) {
@@ -440,6 +479,8 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p, con
         fence_after_sync();
         tmem_free(tm, 256);
     }
+    // A tensor copy that did not land in time must not land after the block ends.
+    if (loads_bad && tid == 0) mbar_wait(&sc.tbar, 0u, 1000000ull);
     if (wait_prev_at_exit && blockIdx.x == gridDim.x - 1) wait_for_predecessor();
 }
 
@@ -490,7 +531,7 @@ constexpr uint32_t TM_DTH = 448, TM_DTL = 480;
 // A recurrence block holds all 512 TMEM columns, so a prep block (which the
 // next segment may start beside it) must never fit on the same SM: their
 // shared memory together exceeds an SM's (228 KB, 1 KB reserved per block).
-static_assert(B_SMEM + A_SMEM + 2 * 1024 > 228 * 1024,
+static_assert(B_SMEM + A_SMEM_LAUNCH + 2 * 1024 > 228 * 1024,
               "a prep block could share an SM with a recurrence block");
 
 // Chunks [seg_lo, seg_hi) of every sequence.  The state enters from the
@@ -1055,8 +1096,21 @@ cudaError_t launch_prefill_tc2p(const PrefillParams &p, const int32_t *cu_host, 
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return cudaGetLastError();
+    // Tensor maps for prep's K, Q and V (the caller's bases and row strides
+    // are 16-byte aligned; token offsets fit in int32).
+    tcp2::PrepMaps maps;
+    memset(&maps, 0, sizeof maps);
+    const uint64_t n_tok = (uint64_t)cu_host[p.n_seq];
+    const bool tma = n_tok > 0 && n_tok < 0x7fffffffull &&
+                     encode_bf16_2d(&maps.k, p.k, (uint64_t)p.H_k * tcp2::D, n_tok,
+                                    (uint64_t)p.k_stride * 2, 64, 64) &&
+                     encode_bf16_2d(&maps.q, p.q, (uint64_t)p.H_k * tcp2::D, n_tok,
+                                    (uint64_t)p.q_stride * 2, 64, 64) &&
+                     encode_bf16_2d(&maps.v, p.v, (uint64_t)p.H_v * tcp2::D, n_tok,
+                                    (uint64_t)p.v_stride * 2, 64, 64);
+    if (!tma && n_tok > 0) return cudaErrorInvalidValue;  // no encoder in the driver
     e = cudaFuncSetAttribute(tcp2::prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)tcp2::A_SMEM);
+                             (int)tcp2::A_SMEM_LAUNCH);
     if (e != cudaSuccess) return e;
     auto kern = out_bf16 ? tcp2::recur_kernel<__nv_bfloat16> : tcp2::recur_kernel<float>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcp2::B_SMEM);
@@ -1073,14 +1127,14 @@ cudaError_t launch_prefill_tc2p(const PrefillParams &p, const int32_t *cu_host, 
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3((unsigned)(units * p.H_v));
             cfg.blockDim = dim3(tcp2::PNT);
-            cfg.dynamicSmemBytes = tcp2::A_SMEM;
+            cfg.dynamicSmemBytes = tcp2::A_SMEM_LAUNCH;
             cfg.stream = s;
             cudaLaunchAttribute attr[1];
             attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
             attr[0].val.programmaticStreamSerializationAllowed = 1;
             cfg.attrs = attr;
             cfg.numAttrs = k > 0 ? 1 : 0;  // later segments overlap the recurrence before them
-            e = cudaLaunchKernelEx(&cfg, tcp2::prep_kernel, p, (const int *)chunk_off, seg_off_k,
+            e = cudaLaunchKernelEx(&cfg, tcp2::prep_kernel, p, maps, (const int *)chunk_off, seg_off_k,
                                    sp.lo[k], records, status, 2 * n_sm, k > 0 ? 1 : 0);
             if (e != cudaSuccess) {
                 (void)cudaGetLastError();

@@ -511,7 +511,7 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p,
 
 constexpr int RNT = 576;                       // 18 warps
 constexpr int OG_BAR = 1, OG_N = 256;
-constexpr uint32_t B_KQ = 0;                   // bf16 [K;Q] (32 KB)
+constexpr uint32_t B_KQ = 0;                   // bf16 [K;Q] (32 KB, as kq_sw lays it out)
 constexpr uint32_t B_W = 32768;                // bf16 W of the current chunk (16 KB)
 constexpr uint32_t B_P = 49152;                // bf16 P hi/lo of the current chunk (16 KB)
 constexpr uint32_t B_SC = 65536;               // 2 x scalars (eg, nqe, dn, eL: 1 KB each)
@@ -520,6 +520,7 @@ constexpr uint32_t B_U = 133120;               // fp32 U of the current chunk (3
 constexpr uint32_t B_OS = 165888;              // fp32 O [r][i] of the chunk being output (32 KB)
 constexpr uint32_t B_BAR = 198656;             // 18 mbarriers, then the TMEM address
 constexpr uint32_t B_SMEM = B_BAR + 160;
+constexpr uint32_t B_SMEM_LAUNCH = B_SMEM + 1024;  // with the alignment slack
 constexpr uint32_t SC_BYTES = REC_STAGED - REC_SCAL;
 // TMEM columns: the fp32 state, -S W^T, two buffers of S Q^T, one of P Delta,
 // and the bf16 copy of S (two values per column) that -S W^T and S Q^T read
@@ -531,24 +532,28 @@ constexpr uint32_t TM_DTH = 448, TM_DTL = 480;
 // A recurrence block holds all 512 TMEM columns, so a prep block (which the
 // next segment may start beside it) must never fit on the same SM: their
 // shared memory together exceeds an SM's (228 KB, 1 KB reserved per block).
-static_assert(B_SMEM + A_SMEM_LAUNCH + 2 * 1024 > 228 * 1024,
+static_assert(B_SMEM_LAUNCH + A_SMEM_LAUNCH + 2 * 1024 > 228 * 1024,
               "a prep block could share an SM with a recurrence block");
 
 // Chunks [seg_lo, seg_hi) of every sequence.  The state enters from the
 // caller's initial state in the first segment (seg_lo == 0), else from
 // `carry`; it leaves to the caller's final state in the segment where the
 // sequence ends, else to `carry` (both [n_seq, H_v, d_v, d_k]).
+// maps: the tensor maps of k and q (those of prep).
 template <typename TOUT>
-__global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, const int *order,
-                                                       const int *chunk_off,
+__global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p,
+                                                       const __grid_constant__ PrepMaps maps,
+                                                       const int *order, const int *chunk_off,
                                                        const unsigned char *records, int *status,
                                                        int seg_lo, int seg_hi, float *carry) {
-    extern __shared__ __align__(1024) unsigned char sm[];
+    extern __shared__ __align__(1024) unsigned char sm_raw[];
+    // The swizzled [K;Q] tile must start on a 1024-byte boundary.
+    unsigned char *sm = sm_raw + ((1024u - (smem_u32(sm_raw) & 1023u)) & 1023u);
     // The next kernel on the stream (the following segment's prep) may start
     // on the SMs this grid leaves free; it reads nothing this grid writes.
     release_dependents();
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + B_BAR);
-    uint64_t *bar_q = bars, *bar_k = bars + 1;   // tiles landed (32 producer lanes each)
+    uint64_t *bar_q = bars, *bar_k = bars + 1;   // tiles landed
     uint64_t *bar_w = bars + 2;                  // W landed
     uint64_t *bar_p = bars + 3;                  // P landed
     uint64_t *bar_sc = bars + 4;                 // [2] scalars landed
@@ -593,8 +598,8 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
 
     if (warp == 0) tmem_alloc(tmem_slot, 512);
     if (tid == 0) {
-        mbar_init(bar_q, 32);
-        mbar_init(bar_k, 32);
+        mbar_init(bar_q, 1);
+        mbar_init(bar_k, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar_sc + b, 1);
             mbar_init(bar_oready + b, 1);
@@ -637,7 +642,11 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
                 fence_smem_to_async();
                 gemm_ta(tm + TM_D, tm + TM_SB, sbase + B_W, 128, 2048, 256, D / 16, ID_D, false);
                 commit(smem_u32(bar_gd));
-                gemm_ta(tm + TM_OI + 64 * b, tm + TM_SB, kq + 16384, 128, 2048, 256, D / 16, ID_KK, false);
+                // B = Q, K-major with the 128-byte swizzle (kq_sw).
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_ta(tm + TM_OI + 64 * b, tm + TM_SB + 8 * kk,
+                           smem_desc_sw128(kq + 8192 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), ID_KK,
+                           kk > 0 ? 1u : 0u);
                 commit(smem_u32(bar_qfree));
                 // The update needs only the decayed Delta^T tiles (TMEM) and the
                 // pre-scaled state; the Delta tiles of P Delta may still be coming.
@@ -648,8 +657,13 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
                 fence_smem_to_async();
                 // S <- e^{gamma_L} S + Dt~^T K (hi + lo, Dt~^T from TMEM); then
                 // O_intra^T = Delta^T P^T (hi*hi + hi*lo + lo*hi) into its buffer.
-                gemm_ta(tm + TM_S, tm + TM_DTH, kq, 2048, 128, 4096, C / 16, ID_S, true);
-                gemm_ta(tm + TM_S, tm + TM_DTL, kq, 2048, 128, 4096, C / 16, ID_S, true);
+                // B = K, MN-major (d_k across the two 64-value atoms 16 KB
+                // apart, 16 tokens = 2 KB a step).
+                for (int kk = 0; kk < C / 16; ++kk) {
+                    const uint64_t bk = smem_desc_sw128(kq + kk * 2048, 16384, 1024);
+                    mma_ta(tm + TM_S, tm + TM_DTH + 8 * kk, bk, ID_S, 1u);
+                    mma_ta(tm + TM_S, tm + TM_DTL + 8 * kk, bk, ID_S, 1u);
+                }
                 commit(smem_u32(bar_gs));
                 // P Delta has one accumulator: chunk c-1's output must have left it.
                 ok = mbar_wait(bar_p, ph, wait_ns) && mbar_wait(bar_dready, ph, wait_ns) &&
@@ -671,24 +685,39 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
         // ------------------------------------------------------ producer
         const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(p.q) + hk * D;
         const __nv_bfloat16 *kg = static_cast<const __nv_bfloat16 *>(p.k) + hk * D;
-        // 64 rows x 256 bytes; lanes cover 8 rows x 4 column chunks (512
-        // contiguous bytes of shared memory) per step.
+        // Copies counted so that an early exit can wait for them.
+        int n_w = 0, n_p = 0, n_u = 0, n_sc[2] = {0, 0}, n_tile[2] = {0, 0};
+        // The K or Q tile of a chunk (kq_sw layout): a full chunk by two tensor
+        // copies; a sequence's ragged last chunk by 16-byte copies that read
+        // zero past its end (this lane waits for its own, then one arrival).
         auto fetch = [&](int64_t c0, int L, bool q_half) {
+            uint64_t *bar = q_half ? bar_q : bar_k;
+            const uint32_t dst = B_KQ + (q_half ? 8192u : 0u);
+            ++n_tile[q_half ? 1 : 0];
+            if (L == C) {
+                if (lane == 0) {
+                    const CUtensorMap *map = q_half ? &maps.q : &maps.k;
+                    bulk_expect(bar, 16384);
+                    tma_load_2d(sbase + dst, map, hk * D, (int)c0, bar);
+                    tma_load_2d(sbase + dst + 16384, map, hk * D + 64, (int)c0, bar);
+                }
+                return;
+            }
             const __nv_bfloat16 *base = q_half ? qg : kg;
             const int64_t stride = q_half ? p.q_stride : p.k_stride;
 #pragma unroll 8
             for (int e = lane; e < 64 * 16; e += 32) {
-                const int r = (e & 7) + 8 * ((e >> 5) & 7);
-                const int jc = ((e >> 3) & 3) + 4 * (e >> 8);
+                const int r = e >> 4, jc = e & 15;
                 const bool in = r < L;
                 const int64_t t = in ? c0 + r : t0;
-                cp_async16(sm + B_KQ + kq_off(r + (q_half ? 64 : 0), 8 * jc),
+                cp_async16(sm + dst + (jc >> 3) * 16384 + r * 128 + (((jc & 7) ^ (r & 7)) << 4),
                            base + t * stride + 8 * jc, in ? 16u : 0u);
             }
-            cp_async_arrive(q_half ? bar_q : bar_k);
+            cp_async_wait_all();
+            fence_smem_to_async();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar);
         };
-        // Bulk copies, each counted so that an early exit can wait for them.
-        int n_w = 0, n_p = 0, n_u = 0, n_sc[2] = {0, 0};
         auto bulk = [&](uint32_t dst, uint32_t src_off, uint32_t bytes, uint64_t *bar, int c) {
             if (lane == 0) {
                 bulk_expect(bar, bytes);
@@ -740,7 +769,6 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
             }
             prefetch(c + 2);
         }
-        cp_async_wait_all();
         // The last chunk's S Q^T commit is the one tcgen05 arrival nobody else
         // waits for; it must land before the CTA ends (after an expired wait,
         // only if its product was issued: it comes within microseconds then).
@@ -750,6 +778,8 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p, co
             if (lane == 0) fail();
             // No bulk copy may land after the CTA ends.
             if (n_w) mbar_wait(bar_w, (uint32_t)(n_w - 1) & 1u, wait_ns);
+            if (n_tile[0]) mbar_wait(bar_k, (uint32_t)(n_tile[0] - 1) & 1u, wait_ns);
+            if (n_tile[1]) mbar_wait(bar_q, (uint32_t)(n_tile[1] - 1) & 1u, wait_ns);
             if (n_p) mbar_wait(bar_p, (uint32_t)(n_p - 1) & 1u, wait_ns);
             if (n_u) mbar_wait(bar_u, (uint32_t)(n_u - 1) & 1u, wait_ns);
             for (int b = 0; b < 2; ++b)
@@ -1056,7 +1086,7 @@ size_t prefill_tc2p_workspace_bytes(int n_seq, int64_t n_chunks, int H_v, int n_
 }
 
 // cu_host: the sequence offsets on the host (segment sizes are planned here).
-// Segment boundaries: 48% and 79% of the longest sequence's chunks, so that
+// Segment boundaries: 40% and 72% of the longest sequence's chunks, so that
 // each later segment's prep (on the SMs the recurrence leaves free) takes
 // about as long as the recurrence of the segment before it.
 cudaError_t launch_prefill_tc2p(const PrefillParams &p, const int32_t *cu_host, int n_seg,
@@ -1071,8 +1101,8 @@ cudaError_t launch_prefill_tc2p(const PrefillParams &p, const int32_t *cu_host, 
     tcp2::SegPlan sp = {};
     sp.n = n_seg < 1 ? 1 : (n_seg > tcp2::MAX_SEG ? tcp2::MAX_SEG : n_seg);
     if (sp.n == 3) {
-        sp.lo[1] = (int)((max_chunks * 48 + 99) / 100);
-        sp.lo[2] = (int)((max_chunks * 79 + 99) / 100);
+        sp.lo[1] = (int)((max_chunks * 40 + 99) / 100);
+        sp.lo[2] = (int)((max_chunks * 72 + 99) / 100);
     } else if (sp.n == 2) {
         sp.lo[1] = (int)((max_chunks * 60 + 99) / 100);
     }
@@ -1113,7 +1143,7 @@ cudaError_t launch_prefill_tc2p(const PrefillParams &p, const int32_t *cu_host, 
                              (int)tcp2::A_SMEM_LAUNCH);
     if (e != cudaSuccess) return e;
     auto kern = out_bf16 ? tcp2::recur_kernel<__nv_bfloat16> : tcp2::recur_kernel<float>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcp2::B_SMEM);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcp2::B_SMEM_LAUNCH);
     if (e != cudaSuccess) return e;
     for (int k = 0; k < sp.n; ++k) {
         int64_t units = 0;
@@ -1143,8 +1173,8 @@ cudaError_t launch_prefill_tc2p(const PrefillParams &p, const int32_t *cu_host, 
         } else if (k > 0) {
             continue;  // no sequence reaches this segment
         }
-        kern<<<(unsigned)((int64_t)p.n_seq * p.H_v), tcp2::RNT, tcp2::B_SMEM, s>>>(
-            p, order, chunk_off, records, status, sp.lo[k], k + 1 == sp.n ? 0x7fffffff : sp.lo[k + 1],
+        kern<<<(unsigned)((int64_t)p.n_seq * p.H_v), tcp2::RNT, tcp2::B_SMEM_LAUNCH, s>>>(
+            p, maps, order, chunk_off, records, status, sp.lo[k], k + 1 == sp.n ? 0x7fffffff : sp.lo[k + 1],
             carry);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;

@@ -227,7 +227,9 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p,
     float *Tscr = reinterpret_cast<float *>(sm + A_T);
     float *gbuf = reinterpret_cast<float *>(sm + A_GB);
 
-    if (warp == 0) tmem_alloc(&sc.tmem, 256);
+    // Thread 0 starts the tile copies first; warp 7 (idle until the first
+    // product) takes the TMEM columns and, later, warms L2 for the successor.
+    if (warp == 7) tmem_alloc(&sc.tmem, 256);
     if (tid == 0) {
         mbar_init(&sc.bar, 1);
         mbar_init(&sc.tbar, 1);
@@ -250,18 +252,6 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p,
         cp_async4(gbuf + tid, (tid < C ? p.g : p.beta) + t * p.gb_stride + hv, in ? 4u : 0u);
     }
     cp_async_commit();
-    if (tid == 0 && blockIdx.x + succ < gridDim.x) {
-        // Warm L2 for the unit most likely to take this block's SM slot next.
-        const int nb = blockIdx.x + succ, hv2 = nb % p.H_v, hk2 = hv2 / p.hv_per_hk;
-        const PrepUnit nu = prep_unit(seg_off, seg_lo, p.n_seq, nb / p.H_v);
-        const int n0 = (int)(p.cu_seqlens[nu.seq] + (int64_t)nu.chunk * C);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            tma_prefetch_2d(&maps.k, hk2 * D + 64 * h, n0);
-            tma_prefetch_2d(&maps.q, hk2 * D + 64 * h, n0);
-            tma_prefetch_2d(&maps.v, hv2 * D + 64 * h, n0);
-        }
-    }
     cp_async_wait<0>();
     // g and beta landed, the barriers' initialisation seen by every thread.
     fence_before_sync();
@@ -282,6 +272,18 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p,
     const bool loads_bad = __syncthreads_or(!loads_ok) != 0;
     fence_after_sync();
     if (loads_bad && tid == 0) atomicExch(status, kTimeoutStatus);
+    if (tid == 7 * 32 && blockIdx.x + succ < gridDim.x) {
+        // Warm L2 for the unit most likely to take this block's SM slot next.
+        const int nb = blockIdx.x + succ, hv2 = nb % p.H_v, hk2 = hv2 / p.hv_per_hk;
+        const PrepUnit nu = prep_unit(seg_off, seg_lo, p.n_seq, nb / p.H_v);
+        const int n0 = (int)(p.cu_seqlens[nu.seq] + (int64_t)nu.chunk * C);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            tma_prefetch_2d(&maps.k, hk2 * D + 64 * h, n0);
+            tma_prefetch_2d(&maps.q, hk2 * D + 64 * h, n0);
+            tma_prefetch_2d(&maps.v, hv2 * D + 64 * h, n0);
+        }
+    }
     const uint32_t tm = sc.tmem;
     const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
     constexpr uint32_t TM_D1 = 0, TM_U = 64, TM_W = 128;
@@ -475,7 +477,7 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p,
     }
     fence_before_sync();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 7) {
         fence_after_sync();
         tmem_free(tm, 256);
     }

@@ -134,21 +134,23 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *cu, int n_seq
 
 // ------------------------------------------------------------ prep kernel
 
-// 256 threads and ~99 KB of shared memory, so two prep CTAs share an SM and
-// hide each other's latencies.
+// 256 threads, ~73 KB of shared memory and 128 TMEM columns, so three prep
+// CTAs share an SM and hide each other's latencies. Regions are reused as
+// their contents die: V lands where Q was once [KK;QK] is done, and TB, then
+// TW, are staged over A once T is built.
 constexpr int PNT = 256;
 constexpr int PSL = 512 / PNT;      // 16-column slices of a 64-column accumulator per thread
-constexpr uint32_t A_KQ = 0;        // bf16 [K;Q] (32 KB)
-constexpr uint32_t A_V = 32768;     // bf16 V (16 KB)
+constexpr uint32_t A_KQ = 0;        // bf16 [K;Q] tiles (32 KB, kq_sw)
+constexpr uint32_t A_V = A_KQ + 8192;  // bf16 V: its two boxes in Q's, 16 KB apart
 constexpr int PLD = 68;             // row stride of the fp32 scratch (16-byte aligned rows)
-constexpr uint32_t A_T = 49152;     // fp32 T [64][PLD]
-constexpr uint32_t A_AX = 66560;    // fp32 A [64][PLD] and X; once T is built, TB/TW (32 KB) over them
+constexpr uint32_t A_T = 32768;     // fp32 T [64][PLD]
+constexpr uint32_t A_AX = 50176;    // fp32 A [64][PLD] and X; once T is built, TB, then TW (16 KB), over A
 constexpr uint32_t A_TBW = A_AX;
-constexpr uint32_t A_GB = 99328;    // g[64], beta[64]
-constexpr uint32_t A_SCAL = 99840;  // scalars, mbarrier
+constexpr uint32_t A_GB = 70656;    // g[64], beta[64]
+constexpr uint32_t A_SCAL = 71168;  // scalars, mbarriers
 constexpr uint32_t A_SMEM = A_SCAL + 3072;
 constexpr uint32_t A_SMEM_LAUNCH = A_SMEM + 1024;  // with the alignment slack
-static_assert(2 * (A_SMEM_LAUNCH + 1024) <= 228 * 1024, "two prep blocks must share an SM");
+static_assert(3 * (A_SMEM_LAUNCH + 1024) <= 228 * 1024, "three prep blocks must share an SM");
 
 struct PrepScalars {
     float gam[C], eg[C], bet[C], nk[C], nq[C], dec[C];
@@ -157,11 +159,14 @@ struct PrepScalars {
     // diagonal 16-block as a product of two factors that are at most one.
     float dtab[4 * C];
     uint64_t bar;
-    uint64_t tbar;  // the K, Q, V tiles landed (tensor-copy path)
+    uint64_t tbar;  // the K and Q tiles landed
+    uint64_t vbar;  // the V tile landed
     uint32_t tmem;
 };
 static_assert(sizeof(PrepScalars) <= A_SMEM - A_SCAL, "prep scalars overflow");
-static_assert(A_T + C * PLD * 4 <= A_AX && A_AX + 32768 <= A_GB, "prep scratch overlap");
+static_assert(A_T + C * PLD * 4 <= A_AX && A_AX + C * PLD * 4 + 3 * 1024 <= A_GB &&
+                  16384 <= C * PLD * 4,
+              "prep scratch overlap");
 
 // Tensor maps of the packed q, k and v (rows = tokens; boxes of 64 elements x
 // 64 tokens, 128-byte swizzle) for the prep kernel's tensor copies.
@@ -198,7 +203,7 @@ __device__ __forceinline__ PrepUnit prep_unit(const int *seg_off, int seg_lo, in
 // exiting, so that this grid completes only after it (the next recurrence
 // segment, queued after this grid, reads the state it carries).
 // K, Q and V come by tensor copies (maps) into 128-byte-swizzled tiles.
-__global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p,
+__global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
                                                      const __grid_constant__ PrepMaps maps,
                                                      const int *chunk_off,
                                                      const int *seg_off, int seg_lo,
@@ -229,20 +234,20 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p,
 
     // Thread 0 starts the tile copies first; warp 7 (idle until the first
     // product) takes the TMEM columns and, later, warms L2 for the successor.
-    if (warp == 7) tmem_alloc(&sc.tmem, 256);
+    if (warp == 7) tmem_alloc(&sc.tmem, 128);
     if (tid == 0) {
         mbar_init(&sc.bar, 1);
         mbar_init(&sc.tbar, 1);
+        mbar_init(&sc.vbar, 1);
         mbar_fence_init();
-        // Six boxes of 64 tokens x 64 values: K and Q (each d half), V.
-        // Tokens past the sequence belong to the next one (zeroed below) or
-        // lie past the tensor (read as zero).
-        bulk_expect(&sc.tbar, 6 * 8192);
+        // Four boxes of 64 tokens x 64 values: K and Q, each d half (V comes
+        // later). Tokens past the sequence belong to the next one (zeroed
+        // below) or lie past the tensor (read as zero).
+        bulk_expect(&sc.tbar, 4 * 8192);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             tma_load_2d(sbase + A_KQ + h * 16384, &maps.k, hk * D + 64 * h, (int)c0, &sc.tbar);
             tma_load_2d(sbase + A_KQ + h * 16384 + 8192, &maps.q, hk * D + 64 * h, (int)c0, &sc.tbar);
-            tma_load_2d(sbase + A_V + h * 8192, &maps.v, hv * D + 64 * h, (int)c0, &sc.tbar);
         }
     }
     if (tid < 2 * C) {
@@ -260,14 +265,16 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p,
     const bool loads_ok = mbar_wait(&sc.tbar, 0u, kWaitNs);
     // Rows past a ragged chunk's end are zero (the products scale them by zero
     // factors too, but the next sequence's values must not reach them).
-    if (loads_ok && L < C) {
+    // nboxes boxes of 8 KB from `at0`, `stride` apart: rows L..63 to zero.
+    auto zero_tail = [&](uint32_t at0, uint32_t stride, int nboxes) {
         const int nz = (C - L) * 8;
-        for (int e = tid; e < 6 * nz; e += PNT) {
+        for (int e = tid; e < nboxes * nz; e += PNT) {
             const int box = e / nz, r = L + ((e - box * nz) >> 3), ch = e & 7;
-            const uint32_t at = box < 4 ? A_KQ + box * 8192 : A_V + (box - 4) * 8192;
-            *reinterpret_cast<uint4 *>(sm + at + r * 128 + ch * 16) = make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4 *>(sm + at0 + box * stride + r * 128 + ch * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
         }
-    }
+    };
+    if (loads_ok && L < C) zero_tail(A_KQ, 8192, 4);
     fence_before_sync();
     const bool loads_bad = __syncthreads_or(!loads_ok) != 0;
     fence_after_sync();
@@ -286,7 +293,9 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p,
     }
     const uint32_t tm = sc.tmem;
     const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
-    constexpr uint32_t TM_D1 = 0, TM_U = 64, TM_W = 128;
+    // [KK;QK] in columns 0..63 until the A/P epilogue has read it; then U
+    // there and W beside it.
+    constexpr uint32_t TM_D1 = 0, TM_U = 0, TM_W = 64;
 
     // Norms (one row of [K;Q] per thread) and the running sums of g.
     if (tid < 128) {
@@ -339,10 +348,15 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p,
     }
 
     uint32_t phase = 0;
-    auto issue_and_wait = [&](auto issue) -> bool {
+    // `ready`: this thread's operands are in place (all must be, or nothing
+    // is issued).
+    auto issue_and_wait = [&](bool ready, auto issue) -> bool {
         fence_smem_to_async();
         fence_before_sync();
-        __syncthreads();
+        if (__syncthreads_or(!ready)) {
+            if (tid == 0) atomicExch(status, kTimeoutStatus);
+            return false;
+        }
         if (tid == 0) {
             fence_after_sync();
             issue();
@@ -359,7 +373,7 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p,
     const uint32_t ID_U = instr_desc<Kind::BF16>(128, 64, true, false);
     const uint32_t kq = sbase + A_KQ;
 
-    bool alive = !loads_bad && issue_and_wait([&] {
+    bool alive = !loads_bad && issue_and_wait(true, [&] {
         // K-major, 128-byte swizzle: a K step is 32 bytes inside a row, the
         // second half of d 16 KB on.
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -367,6 +381,16 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p,
             mma<Kind::BF16>(tm + TM_D1, dk, dk, ID_KK, kk > 0 ? 1u : 0u);
         }
     });
+    // V into Q's boxes, now that [KK;QK] and the norms are done with them.
+    const bool v_issued = alive;
+    if (v_issued && tid == 0) {
+        fence_smem_to_async();
+        bulk_expect(&sc.vbar, 2 * 8192);
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+            tma_load_2d(sbase + A_V + h * 16384, &maps.v, hv * D + 64 * h, (int)c0, &sc.vbar);
+    }
+    bool v_landed = false;
     if (alive) {
         // A (fp32 scratch) and P (hi/lo bf16 straight into the record).  The
         // decay e^{gamma_r - gamma_s}: zero above the diagonal 16-block, a
@@ -414,40 +438,45 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p,
         }
         __syncthreads();
         invert_unit_lower<PNT, PLD>(Ascr, Tscr, Xscr, tid);
-        for (int e = tid; e < C * (C / 8); e += PNT) {
-            const int r = e & 63, s8 = 8 * (e >> 6);
-            float t[8], tb[8], tw[8];
-            *reinterpret_cast<float4 *>(t) = *reinterpret_cast<const float4 *>(Tscr + r * PLD + s8);
-            *reinterpret_cast<float4 *>(t + 4) = *reinterpret_cast<const float4 *>(Tscr + r * PLD + s8 + 4);
+        // T diag(f) as bf16 hi/lo tiles over A (TB with f = beta, then TW with
+        // f = beta e^gamma n_k), each the B operand of one product.
+        auto stage_t = [&](bool w_side) {
+            for (int e = tid; e < C * (C / 8); e += PNT) {
+                const int r = e & 63, s8 = 8 * (e >> 6);
+                float t[8];
+                *reinterpret_cast<float4 *>(t) = *reinterpret_cast<const float4 *>(Tscr + r * PLD + s8);
+                *reinterpret_cast<float4 *>(t + 4) =
+                    *reinterpret_cast<const float4 *>(Tscr + r * PLD + s8 + 4);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int s = s8 + u;
-                tb[u] = t[u] * sc.bet[s];
-                tw[u] = t[u] * sc.bet[s] * sc.eg[s] * sc.nk[s];
+                for (int u = 0; u < 8; ++u) {
+                    const int s = s8 + u;
+                    t[u] *= w_side ? sc.bet[s] * sc.eg[s] * sc.nk[s] : sc.bet[s];
+                }
+                uint4 h, l;
+                split8(t, h, l);
+                *reinterpret_cast<uint4 *>(sm + A_TBW + kmaj(r, s8, C)) = h;
+                *reinterpret_cast<uint4 *>(sm + A_TBW + 8192 + kmaj(r, s8, C)) = l;
             }
-            uint4 h, l;
-            split8(tb, h, l);
-            *reinterpret_cast<uint4 *>(sm + A_TBW + kmaj(r, s8, C)) = h;
-            *reinterpret_cast<uint4 *>(sm + A_TBW + 8192 + kmaj(r, s8, C)) = l;
-            split8(tw, h, l);
-            *reinterpret_cast<uint4 *>(sm + A_TBW + 16384 + kmaj(r, s8, C)) = h;
-            *reinterpret_cast<uint4 *>(sm + A_TBW + 24576 + kmaj(r, s8, C)) = l;
-        }
-        alive = issue_and_wait([&] {
+        };
+        // A = V or K as MN-major (d across the two 64-value atoms 16 KB apart,
+        // the tokens as K, 16 of them = 2 KB a step); B = the staged hi, lo.
+        auto product = [&](uint32_t d_col, uint32_t a_base) {
             const uint32_t tbw = sbase + A_TBW;
-            // V and K as MN-major A (d across 64-value atoms, the tokens as K,
-            // 16 of them = 2 KB a step); B = T diag(beta) (hi, lo) and the
-            // same scaled for W (hi, lo).
             for (int kk = 0; kk < C / 16; ++kk) {
-                const uint64_t av = smem_desc_sw128(sbase + A_V + kk * 2048, 8192, 1024);
-                const uint64_t ak = smem_desc_sw128(kq + kk * 2048, 16384, 1024);
-                const uint32_t acc = kk > 0 ? 1u : 0u;
-                mma<Kind::BF16>(tm + TM_U, av, smem_desc(tbw + kk * 2048, 1024, 128), ID_U, acc);
-                mma<Kind::BF16>(tm + TM_U, av, smem_desc(tbw + 8192 + kk * 2048, 1024, 128), ID_U, 1u);
-                mma<Kind::BF16>(tm + TM_W, ak, smem_desc(tbw + 16384 + kk * 2048, 1024, 128), ID_U, acc);
-                mma<Kind::BF16>(tm + TM_W, ak, smem_desc(tbw + 24576 + kk * 2048, 1024, 128), ID_U, 1u);
+                const uint64_t a = smem_desc_sw128(a_base + kk * 2048, 16384, 1024);
+                mma<Kind::BF16>(tm + d_col, a, smem_desc(tbw + kk * 2048, 1024, 128), ID_U,
+                                kk > 0 ? 1u : 0u);
+                mma<Kind::BF16>(tm + d_col, a, smem_desc(tbw + 8192 + kk * 2048, 1024, 128), ID_U, 1u);
             }
-        });
+        };
+        stage_t(false);
+        v_landed = mbar_wait(&sc.vbar, 0u, kWaitNs);
+        if (v_landed && L < C) zero_tail(A_V, 16384, 2);
+        alive = issue_and_wait(v_landed, [&] { product(TM_U, sbase + A_V); });
+        if (alive) {
+            stage_t(true);
+            alive = issue_and_wait(true, [&] { product(TM_W, kq); });
+        }
     }
     if (alive) {
         // W^T [j][r] -> bf16 MN-major B tile; U^T [i][s] -> fp32 record; scalars.
@@ -479,10 +508,11 @@ __global__ void __launch_bounds__(PNT, 2) prep_kernel(const PrefillParams p,
     __syncthreads();
     if (warp == 7) {
         fence_after_sync();
-        tmem_free(tm, 256);
+        tmem_free(tm, 128);
     }
     // A tensor copy that did not land in time must not land after the block ends.
     if (loads_bad && tid == 0) mbar_wait(&sc.tbar, 0u, 1000000ull);
+    if (v_issued && !v_landed && tid == 0) mbar_wait(&sc.vbar, 0u, 1000000ull);
     if (wait_prev_at_exit && blockIdx.x == gridDim.x - 1) wait_for_predecessor();
 }
 

@@ -119,8 +119,6 @@ constexpr int TG = 8;  // tokens that share one pass over a weight row
 // each warp streams its row past them once per group: one load per 16-byte
 // chunk of the row, the token values read from shared memory.
 __global__ void __launch_bounds__(256) router_kernel(const MoeParams p) {
-    wait_for_predecessor();
-    release_dependents();
     extern __shared__ uint4 xs[];  // [router_tg][hidden / 8]
     const int lane = threadIdx.x & 31;
     const int e = blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -129,6 +127,17 @@ __global__ void __launch_bounds__(256) router_kernel(const MoeParams p) {
     const uint4 *w = reinterpret_cast<const uint4 *>(
         shared_row ? p.w_sgate : p.w_router + (size_t)min(e, p.n_exp - 1) * p.hidden);
     const int nc = p.hidden / 8;
+    // The row's first RPRE chunks per lane come in before the wait on the
+    // previous kernel (which may write x, never the weights).
+    constexpr int RPRE = 8;
+    uint4 wpre[RPRE];
+#pragma unroll
+    for (int u = 0; u < RPRE; ++u) {
+        const int c = lane + 32 * u;
+        wpre[u] = active && c < nc ? __ldg(w + c) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    wait_for_predecessor();
+    release_dependents();
     for (int t0 = 0; t0 < p.n_tok; t0 += p.router_tg) {
         const int ng = min(p.router_tg, p.n_tok - t0);
         __syncthreads();  // the previous group is done with xs
@@ -141,8 +150,17 @@ __global__ void __launch_bounds__(256) router_kernel(const MoeParams p) {
         float acc[TG];
 #pragma unroll
         for (int t = 0; t < TG; ++t) acc[t] = 0.f;
+#pragma unroll
+        for (int u = 0; u < RPRE; ++u) {
+            const int c = lane + 32 * u;
+            if (c < nc) {
+#pragma unroll
+                for (int t = 0; t < TG; ++t)
+                    if (t < ng) acc[t] = dot8_bf16(wpre[u], xs[t * nc + c], acc[t]);
+            }
+        }
 #pragma unroll 8
-        for (int c = lane; c < nc; c += 32) {
+        for (int c = lane + 32 * RPRE; c < nc; c += 32) {
             const uint4 wv = __ldg(w + c);
 #pragma unroll
             for (int t = 0; t < TG; ++t)
@@ -412,16 +430,18 @@ __global__ void __launch_bounds__(256, 2) gate_up_kernel(const MoeParams p) {
 // ------------------------------------------------------------------- down
 // Block (a, i0): output rows i0 .. i0+31 of active expert a's down matrix;
 // warp w takes rows i0 + 4w .. i0 + 4w + 3.  part[pair] = w_pair * W_down h.
+// The routing (expert list, offsets, pair weights) was complete before the
+// gate/up kernel started, and this grid starts after that: a block reads it,
+// and streams in its expert's weight rows, before it waits for h.
 __global__ void __launch_bounds__(256, 2) down_kernel(const MoeParams p) {
-    wait_for_predecessor();
-    release_dependents();
     const int a = blockIdx.y;
-    if (a >= *p.n_active) return;
-    const int e = p.act_expert[a];
+    // Read at L2 (the buffers are rewritten by every layer's routing).
+    if (a >= __ldcg(p.n_active)) return;
+    const int e = __ldcg(p.act_expert + a);
     const bool sh = e == p.n_exp;
     const int I = sh ? p.s_inter : p.inter;
     const __nv_bfloat16 *W = sh ? p.ws_down : p.w_down + (size_t)e * p.hidden * p.inter;
-    const int p0 = p.act_off[a], p1 = p.act_off[a + 1];
+    const int p0 = __ldcg(p.act_off + a), p1 = __ldcg(p.act_off + a + 1);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int hmax = p.inter > p.s_inter ? p.inter : p.s_inter;
     const int row0 = blockIdx.x * DN_ROWS + 4 * warp;
@@ -452,18 +472,26 @@ __global__ void __launch_bounds__(256, 2) down_kernel(const MoeParams p) {
     };
     if (p1 - p0 == 1) {
         // One pair (every routed expert at small batch): the four rows stream
-        // past once, all of a lane's chunks in flight together.
-        if (!wactive) return;
+        // past once, all of a lane's chunks in flight together, issued before
+        // the wait for h.
         constexpr int MAXC = 4;  // chunks per lane: I <= 1024
-        const float *hp = p.h + (size_t)p0 * hmax;
         uint4 wv[4][MAXC];
+#pragma unroll
+        for (int u = 0; u < MAXC; ++u) {
+            const int c = lane + 32 * u;
+            const bool in = wactive && c < nc;
+#pragma unroll
+            for (int r = 0; r < 4; ++r) wv[r][u] = in ? __ldg(wr[r] + c) : make_uint4(0, 0, 0, 0);
+        }
+        wait_for_predecessor();
+        release_dependents();
+        if (!wactive) return;
+        const float *hp = p.h + (size_t)p0 * hmax;
         float4 h0[MAXC], h1[MAXC];
 #pragma unroll
         for (int u = 0; u < MAXC; ++u) {
             const int c = lane + 32 * u;
             const bool in = c < nc;
-#pragma unroll
-            for (int r = 0; r < 4; ++r) wv[r][u] = in ? __ldg(wr[r] + c) : make_uint4(0, 0, 0, 0);
             h0[u] = in ? *reinterpret_cast<const float4 *>(hp + 8 * c) : make_float4(0.f, 0.f, 0.f, 0.f);
             h1[u] = in ? *reinterpret_cast<const float4 *>(hp + 8 * c + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
@@ -478,6 +506,8 @@ __global__ void __launch_bounds__(256, 2) down_kernel(const MoeParams p) {
     // Several pairs (the shared expert, or a popular one): up to DN_G pairs' h
     // staged in shared memory, and each chunk of the four rows applied to all
     // of them once it is loaded.
+    wait_for_predecessor();
+    release_dependents();
     constexpr int DN_G = 8;
     __shared__ __align__(16) float hs[DN_G][1024];
     for (int g0 = p0; g0 < p1; g0 += DN_G) {

@@ -272,10 +272,11 @@ class DecodeE2E:
 
     Each step is one CUDA graph (how a serving loop replays a decode step
     without paying the Python binding's per-call cost): on a side stream it
-    copies the NEXT step's inputs into the other of two device input buffers,
-    while on the main stream its own 18 library calls read the inputs the
-    previous step copied, then its output is copied back.  So every step moves
-    one step's inputs and outputs, and the copies overlap the kernels."""
+    copies the NEXT step's inputs into the other of two device input buffers
+    and the PREVIOUS step's output back to the host, while on the main stream
+    its own 18 library calls read the inputs the previous step copied and
+    write the other of two device output buffers.  So every step moves one
+    step's inputs and one step's output, and the copies overlap the kernels."""
 
     def __init__(self, bench: DecodeBench, host_slots=16):
         self.b = bench
@@ -291,6 +292,7 @@ class DecodeE2E:
         self.d = [{n: torch.empty_like(t[0], device=dev) for n, t in self.h.items()}
                   for _ in range(2)]
         self.h_out = torch.empty(bench.out.shape, dtype=bench.out.dtype).pin_memory()
+        self.d_out = [torch.empty_like(bench.out) for _ in range(2)]
         self.h2d_bytes = sum(t[0].numel() * t[0].element_size() for t in self.h.values())
         self.d2h_bytes = self.h_out.numel() * self.h_out.element_size()
         import types
@@ -305,11 +307,14 @@ class DecodeE2E:
 
     def _enqueue(self, slot):
         main = torch.cuda.current_stream()
+        # The side stream starts once the previous step's kernels are done: its
+        # inputs buffer may be refilled and its output read back.  (An even
+        # slot count makes a slot's parity its step's.)
         self.side.wait_stream(main)
         with torch.cuda.stream(self.side):
             self._copy_in((slot + 1) % self.host_slots)
-        self.b.launch_step(0, x=self.view[slot % 2])
-        self.h_out.copy_(self.b.out, non_blocking=True)
+            self.h_out.copy_(self.d_out[(slot + 1) % 2], non_blocking=True)
+        self.b.launch_step(0, x=self.view[slot % 2], out=self.d_out[slot % 2])
         main.wait_stream(self.side)
 
     def capture(self):
@@ -477,7 +482,7 @@ def prefill_measure(device, lens=None, H_k=P_H, H_v=P_H, seed=2, g_mode="softplu
             "roofline": {"bound": "tensor", "achieved": per_gpu_tflops,
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": per_gpu_tflops / peaks["bf16_tflops"], "traffic": None,
-                         "peak_source": peaks["source"] + " (bf16_tflops, burst)"},
+                         "peak_source": peaks["source"] + " bf16 GEMM, burst (bf16_tflops)"},
             "l2": "flushed (256 MB write) before each repetition", "reps": reps}
 
 
@@ -563,7 +568,7 @@ def attn_decode_measure(device, steps=16, warmup=4, world=1, layers=ATT_LAYERS):
                         "traffic": captured_traffic("attend_kernel"), "kernel": "attend_kernel",
                         "bytes_per_layer": per_layer,
                         "us_per_layer": ms * 1e3 / (steps * L),
-                        "peak_source": peaks["source"] + " (hbm_gbs, of measured copy bandwidth)"}}
+                        "peak_source": peaks["source"] + " copy bandwidth (hbm_gbs)"}}
     del graph, q, gate, k, v, kc, vc, out, ws
     torch.cuda.empty_cache()
     return res
@@ -644,7 +649,7 @@ def moe_decode_measure(device, B=1, steps=32, warmup=4, world=1, slots=16, layer
                      "combine)",
            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                        "peak_source": peaks["source"] + " (hbm_gbs, of measured copy bandwidth)"}}
+                        "peak_source": peaks["source"] + " copy bandwidth (hbm_gbs)"}}
     del graphs, layers, x, out, ws
     torch.cuda.empty_cache()
     return res
@@ -674,7 +679,7 @@ def gva_decode_measure(device, steps=32, warmup=4, world=1):
                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
                         "bytes_per_launch": b.bytes_per_launch,
                         "us_per_launch": per_launch_ms * 1e3,
-                        "peak_source": peaks["source"] + " (hbm_gbs, of measured copy bandwidth)"}}
+                        "peak_source": peaks["source"] + " copy bandwidth (hbm_gbs)"}}
     del b
     torch.cuda.empty_cache()
     return res
@@ -891,13 +896,14 @@ def main():
                      "traffic": captured_traffic("decode_rb_kernel<bf16, bf16>"),
                      "kernel": "decode_rb_kernel<bf16, bf16>",
                      "bytes_per_launch": per_launch_bytes, "us_per_launch": per_launch_ms * 1e3,
-                     "peak_source": peaks["source"] + " (hbm_gbs, of measured copy bandwidth)"},
+                     "peak_source": peaks["source"] + " copy bandwidth (hbm_gbs)"},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": h2d_bytes,
                 "d2h_bytes_per_step": d2h_bytes, "steps": args.e2e_steps,
                 "launch": "one CUDA graph per step: the 18 library calls on inputs the previous "
-                          "step copied from pinned host memory, the next step's inputs copied "
-                          "in meanwhile, the outputs copied back",
+                          "step copied from pinned host memory, while a side stream copies the "
+                          "next step's inputs in and the previous step's outputs back (two "
+                          "device output buffers)",
                 "ms_per_step": ms_e2e / args.e2e_steps},
         "gpu_launches": args.steps * launches_per_step,
         "clocks": clock_info,

@@ -152,12 +152,13 @@ constexpr uint32_t A_SMEM = A_SCAL + 3072;
 constexpr uint32_t A_SMEM_LAUNCH = A_SMEM + 1024;  // with the alignment slack
 static_assert(3 * (A_SMEM_LAUNCH + 1024) <= 228 * 1024, "three prep blocks must share an SM");
 
+constexpr int DTL = C + 4;  // row stride of dtab
 struct PrepScalars {
     float gam[C], eg[C], bet[C], nk[C], nq[C], dec[C];
     // dtab[R][s] = e^{gamma_{16R} - gamma_s} for s < 16R: with the per-row
     // e^{gamma_r - gamma_{16R}} it gives e^{gamma_r - gamma_s} below the
     // diagonal 16-block as a product of two factors that are at most one.
-    float dtab[4 * C];
+    float dtab[4 * DTL];  // rows DTL apart: a warp's two rows sit in different banks
     uint64_t bar;
     uint64_t tbar;  // the K and Q tiles landed
     uint64_t vbar;  // the V tile landed
@@ -344,7 +345,7 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
     if (tid < C) sc.dec[tid] = __expf(sc.gam[L - 1] - sc.gam[tid]);
     {
         const int R = tid >> 6, s = tid & 63;  // PNT == 4 * C entries
-        sc.dtab[tid] = s < 16 * R ? __expf(sc.gam[16 * R] - sc.gam[s]) : 0.f;
+        sc.dtab[R * DTL + s] = s < 16 * R ? __expf(sc.gam[16 * R] - sc.gam[s]) : 0.f;
     }
 
     uint32_t phase = 0;
@@ -405,7 +406,7 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
         tmem_ld16(tm + lane_off + TM_D1 + s0, v);
         if (Sb < R) {
 #pragma unroll
-            for (int c = 0; c < 16; ++c) e[c] = rowf * sc.dtab[R * C + s0 + c];
+            for (int c = 0; c < 16; ++c) e[c] = rowf * sc.dtab[R * DTL + s0 + c];
         } else if (Sb == R) {
 #pragma unroll
             for (int c = 0; c < 16; ++c) e[c] = __expf(gr - sc.gam[s0 + c]);
@@ -414,12 +415,18 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
             for (int c = 0; c < 16; ++c) e[c] = 0.f;
         }
         if (quad < 2) {
+            // 16-byte stores: with rows PLD floats apart, a quarter-warp's eight
+            // rows cover all 32 banks once.
             const float f = sc.bet[rr] * sc.nk[rr];
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
                 const int s = s0 + c;
-                Ascr[rr * PLD + s] = s < rr ? f * e[c] * sc.nk[s] * v[c] : 0.f;
+                v[c] = s < rr ? f * e[c] * sc.nk[s] * v[c] : 0.f;
             }
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4)
+                *reinterpret_cast<float4 *>(Ascr + rr * PLD + s0 + 4 * c4) =
+                    make_float4(v[4 * c4], v[4 * c4 + 1], v[4 * c4 + 2], v[4 * c4 + 3]);
         } else {
             const float f = sc.nq[rr];
 #pragma unroll

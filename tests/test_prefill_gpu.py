@@ -137,6 +137,25 @@ def test_tc_ragged_varlen(lens, heads):
     _check(inp, out, final, torch.bfloat16)
 
 
+@pytest.mark.parametrize("lens", [[100, 64], [36, 300], [200, 1], [800, 50]])
+def test_tc_ragged_tail_never_reads_the_next_sequence(lens):
+    """A sequence's ragged last chunk is loaded as whole 64-token boxes, which reach into the
+    next sequence's rows: with every q, k and v value of the second sequence NaN, the first
+    sequence's outputs and final states are finite and match the oracle (its own inputs
+    only). [800, 50] runs as three segments."""
+    inp = synth.make_inputs(lens, 2, 4, 128, seed=77 + sum(lens), dtype=torch.bfloat16,
+                            s0_std=0.02)
+    t1 = inp.cu_seqlens[1]
+    for name in ("q", "k", "v"):
+        getattr(inp, name)[t1:] = float("nan")
+    out, final = run_prefill(inp, chunk=64)
+    ref = oracle_sequence(inp, 0)
+    o, fs = f64(out[:t1]), f64(final[0:1])
+    # (assert_close also requires every value finite)
+    assert_close(o, ref.y, 2e-3, what="outputs of the first sequence")
+    assert_close(fs, ref.state, 1e-3, what="final states of the first sequence")
+
+
 @pytest.mark.parametrize("scale", [1.0, 128 ** -0.5])
 def test_tc_scale_gate_and_outputs(scale):
     inp = synth.make_inputs([150, 90], 2, 2, 128, seed=31, dtype=torch.bfloat16, s0_std=0.02)

@@ -7,7 +7,8 @@
 // rule named in the Qwen3.5 Chat guide, section "Architektur").  So:
 //
 //   prep kernel:  one CTA per (chunk, value head), every chunk at once, over
-//                 the whole GPU.  Writes, per unit, a 65 KB record to the
+//                 the whole GPU (three CTAs per SM; K, Q and V by tensor
+//                 copies).  Writes, per unit, a 65 KB record to the
 //                 workspace: W (bf16, already in the MMA operand layout),
 //                 P (hi + lo bf16), U (fp32) and the per-token scalars.
 //   recur kernel: one CTA per (sequence, value head), chunks in order, only
@@ -539,11 +540,11 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
 //   warps 8-15  output group, one chunk behind: S Q^T and P Delta out of
 //               double-buffered TMEM, staged through shared memory so that
 //               one warp normalises, gates and stores whole tokens;
-//   warp 16     producer: K and Q tiles (cp.async with zero fill past the
-//               sequence end, counted on an mbarrier), and by bulk copy each
-//               chunk's W, P, U and scalars, every one into its stage as soon
-//               as the previous chunk is done with it (the record is first
-//               prefetched into L2 a chunk ahead);
+//   warp 16     producer: K and Q tiles by tensor copies (a sequence's
+//               ragged last chunk by 16-byte copies that read zero past its
+//               end), and by bulk copy each chunk's W, P, U and scalars, every
+//               one into its stage as soon as the previous chunk is done with
+//               it (the record is first prefetched into L2 a chunk ahead);
 //   warp 17     MMA issue, state path first (-S W^T before S Q^T, the state
 //               update before P Delta), each group committed on its own
 //               barrier so the state group never waits for output products.

@@ -55,7 +55,6 @@ struct MoeParams {
 namespace moe {
 
 constexpr int GU_ROWS = 16;   // intermediate rows per gate_up block (x 2: gate and up)
-constexpr int DN_ROWS = 32;   // output rows per down block
 constexpr int ROUTE_THREADS = 1024;  // also the most experts (one thread each in the scans)
 
 // Dot products of ROWS bf16 rows with one bf16 vector x of n values (n a
@@ -428,12 +427,15 @@ __global__ void __launch_bounds__(256, 2) gate_up_kernel(const MoeParams p) {
 }
 
 // ------------------------------------------------------------------- down
-// Block (a, i0): output rows i0 .. i0+31 of active expert a's down matrix;
-// warp w takes rows i0 + 4w .. i0 + 4w + 3.  part[pair] = w_pair * W_down h.
-// The routing (expert list, offsets, pair weights) was complete before the
-// gate/up kernel started, and this grid starts after that: a block reads it,
-// and streams in its expert's weight rows, before it waits for h.
+// Block (a, i0): output rows i0 .. i0 + 8 RPW - 1 of active expert a's down
+// matrix; warp w takes RPW rows from i0 + RPW w.  part[pair] = w_pair * W_down h.
+// MAXC: 16-byte chunks of a row per lane (I <= 256 MAXC).  The routing (expert
+// list, offsets, pair weights) was complete before the gate/up kernel started,
+// and this grid starts after that: a block reads it, and streams in its
+// expert's weight rows, before it waits for h.
+template <int RPW, int MAXC>
 __global__ void __launch_bounds__(256, 2) down_kernel(const MoeParams p) {
+    static_assert(RPW % 4 == 0, "rows per warp in groups of four");
     const int a = blockIdx.y;
     // Read at L2 (the buffers are rewritten by every layer's routing).
     if (a >= __ldcg(p.n_active)) return;
@@ -444,13 +446,12 @@ __global__ void __launch_bounds__(256, 2) down_kernel(const MoeParams p) {
     const int p0 = __ldcg(p.act_off + a), p1 = __ldcg(p.act_off + a + 1);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int hmax = p.inter > p.s_inter ? p.inter : p.s_inter;
-    const int row0 = blockIdx.x * DN_ROWS + 4 * warp;
+    const int row0 = blockIdx.x * (8 * RPW) + RPW * warp;
     const bool wactive = row0 < p.hidden;
     const int nc = I / 8;
-    const uint4 *wr[4];
-#pragma unroll
-    for (int r = 0; r < 4; ++r)
-        wr[r] = reinterpret_cast<const uint4 *>(W + (size_t)min(row0 + r, p.hidden - 1) * I);
+    auto wrow = [&](int r) {
+        return reinterpret_cast<const uint4 *>(W + (size_t)min(row0 + r, p.hidden - 1) * I);
+    };
     // 8 weights (one 16-byte chunk) against 8 fp32 values of h.
     auto dot8_h = [](const uint4 &w, const float4 &h0, const float4 &h1, float acc) {
         const __nv_bfloat162 *w2 = reinterpret_cast<const __nv_bfloat162 *>(&w);
@@ -462,26 +463,27 @@ __global__ void __launch_bounds__(256, 2) down_kernel(const MoeParams p) {
         }
         return acc;
     };
-    auto store = [&](int i, const float (&acc)[4]) {
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const float a = group_sum<32>(acc[r]);
-            if (lane == 0 && row0 + r < p.hidden)
-                p.part[(size_t)i * p.hidden + row0 + r] = p.pair_w[i] * a;
+    // Rows row0 + rb .. row0 + rb + N - 1 of pair i.
+    auto store = [&](int i, const float *acc, int rb, int N) {
+        for (int r = 0; r < N; ++r) {
+            const float v = group_sum<32>(acc[r]);
+            if (lane == 0 && row0 + rb + r < p.hidden)
+                p.part[(size_t)i * p.hidden + row0 + rb + r] = p.pair_w[i] * v;
         }
     };
     if (p1 - p0 == 1) {
-        // One pair (every routed expert at small batch): the four rows stream
+        // One pair (every routed expert at small batch): the warp's rows stream
         // past once, all of a lane's chunks in flight together, issued before
         // the wait for h.
-        constexpr int MAXC = 4;  // chunks per lane: I <= 1024
-        uint4 wv[4][MAXC];
+        uint4 wv[RPW][MAXC];
 #pragma unroll
-        for (int u = 0; u < MAXC; ++u) {
-            const int c = lane + 32 * u;
-            const bool in = wactive && c < nc;
+        for (int r = 0; r < RPW; ++r) {
+            const uint4 *wr = wrow(r);
 #pragma unroll
-            for (int r = 0; r < 4; ++r) wv[r][u] = in ? __ldg(wr[r] + c) : make_uint4(0, 0, 0, 0);
+            for (int u = 0; u < MAXC; ++u) {
+                const int c = lane + 32 * u;
+                wv[r][u] = wactive && c < nc ? __ldg(wr + c) : make_uint4(0, 0, 0, 0);
+            }
         }
         wait_for_predecessor();
         release_dependents();
@@ -495,17 +497,19 @@ __global__ void __launch_bounds__(256, 2) down_kernel(const MoeParams p) {
             h0[u] = in ? *reinterpret_cast<const float4 *>(hp + 8 * c) : make_float4(0.f, 0.f, 0.f, 0.f);
             h1[u] = in ? *reinterpret_cast<const float4 *>(hp + 8 * c + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        float acc[RPW];
+#pragma unroll
+        for (int r = 0; r < RPW; ++r) acc[r] = 0.f;
 #pragma unroll
         for (int u = 0; u < MAXC; ++u)
 #pragma unroll
-            for (int r = 0; r < 4; ++r) acc[r] = dot8_h(wv[r][u], h0[u], h1[u], acc[r]);
-        store(p0, acc);
+            for (int r = 0; r < RPW; ++r) acc[r] = dot8_h(wv[r][u], h0[u], h1[u], acc[r]);
+        store(p0, acc, 0, RPW);
         return;
     }
     // Several pairs (the shared expert, or a popular one): up to DN_G pairs' h
-    // staged in shared memory, and each chunk of the four rows applied to all
-    // of them once it is loaded.
+    // staged in shared memory, and each chunk of four rows applied to all of
+    // them once it is loaded (the warp's rows four at a time).
     wait_for_predecessor();
     release_dependents();
     constexpr int DN_G = 8;
@@ -520,27 +524,32 @@ __global__ void __launch_bounds__(256, 2) down_kernel(const MoeParams p) {
         }
         __syncthreads();
         if (!wactive) continue;
-        float acc[DN_G][4];
+        for (int rb = 0; rb < RPW && row0 + rb < p.hidden; rb += 4) {
+            const uint4 *wr[4];
 #pragma unroll
-        for (int t = 0; t < DN_G; ++t)
+            for (int r = 0; r < 4; ++r) wr[r] = wrow(rb + r);
+            float acc[DN_G][4];
 #pragma unroll
-            for (int r = 0; r < 4; ++r) acc[t][r] = 0.f;
-        for (int c = lane; c < nc; c += 32) {
-            uint4 wv[4];
+            for (int t = 0; t < DN_G; ++t)
 #pragma unroll
-            for (int r = 0; r < 4; ++r) wv[r] = __ldg(wr[r] + c);
+                for (int r = 0; r < 4; ++r) acc[t][r] = 0.f;
+            for (int c = lane; c < nc; c += 32) {
+                uint4 wv[4];
 #pragma unroll
-            for (int t = 0; t < DN_G; ++t) {  // rows past ng repeat the last pair (unused)
-                const float *hp = hs[min(t, ng - 1)];
-                const float4 a = *reinterpret_cast<const float4 *>(hp + 8 * c);
-                const float4 b = *reinterpret_cast<const float4 *>(hp + 8 * c + 4);
+                for (int r = 0; r < 4; ++r) wv[r] = __ldg(wr[r] + c);
 #pragma unroll
-                for (int r = 0; r < 4; ++r) acc[t][r] = dot8_h(wv[r], a, b, acc[t][r]);
+                for (int t = 0; t < DN_G; ++t) {  // rows past ng repeat the last pair (unused)
+                    const float *hp = hs[min(t, ng - 1)];
+                    const float4 a = *reinterpret_cast<const float4 *>(hp + 8 * c);
+                    const float4 b = *reinterpret_cast<const float4 *>(hp + 8 * c + 4);
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) acc[t][r] = dot8_h(wv[r], a, b, acc[t][r]);
+                }
             }
-        }
 #pragma unroll
-        for (int t = 0; t < DN_G; ++t)
-            if (t < ng) store(g0 + t, acc[t]);
+            for (int t = 0; t < DN_G; ++t)
+                if (t < ng) store(g0 + t, acc[t], rb, 4);
+        }
     }
 }
 
@@ -671,9 +680,13 @@ cudaError_t launch_moe_args(const gdr_moe_args *a, void *workspace, cudaStream_t
     if ((e = launch(moe::gate_up_kernel, dim3((imax + moe::GU_ROWS - 1) / moe::GU_ROWS, max_active),
                     256, 0)) != cudaSuccess)
         return e;
-    if ((e = launch(moe::down_kernel, dim3((p.hidden + moe::DN_ROWS - 1) / moe::DN_ROWS, max_active),
-                    256, 0)) != cudaSuccess)
-        return e;
+    // Eight rows per warp while a row fits in two chunks per lane (I <= 512):
+    // twice the bytes in flight per block, half the blocks.
+    if (imax <= 512)
+        e = launch(moe::down_kernel<8, 2>, dim3((p.hidden + 63) / 64, max_active), 256, 0);
+    else
+        e = launch(moe::down_kernel<4, 4>, dim3((p.hidden + 31) / 32, max_active), 256, 0);
+    if (e != cudaSuccess) return e;
     const dim3 cgrid(p.n_tok, (p.hidden + 255) / 256);
     if (a->out_dtype == GDR_BF16)
         e = launch(moe::combine_kernel<__nv_bfloat16>, cgrid, 256, 0);

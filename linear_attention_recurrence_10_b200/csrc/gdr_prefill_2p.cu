@@ -29,18 +29,13 @@ namespace tcp2 {
 using namespace gdr::tcp;
 
 
-// Per-(chunk, value head) record in the workspace.
-// The first REC_STAGED bytes (W, P, scalars) are staged in shared memory by the
-// recurrence; U is read from here straight into registers.
+// Per-(chunk, value head) record in the workspace, staged in shared memory by
+// the recurrence by bulk copies.
 constexpr uint32_t REC_W = 0;        // bf16 W, MN-major B tile (w_off), 16 KB
 constexpr uint32_t REC_P = 16384;    // P hi, then lo, K-major [r][s] (kmaj R=64), 8 KB each
 constexpr uint32_t REC_SCAL = 32768; // fp32 eg[64] | nqe[64] | dn[64] | eL | pad
-constexpr uint32_t REC_STAGED = 33792;
-constexpr uint32_t REC_U = 33792;    // fp32 U: byte (s/4)*2048 + i*16 + (s%4)*4, 32 KB
-constexpr uint32_t REC_BYTES = 66560;
-__host__ __device__ constexpr uint32_t u_off(int s, int i) {
-    return (uint32_t)((s >> 2) * 2048 + i * 16 + (s & 3) * 4);
-}
+constexpr uint32_t REC_TB = 33792;   // T diag(beta) hi, then lo, K-major [s][r] (kmaj R=64), 8 KB each
+constexpr uint32_t REC_BYTES = 50176;
 
 // The prefill may run as up to MAX_SEG segments of chunk indices [lo_k, lo_k+1)
 // of every sequence, so that the prep of segment k+1 overlaps the recurrence
@@ -136,16 +131,14 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *cu, int n_seq
 // ------------------------------------------------------------ prep kernel
 
 // 256 threads, ~73 KB of shared memory and 128 TMEM columns, so three prep
-// CTAs share an SM and hide each other's latencies. Regions are reused as
-// their contents die: V lands where Q was once [KK;QK] is done, and TB, then
-// TW, are staged over A once T is built.
+// CTAs share an SM and hide each other's latencies. TW is staged over A once
+// T is built (TB goes straight into the record).
 constexpr int PNT = 256;
 constexpr int PSL = 512 / PNT;      // 16-column slices of a 64-column accumulator per thread
 constexpr uint32_t A_KQ = 0;        // bf16 [K;Q] tiles (32 KB, kq_sw)
-constexpr uint32_t A_V = A_KQ + 8192;  // bf16 V: its two boxes in Q's, 16 KB apart
 constexpr int PLD = 68;             // row stride of the fp32 scratch (16-byte aligned rows)
 constexpr uint32_t A_T = 32768;     // fp32 T [64][PLD]
-constexpr uint32_t A_AX = 50176;    // fp32 A [64][PLD] and X; once T is built, TB, then TW (16 KB), over A
+constexpr uint32_t A_AX = 50176;    // fp32 A [64][PLD] and X; once T is built, TW (16 KB) over A
 constexpr uint32_t A_TBW = A_AX;
 constexpr uint32_t A_GB = 70656;    // g[64], beta[64]
 constexpr uint32_t A_SCAL = 71168;  // scalars, mbarriers
@@ -162,7 +155,6 @@ struct PrepScalars {
     float dtab[4 * DTL];  // rows DTL apart: a warp's two rows sit in different banks
     uint64_t bar;
     uint64_t tbar;  // the K and Q tiles landed
-    uint64_t vbar;  // the V tile landed
     uint32_t tmem;
 };
 static_assert(sizeof(PrepScalars) <= A_SMEM - A_SCAL, "prep scalars overflow");
@@ -240,11 +232,10 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
     if (tid == 0) {
         mbar_init(&sc.bar, 1);
         mbar_init(&sc.tbar, 1);
-        mbar_init(&sc.vbar, 1);
         mbar_fence_init();
-        // Four boxes of 64 tokens x 64 values: K and Q, each d half (V comes
-        // later). Tokens past the sequence belong to the next one (zeroed
-        // below) or lie past the tensor (read as zero).
+        // Four boxes of 64 tokens x 64 values: K and Q, each d half. Tokens
+        // past the sequence belong to the next one (zeroed below) or lie past
+        // the tensor (read as zero).
         bulk_expect(&sc.tbar, 4 * 8192);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -290,14 +281,12 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
         for (int h = 0; h < 2; ++h) {
             tma_prefetch_2d(&maps.k, hk2 * D + 64 * h, n0);
             tma_prefetch_2d(&maps.q, hk2 * D + 64 * h, n0);
-            tma_prefetch_2d(&maps.v, hv2 * D + 64 * h, n0);
         }
     }
     const uint32_t tm = sc.tmem;
     const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
-    // [KK;QK] in columns 0..63 until the A/P epilogue has read it; then U
-    // there and W beside it.
-    constexpr uint32_t TM_D1 = 0, TM_U = 0, TM_W = 64;
+    // [KK;QK] in columns 0..63, W^T beside it.
+    constexpr uint32_t TM_D1 = 0, TM_W = 64;
 
     // Norms (one row of [K;Q] per thread) and the running sums of g.
     if (tid < 128) {
@@ -383,16 +372,6 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
             mma<Kind::BF16>(tm + TM_D1, dk, dk, ID_KK, kk > 0 ? 1u : 0u);
         }
     });
-    // V into Q's boxes, now that [KK;QK] and the norms are done with them.
-    const bool v_issued = alive;
-    if (v_issued && tid == 0) {
-        fence_smem_to_async();
-        bulk_expect(&sc.vbar, 2 * 8192);
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-            tma_load_2d(sbase + A_V + h * 16384, &maps.v, hv * D + 64 * h, (int)c0, &sc.vbar);
-    }
-    bool v_landed = false;
     if (alive) {
         // A (fp32 scratch) and P (hi/lo bf16 straight into the record).  The
         // decay e^{gamma_r - gamma_s}: zero above the diagonal 16-block, a
@@ -446,9 +425,10 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
         }
         __syncthreads();
         invert_unit_lower<PNT, PLD>(Ascr, Tscr, Xscr, tid);
-        // T diag(f) as bf16 hi/lo tiles over A (TB with f = beta, then TW with
-        // f = beta e^gamma n_k), each the B operand of one product.
-        auto stage_t = [&](bool w_side) {
+        // T diag(f) as bf16 hi/lo tiles at dst: TB (f = beta) into the record,
+        // the B operand of the recurrence's U product; TW (f = beta e^gamma
+        // n_k) over A, the B operand of W's.
+        auto stage_t = [&](bool w_side, unsigned char *dst) {
             for (int e = tid; e < C * (C / 8); e += PNT) {
                 const int r = e & 63, s8 = 8 * (e >> 6);
                 float t[8];
@@ -462,46 +442,35 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
                 }
                 uint4 h, l;
                 split8(t, h, l);
-                *reinterpret_cast<uint4 *>(sm + A_TBW + kmaj(r, s8, C)) = h;
-                *reinterpret_cast<uint4 *>(sm + A_TBW + 8192 + kmaj(r, s8, C)) = l;
+                *reinterpret_cast<uint4 *>(dst + kmaj(r, s8, C)) = h;
+                *reinterpret_cast<uint4 *>(dst + 8192 + kmaj(r, s8, C)) = l;
             }
         };
-        // A = V or K as MN-major (d across the two 64-value atoms 16 KB apart,
-        // the tokens as K, 16 of them = 2 KB a step); B = the staged hi, lo.
-        auto product = [&](uint32_t d_col, uint32_t a_base) {
+        stage_t(false, rec + REC_TB);
+        stage_t(true, sm + A_TBW);
+        // W^T = K^T TW^T: K as MN-major A (d across the two 64-value atoms 16 KB
+        // apart, the tokens as K, 16 of them = 2 KB a step); B = TW hi, lo.
+        alive = issue_and_wait(true, [&] {
             const uint32_t tbw = sbase + A_TBW;
             for (int kk = 0; kk < C / 16; ++kk) {
-                const uint64_t a = smem_desc_sw128(a_base + kk * 2048, 16384, 1024);
-                mma<Kind::BF16>(tm + d_col, a, smem_desc(tbw + kk * 2048, 1024, 128), ID_U,
+                const uint64_t a = smem_desc_sw128(kq + kk * 2048, 16384, 1024);
+                mma<Kind::BF16>(tm + TM_W, a, smem_desc(tbw + kk * 2048, 1024, 128), ID_U,
                                 kk > 0 ? 1u : 0u);
-                mma<Kind::BF16>(tm + d_col, a, smem_desc(tbw + 8192 + kk * 2048, 1024, 128), ID_U, 1u);
+                mma<Kind::BF16>(tm + TM_W, a, smem_desc(tbw + 8192 + kk * 2048, 1024, 128), ID_U, 1u);
             }
-        };
-        stage_t(false);
-        v_landed = mbar_wait(&sc.vbar, 0u, kWaitNs);
-        if (v_landed && L < C) zero_tail(A_V, 16384, 2);
-        alive = issue_and_wait(v_landed, [&] { product(TM_U, sbase + A_V); });
-        if (alive) {
-            stage_t(true);
-            alive = issue_and_wait(true, [&] { product(TM_W, kq); });
-        }
+        });
     }
     if (alive) {
-        // W^T [j][r] -> bf16 MN-major B tile; U^T [i][s] -> fp32 record; scalars.
-        const int x = 32 * quad + lane;  // j for W, i for U
+        // W^T [j][r] -> bf16 MN-major B tile; scalars.
+        const int x = 32 * quad + lane;  // j
 #pragma unroll
         for (int sl = 0; sl < PSL; ++sl) {
         const int c0l = 16 * (part * PSL + sl);
-        float w[16], u[16];
+        float w[16];
         tmem_ld16(tm + lane_off + TM_W + c0l, w);
-        tmem_ld16(tm + lane_off + TM_U + c0l, u);
 #pragma unroll
         for (int r8 = 0; r8 < 2; ++r8)
             *reinterpret_cast<uint4 *>(rec + REC_W + w_off(x, c0l + 8 * r8)) = pack8(w + 8 * r8);
-#pragma unroll
-        for (int s4 = 0; s4 < 4; ++s4)
-            *reinterpret_cast<float4 *>(rec + REC_U + u_off(c0l + 4 * s4, x)) =
-                make_float4(u[4 * s4], u[4 * s4 + 1], u[4 * s4 + 2], u[4 * s4 + 3]);
         }
         float *scal = reinterpret_cast<float *>(rec + REC_SCAL);
         if (tid < C) {
@@ -520,7 +489,6 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
     }
     // A tensor copy that did not land in time must not land after the block ends.
     if (loads_bad && tid == 0) mbar_wait(&sc.tbar, 0u, 1000000ull);
-    if (v_issued && !v_landed && tid == 0) mbar_wait(&sc.vbar, 0u, 1000000ull);
     if (wait_prev_at_exit && blockIdx.x == gridDim.x - 1) wait_for_predecessor();
 }
 
@@ -556,15 +524,16 @@ constexpr uint32_t B_W = 32768;                // bf16 W of the current chunk (1
 constexpr uint32_t B_P = 49152;                // bf16 P hi/lo of the current chunk (16 KB)
 constexpr uint32_t B_SC = 65536;               // 2 x scalars (eg, nqe, dn, eL: 1 KB each)
 constexpr uint32_t B_DL = 67584;               // Delta hi/lo (32 KB)
-constexpr uint32_t B_U = 133120;               // fp32 U of the current chunk (32 KB, record layout)
+constexpr uint32_t B_V = 133120;               // bf16 V of the current chunk (16 KB, two 128-byte-swizzled boxes)
+constexpr uint32_t B_TB = 149504;              // T diag(beta) hi/lo of the current chunk (16 KB, record layout)
 constexpr uint32_t B_OS = 165888;              // fp32 O [r][i] of the chunk being output (32 KB)
 constexpr uint32_t B_BAR = 198656;             // 18 mbarriers, then the TMEM address
 constexpr uint32_t B_SMEM = B_BAR + 160;
 constexpr uint32_t B_SMEM_LAUNCH = B_SMEM + 1024;  // with the alignment slack
-constexpr uint32_t SC_BYTES = REC_STAGED - REC_SCAL;
-// TMEM columns: the fp32 state, -S W^T, two buffers of S Q^T, one of P Delta,
-// and the bf16 copy of S (two values per column) that -S W^T and S Q^T read
-// as their A operand.
+constexpr uint32_t SC_BYTES = REC_TB - REC_SCAL;
+// TMEM columns: the fp32 state, Delta^T = U^T - S W^T (the U product first,
+// then -S W^T onto it), two buffers of S Q^T, one of P Delta, and the bf16 copy
+// of S (two values per column) that -S W^T and S Q^T read as their A operand.
 constexpr uint32_t TM_S = 0, TM_D = 128, TM_OI = 192, TM_O2 = 320, TM_SB = 384;
 // ... and the decayed Delta^T tiles (hi, lo; two values per column), the A
 // operand of the state update.
@@ -597,7 +566,7 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p,
     uint64_t *bar_w = bars + 2;                  // W landed
     uint64_t *bar_p = bars + 3;                  // P landed
     uint64_t *bar_sc = bars + 4;                 // [2] scalars landed
-    uint64_t *bar_u = bars + 6;                  // U landed
+    uint64_t *bar_u = bars + 6;                  // V and T diag(beta) landed
     uint64_t *bar_gd = bars + 7;                 // -S W^T done (W may be refilled)
     uint64_t *bar_qfree = bars + 8;              // S Q^T done (Q may be refilled)
     uint64_t *bar_gs = bars + 9;                 // state update done (K may be refilled)
@@ -670,7 +639,25 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p,
             const uint32_t ID_D = instr_desc<Kind::BF16>(128, 64, false, true, true);  // -S, B = W MN-major
             const uint32_t ID_S = instr_desc<Kind::BF16>(128, 128, false, true);       // B = K, MN-major
             const uint32_t kq = sbase + B_KQ;
-            bool ok = true;
+            // U^T = V^T (T diag(beta))^T into the Delta accumulator: A = V,
+            // MN-major (d_v across the two 64-value boxes 8 KB apart, 16 tokens
+            // = 2 KB a step); B = T diag(beta) hi, lo.  The -S W^T that follows
+            // accumulates onto it (same accumulator and shape: issued in order).
+            const uint32_t ID_U = instr_desc<Kind::BF16>(128, 64, true, false);
+            auto issue_u = [&]() {
+                for (int kk = 0; kk < C / 16; ++kk) {
+                    const uint64_t av = smem_desc_sw128(sbase + B_V + kk * 2048, 8192, 1024);
+                    mma<Kind::BF16>(tm + TM_D, av, smem_desc(sbase + B_TB + kk * 2048, 1024, 128), ID_U,
+                                    kk > 0 ? 1u : 0u);
+                    mma<Kind::BF16>(tm + TM_D, av, smem_desc(sbase + B_TB + 8192 + kk * 2048, 1024, 128),
+                                    ID_U, 1u);
+                }
+            };
+            bool ok = mbar_wait(bar_u, 0u, wait_ns);
+            if (ok) {
+                fence_after_sync();
+                issue_u();
+            }
             for (int c = 0; c < n_chunks && ok; ++c) {
                 const int b = c & 1;
                 const uint32_t ph = (uint32_t)c & 1u;
@@ -680,7 +667,7 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p,
                 if (!ok) break;
                 fence_after_sync();
                 fence_smem_to_async();
-                gemm_ta(tm + TM_D, tm + TM_SB, sbase + B_W, 128, 2048, 256, D / 16, ID_D, false);
+                gemm_ta(tm + TM_D, tm + TM_SB, sbase + B_W, 128, 2048, 256, D / 16, ID_D, true);
                 commit(smem_u32(bar_gd));
                 // B = Q, K-major with the 128-byte swizzle (kq_sw).
                 for (int kk = 0; kk < D / 16; ++kk)
@@ -705,6 +692,14 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p,
                     mma_ta(tm + TM_S, tm + TM_DTL + 8 * kk, bk, ID_S, 1u);
                 }
                 commit(smem_u32(bar_gs));
+                // The next chunk's U product, now that this chunk's Delta has
+                // been read out of its accumulator (dtready, waited above).
+                if (c + 1 < n_chunks) {
+                    ok = mbar_wait(bar_u, (uint32_t)(c + 1) & 1u, wait_ns);
+                    if (!ok) break;
+                    fence_after_sync();
+                    issue_u();
+                }
                 // P Delta has one accumulator: chunk c-1's output must have left it.
                 ok = mbar_wait(bar_p, ph, wait_ns) && mbar_wait(bar_dready, ph, wait_ns) &&
                      (c < 1 || mbar_wait(bar_ofree + ((c - 1) & 1), (uint32_t)((c - 1) >> 1) & 1u, wait_ns));
@@ -767,6 +762,33 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p,
         auto prefetch = [&](int c) {
             if (lane == 0 && c < n_chunks) bulk_prefetch_l2(rec0 + (size_t)c * rec_step, REC_BYTES);
         };
+        // V of chunk c (two 128-byte-swizzled boxes: tensor copies, or for a
+        // ragged last chunk 16-byte copies that read zero past its end, waited
+        // for here) and its T diag(beta) tiles from the record, on bar_u.
+        auto fetch_vt = [&](int64_t c0, int L, int c) {
+            if (L < C) {
+                const __nv_bfloat16 *vb = static_cast<const __nv_bfloat16 *>(p.v) + hv * D;
+#pragma unroll 8
+                for (int e = lane; e < 64 * 16; e += 32) {
+                    const int r = e >> 4, jc = e & 15;
+                    const bool in = r < L;
+                    const int64_t t = in ? c0 + r : t0;
+                    cp_async16(sm + B_V + (jc >> 3) * 8192 + r * 128 + (((jc & 7) ^ (r & 7)) << 4),
+                               vb + t * p.v_stride + 8 * jc, in ? 16u : 0u);
+                }
+                cp_async_wait_all();
+                fence_smem_to_async();
+                __syncwarp();
+            }
+            if (lane == 0) {
+                bulk_expect(bar_u, L == C ? 32768u : 16384u);
+                if (L == C) {
+                    tma_load_2d(sbase + B_V, &maps.v, hv * D, (int)c0, bar_u);
+                    tma_load_2d(sbase + B_V + 8192, &maps.v, hv * D + 64, (int)c0, bar_u);
+                }
+                bulk_copy(sm + B_TB, rec0 + (size_t)c * rec_step + REC_TB, 16384, bar_u);
+            }
+        };
         bool ok = true;
         prefetch(0);
         prefetch(1);
@@ -784,10 +806,11 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p,
             fetch(c0, L, true);
             bulk(B_W, REC_W, REC_P - REC_W, bar_w, c);
             ++n_w;
-            // U once chunk c-1's Delta epilogue is done with the stage.
-            if (c > 0) ok = mbar_wait(bar_dready, pp, wait_ns);
+            // V and T diag(beta) of chunk c once chunk c-1's U product (under
+            // the same commit as its -S W^T) is done with the stage.
+            if (c > 0) ok = mbar_wait(bar_gd, pp, wait_ns);
             if (!ok) break;
-            bulk(B_U, REC_U, REC_BYTES - REC_U, bar_u, c);
+            fetch_vt(c0, L, c);
             ++n_u;
             // K once chunk c-1's state update is done.  A diagnostic call may
             // withhold chunk 0's K tile, so that the waits on it run out.
@@ -898,7 +921,7 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p,
         for (; c < n_chunks && ok; ++c) {
             const float *sc = scal(c);  // landed: it gave this chunk's e^{gamma_L}
             // Delta^T = U^T - S W^T as hi/lo tiles, and its decayed, k-normalised copy.
-            ok = wait_all(bar_gd, (uint32_t)c & 1u) && wait_all(bar_u, (uint32_t)c & 1u);
+            ok = wait_all(bar_gd, (uint32_t)c & 1u);
             if (!ok) break;
             fence_after_sync();
             // Decayed Delta^T first: it is all the state update waits for.
@@ -911,9 +934,8 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p,
                 tmem_ld16(tm + lane_off + TM_D + s0, dv[h16]);
 #pragma unroll
                 for (int s4 = 0; s4 < 4; ++s4) {
-                    const float4 u = *reinterpret_cast<const float4 *>(sm + B_U + u_off(s0 + 4 * s4, i));
+                    // (Delta^T itself: the U product with -S W^T accumulated onto it)
                     const float4 dn = *reinterpret_cast<const float4 *>(sc + 2 * C + s0 + 4 * s4);
-                    v[4 * s4] += u.x; v[4 * s4 + 1] += u.y; v[4 * s4 + 2] += u.z; v[4 * s4 + 3] += u.w;
                     w[4 * s4] = v[4 * s4] * dn.x; w[4 * s4 + 1] = v[4 * s4 + 1] * dn.y;
                     w[4 * s4 + 2] = v[4 * s4 + 2] * dn.z; w[4 * s4 + 3] = v[4 * s4 + 3] * dn.w;
                 }

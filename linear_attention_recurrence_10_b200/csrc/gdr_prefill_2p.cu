@@ -2,17 +2,19 @@
 // as two kernels, for calls whose workspace has room for per-chunk results.
 //
 // Most of a chunk's work does not depend on the state entering it: the gates,
-// the q/k norms, A and P, the inverse T = (I + A)^{-1}, U = T diag(beta) V and
-// W = T diag(beta e^gamma n) K (the chunkwise WY / UT form of the gated delta
-// rule named in the Qwen3.5 Chat guide, section "Architektur").  So:
+// the q/k norms, A and P, the inverse T = (I + A)^{-1}, T diag(beta) (U is
+// T diag(beta) V) and W = T diag(beta e^gamma n) K (the chunkwise WY / UT form
+// of the gated delta rule named in the Qwen3.5 Chat guide, section
+// "Architektur").  So:
 //
 //   prep kernel:  one CTA per (chunk, value head), every chunk at once, over
-//                 the whole GPU (three CTAs per SM; K, Q and V by tensor
-//                 copies).  Writes, per unit, a 65 KB record to the
-//                 workspace: W (bf16, already in the MMA operand layout),
-//                 P (hi + lo bf16), U (fp32) and the per-token scalars.
+//                 the whole GPU (three CTAs per SM; K and Q by tensor copies).
+//                 Writes, per unit, a 49 KB record to the workspace: W (bf16,
+//                 already in the MMA operand layout), P and T diag(beta) (hi +
+//                 lo bf16) and the per-token scalars.
 //   recur kernel: one CTA per (sequence, value head), chunks in order, only
 //                 the state-dependent part:
+//                   U^T     = V^T (T diag(beta))^T      (off the chain)
 //                   Delta^T = U^T - S W^T
 //                   O^T     = diag-scaled S Q^T + Delta^T P^T
 //                   S       = e^{gamma_L} S + (Delta^T diag(e^{gamma_L-gamma} n)) K
@@ -510,12 +512,14 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
 //               one warp normalises, gates and stores whole tokens;
 //   warp 16     producer: K and Q tiles by tensor copies (a sequence's
 //               ragged last chunk by 16-byte copies that read zero past its
-//               end), and by bulk copy each chunk's W, P, U and scalars, every
-//               one into its stage as soon as the previous chunk is done with
-//               it (the record is first prefetched into L2 a chunk ahead);
+//               end), V the same way, and by bulk copy each chunk's W, P,
+//               T diag(beta) and scalars, every one into its stage as soon as
+//               the previous chunk is done with it (the record is first
+//               prefetched into L2 a chunk ahead);
 //   warp 17     MMA issue, state path first (-S W^T before S Q^T, the state
-//               update before P Delta), each group committed on its own
-//               barrier so the state group never waits for output products.
+//               update, then the next chunk's U product, before P Delta), each
+//               group committed on its own barrier so the state group never
+//               waits for output products.
 
 constexpr int RNT = 576;                       // 18 warps
 constexpr int OG_BAR = 1, OG_N = 256;

@@ -763,8 +763,20 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p,
                 bulk_copy(sm + dst, rec0 + (size_t)c * rec_step + src_off, bytes, bar);
             }
         };
+        // Chunk c's record, and its K, Q and V tiles (full chunks), into L2.
         auto prefetch = [&](int c) {
-            if (lane == 0 && c < n_chunks) bulk_prefetch_l2(rec0 + (size_t)c * rec_step, REC_BYTES);
+            if (lane == 0 && c < n_chunks) {
+                bulk_prefetch_l2(rec0 + (size_t)c * rec_step, REC_BYTES);
+                if (chunk_len(c) == C) {
+                    const int t = (int)(t0 + (int64_t)c * C);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        tma_prefetch_2d(&maps.k, hk * D + 64 * h, t);
+                        tma_prefetch_2d(&maps.q, hk * D + 64 * h, t);
+                        tma_prefetch_2d(&maps.v, hv * D + 64 * h, t);
+                    }
+                }
+            }
         };
         // V of chunk c (two 128-byte-swizzled boxes: tensor copies, or for a
         // ragged last chunk 16-byte copies that read zero past its end, waited
@@ -804,18 +816,18 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p,
             const int64_t c0 = t0 + (int64_t)c * C;
             const int L = chunk_len(c);
             const uint32_t pp = (uint32_t)(c - 1) & 1u;  // phase of chunk c-1's events
-            // Q and W of chunk c once chunk c-1's S Q^T (issued after -S W^T) is done.
-            if (c > 0) ok = mbar_wait(bar_qfree, pp, wait_ns);
-            if (!ok) break;
-            fetch(c0, L, true);
-            bulk(B_W, REC_W, REC_P - REC_W, bar_w, c);
-            ++n_w;
             // V and T diag(beta) of chunk c once chunk c-1's U product (under
             // the same commit as its -S W^T) is done with the stage.
             if (c > 0) ok = mbar_wait(bar_gd, pp, wait_ns);
             if (!ok) break;
             fetch_vt(c0, L, c);
             ++n_u;
+            // Q and W of chunk c once chunk c-1's S Q^T (issued after -S W^T) is done.
+            if (c > 0) ok = mbar_wait(bar_qfree, pp, wait_ns);
+            if (!ok) break;
+            fetch(c0, L, true);
+            bulk(B_W, REC_W, REC_P - REC_W, bar_w, c);
+            ++n_w;
             // K once chunk c-1's state update is done.  A diagnostic call may
             // withhold chunk 0's K tile, so that the waits on it run out.
             if (c > 0) ok = mbar_wait(bar_gs, pp, wait_ns);

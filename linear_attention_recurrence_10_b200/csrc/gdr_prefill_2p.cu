@@ -514,8 +514,8 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
 //               ragged last chunk by 16-byte copies that read zero past its
 //               end), V the same way, and by bulk copy each chunk's W, P,
 //               T diag(beta) and scalars, every one into its stage as soon as
-//               the previous chunk is done with it (the record is first
-//               prefetched into L2 a chunk ahead);
+//               the previous chunk is done with it (no L2 prefetch: it shared
+//               the copy engine with these loads and measured slower);
 //   warp 17     MMA issue, state path first (-S W^T before S Q^T, the state
 //               update, then the next chunk's U product, before P Delta), each
 //               group committed on its own barrier so the state group never
@@ -772,21 +772,6 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p,
                 bulk_copy(sm + dst, rec0 + (size_t)c * rec_step + src_off, bytes, bar);
             }
         };
-        // Chunk c's record, and its K, Q and V tiles (full chunks), into L2.
-        auto prefetch = [&](int c) {
-            if (lane == 0 && c < n_chunks) {
-                bulk_prefetch_l2(rec0 + (size_t)c * rec_step, REC_BYTES);
-                if (chunk_len(c) == C) {
-                    const int t = (int)(t0 + (int64_t)c * C);
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        tma_prefetch_2d(&maps.k, hk * D + 64 * h, t);
-                        tma_prefetch_2d(&maps.q, hk * D + 64 * h, t);
-                        tma_prefetch_2d(&maps.v, hv * D + 64 * h, t);
-                    }
-                }
-            }
-        };
         // V of chunk c (two 128-byte-swizzled boxes: tensor copies, or for a
         // ragged last chunk 16-byte copies that read zero past its end, waited
         // for here) and its T diag(beta) tiles from the record, on bar_u.
@@ -815,8 +800,6 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p,
             }
         };
         bool ok = true;
-        prefetch(0);
-        prefetch(1);
         for (int c = 0; c < n_chunks && c < 2; ++c) {
             bulk(B_SC + (c & 1) * SC_BYTES, REC_SCAL, SC_BYTES, bar_sc + (c & 1), c);
             ++n_sc[c & 1];
@@ -848,14 +831,13 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p,
             bulk(B_P, REC_P, REC_SCAL - REC_P, bar_p, c);
             ++n_p;
             // Scalars of chunk c+1 replace chunk c-1's once the output group is
-            // done with them; the record after that goes to L2.
+            // done with them.
             if (c >= 1 && c + 1 < n_chunks) {
                 ok = mbar_wait(bar_ofree + ((c + 1) & 1), (uint32_t)((c - 1) >> 1) & 1u, wait_ns);
                 if (!ok) break;
                 bulk(B_SC + ((c + 1) & 1) * SC_BYTES, REC_SCAL, SC_BYTES, bar_sc + ((c + 1) & 1), c + 1);
                 ++n_sc[(c + 1) & 1];
             }
-            prefetch(c + 2);
         }
         // The last chunk's S Q^T commit is the one tcgen05 arrival nobody else
         // waits for; it must land before the CTA ends (after an expired wait,

@@ -326,18 +326,6 @@ __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-// Ask L2 to fetch the 128-byte line holding `p` (no result, nothing to wait for).
-__device__ __forceinline__ void prefetch_l2(const void *p) {
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
-
-// Start moving `bytes` (a multiple of 16, 16-byte aligned) of global memory
-// into L2; nothing is written anywhere and nothing needs to be waited for.
-__device__ __forceinline__ void bulk_prefetch_l2(const void *gmem_src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gmem_src), "r"(bytes)
-                 : "memory");
-}
-
 // A plain arrival (release semantics) on the barrier.
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");

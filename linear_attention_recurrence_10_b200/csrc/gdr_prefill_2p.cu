@@ -521,14 +521,17 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
 //               group committed on its own barrier so the state group never
 //               waits for output products.
 
-// The gate z sigma(z), with sigma(z) = (1 + tanh(z / 2)) / 2: one
-// special-function op (tanh.approx, relative error below 2^-10.9) where
-// e^{-z} and a reciprocal take two; the output warps run 32 per lane a chunk.
-__device__ __forceinline__ float silu_tanh(float z) {
+// tanh.approx (relative error below 2^-10.9): with sigma(z) = (1 + tanh(z/2))
+// / 2 the gate z sigma(z) costs one special-function op where e^{-z} and a
+// reciprocal take two; the output warps run 32 per lane a chunk.
+__device__ __forceinline__ float tanh_approx(float x) {
     float t;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * z));
-    return z * fmaf(0.5f, t, 0.5f);
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(x));
+    return t;
 }
+// The output warps' element-wise fp32 work runs in pairs (sm_100's two-wide
+// FMA and multiply; each lane rounds as the scalar op does).
+__device__ __forceinline__ float2 f2(float x, float y) { return make_float2(x, y); }
 
 constexpr int RNT = 576;                       // 18 warps
 constexpr int OG_BAR = 1, OG_N = 256;
@@ -1051,10 +1054,14 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p,
                     for (int k4 = 0; k4 < 4; ++k4) {
                         const int r = r0 + 16 * h16 + 4 * k4;
                         const float4 m = *reinterpret_cast<const float4 *>(sc + C + r);
-                        Os[r * D + i] = fmaf(m.x, a[4 * k4], d[4 * k4]);
-                        Os[(r + 1) * D + i] = fmaf(m.y, a[4 * k4 + 1], d[4 * k4 + 1]);
-                        Os[(r + 2) * D + i] = fmaf(m.z, a[4 * k4 + 2], d[4 * k4 + 2]);
-                        Os[(r + 3) * D + i] = fmaf(m.w, a[4 * k4 + 3], d[4 * k4 + 3]);
+                        const float2 o01 = __ffma2_rn(f2(m.x, m.y), f2(a[4 * k4], a[4 * k4 + 1]),
+                                                      f2(d[4 * k4], d[4 * k4 + 1]));
+                        const float2 o23 = __ffma2_rn(f2(m.z, m.w), f2(a[4 * k4 + 2], a[4 * k4 + 3]),
+                                                      f2(d[4 * k4 + 2], d[4 * k4 + 3]));
+                        Os[r * D + i] = o01.x;
+                        Os[(r + 1) * D + i] = o01.y;
+                        Os[(r + 2) * D + i] = o23.x;
+                        Os[(r + 3) * D + i] = o23.y;
                     }
                 }
             }
@@ -1075,7 +1082,11 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p,
                 // lanes; xor 8 and 16 finish the sum (9 shuffles for 8 tokens).
                 float ps[8];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) ps[u] = dot4(o4[u], o4[u]);
+                for (int u = 0; u < 8; ++u) {
+                    const float2 xy = f2(o4[u].x, o4[u].y), zw = f2(o4[u].z, o4[u].w);
+                    const float2 q = __ffma2_rn(zw, zw, __fmul2_rn(xy, xy));
+                    ps[u] = q.x + q.y;
+                }
 #pragma unroll
                 for (int st = 4; st >= 1; st >>= 1) {
                     const bool upper = (lane & st) != 0;
@@ -1096,13 +1107,18 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p,
                 const int r = 8 * og + u;
                 float4 y = o4[u];
                 if (zg) {
+                    // y = (o rstd) (w z / 2) (1 + tanh(z / 2)), two values at a time.
                     const float rstd = __shfl_sync(0xffffffffu, rstd_l, u);
                     const float2 za = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&zr[u].x));
                     const float2 zb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&zr[u].y));
-                    y.x *= rstd * w4.x * silu_tanh(za.x);
-                    y.y *= rstd * w4.y * silu_tanh(za.y);
-                    y.z *= rstd * w4.z * silu_tanh(zb.x);
-                    y.w *= rstd * w4.w * silu_tanh(zb.y);
+                    const float2 ha = __fmul2_rn(za, f2(0.5f, 0.5f)), hb = __fmul2_rn(zb, f2(0.5f, 0.5f));
+                    const float2 ta = f2(tanh_approx(ha.x), tanh_approx(ha.y));
+                    const float2 tb = f2(tanh_approx(hb.x), tanh_approx(hb.y));
+                    const float2 ua = __fmul2_rn(f2(w4.x, w4.y), ha), ub = __fmul2_rn(f2(w4.z, w4.w), hb);
+                    const float2 ga = __ffma2_rn(ua, ta, ua), gb = __ffma2_rn(ub, tb, ub);
+                    const float2 ya = __fmul2_rn(__fmul2_rn(f2(y.x, y.y), f2(rstd, rstd)), ga);
+                    const float2 yb = __fmul2_rn(__fmul2_rn(f2(y.z, y.w), f2(rstd, rstd)), gb);
+                    y = make_float4(ya.x, ya.y, yb.x, yb.y);
                 }
                 if (r < L) Elem<TOUT>::store4(out + (c0 + r) * p.out_stride + hv * D + 4 * lane, y);
             }

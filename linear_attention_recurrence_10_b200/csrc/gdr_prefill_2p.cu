@@ -380,6 +380,28 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
         // row factor times a table entry below it, exact on it.
         const int rr = 32 * (quad & 1) + lane, R = rr >> 4;
         const float gr = sc.gam[rr];
+        // v[c] <- f e[c] n_k[s0+c] v[c] on or below the diagonal (strictly
+        // below for A), else 0; pairs by two-wide multiplies, n_k by 16 bytes.
+        auto scale_row = [&](float (&v)[16], const float (&e)[16], float f, int s0, int rr,
+                             bool diag) {
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                const float4 nk = *reinterpret_cast<const float4 *>(sc.nk + s0 + 4 * c4);
+                const float2 ff = make_float2(f, f);
+                const float2 a = __fmul2_rn(__fmul2_rn(ff, make_float2(e[4 * c4], e[4 * c4 + 1])),
+                                            __fmul2_rn(make_float2(nk.x, nk.y),
+                                                       make_float2(v[4 * c4], v[4 * c4 + 1])));
+                const float2 b = __fmul2_rn(__fmul2_rn(ff, make_float2(e[4 * c4 + 2], e[4 * c4 + 3])),
+                                            __fmul2_rn(make_float2(nk.z, nk.w),
+                                                       make_float2(v[4 * c4 + 2], v[4 * c4 + 3])));
+                const float r4[4] = {a.x, a.y, b.x, b.y};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int s = s0 + 4 * c4 + u;
+                    v[4 * c4 + u] = (diag ? s <= rr : s < rr) ? r4[u] : 0.f;
+                }
+            }
+        };
         const float rowf = R > 0 ? __expf(gr - sc.gam[16 * R]) : 1.f;
 #pragma unroll
         for (int sl = 0; sl < PSL; ++sl) {
@@ -388,7 +410,12 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
         tmem_ld16(tm + lane_off + TM_D1 + s0, v);
         if (Sb < R) {
 #pragma unroll
-            for (int c = 0; c < 16; ++c) e[c] = rowf * sc.dtab[R * DTL + s0 + c];
+            for (int c4 = 0; c4 < 4; ++c4) {
+                const float4 t = *reinterpret_cast<const float4 *>(sc.dtab + R * DTL + s0 + 4 * c4);
+                const float2 a = __fmul2_rn(make_float2(rowf, rowf), make_float2(t.x, t.y));
+                const float2 b = __fmul2_rn(make_float2(rowf, rowf), make_float2(t.z, t.w));
+                e[4 * c4] = a.x; e[4 * c4 + 1] = a.y; e[4 * c4 + 2] = b.x; e[4 * c4 + 3] = b.y;
+            }
         } else if (Sb == R) {
 #pragma unroll
             for (int c = 0; c < 16; ++c) e[c] = __expf(gr - sc.gam[s0 + c]);
@@ -400,22 +427,13 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
             // 16-byte stores: with rows PLD floats apart, a quarter-warp's eight
             // rows cover all 32 banks once.
             const float f = sc.bet[rr] * sc.nk[rr];
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                const int s = s0 + c;
-                v[c] = s < rr ? f * e[c] * sc.nk[s] * v[c] : 0.f;
-            }
+            scale_row(v, e, f, s0, rr, false);
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4)
                 *reinterpret_cast<float4 *>(Ascr + rr * PLD + s0 + 4 * c4) =
                     make_float4(v[4 * c4], v[4 * c4 + 1], v[4 * c4 + 2], v[4 * c4 + 3]);
         } else {
-            const float f = sc.nq[rr];
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                const int s = s0 + c;
-                v[c] = s <= rr ? f * e[c] * sc.nk[s] * v[c] : 0.f;
-            }
+            scale_row(v, e, sc.nq[rr], s0, rr, true);
 #pragma unroll
             for (int c8 = 0; c8 < 2; ++c8) {
                 uint4 h, l;

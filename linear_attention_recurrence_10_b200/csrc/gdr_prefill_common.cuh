@@ -110,7 +110,8 @@ __device__ __forceinline__ void offdiag_stage(const float *Ascr, float *Tscr, fl
 // The same distance stage with 16-byte aligned rows (LD % 4 == 0): each thread
 // computes a strip of four adjacent outputs, so every operand load is a
 // 16-byte vector that feeds four (row operand) or sixteen (column operand)
-// FMAs instead of one.  X is kept as dense 16 x 16 blocks.
+// FMAs instead of one, issued as two-wide FMAs (sm_100; each lane rounds as
+// fmaf does).  X is kept as dense 16 x 16 blocks.
 template <int DIST, int NT, int LD>
 __device__ __forceinline__ void offdiag_stage_strips(const float *Ascr, float *Tscr, float *Xscr,
                                                      int tid) {
@@ -120,7 +121,7 @@ __device__ __forceinline__ void offdiag_stage_strips(const float *Ascr, float *T
         const int j = e >> 6, i = j + DIST, rr = (e >> 2) & 15, c4 = 4 * (e & 3);
         const float *arow = Ascr + (16 * i + rr) * LD + 16 * j;
         const float *tcol = Tscr + 16 * j * LD + 16 * j + c4;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float2 lo = make_float2(0.f, 0.f), hi = make_float2(0.f, 0.f);  // the strip's four sums
 #pragma unroll
         for (int k4 = 0; k4 < 4 * DIST; ++k4) {
             const float4 a = *reinterpret_cast<const float4 *>(arow + 4 * k4);
@@ -128,20 +129,19 @@ __device__ __forceinline__ void offdiag_stage_strips(const float *Ascr, float *T
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const float4 t = *reinterpret_cast<const float4 *>(tcol + (4 * k4 + u) * LD);
-                acc.x = fmaf(av[u], t.x, acc.x);
-                acc.y = fmaf(av[u], t.y, acc.y);
-                acc.z = fmaf(av[u], t.z, acc.z);
-                acc.w = fmaf(av[u], t.w, acc.w);
+                const float2 au = make_float2(av[u], av[u]);
+                lo = __ffma2_rn(au, make_float2(t.x, t.y), lo);
+                hi = __ffma2_rn(au, make_float2(t.z, t.w), hi);
             }
         }
-        *reinterpret_cast<float4 *>(Xscr + (j << 8) + rr * 16 + c4) = acc;
+        *reinterpret_cast<float4 *>(Xscr + (j << 8) + rr * 16 + c4) = make_float4(lo.x, lo.y, hi.x, hi.y);
     }
     __syncthreads();
     for (int e = tid; e < NSTRIP; e += NT) {
         const int j = e >> 6, i = j + DIST, rr = (e >> 2) & 15, c4 = 4 * (e & 3);
         const float *trow = Tscr + (16 * i + rr) * LD + 16 * i;
         const float *xblk = Xscr + (j << 8) + c4;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float2 lo = make_float2(0.f, 0.f), hi = make_float2(0.f, 0.f);
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4) {
             const float4 t = *reinterpret_cast<const float4 *>(trow + 4 * k4);
@@ -149,14 +149,13 @@ __device__ __forceinline__ void offdiag_stage_strips(const float *Ascr, float *T
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const float4 x = *reinterpret_cast<const float4 *>(xblk + (4 * k4 + u) * 16);
-                acc.x = fmaf(tv[u], x.x, acc.x);
-                acc.y = fmaf(tv[u], x.y, acc.y);
-                acc.z = fmaf(tv[u], x.z, acc.z);
-                acc.w = fmaf(tv[u], x.w, acc.w);
+                const float2 tu = make_float2(tv[u], tv[u]);
+                lo = __ffma2_rn(tu, make_float2(x.x, x.y), lo);
+                hi = __ffma2_rn(tu, make_float2(x.z, x.w), hi);
             }
         }
         *reinterpret_cast<float4 *>(Tscr + (16 * i + rr) * LD + 16 * j + c4) =
-            make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+            make_float4(-lo.x, -lo.y, -hi.x, -hi.y);
     }
     __syncthreads();
 }
@@ -176,8 +175,20 @@ __device__ __forceinline__ void invert_unit_lower(const float *Ascr, float *Tscr
         for (int r = 0; r < 16; ++r) x[r] = (r == c) ? 1.f : 0.f;
 #pragma unroll
         for (int s = 0; s < 15; ++s) {
+            // Rows in pairs (two-wide FMA); fmaf(a, -x, y) is fmaf(-a, x, y) exactly.
+            const float2 nx = make_float2(-x[s], -x[s]);
 #pragma unroll
-            for (int r = s + 1; r < 16; ++r) x[r] = fmaf(-Ascr[(base + r) * LD + base + s], x[s], x[r]);
+            for (int r = s + 1; r < 16; r += 2) {
+                if (r + 1 < 16) {
+                    const float2 y = __ffma2_rn(make_float2(Ascr[(base + r) * LD + base + s],
+                                                            Ascr[(base + r + 1) * LD + base + s]),
+                                               nx, make_float2(x[r], x[r + 1]));
+                    x[r] = y.x;
+                    x[r + 1] = y.y;
+                } else {
+                    x[r] = fmaf(Ascr[(base + r) * LD + base + s], nx.x, x[r]);
+                }
+            }
         }
 #pragma unroll
         for (int r = 0; r < 16; ++r) Tscr[(base + r) * LD + base + c] = x[r];

@@ -151,6 +151,7 @@ static_assert(3 * (A_SMEM_LAUNCH + 1024) <= 228 * 1024, "three prep blocks must 
 constexpr int DTL = C + 4;  // row stride of dtab
 struct PrepScalars {
     float gam[C], eg[C], bet[C], nk[C], nq[C], dec[C];
+    float tw[C];  // beta e^gamma n_k: the column factor of TW
     // dtab[R][s] = e^{gamma_{16R} - gamma_s} for s < 16R: with the per-row
     // e^{gamma_r - gamma_{16R}} it gives e^{gamma_r - gamma_s} below the
     // diagonal 16-block as a product of two factors that are at most one.
@@ -334,7 +335,10 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
         sc.eg[lane + 32] = __expf(gb);
     }
     __syncthreads();
-    if (tid < C) sc.dec[tid] = __expf(sc.gam[L - 1] - sc.gam[tid]);
+    if (tid < C) {
+        sc.dec[tid] = __expf(sc.gam[L - 1] - sc.gam[tid]);
+        sc.tw[tid] = sc.bet[tid] * sc.eg[tid] * sc.nk[tid];
+    }
     {
         const int R = tid >> 6, s = tid & 63;  // PNT == 4 * C entries
         sc.dtab[R * DTL + s] = s < 16 * R ? __expf(sc.gam[16 * R] - sc.gam[s]) : 0.f;
@@ -455,10 +459,13 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
                 *reinterpret_cast<float4 *>(t) = *reinterpret_cast<const float4 *>(Tscr + r * PLD + s8);
                 *reinterpret_cast<float4 *>(t + 4) =
                     *reinterpret_cast<const float4 *>(Tscr + r * PLD + s8 + 4);
+                const float *fs = (w_side ? sc.tw : sc.bet) + s8;
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int s = s8 + u;
-                    t[u] *= w_side ? sc.bet[s] * sc.eg[s] * sc.nk[s] : sc.bet[s];
+                for (int u4 = 0; u4 < 2; ++u4) {
+                    const float4 f = *reinterpret_cast<const float4 *>(fs + 4 * u4);
+                    const float2 a = __fmul2_rn(make_float2(t[4 * u4], t[4 * u4 + 1]), make_float2(f.x, f.y));
+                    const float2 b = __fmul2_rn(make_float2(t[4 * u4 + 2], t[4 * u4 + 3]), make_float2(f.z, f.w));
+                    t[4 * u4] = a.x; t[4 * u4 + 1] = a.y; t[4 * u4 + 2] = b.x; t[4 * u4 + 3] = b.y;
                 }
                 uint4 h, l;
                 split8(t, h, l);

@@ -62,7 +62,9 @@ __device__ __forceinline__ void split8(const float *v, uint4 &hi, uint4 &lo) {
     for (int u = 0; u < 4; ++u) {
         const __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * u], v[2 * u + 1]);
         const float2 f = __bfloat1622float2(b);
-        const __nv_bfloat162 r = __floats2bfloat162_rn(v[2 * u] - f.x, v[2 * u + 1] - f.y);
+        // x - hi for both lanes at once (sm_100's two-wide add; exact here).
+        const float2 d = __fadd2_rn(make_float2(v[2 * u], v[2 * u + 1]), make_float2(-f.x, -f.y));
+        const __nv_bfloat162 r = __floats2bfloat162_rn(d.x, d.y);
         h[u] = *reinterpret_cast<const uint32_t *>(&b);
         l[u] = *reinterpret_cast<const uint32_t *>(&r);
     }

@@ -525,7 +525,7 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
 // state path is serial: Delta = U - W S^T needs the state entering the chunk,
 // and the next state needs Delta.  The output of a chunk (O = (m e^gamma) Q S^T
 // + P Delta, then RMSNormGated) feeds nothing later, so the CTA is split into
-// four roles that run concurrently and hand work over on mbarriers:
+// five roles that run concurrently and hand work over on mbarriers:
 //   warps 0-7   state group: the Delta epilogue -- first the decayed,
 //               k-normalised copy of Delta^T as hi/lo tiles in TMEM, all the
 //               state update waits for, then Delta's hi/lo tiles for P Delta --
@@ -535,12 +535,14 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
 //   warps 8-15  output group, one chunk behind: S Q^T and P Delta out of
 //               double-buffered TMEM, staged through shared memory so that
 //               one warp normalises, gates and stores whole tokens;
-//   warp 16     producer: K and Q tiles by tensor copies (a sequence's
-//               ragged last chunk by 16-byte copies that read zero past its
-//               end), V the same way, and by bulk copy each chunk's W, P,
-//               T diag(beta) and scalars, every one into its stage as soon as
-//               the previous chunk is done with it (no L2 prefetch: it shared
-//               the copy engine with these loads and measured slower);
+//   warp 16     producer for the state path: K and Q tiles by tensor copies
+//               (a sequence's ragged last chunk by 16-byte copies that read
+//               zero past its end), V the same way, and by bulk copy each
+//               chunk's W and T diag(beta), every one into its stage as soon
+//               as the previous chunk is done with it (no L2 prefetch: it
+//               shared the copy engine with these loads and measured slower);
+//   warp 18     producer for the output side: P and the per-token scalars,
+//               whose stages the output group frees;
 //   warp 17     MMA issue, state path first (-S W^T before S Q^T, the state
 //               update, then the next chunk's U product, before P Delta), each
 //               group committed on its own barrier so the state group never
@@ -558,7 +560,7 @@ __device__ __forceinline__ float tanh_approx(float x) {
 // FMA and multiply; each lane rounds as the scalar op does).
 __device__ __forceinline__ float2 f2(float x, float y) { return make_float2(x, y); }
 
-constexpr int RNT = 576;                       // 18 warps
+constexpr int RNT = 608;                       // 19 warps
 constexpr int OG_BAR = 1, OG_N = 256;
 constexpr uint32_t B_KQ = 0;                   // bf16 [K;Q] (32 KB, as kq_sw lays it out)
 constexpr uint32_t B_W = 32768;                // bf16 W of the current chunk (16 KB)
@@ -762,7 +764,7 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p,
         const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(p.q) + hk * D;
         const __nv_bfloat16 *kg = static_cast<const __nv_bfloat16 *>(p.k) + hk * D;
         // Copies counted so that an early exit can wait for them.
-        int n_w = 0, n_p = 0, n_u = 0, n_sc[2] = {0, 0}, n_tile[2] = {0, 0};
+        int n_w = 0, n_u = 0, n_tile[2] = {0, 0};
         // The K or Q tile of a chunk (kq_sw layout): a full chunk by two tensor
         // copies; a sequence's ragged last chunk by 16-byte copies that read
         // zero past its end (this lane waits for its own, then one arrival).
@@ -828,10 +830,6 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p,
             }
         };
         bool ok = true;
-        for (int c = 0; c < n_chunks && c < 2; ++c) {
-            bulk(B_SC + (c & 1) * SC_BYTES, REC_SCAL, SC_BYTES, bar_sc + (c & 1), c);
-            ++n_sc[c & 1];
-        }
         for (int c = 0; c < n_chunks && ok; ++c) {
             const int64_t c0 = t0 + (int64_t)c * C;
             const int L = chunk_len(c);
@@ -853,6 +851,39 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p,
             if (c > 0) ok = mbar_wait(bar_gs, pp, wait_ns);
             if (!ok) break;
             if (!(p.withhold_first_k && c == 0)) fetch(c0, L, false);
+        }
+        // The last chunk's S Q^T commit is the one tcgen05 arrival nobody else
+        // waits for; it must land before the CTA ends (after an expired wait,
+        // only if its product was issued: it comes within microseconds then).
+        if (lane == 0 && n_chunks > 0)
+            mbar_wait(bar_qfree, (uint32_t)(n_chunks - 1) & 1u, ok ? wait_ns : 1000000ull);
+        if (!ok) {
+            if (lane == 0) fail();
+            // No bulk copy may land after the CTA ends.
+            if (n_w) mbar_wait(bar_w, (uint32_t)(n_w - 1) & 1u, wait_ns);
+            if (n_tile[0]) mbar_wait(bar_k, (uint32_t)(n_tile[0] - 1) & 1u, wait_ns);
+            if (n_tile[1]) mbar_wait(bar_q, (uint32_t)(n_tile[1] - 1) & 1u, wait_ns);
+            if (n_u) mbar_wait(bar_u, (uint32_t)(n_u - 1) & 1u, wait_ns);
+        }
+        __syncwarp();
+    } else if (warp == 18) {
+        // --------------------------------------------- output-side producer
+        // P and the per-token scalars.  Their stages are freed by the output
+        // group, a chunk behind; on a warp of their own these waits no longer
+        // hold up the copies the state path waits for.
+        int n_p = 0, n_sc[2] = {0, 0};
+        auto bulk = [&](uint32_t dst, uint32_t src_off, uint32_t bytes, uint64_t *bar, int c) {
+            if (lane == 0) {
+                bulk_expect(bar, bytes);
+                bulk_copy(sm + dst, rec0 + (size_t)c * rec_step + src_off, bytes, bar);
+            }
+        };
+        bool ok = true;
+        for (int c = 0; c < n_chunks && c < 2; ++c) {
+            bulk(B_SC + (c & 1) * SC_BYTES, REC_SCAL, SC_BYTES, bar_sc + (c & 1), c);
+            ++n_sc[c & 1];
+        }
+        for (int c = 0; c < n_chunks && ok; ++c) {
             // P once chunk c-1's P Delta is done.
             if (c > 0) ok = mbar_wait(bar_oready + ((c - 1) & 1), (uint32_t)((c - 1) >> 1) & 1u, wait_ns);
             if (!ok) break;
@@ -867,19 +898,10 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p,
                 ++n_sc[(c + 1) & 1];
             }
         }
-        // The last chunk's S Q^T commit is the one tcgen05 arrival nobody else
-        // waits for; it must land before the CTA ends (after an expired wait,
-        // only if its product was issued: it comes within microseconds then).
-        if (lane == 0 && n_chunks > 0)
-            mbar_wait(bar_qfree, (uint32_t)(n_chunks - 1) & 1u, ok ? wait_ns : 1000000ull);
         if (!ok) {
             if (lane == 0) fail();
             // No bulk copy may land after the CTA ends.
-            if (n_w) mbar_wait(bar_w, (uint32_t)(n_w - 1) & 1u, wait_ns);
-            if (n_tile[0]) mbar_wait(bar_k, (uint32_t)(n_tile[0] - 1) & 1u, wait_ns);
-            if (n_tile[1]) mbar_wait(bar_q, (uint32_t)(n_tile[1] - 1) & 1u, wait_ns);
             if (n_p) mbar_wait(bar_p, (uint32_t)(n_p - 1) & 1u, wait_ns);
-            if (n_u) mbar_wait(bar_u, (uint32_t)(n_u - 1) & 1u, wait_ns);
             for (int b = 0; b < 2; ++b)
                 if (n_sc[b]) mbar_wait(bar_sc + b, (uint32_t)(n_sc[b] - 1) & 1u, wait_ns);
         }

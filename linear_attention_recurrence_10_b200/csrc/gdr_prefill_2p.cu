@@ -1218,7 +1218,7 @@ size_t prefill_tc2p_workspace_bytes(int n_seq, int64_t n_chunks, int H_v, int n_
 }
 
 // cu_host: the sequence offsets on the host (segment sizes are planned here).
-// Segment boundaries: 40% and 72% of the longest sequence's chunks, so that
+// Segment boundaries: 34% and 66% of the longest sequence's chunks, so that
 // each later segment's prep (on the SMs the recurrence leaves free) takes
 // about as long as the recurrence of the segment before it.
 cudaError_t launch_prefill_tc2p(const PrefillParams &p, const int32_t *cu_host, int n_seg,
@@ -1233,8 +1233,8 @@ cudaError_t launch_prefill_tc2p(const PrefillParams &p, const int32_t *cu_host, 
     tcp2::SegPlan sp = {};
     sp.n = n_seg < 1 ? 1 : (n_seg > tcp2::MAX_SEG ? tcp2::MAX_SEG : n_seg);
     if (sp.n == 3) {
-        sp.lo[1] = (int)((max_chunks * 40 + 99) / 100);
-        sp.lo[2] = (int)((max_chunks * 72 + 99) / 100);
+        sp.lo[1] = (int)((max_chunks * 34 + 99) / 100);
+        sp.lo[2] = (int)((max_chunks * 66 + 99) / 100);
     } else if (sp.n == 2) {
         sp.lo[1] = (int)((max_chunks * 60 + 99) / 100);
     }

@@ -529,9 +529,9 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
 //   warps 0-7   state group: the Delta epilogue -- first the decayed,
 //               k-normalised copy of Delta^T as hi/lo tiles in TMEM, all the
 //               state update waits for, then Delta's hi/lo tiles for P Delta --
-//               and, once the update is done, the bf16 copy of S that the next
-//               chunk's first products wait for, then the state pre-scaled by
-//               the next chunk's e^{gamma_L}, which only its update waits for;
+//               and, once the update is done, from one read of the state, the
+//               bf16 copy of S that the next chunk's first products wait for
+//               and the state pre-scaled by the next chunk's e^{gamma_L};
 //   warps 8-15  output group, one chunk behind: S Q^T and P Delta out of
 //               double-buffered TMEM, staged through shared memory so that
 //               one warp normalises, gates and stores whole tokens;
@@ -1025,28 +1025,25 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p,
             publish(bar_dready);
 
             // Once the state update is done: the next chunk's bf16 S (what its
-            // first products wait for), then the state scaled for its update.
+            // first products wait for) and the state scaled for its update.
             ok = wait_all(bar_gs, (uint32_t)c & 1u);
             if (!ok || c + 1 == n_chunks) continue;
             ok = wait_all(bar_sc + ((c + 1) & 1), (uint32_t)((c + 1) >> 1) & 1u);
             if (!ok) continue;
             fence_after_sync();
             const float eL = scal(c + 1)[3 * C];
+            // One read of each half row: its bf16 copy, then the pre-scaled
+            // state in place (published together; reading the row twice, to
+            // publish the copy first, measured slower).
 #pragma unroll 1
             for (int jj = 0; jj < 2; ++jj) {
                 const int j0 = 64 * half + 32 * jj;
                 float v[32];
                 tmem_ld32(tm + lane_off + TM_S + j0, v);
                 stage_bf16(v, j0);
-            }
-            publish(bar_sready);
-#pragma unroll 1
-            for (int jj = 0; jj < 2; ++jj) {
-                const int j0 = 64 * half + 32 * jj;
-                float v[32];
-                tmem_ld32(tm + lane_off + TM_S + j0, v);
                 stage_scaled(v, j0, eL);
             }
+            publish(bar_sready);
             publish(bar_scaled);
         }
         state_ok = ok && n_chunks > 0 && c == n_chunks;

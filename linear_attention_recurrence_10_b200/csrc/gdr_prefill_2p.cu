@@ -177,8 +177,6 @@ __device__ __forceinline__ uint32_t kq_sw(int row, int jc) {
     return (uint32_t)((jc >> 3) * 16384 + row * 128 + (((jc & 7) ^ (row & 7)) << 4));
 }
 
-// `succ`: block index distance to the unit that most likely takes this block's
-// SM slot next (resident blocks per SM x SMs); its inputs are prefetched to L2.
 // The block's unit within a segment: the sequence (the last s with
 // seg_off[s] <= unit) and its chunk index (from the segment's first chunk).
 struct PrepUnit {
@@ -204,7 +202,7 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
                                                      const __grid_constant__ PrepMaps maps,
                                                      const int *chunk_off,
                                                      const int *seg_off, int seg_lo,
-                                                     unsigned char *records, int *status, int succ,
+                                                     unsigned char *records, int *status,
                                                      int wait_prev_at_exit) {
     extern __shared__ __align__(1024) unsigned char sm_raw[];
     // The swizzled tiles must start on a 1024-byte boundary (A_SMEM_LAUNCH
@@ -230,7 +228,8 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
     float *gbuf = reinterpret_cast<float *>(sm + A_GB);
 
     // Thread 0 starts the tile copies first; warp 7 (idle until the first
-    // product) takes the TMEM columns and, later, warms L2 for the successor.
+    // product) takes the TMEM columns.  (Warming L2 for the unit that next
+    // takes this block's slot measured slower: the copy engine is shared.)
     if (warp == 7) tmem_alloc(&sc.tmem, 128);
     if (tid == 0) {
         mbar_init(&sc.bar, 1);
@@ -275,17 +274,6 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
     const bool loads_bad = __syncthreads_or(!loads_ok) != 0;
     fence_after_sync();
     if (loads_bad && tid == 0) atomicExch(status, kTimeoutStatus);
-    if (tid == 7 * 32 && blockIdx.x + succ < gridDim.x) {
-        // Warm L2 for the unit most likely to take this block's SM slot next.
-        const int nb = blockIdx.x + succ, hv2 = nb % p.H_v, hk2 = hv2 / p.hv_per_hk;
-        const PrepUnit nu = prep_unit(seg_off, seg_lo, p.n_seq, nb / p.H_v);
-        const int n0 = (int)(p.cu_seqlens[nu.seq] + (int64_t)nu.chunk * C);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            tma_prefetch_2d(&maps.k, hk2 * D + 64 * h, n0);
-            tma_prefetch_2d(&maps.q, hk2 * D + 64 * h, n0);
-        }
-    }
     const uint32_t tm = sc.tmem;
     const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
     // [KK;QK] in columns 0..63, W^T beside it.
@@ -1251,10 +1239,6 @@ cudaError_t launch_prefill_tc2p(const PrefillParams &p, const int32_t *cu_host, 
                                           seg_off);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    int dev = 0, n_sm = 148;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return cudaGetLastError();
     // Tensor maps for prep's K, Q and V (the caller's bases and row strides
     // are 16-byte aligned; token offsets fit in int32).
     tcp2::PrepMaps maps;
@@ -1294,7 +1278,7 @@ cudaError_t launch_prefill_tc2p(const PrefillParams &p, const int32_t *cu_host, 
             cfg.attrs = attr;
             cfg.numAttrs = k > 0 ? 1 : 0;  // later segments overlap the recurrence before them
             e = cudaLaunchKernelEx(&cfg, tcp2::prep_kernel, p, maps, (const int *)chunk_off, seg_off_k,
-                                   sp.lo[k], records, status, 2 * n_sm, k > 0 ? 1 : 0);
+                                   sp.lo[k], records, status, k > 0 ? 1 : 0);
             if (e != cudaSuccess) {
                 (void)cudaGetLastError();
                 return e;

@@ -308,14 +308,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t smem_dst, const void *tmap,
         "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar))
         : "memory");
 }
-// Start moving the box at (x, y) of the tensor map at `tmap` into L2 (no
-// result, nothing to wait for; x as for tma_load_2d).
-__device__ __forceinline__ void tma_prefetch_2d(const void *tmap, int x, int y) {
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                     reinterpret_cast<uint64_t>(tmap)),
-                 "r"(x), "r"(y)
-                 : "memory");
-}
 // Bring a tensor map into the descriptor cache ahead of its first use.
 __device__ __forceinline__ void tma_prefetch_map(const void *tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");

@@ -224,8 +224,9 @@ def test_prefill_workspace_required(lib):
     n = ctypes.c_size_t(0)
     assert lib.gdr_prefill_workspace_size(ctypes.byref(a), ctypes.byref(n)) == OK
     assert n.value >= 16 + 4 * a.n_seq
-    # 3 sequences of 5, 0, 9 tokens = 2 chunks of 64 for each of 4 value heads.
-    assert n.value >= 2 * 4 * 65536
+    # 3 sequences of 5, 0, 9 tokens = 2 chunks of 64 for each of 4 value heads,
+    # each with a record holding at least W, P and T diag(beta) (16 KB tiles).
+    assert n.value >= 2 * 4 * 3 * 16384
     assert lib.gdr_prefill_chunked(ctypes.byref(a), None, 0, None) == WORKSPACE
     # Below the one-kernel minimum (16 + 4 n_seq, rounded up to 256 bytes).
     assert lib.gdr_prefill_chunked(ctypes.byref(a), FAKE + (12 << 32), 255, None) == WORKSPACE

@@ -20,8 +20,9 @@
 //                   S       = e^{gamma_L} S + (Delta^T diag(e^{gamma_L-gamma} n)) K
 //                   y       = RMSNormGated(O)
 //
-// Arithmetic, operand precisions (bf16 MMAs, hi + lo pairs for T, P, Delta)
-// and layouts are those of the one-kernel version in gdr_prefill_tc.cu.
+// Operand precisions (bf16 MMAs, hi + lo pairs for T, P, Delta) are those of
+// the one-kernel version in gdr_prefill_tc.cu; the output gate here takes its
+// sigmoid from tanh.approx (tanh_approx below) where that version divides.
 #include "gdr_prefill_common.cuh"
 #include "gdr_tmap.cuh"
 

@@ -74,6 +74,9 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *cu, int n_seq
                                                     int *seg_off) {
     __shared__ int part[1024];
     const int tid = threadIdx.x;
+    // The first prep grid may be scheduled now; it waits for this grid before
+    // it reads what this grid writes.
+    release_dependents();
     if (tid == 0) *status = 0;
     for (int s = tid; s < n_seq; s += 1024) {
         const int ls = cu[s + 1] - cu[s];
@@ -198,13 +201,16 @@ __device__ __forceinline__ PrepUnit prep_unit(const int *seg_off, int seg_lo, in
 // segment's recurrence; the block of the highest index waits for it before
 // exiting, so that this grid completes only after it (the next recurrence
 // segment, queued after this grid, reads the state it carries).
+// wait_prev_at_start: launched as a programmatic dependent of the plan
+// kernel (the first segment); every block waits for it before reading the
+// order and offsets it writes.
 // K, Q and V come by tensor copies (maps) into 128-byte-swizzled tiles.
 __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
                                                      const __grid_constant__ PrepMaps maps,
                                                      const int *chunk_off,
                                                      const int *seg_off, int seg_lo,
                                                      unsigned char *records, int *status,
-                                                     int wait_prev_at_exit) {
+                                                     int wait_prev_at_exit, int wait_prev_at_start) {
     extern __shared__ __align__(1024) unsigned char sm_raw[];
     // The swizzled tiles must start on a 1024-byte boundary (A_SMEM_LAUNCH
     // leaves room to round up).
@@ -214,6 +220,7 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
     const int quad = warp & 3, part = warp >> 2;
     const int hv = blockIdx.x % p.H_v;
     const int hk = hv / p.hv_per_hk;
+    if (wait_prev_at_start) wait_for_predecessor();
     const PrepUnit pu = prep_unit(seg_off, seg_lo, p.n_seq, blockIdx.x / p.H_v);
     const int seq = pu.seq;
     const int gchunk = chunk_off[seq] + pu.chunk;
@@ -1277,9 +1284,12 @@ cudaError_t launch_prefill_tc2p(const PrefillParams &p, const int32_t *cu_host, 
             attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
             attr[0].val.programmaticStreamSerializationAllowed = 1;
             cfg.attrs = attr;
-            cfg.numAttrs = k > 0 ? 1 : 0;  // later segments overlap the recurrence before them
+            // Programmatic dependents: the first segment's prep of the plan
+            // kernel, the later ones of the recurrence before them (which they
+            // overlap).
+            cfg.numAttrs = 1;
             e = cudaLaunchKernelEx(&cfg, tcp2::prep_kernel, p, maps, (const int *)chunk_off, seg_off_k,
-                                   sp.lo[k], records, status, k > 0 ? 1 : 0);
+                                   sp.lo[k], records, status, k > 0 ? 1 : 0, k == 0 ? 1 : 0);
             if (e != cudaSuccess) {
                 (void)cudaGetLastError();
                 return e;

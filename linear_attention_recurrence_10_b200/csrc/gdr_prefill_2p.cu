@@ -643,6 +643,14 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p,
     // shortens it) and the CTA then unwinds: status word, copies, TMEM.
     const uint64_t wait_ns = p.wait_ns ? p.wait_ns : kWaitNs;
     auto scal = [&](int c) { return reinterpret_cast<const float *>(sm + B_SC + (c & 1) * SC_BYTES); };
+    // Bytes [src_off, src_off + bytes) of chunk c's record into shared memory at
+    // dst, landing on bar (issued by lane 0 of a producer warp).
+    auto bulk = [&](uint32_t dst, uint32_t src_off, uint32_t bytes, uint64_t *bar, int c) {
+        if (lane == 0) {
+            bulk_expect(bar, bytes);
+            bulk_copy(sm + dst, rec0 + (size_t)c * rec_step + src_off, bytes, bar);
+        }
+    };
 
     if (warp == 0) tmem_alloc(tmem_slot, 512);
     if (tid == 0) {
@@ -792,12 +800,6 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p,
             __syncwarp();
             if (lane == 0) mbar_arrive(bar);
         };
-        auto bulk = [&](uint32_t dst, uint32_t src_off, uint32_t bytes, uint64_t *bar, int c) {
-            if (lane == 0) {
-                bulk_expect(bar, bytes);
-                bulk_copy(sm + dst, rec0 + (size_t)c * rec_step + src_off, bytes, bar);
-            }
-        };
         // V of chunk c (two 128-byte-swizzled boxes: tensor copies, or for a
         // ragged last chunk 16-byte copies that read zero past its end, waited
         // for here) and its T diag(beta) tiles from the record, on bar_u.
@@ -868,12 +870,6 @@ __global__ void __launch_bounds__(RNT, 1) recur_kernel(const PrefillParams p,
         // group, a chunk behind; on a warp of their own these waits no longer
         // hold up the copies the state path waits for.
         int n_p = 0, n_sc[2] = {0, 0};
-        auto bulk = [&](uint32_t dst, uint32_t src_off, uint32_t bytes, uint64_t *bar, int c) {
-            if (lane == 0) {
-                bulk_expect(bar, bytes);
-                bulk_copy(sm + dst, rec0 + (size_t)c * rec_step + src_off, bytes, bar);
-            }
-        };
         bool ok = true;
         for (int c = 0; c < n_chunks && c < 2; ++c) {
             bulk(B_SC + (c & 1) * SC_BYTES, REC_SCAL, SC_BYTES, bar_sc + (c & 1), c);

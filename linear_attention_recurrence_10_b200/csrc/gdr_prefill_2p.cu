@@ -289,7 +289,8 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
 
     // Norms (one row of [K;Q] per thread) and the running sums of g.
     if (tid < 128) {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        // Sums of squares in pairs (two-wide FMA), four pair accumulators.
+        float2 acc[4] = {};
 #pragma unroll
         for (int jc = 0; jc < 16; ++jc) {
             const uint4 raw =
@@ -298,10 +299,11 @@ __global__ void __launch_bounds__(PNT, 3) prep_kernel(const PrefillParams p,
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const float2 f = __bfloat1622float2(h2[u]);
-                acc[u] = fmaf(f.x, f.x, fmaf(f.y, f.y, acc[u]));
+                acc[u] = __ffma2_rn(f, f, acc[u]);
             }
         }
-        const float ss = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        const float ss = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
+                         ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
         const int r = tid & 63;
         const float f = p.qk_l2norm ? rsqrtf(ss + p.eps_l2) : 1.0f;
         if (tid < 64) sc.nk[r] = r < L ? f : 0.f;

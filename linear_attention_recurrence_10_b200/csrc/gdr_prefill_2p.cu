@@ -572,6 +572,13 @@ constexpr uint32_t B_BAR = 198656;             // 18 mbarriers, then the TMEM ad
 constexpr uint32_t B_SMEM = B_BAR + 160;
 constexpr uint32_t B_SMEM_LAUNCH = B_SMEM + 1024;  // with the alignment slack
 constexpr uint32_t SC_BYTES = REC_TB - REC_SCAL;
+// The stages in order and apart; 18 mbarriers and the TMEM address after them.
+static_assert(B_KQ + 32768 <= B_W && B_W + 16384 <= B_P && B_P + 16384 <= B_SC &&
+                  B_SC + 2 * SC_BYTES <= B_DL && B_DL + 32768 <= B_V && B_V + 16384 <= B_TB &&
+                  B_TB + 16384 <= B_OS && B_OS + C * D * 4 <= B_BAR &&
+                  B_BAR + 18 * 8 + 4 <= B_SMEM && B_SMEM_LAUNCH <= 227 * 1024,
+              "recurrence shared-memory layout");
+static_assert(B_KQ % 1024 == 0 && B_V % 1024 == 0, "128-byte-swizzled tiles start on 1024 bytes");
 // TMEM columns: the fp32 state, Delta^T = U^T - S W^T (the U product first,
 // then -S W^T onto it), two buffers of S Q^T, one of P Delta, and the bf16 copy
 // of S (two values per column) that -S W^T and S Q^T read as their A operand.
